@@ -1,0 +1,299 @@
+"""fp64 CPU oracle for block-sparse video self-attention -- TEST INFRASTRUCTURE.
+
+Only the tests, ``__graft_entry__.smoke()`` and the benchmark's CPU-baseline
+leg may import this package.  It shares no code with the CUDA library and
+never calls it.  The arithmetic lives in ``vsa_oracle.c`` (plain C, double
+precision); this module only moves numpy arrays in and out and loops over
+(batch, head), in the order the "Adaptive tiling (SPADE)" Recipe composes the
+steps: choose a tiling per head, permute, score, select, attend, permute back.
+
+Inputs are taken as float32 numpy arrays (or torch tensors), which carry bf16
+and fp32 values exactly.
+"""
+
+from __future__ import annotations
+
+import ctypes
+import os
+from typing import Optional, Sequence
+
+import numpy as np
+
+from . import build as _build
+
+_lib = None
+
+
+def lib():
+    global _lib
+    if _lib is None:
+        path = _build.build()
+        L = ctypes.CDLL(path)
+        P = ctypes.c_void_p
+        i64, i32, dbl = ctypes.c_int64, ctypes.c_int, ctypes.c_double
+        L.orc_tile_labels.argtypes = [i32] * 6 + [P]
+        L.orc_tile_permutation.argtypes = [i32] * 6 + [P]
+        L.orc_permute_rows.argtypes = [P, i64, i32, P, P]
+        L.orc_unpermute_rows.argtypes = [P, i64, i32, P, P]
+        L.orc_tile_sics.argtypes = [P] + [i32] * 7 + [P]
+        L.orc_select_tiling.argtypes = [P, i32, i32, i32, i32, P, i32, P]
+        L.orc_select_tiling.restype = i32
+        L.orc_block_minmax.argtypes = [P, i64, i32, i32, P, P]
+        L.orc_block_scores.argtypes = [P, P, P, P, i64, i32, P]
+        L.orc_topk_block_list.argtypes = [P, i64, i32, i32, i32, i32, P, P]
+        L.orc_topk_block_list.restype = i32
+        L.orc_tile_neighbourhood_list.argtypes = [i32] * 11 + [P, P, P]
+        L.orc_tile_neighbourhood_list.restype = i32
+        L.orc_window_attention.argtypes = [P, P, P, i64, i32, i32, i32, dbl, i32, P, i64, P]
+        L.orc_block_sparse_attention.argtypes = [P, P, P, i64, i32, i32, P, P, i32, i32, dbl, P, i64, P]
+        L.orc_window_key_ranges.argtypes = [i64] * 5 + [P]
+        L.orc_window_key_ranges.restype = i32
+        _lib = L
+    return _lib
+
+
+def _f32(x) -> np.ndarray:
+    if hasattr(x, "detach"):
+        x = x.detach().to("cpu").float().numpy()
+    return np.ascontiguousarray(x, dtype=np.float32)
+
+
+def _ptr(a: np.ndarray):
+    return a.ctypes.data_as(ctypes.c_void_p)
+
+
+def default_scale(D: int, scale: Optional[float]) -> float:
+    """_default_scale: the explicit scale, else D ** -0.5."""
+    if scale is not None and scale > 0:
+        return float(scale)
+    if D <= 0:
+        raise ValueError("head_dim must be positive")
+    return float(D) ** -0.5
+
+
+# --------------------------------------------------------------------------
+# permutation
+# --------------------------------------------------------------------------
+
+def tile_labels(grid, tile) -> np.ndarray:
+    T, H, W = grid
+    out = np.empty(T * H * W, dtype=np.int64)
+    lib().orc_tile_labels(T, H, W, *tile, _ptr(out))
+    return out
+
+
+def tile_permutation(grid, tile) -> np.ndarray:
+    T, H, W = grid
+    out = np.empty(T * H * W, dtype=np.int64)
+    lib().orc_tile_permutation(T, H, W, *tile, _ptr(out))
+    return out
+
+
+def permute_rows(x, perm) -> np.ndarray:
+    x = _f32(x)
+    S, D = x.shape
+    y = np.empty_like(x)
+    lib().orc_permute_rows(_ptr(x), S, D, _ptr(np.ascontiguousarray(perm, np.int64)), _ptr(y))
+    return y
+
+
+def unpermute_rows(y, perm) -> np.ndarray:
+    y = _f32(y)
+    S, D = y.shape
+    x = np.empty_like(y)
+    lib().orc_unpermute_rows(_ptr(y), S, D, _ptr(np.ascontiguousarray(perm, np.int64)), _ptr(x))
+    return x
+
+
+# --------------------------------------------------------------------------
+# tiling choice
+# --------------------------------------------------------------------------
+
+def tile_sics(q, grid, tile) -> np.ndarray:
+    """SICS of every tile of one tiling, for one head's q [S, D]."""
+    q = _f32(q)
+    T, H, W = grid
+    n = (T * H * W) // (tile[0] * tile[1] * tile[2])
+    out = np.empty(n, dtype=np.float64)
+    lib().orc_tile_sics(_ptr(q), T, H, W, q.shape[1], *tile, _ptr(out))
+    return out
+
+
+def select_tiling(q, grid, tiles):
+    """(choice, cohesion[n_tiles]) for one head's q [S, D]."""
+    q = _f32(q)
+    T, H, W = grid
+    t = np.ascontiguousarray(np.array(tiles, dtype=np.int32).reshape(-1))
+    sc = np.empty(len(tiles), dtype=np.float64)
+    c = lib().orc_select_tiling(_ptr(q), T, H, W, q.shape[1], _ptr(t), len(tiles), _ptr(sc))
+    return int(c), sc
+
+
+# --------------------------------------------------------------------------
+# summaries, scores, top-k, structured lists
+# --------------------------------------------------------------------------
+
+def block_minmax(xp, block: int):
+    xp = _f32(xp)
+    S, D = xp.shape
+    nb = S // block
+    mx = np.empty((nb, D), np.float64)
+    mn = np.empty((nb, D), np.float64)
+    lib().orc_block_minmax(_ptr(xp), S, D, block, _ptr(mx), _ptr(mn))
+    return mx, mn
+
+
+def block_scores(qmax, qmin, kmax, kmin) -> np.ndarray:
+    a = [np.ascontiguousarray(x, np.float64) for x in (qmax, qmin, kmax, kmin)]
+    nb, D = a[0].shape
+    s = np.empty((nb, nb), np.float64)
+    lib().orc_block_scores(*(_ptr(x) for x in a), nb, D, _ptr(s))
+    return s
+
+
+def list_cap(nb: int, k: int, n_sink: int, diag_halfwidth: int) -> int:
+    return min(nb, k + n_sink + 2 * diag_halfwidth + 1)
+
+
+def topk_block_list(score, k: int, n_sink: int = 1, diag_halfwidth: int = 0,
+                    cap: Optional[int] = None):
+    s = np.ascontiguousarray(score, np.float64)
+    nb = s.shape[0]
+    cap = cap if cap is not None else list_cap(nb, k, n_sink, diag_halfwidth)
+    idx = np.empty((nb, cap), np.int32)
+    cnt = np.empty(nb, np.int32)
+    rc = lib().orc_topk_block_list(_ptr(s), nb, k, n_sink, diag_halfwidth, cap, _ptr(idx), _ptr(cnt))
+    if rc != 0:
+        raise ValueError("cap too small for the top-k list")
+    return idx, cnt
+
+
+STRUCTURED_KINDS = ("spatial", "temporal", "sliding_tile")
+
+
+def structured_tile(kind: str, grid, tile=(4, 8, 8), radius=(1, 1, 1)):
+    """(tile, radius) of a structured mask: spatial_only = same frame,
+    temporal_only = same (h, w), sliding_tile = tile neighbourhood."""
+    T, H, W = grid
+    if kind == "spatial":
+        return (1, H, W), (0, 0, 0)
+    if kind == "temporal":
+        return (T, 1, 1), (0, 0, 0)
+    if kind == "sliding_tile":
+        return tuple(tile), tuple(radius)
+    raise ValueError(kind)
+
+
+def tile_neighbourhood_list(grid, tile, radius, block: int, cap: Optional[int] = None):
+    T, H, W = grid
+    S = T * H * W
+    nb = S // block
+    if cap is None:
+        cap = nb
+    idx = np.empty((nb, cap), np.int32)
+    cnt = np.empty(nb, np.int32)
+    g = ctypes.c_int(0)
+    rc = lib().orc_tile_neighbourhood_list(T, H, W, *tile, *radius, block, cap,
+                                           _ptr(idx), _ptr(cnt), ctypes.byref(g))
+    if rc != 0:
+        raise ValueError(f"unsupported tile/radius/block combination (rc={rc})")
+    used = int(cnt.max())
+    return idx[:, :used].copy() if cap == nb else idx, cnt, int(g.value)
+
+
+# --------------------------------------------------------------------------
+# attention
+# --------------------------------------------------------------------------
+
+def _rows(rows, S):
+    if rows is None:
+        return np.arange(S, dtype=np.int64)
+    return np.ascontiguousarray(rows, np.int64)
+
+
+def window_attention(q, k, v, window: int, sink: int = 0, scale=None, rows=None):
+    """windowed_attention for one head [S, D]; returns rows x D doubles."""
+    q, k, v = _f32(q), _f32(k), _f32(v)
+    S, D = q.shape
+    r = _rows(rows, S)
+    out = np.empty((len(r), D), np.float64)
+    lib().orc_window_attention(_ptr(q), _ptr(k), _ptr(v), S, D, window, sink,
+                               default_scale(D, scale), 0, _ptr(r), len(r), _ptr(out))
+    return out
+
+
+def dense_attention(q, k, v, scale=None, rows=None):
+    """full_attention for one head [S, D]."""
+    q, k, v = _f32(q), _f32(k), _f32(v)
+    S, D = q.shape
+    r = _rows(rows, S)
+    out = np.empty((len(r), D), np.float64)
+    lib().orc_window_attention(_ptr(q), _ptr(k), _ptr(v), S, D, 1, 0,
+                               default_scale(D, scale), 1, _ptr(r), len(r), _ptr(out))
+    return out
+
+
+def block_sparse_attention(qp, kp, vp, idx, cnt, block: int, group_size: int = 0,
+                           scale=None, rows=None):
+    """Block-list attention for one head in the permuted order."""
+    qp, kp, vp = _f32(qp), _f32(kp), _f32(vp)
+    S, D = qp.shape
+    idx = np.ascontiguousarray(idx, np.int32)
+    cnt = np.ascontiguousarray(cnt, np.int32)
+    r = _rows(rows, S)
+    out = np.empty((len(r), D), np.float64)
+    lib().orc_block_sparse_attention(_ptr(qp), _ptr(kp), _ptr(vp), S, D, block,
+                                     _ptr(idx), _ptr(cnt), idx.shape[1], group_size,
+                                     default_scale(D, scale), _ptr(r), len(r), _ptr(out))
+    return out
+
+
+def window_key_ranges(qs: int, qe: int, S: int, half: int, sink: int):
+    out = np.zeros(4, np.int64)
+    n = lib().orc_window_key_ranges(qs, qe, S, half, sink, _ptr(out))
+    return [(int(out[2 * i]), int(out[2 * i + 1])) for i in range(n)]
+
+
+# --------------------------------------------------------------------------
+# the SPADE composition for one head
+# --------------------------------------------------------------------------
+
+def spade_head(q, k, v, grid, tiles, k_blocks: int, n_sink: int = 1,
+               diag_halfwidth: int = 0, scale=None, query_blocks=None):
+    """Adaptive tiling -> permutation -> min/max scores -> top-k + sink +
+    diagonal -> block-sparse attention -> inverse permutation, for one head.
+
+    Returns a dict with every intermediate.  With ``query_blocks`` only those
+    query blocks (in the permuted order) are attended; ``out_perm`` then holds
+    just their rows and ``out`` is None.
+    """
+    q, k, v = _f32(q), _f32(k), _f32(v)
+    choice, cohesion = select_tiling(q, grid, tiles) if len(tiles) > 1 else (0, None)
+    tile = tiles[choice]
+    block = tile[0] * tile[1] * tile[2]
+    perm = tile_permutation(grid, tile)
+    qp, kp, vp = (permute_rows(x, perm) for x in (q, k, v))
+    qmax, qmin = block_minmax(qp, block)
+    kmax, kmin = block_minmax(kp, block)
+    score = block_scores(qmax, qmin, kmax, kmin)
+    idx, cnt = topk_block_list(score, k_blocks, n_sink, diag_halfwidth)
+    res = dict(choice=choice, cohesion=cohesion, perm=perm, block=block,
+               qmax=qmax, qmin=qmin, kmax=kmax, kmin=kmin, score=score,
+               idx=idx, cnt=cnt)
+    if query_blocks is None:
+        op = block_sparse_attention(qp, kp, vp, idx, cnt, block, 0, scale)
+        res["out_perm"] = op
+        res["out"] = _unpermute64(op, perm)
+    else:
+        rows = np.concatenate([np.arange(b * block, (b + 1) * block) for b in query_blocks])
+        res["out_perm"] = block_sparse_attention(qp, kp, vp, idx, cnt, block, 0, scale, rows)
+        res["rows"] = rows
+        res["out"] = None
+    return res
+
+
+def _unpermute64(y: np.ndarray, perm: np.ndarray) -> np.ndarray:
+    """x[perm[p]] = y[p] for double rows (the inverse permutation)."""
+    x = np.empty_like(y)
+    x[perm] = y
+    return x

@@ -1,0 +1,401 @@
+"""Pins of the fp64 oracle to what the pages and the mathematics fix.
+
+Each test checks the oracle against something other than itself: worked
+examples done by hand (tests/golden), coordinate properties that determine a
+result uniquely, brute force over tiny inputs, or special cases that reduce to
+a library routine (torch scaled_dot_product_attention in fp64, numpy).
+"""
+
+import itertools
+import json
+import math
+import os
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from workloads import integer_grid, smooth_qkv
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
+
+
+def _coords(grid):
+    T, H, W = grid
+    i = np.arange(T * H * W)
+    return i // (H * W), (i // W) % H, i % W
+
+
+def _sdpa64(q, k, v, scale, mask=None):
+    """torch SDPA in fp64 on the CPU; mask is a bool [S, S] (True = visible)."""
+    q, k, v = (torch.as_tensor(np.asarray(x, np.float64))[None, None] for x in (q, k, v))
+    m = None if mask is None else torch.as_tensor(mask)[None, None]
+    o = torch.nn.functional.scaled_dot_product_attention(q, k, v, attn_mask=m, scale=scale)
+    return o[0, 0].numpy()
+
+
+# --------------------------------------------------------------------------
+# permutation (ADR step 6; SPADE Recipe: argsort of tile labels)
+# --------------------------------------------------------------------------
+
+@pytest.mark.parametrize("grid,tile", [((4, 8, 8), (2, 4, 4)), ((3, 4, 6), (1, 2, 3)),
+                                       ((4, 6, 10), (4, 1, 1)), ((2, 4, 4), (1, 4, 4)),
+                                       ((6, 6, 8), (3, 2, 4))])
+def test_permutation_determined_by_coordinates(grid, tile):
+    """Runs of tile-volume positions hold exactly one tile each, tiles in
+    row-major tile order, tokens inside a tile in ascending T-major order,
+    and every token appears once."""
+    perm = oracle.tile_permutation(grid, tile)
+    S = grid[0] * grid[1] * grid[2]
+    vol = tile[0] * tile[1] * tile[2]
+    assert sorted(perm.tolist()) == list(range(S))
+    t, h, w = _coords(grid)
+    ntile = (grid[1] // tile[1], grid[2] // tile[2])
+    for r in range(S // vol):
+        run = perm[r * vol:(r + 1) * vol]
+        ct, ch, cw = t[run] // tile[0], h[run] // tile[1], w[run] // tile[2]
+        assert len(set(zip(ct, ch, cw))) == 1
+        assert (ct[0] * ntile[0] + ch[0]) * ntile[1] + cw[0] == r
+        assert np.all(np.diff(run) > 0)
+
+
+def test_unpermute_inverts_permute():
+    grid, tile = (4, 8, 8), (2, 4, 4)
+    x = integer_grid((256, 64), seed=5, dtype=torch.float32).numpy()
+    perm = oracle.tile_permutation(grid, tile)
+    y = oracle.permute_rows(x, perm)
+    assert np.array_equal(oracle.unpermute_rows(y, perm), x)
+    assert np.array_equal(y, x[perm])
+    assert not np.array_equal(y, x)
+
+
+def test_identity_permutation_for_whole_frames():
+    """A (1, H, W) tile is a whole frame: T-major order is already tile order."""
+    perm = oracle.tile_permutation((5, 4, 6), (1, 4, 6))
+    assert np.array_equal(perm, np.arange(120))
+
+
+# --------------------------------------------------------------------------
+# SICS and the tiling choice (SPADE step 1; block_self_similarity; select_tiling)
+# --------------------------------------------------------------------------
+
+def test_sics_golden():
+    g = json.load(open(os.path.join(GOLDEN, "sics_tiny.json")))
+    got = oracle.tile_sics(np.array(g["q"], np.float32), tuple(g["grid"]), tuple(g["tile"]))
+    np.testing.assert_allclose(got, g["tile_sics"], rtol=0, atol=1e-15)
+
+
+def _pairwise_mean_cos(x):
+    """Brute force: mean cosine over distinct ordered pairs of non-zero rows."""
+    x = np.asarray(x, np.float64)
+    x = x[np.linalg.norm(x, axis=1) > 0]
+    m = len(x)
+    if m < 2:
+        return 0.0
+    tot = 0.0
+    for i in range(m):
+        for j in range(m):
+            if i != j:
+                tot += x[i] @ x[j] / (np.linalg.norm(x[i]) * np.linalg.norm(x[j]))
+    return tot / (m * (m - 1))
+
+
+@pytest.mark.parametrize("grid,tile", [((2, 4, 4), (1, 2, 2)), ((4, 4, 4), (2, 2, 1)),
+                                       ((2, 2, 8), (2, 2, 4))])
+def test_sics_brute_force(grid, tile):
+    S = grid[0] * grid[1] * grid[2]
+    q = np.random.default_rng(3).normal(size=(S, 8)).astype(np.float32)
+    q[5] = 0.0  # one zero-norm query, excluded
+    got = oracle.tile_sics(q, grid, tile)
+    t, h, w = _coords(grid)
+    nth, ntw = grid[1] // tile[1], grid[2] // tile[2]
+    lab = ((t // tile[0]) * nth + h // tile[1]) * ntw + w // tile[2]
+    want = [_pairwise_mean_cos(q[lab == c]) for c in range(len(got))]
+    np.testing.assert_allclose(got, want, rtol=1e-12, atol=1e-12)
+
+
+def test_sics_special_cases():
+    # constant direction: 1; m = 2: the plain cosine
+    grid, tile = (1, 1, 4), (1, 1, 2)
+    q = np.array([[1, 2, 3], [2, 4, 6], [1, 0, 1], [0, 1, 1]], np.float32)
+    got = oracle.tile_sics(q, grid, tile)
+    assert got[0] == pytest.approx(1.0, abs=1e-15)
+    assert got[1] == pytest.approx(0.5, abs=1e-15)  # cos((1,0,1),(0,1,1)) = 1/2
+
+
+def test_select_tiling_picks_the_cohesive_tiling_and_breaks_ties_low():
+    grid = (4, 4, 4)
+    t, h, w = _coords(grid)
+    rng = np.random.default_rng(0)
+    # every frame is one direction, frames differ: whole-frame tiles are cohesive
+    dirs = rng.normal(size=(4, 16))
+    q = dirs[t].astype(np.float32)
+    tiles = [(4, 1, 1), (1, 4, 4), (2, 2, 2)]
+    choice, sc = oracle.select_tiling(q, grid, tiles)
+    assert choice == 1 and sc[1] == pytest.approx(1.0)
+    # identical candidates tie exactly: the lower index wins
+    choice, sc = oracle.select_tiling(q, grid, [(2, 2, 2), (2, 2, 2), (1, 4, 4)])
+    assert choice == 2
+    choice, sc = oracle.select_tiling(q, grid, [(2, 2, 2), (2, 2, 2)])
+    assert choice == 0 and sc[0] == sc[1]
+
+
+def test_self_pair_reading_gives_the_same_choice():
+    """Counting self-pairs maps SICS to (m-1)/m * SICS + 1/m: monotone for a
+    common tile volume, so the choice does not depend on that reading."""
+    grid = (4, 8, 8)
+    q, _, _ = smooth_qkv(1, 2, grid, 32, seed=11, kinds=["spatial", "temporal"],
+                         dtype=torch.float32)
+    tiles = [(1, 4, 8), (2, 4, 4), (4, 2, 4)]
+    for hd in range(2):
+        c, sc = oracle.select_tiling(q[0, hd], grid, tiles)
+        m = 32
+        alt = (m - 1) / m * sc + 1 / m
+        assert int(np.argmax(alt)) == c
+
+
+# --------------------------------------------------------------------------
+# summaries and scores (SPADE step 3; minmax_block_scores)
+# --------------------------------------------------------------------------
+
+def test_block_scores_golden():
+    g = json.load(open(os.path.join(GOLDEN, "block_scores_tiny.json")))
+    qmax, qmin = oracle.block_minmax(np.array(g["q"], np.float32), g["block"])
+    kmax, kmin = oracle.block_minmax(np.array(g["k"], np.float32), g["block"])
+    assert np.array_equal(qmax, g["q_max"]) and np.array_equal(qmin, g["q_min"])
+    assert np.array_equal(kmax, g["k_max"]) and np.array_equal(kmin, g["k_min"])
+    s = oracle.block_scores(qmax, qmin, kmax, kmin)
+    assert np.array_equal(s, g["scores"])
+    idx, cnt = oracle.topk_block_list(s, 1, n_sink=0, diag_halfwidth=-1, cap=1)
+    assert idx.tolist() == g["top1_plain"]
+    idx, cnt = oracle.topk_block_list(s, 1, n_sink=1, diag_halfwidth=0, cap=2)
+    assert idx.tolist() == g["top1_sink_diag"] and cnt.tolist() == [2, 2]
+
+
+def test_block_minmax_against_numpy():
+    x = integer_grid((512, 64), seed=9, dtype=torch.float32).numpy()
+    mx, mn = oracle.block_minmax(x, 32)
+    r = x.reshape(16, 32, 64).astype(np.float64)
+    assert np.array_equal(mx, r.max(1)) and np.array_equal(mn, r.min(1))
+
+
+def test_singleton_blocks_reduce_to_twice_the_dot_product():
+    """With one token per block, q_max = q_min = q and k_max = k_min = k, so
+    the score is 2 q . k."""
+    x = integer_grid((2, 40, 16), seed=4, dtype=torch.float32).numpy()
+    qmax, qmin = oracle.block_minmax(x[0], 1)
+    kmax, kmin = oracle.block_minmax(x[1], 1)
+    s = oracle.block_scores(qmax, qmin, kmax, kmin)
+    want = 2.0 * x[0].astype(np.float64) @ x[1].astype(np.float64).T
+    assert np.array_equal(s, want)
+
+
+def test_scores_symmetric_in_the_key_summaries_and_positively_homogeneous():
+    rng = np.random.default_rng(1)
+    a, b, c, d = (rng.normal(size=(6, 8)) for _ in range(4))
+    s = oracle.block_scores(a, b, c, d)
+    assert np.array_equal(s, oracle.block_scores(a, b, d, c))
+    np.testing.assert_allclose(oracle.block_scores(2 * a, 2 * b, c, d), 2 * s, rtol=1e-14)
+    assert not np.allclose(s, oracle.block_scores(a, b, -c, -d))
+
+
+# --------------------------------------------------------------------------
+# top-k + sink + diagonal (SPADE step 4; top_k_block_mask; recipe note)
+# --------------------------------------------------------------------------
+
+def _brute_topk(row, k):
+    """The unique k-subset whose every member outranks every non-member,
+    ranking by larger score, then lower index."""
+    nb = len(row)
+    key = lambda j: (-row[j], j)
+    found = []
+    for sub in itertools.combinations(range(nb), k):
+        rest = [j for j in range(nb) if j not in sub]
+        if not rest or max(key(j) for j in sub) < min(key(j) for j in rest):
+            found.append(set(sub))
+    assert len(found) == 1
+    return found[0]
+
+
+@pytest.mark.parametrize("seed", range(6))
+def test_topk_brute_force_with_ties(seed):
+    nb = 7
+    rng = np.random.default_rng(seed)
+    s = rng.integers(-2, 3, size=(nb, nb)).astype(np.float64)  # many ties
+    for k, n_sink, dhw in [(1, 0, -1), (2, 1, 0), (3, 2, 1), (nb, 1, 0)]:
+        idx, cnt = oracle.topk_block_list(s, k, n_sink, dhw, cap=nb)
+        for i in range(nb):
+            want = _brute_topk(s[i], k)
+            want |= {j for j in range(nb) if j < n_sink or abs(j - i) <= dhw}
+            got = idx[i, :cnt[i]].tolist()
+            assert got == sorted(want)
+            assert (idx[i, cnt[i]:] == -1).all()
+
+
+def test_sink_and_diagonal_always_present():
+    nb = 40
+    s = np.random.default_rng(2).normal(size=(nb, nb))
+    s[:, 0] = -1e9                      # the sink block never wins on score
+    np.fill_diagonal(s, -1e9)           # nor does the diagonal
+    idx, cnt = oracle.topk_block_list(s, 5, n_sink=1, diag_halfwidth=0)
+    for i in range(nb):
+        row = idx[i, :cnt[i]].tolist()
+        assert 0 in row and i in row
+        assert cnt[i] == (6 if i == 0 else 7)
+
+
+# --------------------------------------------------------------------------
+# structured masks (ADR step 1)
+# --------------------------------------------------------------------------
+
+def _expand_list_to_tmajor(idx, cnt, g, block, perm):
+    """Element mask in T-major order from a block list in the permuted order."""
+    S = len(perm)
+    m = np.zeros((S, S), bool)
+    for i in range(S // block):
+        for c in range(cnt[i]):
+            j = idx[i, c]
+            m[i * block:(i + 1) * block, j * block:(j + 1) * block] = True
+    if g > 0:
+        p = np.arange(S)
+        m &= (p[:, None] // g) == (p[None, :] // g)
+    out = np.zeros_like(m)
+    out[np.ix_(perm, perm)] = m
+    return out
+
+
+@pytest.mark.parametrize("grid,block", [((4, 4, 8), 32), ((2, 4, 8), 16), ((8, 4, 4), 16)])
+def test_spatial_and_temporal_lists_are_exactly_frame_and_pixel_masks(grid, block):
+    t, h, w = _coords(grid)
+    for kind, want in [("spatial", t[:, None] == t[None, :]),
+                       ("temporal", (h[:, None] == h[None, :]) & (w[:, None] == w[None, :]))]:
+        tile, rad = oracle.structured_tile(kind, grid)
+        idx, cnt, g = oracle.tile_neighbourhood_list(grid, tile, rad, block)
+        perm = oracle.tile_permutation(grid, tile)
+        got = _expand_list_to_tmajor(idx, cnt, g, block, perm)
+        assert np.array_equal(got, want), kind
+
+
+def test_sliding_tile_list_is_the_clipped_tile_neighbourhood():
+    grid, tile, block = (6, 12, 12), (2, 4, 4), 16
+    idx, cnt, g = oracle.tile_neighbourhood_list(grid, tile, (1, 1, 1), block)
+    perm = oracle.tile_permutation(grid, tile)
+    got = _expand_list_to_tmajor(idx, cnt, g, block, perm)
+    t, h, w = _coords(grid)
+    ct, ch, cw = t // 2, h // 4, w // 4
+    want = ((np.abs(ct[:, None] - ct[None, :]) <= 1) & (np.abs(ch[:, None] - ch[None, :]) <= 1)
+            & (np.abs(cw[:, None] - cw[None, :]) <= 1))
+    assert g == 0 and np.array_equal(got, want)
+    # a corner tile has 2*2*2 neighbours, an interior one 3*3*3; 2 blocks per tile
+    assert cnt.min() == 2 * 8 and cnt.max() == 2 * 27
+    for i in range(len(cnt)):
+        assert np.all(np.diff(idx[i, :cnt[i]]) > 0)
+
+
+# --------------------------------------------------------------------------
+# attention (windowed_attention / full_attention; recipe note: dropped blocks)
+# --------------------------------------------------------------------------
+
+def _qkv(S, D, seed):
+    q, k, v = (integer_grid((S, D), seed + o, torch.float32).numpy() for o in range(3))
+    return q, k, v
+
+
+@pytest.mark.parametrize("window", [64, 200, 257])
+def test_window_at_least_S_is_dense_sdpa(window):
+    q, k, v = _qkv(64, 16, 20)
+    scale = 16 ** -0.5
+    got = oracle.window_attention(q, k, v, window=window, sink=3)
+    want = _sdpa64(q, k, v, scale)
+    np.testing.assert_allclose(got, want, rtol=0, atol=1e-12)
+    np.testing.assert_allclose(oracle.dense_attention(q, k, v), want, rtol=0, atol=1e-12)
+
+
+@pytest.mark.parametrize("S,window,sink", [(64, 1, 0), (64, 9, 0), (64, 10, 5), (50, 31, 7),
+                                           (64, 63, 64), (37, 2, 37)])
+def test_window_matches_sdpa_with_the_docstring_mask(S, window, sink):
+    """Mask built from the module docstring's statement: sinks j in [0, sink)
+    and local j in [max(0, i - half), min(S, i + half + 1))."""
+    q, k, v = _qkv(S, 16, 30)
+    half = window // 2
+    m = np.zeros((S, S), bool)
+    for i in range(S):
+        m[i, :sink] = True
+        m[i, max(0, i - half):min(S, i + half + 1)] = True
+    got = oracle.window_attention(q, k, v, window=window, sink=sink, scale=0.3)
+    np.testing.assert_allclose(got, _sdpa64(q, k, v, 0.3, m), rtol=0, atol=1e-12)
+
+
+def test_window_formula_covers_everything_from_2S_minus_1():
+    """|i - j| <= floor(window/2) reaches every key once window >= 2S - 1."""
+    S = 40
+    q, k, v = _qkv(S, 8, 40)
+    half = (2 * S - 1) // 2
+    assert all(abs(i - j) <= half for i in range(S) for j in range(S))
+    got = oracle.window_attention(q, k, v, window=2 * S - 1, sink=0)
+    np.testing.assert_allclose(got, _sdpa64(q, k, v, 8 ** -0.5), atol=1e-12, rtol=0)
+
+
+def test_default_scale_is_inverse_sqrt_head_dim():
+    q, k, v = _qkv(32, 16, 50)
+    np.testing.assert_array_equal(oracle.dense_attention(q, k, v),
+                                  oracle.dense_attention(q, k, v, scale=0.25))
+    assert oracle.default_scale(64, None) == 0.125
+
+
+@pytest.mark.parametrize("S,chunk,half,sink", [(300, 128, 32, 16), (300, 64, 100, 0),
+                                               (513, 512, 7, 300), (90, 7, 3, 10)])
+def test_key_ranges_cover_exactly_the_chunk_union(S, chunk, half, sink):
+    """_key_ranges_for_block returns exactly the union, over the chunk's rows,
+    of the per-element visible keys, without overlap."""
+    for qs in range(0, S, chunk):
+        qe = min(S, qs + chunk)
+        ranges = oracle.window_key_ranges(qs, qe, S, half, sink)
+        got = [j for a, b in ranges for j in range(a, b)]
+        assert len(got) == len(set(got))
+        want = {j for i in range(qs, qe) for j in range(S) if j < sink or abs(i - j) <= half}
+        assert set(got) == want
+
+
+def test_block_list_attention_equals_sdpa_with_the_expanded_mask():
+    S, D, block = 96, 16, 16
+    q, k, v = _qkv(S, D, 60)
+    nb = S // block
+    rng = np.random.default_rng(7)
+    idx = np.full((nb, 4), -1, np.int32)
+    cnt = np.zeros(nb, np.int32)
+    m = np.zeros((S, S), bool)
+    for i in range(nb):
+        sel = sorted(set(rng.choice(nb, 3, replace=False).tolist()) | {i})
+        cnt[i] = len(sel)
+        idx[i, :len(sel)] = sel
+        for j in sel:
+            m[i * block:(i + 1) * block, j * block:(j + 1) * block] = True
+    got = oracle.block_sparse_attention(q, k, v, idx, cnt, block, 0, 0.2)
+    np.testing.assert_allclose(got, _sdpa64(q, k, v, 0.2, m), atol=1e-12, rtol=0)
+    # group mask: only keys of the query's own group of 4 tokens
+    g = 4
+    p = np.arange(S)
+    got = oracle.block_sparse_attention(q, k, v, idx, cnt, block, g, 0.2)
+    want = _sdpa64(q, k, v, 0.2, m & ((p[:, None] // g) == (p[None, :] // g)))
+    np.testing.assert_allclose(got, want, atol=1e-12, rtol=0)
+
+
+def test_all_blocks_budget_equals_dense_attention():
+    """k = number of blocks keeps every block: the SPADE composition must then
+    be dense attention in the original T-major order."""
+    grid = (4, 8, 8)
+    q, k, v = (integer_grid((256, 64), 70 + o, torch.float32).numpy() for o in range(3))
+    tiles = [(2, 4, 4), (1, 8, 4), (4, 2, 4)]
+    res = oracle.spade_head(q, k, v, grid, tiles, k_blocks=8)
+    assert (res["cnt"] == 8).all()
+    np.testing.assert_allclose(res["out"], _sdpa64(q, k, v, 64 ** -0.5), atol=1e-12, rtol=0)
+
+
+def test_sampled_rows_match_full_rows():
+    grid = (4, 8, 8)
+    q, k, v = (integer_grid((256, 64), 80 + o, torch.float32).numpy() for o in range(3))
+    full = oracle.spade_head(q, k, v, grid, [(2, 4, 4)], k_blocks=2)
+    part = oracle.spade_head(q, k, v, grid, [(2, 4, 4)], k_blocks=2, query_blocks=[0, 5, 7])
+    np.testing.assert_array_equal(part["out_perm"], full["out_perm"][part["rows"]])
