@@ -1,0 +1,372 @@
+// api.cu -- the C ABI of libvsa: argument validation (before any launch),
+// error reporting and dispatch to the kernels.
+//
+// Validation follows the pages' rules ("fastvideo/mlx_runtime/
+// windowed_attention.py": _validate_qkv, windowed_attention argument checks,
+// _default_scale; "Adaptive tiling (SPADE)", Deviations: divisible grids
+// only) and the limits of this implementation.
+#include <stdarg.h>
+#include <stdio.h>
+
+#include <string>
+
+#include "common.cuh"
+#include "internal.h"
+
+namespace vsa {
+
+namespace {
+thread_local std::string g_last_error;
+__device__ int g_status_word = 0;  // first device-side failure (see common.cuh)
+}  // namespace
+
+vsa_status fail(vsa_status s, const char *fmt, ...) {
+    char buf[512];
+    va_list ap;
+    va_start(ap, fmt);
+    vsnprintf(buf, sizeof(buf), fmt, ap);
+    va_end(ap);
+    g_last_error = buf;
+    return s;
+}
+
+vsa_status check_cuda(cudaError_t e, const char *what) {
+    if (e == cudaSuccess) return VSA_OK;
+    return fail(VSA_ERR_CUDA, "%s: %s", what, cudaGetErrorString(e));
+}
+
+int *device_status_word() {
+    static int *ptrs[128] = {};
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 128) return nullptr;
+    if (!ptrs[dev]) {
+        void *p = nullptr;
+        if (cudaGetSymbolAddress(&p, g_status_word) != cudaSuccess) return nullptr;
+        ptrs[dev] = static_cast<int *>(p);
+    }
+    return ptrs[dev];
+}
+
+}  // namespace vsa
+
+using namespace vsa;
+
+namespace {
+
+bool aligned16(const void *p) { return p != nullptr && (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+bool aligned4(const void *p) { return p != nullptr && (reinterpret_cast<uintptr_t>(p) & 3u) == 0; }
+int esize_of(vsa_dtype d) { return d == VSA_BF16 ? 2 : d == VSA_F32 ? 4 : 0; }
+cudaStream_t as_stream(void *s) { return static_cast<cudaStream_t>(s); }
+
+#define VSA_REQUIRE(cond, ...)                                   \
+    do {                                                         \
+        if (!(cond)) return fail(VSA_ERR_INVALID_ARGUMENT, __VA_ARGS__); \
+    } while (0)
+
+vsa_status check_grid(vsa_dims3 grid, int S) {
+    VSA_REQUIRE(grid.t > 0 && grid.h > 0 && grid.w > 0, "grid dimensions must be positive, got (%d, %d, %d)",
+                grid.t, grid.h, grid.w);
+    VSA_REQUIRE(static_cast<long long>(grid.t) * grid.h * grid.w == S,
+                "grid (%d, %d, %d) has %lld tokens but S = %d", grid.t, grid.h, grid.w,
+                static_cast<long long>(grid.t) * grid.h * grid.w, S);
+    return VSA_OK;
+}
+
+vsa_status check_tiles(vsa_dims3 grid, const vsa_dims3 *tiles, int n_tiles, TileSet *ts) {
+    VSA_REQUIRE(tiles != nullptr, "tiles must not be NULL");
+    VSA_REQUIRE(n_tiles >= 1 && n_tiles <= 8, "n_tiles must be in [1, 8], got %d", n_tiles);
+    ts->n = n_tiles;
+    for (int c = 0; c < n_tiles; ++c) {
+        const vsa_dims3 t = tiles[c];
+        VSA_REQUIRE(t.t > 0 && t.h > 0 && t.w > 0, "tile %d must be positive, got (%d, %d, %d)", c, t.t, t.h, t.w);
+        VSA_REQUIRE(grid.t % t.t == 0 && grid.h % t.h == 0 && grid.w % t.w == 0,
+                    "tile %d (%d, %d, %d) does not divide the grid (%d, %d, %d)", c, t.t, t.h, t.w, grid.t,
+                    grid.h, grid.w);
+        ts->t[c] = t.t;
+        ts->h[c] = t.h;
+        ts->w[c] = t.w;
+    }
+    for (int c = n_tiles; c < 8; ++c) ts->t[c] = ts->h[c] = ts->w[c] = 1;
+    return VSA_OK;
+}
+
+vsa_status check_bhsd(int B, int n_heads, int S, int D) {
+    VSA_REQUIRE(B >= 1 && n_heads >= 1, "B and n_heads must be >= 1, got %d, %d", B, n_heads);
+    VSA_REQUIRE(S >= 1, "sequence length S must be > 0, got %d", S);
+    VSA_REQUIRE(D >= 1, "head dim D must be > 0, got %d", D);
+    VSA_REQUIRE(static_cast<long long>(B) * n_heads <= 65535, "B * n_heads must be <= 65535");
+    return VSA_OK;
+}
+
+vsa_status check_d(int D) {
+    if (D != 64 && D != 128) return fail(VSA_ERR_UNSUPPORTED, "head dim D must be 64 or 128, got %d", D);
+    return VSA_OK;
+}
+
+bool overlaps(const void *a, const void *b, size_t n) {
+    const uintptr_t x = reinterpret_cast<uintptr_t>(a), y = reinterpret_cast<uintptr_t>(b);
+    return x < y + n && y < x + n;
+}
+
+#define VSA_TRY(expr)                     \
+    do {                                  \
+        vsa_status _s = (expr);           \
+        if (_s != VSA_OK) return _s;      \
+    } while (0)
+
+int *status_or_null() { return device_status_word(); }
+
+}  // namespace
+
+extern "C" {
+
+const char *vsa_last_error(void) { return g_last_error.c_str(); }
+
+vsa_status vsa_device_status(void *stream) {
+    cudaError_t e = cudaStreamSynchronize(as_stream(stream));
+    if (e != cudaSuccess) return check_cuda(e, "cudaStreamSynchronize");
+    int v = 0;
+    e = cudaMemcpyFromSymbol(&v, g_status_word, sizeof(int));
+    if (e != cudaSuccess) return check_cuda(e, "reading the device status word");
+    const int zero = 0;
+    e = cudaMemcpyToSymbol(g_status_word, &zero, sizeof(int));
+    if (e != cudaSuccess) return check_cuda(e, "clearing the device status word");
+    if (v == DEV_RUNTIME) return fail(VSA_ERR_RUNTIME, "a device-side check failed (invalid block list, choice or empty key set)");
+    if (v == DEV_TIMEOUT) return fail(VSA_ERR_TIMEOUT, "a bounded wait inside a kernel gave up");
+    if (v != 0) return fail(VSA_ERR_RUNTIME, "device status word holds %d", v);
+    return VSA_OK;
+}
+
+size_t vsa_select_tiling_workspace_size(int B, int n_heads, vsa_dims3 grid, const vsa_dims3 *tiles, int n_tiles) {
+    TileSet ts;
+    if (B < 1 || n_heads < 1 || grid.t < 1 || grid.h < 1 || grid.w < 1) return 0;
+    if (check_tiles(grid, tiles, n_tiles, &ts) != VSA_OK) return 0;
+    SelectGeom g;
+    if (!select_geometry(grid.t, grid.h, grid.w, ts, &g)) return 0;
+    const size_t bytes = static_cast<size_t>(B) * n_heads * g.n_regions * n_tiles * sizeof(float);
+    return (bytes + 255) & ~static_cast<size_t>(255);
+}
+
+vsa_status vsa_select_tiling(const void *q, vsa_dtype dtype, int B, int n_heads, int S, int D, vsa_dims3 grid,
+                             const vsa_dims3 *tiles, int n_tiles, int32_t *choice, float *sics, void *workspace,
+                             size_t workspace_bytes, void *stream) {
+    VSA_REQUIRE(esize_of(dtype) != 0, "dtype must be VSA_BF16 or VSA_F32");
+    VSA_TRY(check_bhsd(B, n_heads, S, D));
+    VSA_TRY(check_d(D));
+    VSA_REQUIRE(aligned16(q), "q must be a non-NULL 16-byte aligned device pointer");
+    VSA_REQUIRE(aligned4(choice), "choice must be a non-NULL 4-byte aligned device pointer");
+    VSA_REQUIRE(sics == nullptr || aligned4(sics), "sics must be NULL or 4-byte aligned");
+    VSA_TRY(check_grid(grid, S));
+    TileSet ts;
+    VSA_TRY(check_tiles(grid, tiles, n_tiles, &ts));
+    SelectGeom g;
+    if (!select_geometry(grid.t, grid.h, grid.w, ts, &g))
+        return fail(VSA_ERR_UNSUPPORTED,
+                    "the candidate tiles' lcm region holds %d cells of their gcd tile (at most 256 supported)",
+                    g.cells);
+    const size_t need = vsa_select_tiling_workspace_size(B, n_heads, grid, tiles, n_tiles);
+    VSA_REQUIRE(aligned16(workspace), "workspace must be a non-NULL 16-byte aligned device pointer");
+    VSA_REQUIRE(workspace_bytes >= need, "workspace holds %zu bytes, %zu needed", workspace_bytes, need);
+    return check_cuda(launch_select_tiling(q, esize_of(dtype), B * n_heads, S, D, grid.t, grid.h, grid.w, ts, g,
+                                           choice, sics, static_cast<float *>(workspace), status_or_null(),
+                                           as_stream(stream)),
+                      "select_tiling launch");
+}
+
+static vsa_status permute_common(const void *src, void *dst, vsa_dtype dtype, int B, int n_heads, int S, int D,
+                                 vsa_dims3 grid, const vsa_dims3 *tiles, int n_tiles, const int32_t *choice,
+                                 bool inverse, void *stream) {
+    VSA_REQUIRE(esize_of(dtype) != 0, "dtype must be VSA_BF16 or VSA_F32");
+    VSA_TRY(check_bhsd(B, n_heads, S, D));
+    VSA_TRY(check_d(D));
+    VSA_REQUIRE(aligned16(src) && aligned16(dst), "x and y must be non-NULL 16-byte aligned device pointers");
+    const size_t bytes = static_cast<size_t>(B) * n_heads * S * D * esize_of(dtype);
+    VSA_REQUIRE(!overlaps(src, dst, bytes), "x and y must not overlap");
+    VSA_REQUIRE(choice == nullptr || aligned4(choice), "choice must be NULL or 4-byte aligned");
+    VSA_TRY(check_grid(grid, S));
+    TileSet ts;
+    VSA_TRY(check_tiles(grid, tiles, n_tiles, &ts));
+    return check_cuda(launch_permute(src, dst, esize_of(dtype), B * n_heads, S, D, grid.t, grid.h, grid.w, ts,
+                                     choice, inverse, status_or_null(), as_stream(stream)),
+                      inverse ? "unpermute launch" : "permute launch");
+}
+
+vsa_status vsa_permute(const void *x, void *y, vsa_dtype dtype, int B, int n_heads, int S, int D, vsa_dims3 grid,
+                       const vsa_dims3 *tiles, int n_tiles, const int32_t *choice, void *stream) {
+    return permute_common(x, y, dtype, B, n_heads, S, D, grid, tiles, n_tiles, choice, false, stream);
+}
+
+vsa_status vsa_unpermute(const void *y, void *x, vsa_dtype dtype, int B, int n_heads, int S, int D, vsa_dims3 grid,
+                         const vsa_dims3 *tiles, int n_tiles, const int32_t *choice, void *stream) {
+    return permute_common(y, x, dtype, B, n_heads, S, D, grid, tiles, n_tiles, choice, true, stream);
+}
+
+vsa_status vsa_block_summaries(const void *x_perm, vsa_dtype dtype, int B, int n_heads, int S, int D, int block,
+                               void *x_max, void *x_min, void *stream) {
+    VSA_REQUIRE(esize_of(dtype) != 0, "dtype must be VSA_BF16 or VSA_F32");
+    VSA_TRY(check_bhsd(B, n_heads, S, D));
+    VSA_TRY(check_d(D));
+    VSA_REQUIRE(block == 16 || block == 32 || block == 64 || block == 128 || block == 256,
+                "block must be one of 16, 32, 64, 128, 256, got %d", block);
+    VSA_REQUIRE(S % block == 0, "block (%d) must divide S (%d)", block, S);
+    VSA_REQUIRE(aligned16(x_perm) && aligned16(x_max) && aligned16(x_min),
+                "x_perm, x_max and x_min must be non-NULL 16-byte aligned device pointers");
+    return check_cuda(launch_summaries(x_perm, esize_of(dtype), B * n_heads, S, D, block, x_max, x_min,
+                                       as_stream(stream)),
+                      "block_summaries launch");
+}
+
+vsa_status vsa_block_scores(const void *q_max, const void *q_min, const void *k_max, const void *k_min,
+                            vsa_dtype dtype, int B, int n_heads, int nb, int D, float *scores, void *stream) {
+    VSA_REQUIRE(esize_of(dtype) != 0, "dtype must be VSA_BF16 or VSA_F32");
+    VSA_TRY(check_bhsd(B, n_heads, nb, D));
+    VSA_TRY(check_d(D));
+    VSA_REQUIRE(aligned16(q_max) && aligned16(q_min) && aligned16(k_max) && aligned16(k_min),
+                "summaries must be non-NULL 16-byte aligned device pointers");
+    VSA_REQUIRE(aligned4(scores), "scores must be a non-NULL 4-byte aligned device pointer");
+    VSA_REQUIRE(static_cast<long long>(nb) <= 65535LL * 64, "nb too large");
+    return check_cuda(launch_scores(q_max, q_min, k_max, k_min, esize_of(dtype), B * n_heads, nb, D, scores,
+                                    as_stream(stream)),
+                      "block_scores launch");
+}
+
+vsa_status vsa_topk_block_mask(const float *scores, int B, int n_heads, int nb, int k, int n_sink_blocks,
+                               int diag_halfwidth, int32_t *idx, int32_t *cnt, int cap, void *stream) {
+    VSA_REQUIRE(B >= 1 && n_heads >= 1, "B and n_heads must be >= 1");
+    VSA_REQUIRE(nb >= 1, "nb must be >= 1, got %d", nb);
+    VSA_REQUIRE(k >= 1 && k <= nb, "k must be in [1, nb] = [1, %d], got %d", nb, k);
+    VSA_REQUIRE(n_sink_blocks >= 0 && n_sink_blocks <= nb, "n_sink_blocks must be in [0, nb], got %d",
+                n_sink_blocks);
+    VSA_REQUIRE(diag_halfwidth >= -1, "diag_halfwidth must be >= -1 (-1 = no diagonal), got %d", diag_halfwidth);
+    long long most = static_cast<long long>(k) + n_sink_blocks + (diag_halfwidth >= 0 ? 2LL * diag_halfwidth + 1 : 0);
+    if (most > nb) most = nb;
+    VSA_REQUIRE(cap >= most, "cap (%d) must be >= min(nb, k + n_sink + 2*diag_halfwidth + 1) = %lld", cap, most);
+    VSA_REQUIRE(aligned4(scores) && aligned4(idx) && aligned4(cnt),
+                "scores, idx and cnt must be non-NULL 4-byte aligned device pointers");
+    return check_cuda(launch_topk(scores, B * n_heads, nb, k, n_sink_blocks, diag_halfwidth, idx, cnt, cap,
+                                  as_stream(stream)),
+                      "topk launch");
+}
+
+vsa_status vsa_structured_block_list(vsa_mask_kind kind, vsa_dims3 grid, vsa_dims3 tile, vsa_dims3 radius, int block,
+                                     int32_t *idx, int32_t *cnt, int cap, int *group_size_out, void *stream) {
+    VSA_REQUIRE(grid.t > 0 && grid.h > 0 && grid.w > 0, "grid dimensions must be positive");
+    const long long S = static_cast<long long>(grid.t) * grid.h * grid.w;
+    VSA_REQUIRE(S < (1LL << 31), "grid too large");
+    if (kind == VSA_MASK_SPATIAL) {
+        tile = vsa_dims3{1, grid.h, grid.w};
+        radius = vsa_dims3{0, 0, 0};
+    } else if (kind == VSA_MASK_TEMPORAL) {
+        tile = vsa_dims3{grid.t, 1, 1};
+        radius = vsa_dims3{0, 0, 0};
+    } else {
+        VSA_REQUIRE(kind == VSA_MASK_SLIDING_TILE, "unknown mask kind %d", static_cast<int>(kind));
+    }
+    VSA_REQUIRE(tile.t > 0 && tile.h > 0 && tile.w > 0, "tile must be positive");
+    VSA_REQUIRE(grid.t % tile.t == 0 && grid.h % tile.h == 0 && grid.w % tile.w == 0,
+                "tile (%d, %d, %d) does not divide the grid (%d, %d, %d)", tile.t, tile.h, tile.w, grid.t, grid.h,
+                grid.w);
+    VSA_REQUIRE(radius.t >= 0 && radius.h >= 0 && radius.w >= 0, "radius must be >= 0");
+    VSA_REQUIRE(block == 32 || block == 64 || block == 128, "block must be 32, 64 or 128, got %d", block);
+    VSA_REQUIRE(S % block == 0, "block (%d) must divide S (%lld)", block, S);
+    VSA_REQUIRE(aligned4(idx) && aligned4(cnt), "idx and cnt must be non-NULL 4-byte aligned device pointers");
+    VSA_REQUIRE(group_size_out != nullptr, "group_size_out must not be NULL");
+    const long long vol = static_cast<long long>(tile.t) * tile.h * tile.w;
+    long long longest;
+    int group;
+    if (vol % block == 0) {
+        const long long nt[3] = {grid.t / tile.t, grid.h / tile.h, grid.w / tile.w};
+        const long long r[3] = {radius.t, radius.h, radius.w};
+        longest = vol / block;
+        for (int a = 0; a < 3; ++a) longest *= (2 * r[a] + 1 < nt[a] ? 2 * r[a] + 1 : nt[a]);
+        group = 0;
+    } else if (block % vol == 0 && radius.t == 0 && radius.h == 0 && radius.w == 0) {
+        longest = 1;
+        group = static_cast<int>(vol);
+    } else {
+        return fail(VSA_ERR_UNSUPPORTED,
+                    "tile volume %lld and block %d: need a tile that is a whole number of blocks, or radius 0 and "
+                    "a block that is a whole number of tiles",
+                    vol, block);
+    }
+    VSA_REQUIRE(cap >= longest, "cap (%d) must be >= the longest list (%lld)", cap, longest);
+    *group_size_out = group;
+    return check_cuda(launch_structured(grid.t, grid.h, grid.w, tile.t, tile.h, tile.w, radius.t, radius.h,
+                                        radius.w, block, idx, cnt, cap, as_stream(stream)),
+                      "structured_block_list launch");
+}
+
+static vsa_status check_attention_common(const void *q, const void *k, const void *v, void *o, vsa_dtype out_dtype,
+                                         int B, int n_heads, int S, int D, float scale) {
+    VSA_TRY(check_bhsd(B, n_heads, S, D));
+    VSA_TRY(check_d(D));
+    VSA_REQUIRE(out_dtype == VSA_BF16 || out_dtype == VSA_F32, "out_dtype must be VSA_BF16 or VSA_F32");
+    VSA_REQUIRE(aligned16(q) && aligned16(k) && aligned16(v) && aligned16(o),
+                "q, k, v and o must be non-NULL 16-byte aligned device pointers");
+    const size_t obytes = static_cast<size_t>(B) * n_heads * S * D * esize_of(out_dtype);
+    const size_t ibytes = static_cast<size_t>(B) * n_heads * S * D * 2;
+    VSA_REQUIRE(!overlaps(o, q, obytes > ibytes ? obytes : ibytes) && !overlaps(o, k, obytes > ibytes ? obytes : ibytes) &&
+                    !overlaps(o, v, obytes > ibytes ? obytes : ibytes),
+                "o must not overlap q, k or v");
+    VSA_REQUIRE(scale == scale && scale < 3.0e38f, "scale must be finite");
+    return VSA_OK;
+}
+
+vsa_status vsa_block_sparse_attention(const void *q, const void *k, const void *v, void *o, vsa_dtype out_dtype,
+                                      int B, int n_heads, int S, int D, int block, const int32_t *idx,
+                                      const int32_t *cnt, int cap, int list_per_head, int group_size, float scale,
+                                      void *stream) {
+    VSA_TRY(check_attention_common(q, k, v, o, out_dtype, B, n_heads, S, D, scale));
+    VSA_REQUIRE(block == 32 || block == 64 || block == 128, "block must be 32, 64 or 128, got %d", block);
+    VSA_REQUIRE(S % block == 0, "block (%d) must divide S (%d)", block, S);
+    VSA_REQUIRE(aligned4(idx) && aligned4(cnt), "idx and cnt must be non-NULL 4-byte aligned device pointers");
+    VSA_REQUIRE(cap >= 1, "cap must be >= 1, got %d", cap);
+    VSA_REQUIRE(group_size >= 0, "group_size must be >= 0, got %d", group_size);
+    AttnLaunch L{};
+    L.q = q; L.k = k; L.v = v; L.o = o;
+    L.out_f32 = out_dtype == VSA_F32;
+    L.BH = B * n_heads; L.S = S; L.D = D;
+    L.block = block;
+    L.window = false;
+    L.idx = idx; L.cnt = cnt; L.cap = cap; L.list_per_head = list_per_head ? 1 : 0;
+    L.group = group_size; L.nb = S / block;
+    L.scale = scale > 0.f ? scale : 1.0f / sqrtf(static_cast<float>(D));
+    return launch_attention(L, status_or_null(), as_stream(stream));
+}
+
+vsa_status vsa_window_attention(const void *q, const void *k, const void *v, void *o, vsa_dtype out_dtype, int B,
+                                int n_heads, int S, int D, int window, int sink, float scale, int chunk,
+                                void *stream) {
+    VSA_TRY(check_attention_common(q, k, v, o, out_dtype, B, n_heads, S, D, scale));
+    VSA_REQUIRE(window >= 1, "window must be >= 1, got %d", window);
+    VSA_REQUIRE(sink >= 0, "sink must be >= 0, got %d", sink);
+    VSA_REQUIRE(sink <= S, "sink (%d) cannot exceed sequence length (%d)", sink, S);
+    VSA_REQUIRE(chunk >= 0, "chunk_size must be >= 1 (or 0 for the default), got %d", chunk);
+    AttnLaunch L{};
+    L.q = q; L.k = k; L.v = v; L.o = o;
+    L.out_f32 = out_dtype == VSA_F32;
+    L.BH = B * n_heads; L.S = S; L.D = D;
+    L.block = 128;
+    L.window = true;
+    L.dense = window >= S ? 1 : 0;
+    L.half = window / 2;
+    L.sink = sink;
+    L.scale = scale > 0.f ? scale : 1.0f / sqrtf(static_cast<float>(D));
+    return launch_attention(L, status_or_null(), as_stream(stream));
+}
+
+vsa_status vsa_cast_f32_to_bf16(const float *x, void *y, int64_t n, void *stream) {
+    VSA_REQUIRE(n >= 0, "n must be >= 0");
+    if (n == 0) return VSA_OK;
+    VSA_REQUIRE(aligned16(x), "x must be a non-NULL 16-byte aligned device pointer");
+    VSA_REQUIRE(y != nullptr && (reinterpret_cast<uintptr_t>(y) & 7u) == 0, "y must be a non-NULL 8-byte aligned device pointer");
+    return check_cuda(launch_cast_f32_bf16(x, y, n, as_stream(stream)), "cast launch");
+}
+
+vsa_status vsa_debug_wait_timeout(int64_t timeout_ns, void *stream) {
+    VSA_REQUIRE(timeout_ns >= 0 && timeout_ns <= 10000000000LL, "timeout_ns must be in [0, 1e10]");
+    return check_cuda(launch_wait_timeout(static_cast<uint64_t>(timeout_ns), status_or_null(), as_stream(stream)),
+                      "wait_timeout launch");
+}
+
+}  // extern "C"

@@ -1,0 +1,67 @@
+// internal.h -- host-side declarations shared by the libvsa translation units.
+#pragma once
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "../../include/vsa.h"
+
+namespace vsa {
+
+// Record a message for vsa_last_error() and return `s`.
+vsa_status fail(vsa_status s, const char *fmt, ...);
+// Map a CUDA error to VSA_ERR_CUDA (with its message), or VSA_OK.
+vsa_status check_cuda(cudaError_t e, const char *what);
+// Device address of the status word of the current device.
+int *device_status_word();
+
+struct TileSet {
+    int n;
+    int t[8], h[8], w[8];
+};
+
+// Launchers (arguments already validated by the C ABI layer).
+cudaError_t launch_permute(const void *src, void *dst, int esize, int BH, int S, int D, int T, int H, int W,
+                           const TileSet &tiles, const int32_t *choice, bool inverse, int *status,
+                           cudaStream_t st);
+cudaError_t launch_cast_f32_bf16(const float *x, void *y, int64_t n, cudaStream_t st);
+cudaError_t launch_summaries(const void *x, int esize, int BH, int S, int D, int block, void *xmax, void *xmin,
+                             cudaStream_t st);
+cudaError_t launch_scores(const void *qmax, const void *qmin, const void *kmax, const void *kmin, int esize, int BH,
+                          int nb, int D, float *scores, cudaStream_t st);
+cudaError_t launch_topk(const float *scores, int BH, int nb, int k, int n_sink, int diag_hw, int32_t *idx,
+                        int32_t *cnt, int cap, cudaStream_t st);
+cudaError_t launch_structured(int T, int H, int W, int tt, int th, int tw, int rt, int rh, int rw, int block,
+                              int32_t *idx, int32_t *cnt, int cap, cudaStream_t st);
+
+struct SelectGeom {
+    int Rt, Rh, Rw;   // region = per-axis lcm of the candidate tiles
+    int Ct, Ch, Cw;   // cell = per-axis gcd of the candidate tiles
+    int n_regions;    // regions per (b, head)
+    int cells;        // cells per region
+};
+bool select_geometry(int T, int H, int W, const TileSet &tiles, SelectGeom *g);
+cudaError_t launch_select_tiling(const void *q, int esize, int BH, int S, int D, int T, int H, int W,
+                                 const TileSet &tiles, const SelectGeom &g, int32_t *choice, float *sics,
+                                 float *partial, int *status, cudaStream_t st);
+
+struct AttnLaunch {
+    const void *q, *k, *v;
+    void *o;
+    int out_f32;
+    int BH, S, D;
+    int block;          // rows per query tile = keys per key tile
+    bool window;
+    // block-list mode
+    const int32_t *idx, *cnt;
+    int cap, list_per_head, group, nb;
+    // window mode
+    int half, sink, dense;
+    float scale;
+};
+vsa_status launch_attention(const AttnLaunch &a, int *status, cudaStream_t st);
+
+cudaError_t launch_wait_timeout(uint64_t limit_ns, int *status, cudaStream_t st);
+
+}  // namespace vsa

@@ -1,0 +1,263 @@
+// select_tiling.cu -- per-(batch, head) choice of the most cohesive tiling.
+//
+// "Adaptive tiling (SPADE)", The idea, step 1 and select_tiling /
+// block_self_similarity: the cohesion of a tiling is the mean over its tiles
+// of the tile's SICS, the mean cosine over distinct pairs of its non-zero
+// queries, (|sum of unit queries|^2 - m) / (m (m - 1)); the choice is the
+// most cohesive candidate, ties to the lower index.
+//
+// Q is read once for all candidates.  The grid is cut into regions of the
+// per-axis lcm of the candidate tiles (every candidate tiles a region
+// exactly) and each region into cells of the per-axis gcd (every tile is a
+// union of cells).  Pass 1: one CTA per (region, bh) normalises each query
+// once, sums unit vectors per cell, then per candidate tile sums its cells
+// and turns the norm into the tile's SICS; it writes per-candidate sums of
+// tile SICS for its region.  Pass 2: one warp per bh adds the regions in a
+// fixed order, divides by the tile count and takes the argmax.
+#include "common.cuh"
+#include "internal.h"
+
+namespace vsa {
+
+namespace {
+
+constexpr int kThreads = 256;
+constexpr int kWarps = kThreads / 32;
+constexpr int kMaxCells = 256;
+
+int gcd(int a, int b) { return b == 0 ? a : gcd(b, a % b); }
+int lcm(int a, int b) { return a / gcd(a, b) * b; }
+
+struct SelArgs {
+    const uint8_t *q;
+    int S, H, W, D, esize;
+    TileSet tiles;
+    int Rt, Rh, Rw, Ct, Ch, Cw;
+    int nrt, nrh, nrw;  // regions per axis
+    int cells;
+    float *partial;     // [BH][n_regions][tiles.n]
+};
+
+template <typename T, int LPT>  // LPT: lanes (16 bytes each) per query row
+__global__ void __launch_bounds__(kThreads) sics_partial_kernel(const SelArgs a) {
+    constexpr int EPL = 16 / sizeof(T);  // elements per lane
+    constexpr int TPI = 32 / LPT;        // query rows per warp pass
+    extern __shared__ float sm[];
+    float *cell_sum = sm;                               // [cells][D]
+    float *cell_cnt = cell_sum + a.cells * a.D;         // [cells]
+    float *tile_val = cell_cnt + a.cells;               // [items]
+    const int region = blockIdx.x, bh = blockIdx.y;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int rt = region / (a.nrh * a.nrw), rh = (region / a.nrw) % a.nrh, rw = region % a.nrw;
+    const int t0 = rt * a.Rt, h0 = rh * a.Rh, w0 = rw * a.Rw;
+    const int nct = a.Rt / a.Ct, nch = a.Rh / a.Ch, ncw = a.Rw / a.Cw;
+    const int cvol = a.Ct * a.Ch * a.Cw;
+    const size_t head = static_cast<size_t>(bh) * a.S;
+
+    for (int cell = warp; cell < a.cells; cell += kWarps) {
+        const int ct = cell / (nch * ncw), ch = (cell / ncw) % nch, cw = cell % ncw;
+        const int tb = t0 + ct * a.Ct, hb = h0 + ch * a.Ch, wb = w0 + cw * a.Cw;
+        float acc[EPL];
+        #pragma unroll
+        for (int e = 0; e < EPL; ++e) acc[e] = 0.f;
+        float m = 0.f;
+        #pragma unroll 2
+        for (int tok0 = 0; tok0 < cvol; tok0 += TPI) {  // uniform trip count: shuffles below
+            const int tok = tok0 + lane / LPT;
+            const bool valid = tok < cvol;
+            const int dt = tok / (a.Ch * a.Cw), r2 = tok - dt * (a.Ch * a.Cw);
+            const int dh = r2 / a.Cw, dw = r2 - dh * a.Cw;
+            const size_t token = static_cast<size_t>((tb + dt) * a.H + hb + dh) * a.W + wb + dw;
+            uint4 raw = make_uint4(0u, 0u, 0u, 0u);
+            if (valid)
+                raw = __ldcs(reinterpret_cast<const uint4 *>(a.q + ((head + token) * a.D) * sizeof(T)) + (lane % LPT));
+            float x[EPL];
+            if constexpr (sizeof(T) == 2) {
+                const __nv_bfloat162 *hv = reinterpret_cast<const __nv_bfloat162 *>(&raw);
+                #pragma unroll
+                for (int e = 0; e < EPL / 2; ++e) {
+                    const float2 f = __bfloat1622float2(hv[e]);
+                    x[2 * e] = f.x;
+                    x[2 * e + 1] = f.y;
+                }
+            } else {
+                const float *fv = reinterpret_cast<const float *>(&raw);
+                #pragma unroll
+                for (int e = 0; e < EPL; ++e) x[e] = fv[e];
+            }
+            float ss = 0.f;
+            #pragma unroll
+            for (int e = 0; e < EPL; ++e) ss = fmaf(x[e], x[e], ss);
+            #pragma unroll
+            for (int off = LPT / 2; off > 0; off >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, off);
+            if (ss > 0.f) {
+                const float inv = rsqrtf(ss);
+                #pragma unroll
+                for (int e = 0; e < EPL; ++e) acc[e] = fmaf(x[e], inv, acc[e]);
+                m += 1.f;
+            }
+        }
+        #pragma unroll
+        for (int off = LPT; off < 32; off <<= 1) {
+            #pragma unroll
+            for (int e = 0; e < EPL; ++e) acc[e] += __shfl_xor_sync(0xffffffffu, acc[e], off);
+            m += __shfl_xor_sync(0xffffffffu, m, off);
+        }
+        if (lane < LPT) {
+            #pragma unroll
+            for (int e = 0; e < EPL; ++e) cell_sum[cell * a.D + lane * EPL + e] = acc[e];
+        }
+        if (lane == 0) cell_cnt[cell] = m;
+    }
+    __syncthreads();
+
+    // candidate tiles inside this region: item -> (candidate c, tile index)
+    int items = 0;
+    for (int c = 0; c < a.tiles.n; ++c)
+        items += (a.Rt / a.tiles.t[c]) * (a.Rh / a.tiles.h[c]) * (a.Rw / a.tiles.w[c]);
+    for (int item = warp; item < items; item += kWarps) {
+        int c = 0, rem = item;
+        while (true) {
+            const int n = (a.Rt / a.tiles.t[c]) * (a.Rh / a.tiles.h[c]) * (a.Rw / a.tiles.w[c]);
+            if (rem < n) break;
+            rem -= n;
+            ++c;
+        }
+        const int tt = a.tiles.t[c], th = a.tiles.h[c], tw = a.tiles.w[c];
+        const int nth = a.Rh / th, ntw = a.Rw / tw;
+        const int at = rem / (nth * ntw), ah = (rem / ntw) % nth, aw = rem % ntw;
+        // cells of this tile, in cell coordinates
+        const int c0t = at * tt / a.Ct, c0h = ah * th / a.Ch, c0w = aw * tw / a.Cw;
+        const int kt = tt / a.Ct, kh = th / a.Ch, kw = tw / a.Cw;
+        float sq = 0.f, m = 0.f;
+        for (int d = lane; d < a.D; d += 32) {
+            float s = 0.f;
+            for (int x = 0; x < kt; ++x)
+                for (int y = 0; y < kh; ++y)
+                    for (int z = 0; z < kw; ++z)
+                        s += cell_sum[(((c0t + x) * nch + c0h + y) * ncw + c0w + z) * a.D + d];
+            sq = fmaf(s, s, sq);
+        }
+        for (int x = 0; x < kt; ++x)
+            for (int y = 0; y < kh; ++y)
+                for (int z = 0; z < kw; ++z) m += cell_cnt[((c0t + x) * nch + c0h + y) * ncw + c0w + z];
+        #pragma unroll
+        for (int off = 16; off > 0; off >>= 1) sq += __shfl_down_sync(0xffffffffu, sq, off);
+        if (lane == 0) tile_val[item] = m >= 2.f ? (sq - m) / (m * (m - 1.f)) : 0.f;
+    }
+    __syncthreads();
+    if (threadIdx.x < a.tiles.n) {
+        const int c = threadIdx.x;
+        int first = 0;
+        for (int cc = 0; cc < c; ++cc)
+            first += (a.Rt / a.tiles.t[cc]) * (a.Rh / a.tiles.h[cc]) * (a.Rw / a.tiles.w[cc]);
+        const int n = (a.Rt / a.tiles.t[c]) * (a.Rh / a.tiles.h[c]) * (a.Rw / a.tiles.w[c]);
+        float s = 0.f;
+        for (int i = 0; i < n; ++i) s += tile_val[first + i];
+        const int n_regions = a.nrt * a.nrh * a.nrw;
+        a.partial[(static_cast<size_t>(bh) * n_regions + region) * a.tiles.n + c] = s;
+    }
+}
+
+struct FinalArgs {
+    const float *partial;
+    int BH, n_regions, n_tiles;
+    float tiles_total[8];  // tiles of candidate c over the whole grid
+    int32_t *choice;
+    float *sics;
+};
+
+__global__ void sics_final_kernel(const FinalArgs a) {
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int bh = blockIdx.x * (blockDim.x / 32) + warp;
+    if (bh >= a.BH) return;
+    float best = 0.f;
+    int best_c = 0;
+    for (int c = 0; c < a.n_tiles; ++c) {
+        float s = 0.f;
+        for (int r = lane; r < a.n_regions; r += 32)
+            s += a.partial[(static_cast<size_t>(bh) * a.n_regions + r) * a.n_tiles + c];
+        #pragma unroll
+        for (int off = 16; off > 0; off >>= 1) s += __shfl_down_sync(0xffffffffu, s, off);
+        s = __shfl_sync(0xffffffffu, s, 0);
+        const float mean = s / a.tiles_total[c];
+        if (c == 0 || mean > best) {
+            best = mean;
+            best_c = c;
+        }
+        if (lane == 0 && a.sics) a.sics[static_cast<size_t>(bh) * a.n_tiles + c] = mean;
+    }
+    if (lane == 0) a.choice[bh] = best_c;
+}
+
+}  // namespace
+
+bool select_geometry(int T, int H, int W, const TileSet &tiles, SelectGeom *g) {
+    int Rt = 1, Rh = 1, Rw = 1, Ct = tiles.t[0], Ch = tiles.h[0], Cw = tiles.w[0];
+    for (int c = 0; c < tiles.n; ++c) {
+        Rt = lcm(Rt, tiles.t[c]);
+        Rh = lcm(Rh, tiles.h[c]);
+        Rw = lcm(Rw, tiles.w[c]);
+        Ct = gcd(Ct, tiles.t[c]);
+        Ch = gcd(Ch, tiles.h[c]);
+        Cw = gcd(Cw, tiles.w[c]);
+    }
+    g->Rt = Rt; g->Rh = Rh; g->Rw = Rw;
+    g->Ct = Ct; g->Ch = Ch; g->Cw = Cw;
+    if (T % Rt || H % Rh || W % Rw) return false;
+    g->n_regions = (T / Rt) * (H / Rh) * (W / Rw);
+    g->cells = (Rt / Ct) * (Rh / Ch) * (Rw / Cw);
+    return g->cells <= kMaxCells;
+}
+
+cudaError_t launch_select_tiling(const void *q, int esize, int BH, int S, int D, int T, int H, int W,
+                                 const TileSet &tiles, const SelectGeom &g, int32_t *choice, float *sics,
+                                 float *partial, int *status, cudaStream_t st) {
+    (void)status;
+    SelArgs a;
+    a.q = static_cast<const uint8_t *>(q);
+    a.S = S; a.H = H; a.W = W; a.D = D; a.esize = esize;
+    a.tiles = tiles;
+    a.Rt = g.Rt; a.Rh = g.Rh; a.Rw = g.Rw;
+    a.Ct = g.Ct; a.Ch = g.Ch; a.Cw = g.Cw;
+    a.nrt = T / g.Rt; a.nrh = H / g.Rh; a.nrw = W / g.Rw;
+    a.cells = g.cells;
+    a.partial = partial;
+    int items = 0;
+    for (int c = 0; c < tiles.n; ++c)
+        items += (g.Rt / tiles.t[c]) * (g.Rh / tiles.h[c]) * (g.Rw / tiles.w[c]);
+    const size_t smem = (static_cast<size_t>(g.cells) * D + g.cells + items) * sizeof(float);
+    dim3 grid(g.n_regions, BH);
+    const int lpt = D * esize / 16;
+    cudaError_t e = cudaSuccess;
+#define VSA_SICS_LAUNCH(TYPE, L)                                                                           \
+    do {                                                                                                   \
+        e = cudaFuncSetAttribute(sics_partial_kernel<TYPE, L>, cudaFuncAttributeMaxDynamicSharedMemorySize, \
+                                 static_cast<int>(smem));                                                  \
+        if (e != cudaSuccess) return e;                                                                    \
+        sics_partial_kernel<TYPE, L><<<grid, kThreads, smem, st>>>(a);                                     \
+    } while (0)
+    if (esize == 2) {
+        if (lpt == 8) VSA_SICS_LAUNCH(__nv_bfloat16, 8);
+        else VSA_SICS_LAUNCH(__nv_bfloat16, 16);
+    } else {
+        if (lpt == 16) VSA_SICS_LAUNCH(float, 16);
+        else VSA_SICS_LAUNCH(float, 32);
+    }
+#undef VSA_SICS_LAUNCH
+    e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+    FinalArgs f;
+    f.partial = partial;
+    f.BH = BH;
+    f.n_regions = g.n_regions;
+    f.n_tiles = tiles.n;
+    for (int c = 0; c < 8; ++c)
+        f.tiles_total[c] = c < tiles.n ? static_cast<float>(S / (tiles.t[c] * tiles.h[c] * tiles.w[c])) : 1.f;
+    f.choice = choice;
+    f.sics = sics;
+    sics_final_kernel<<<(BH + 7) / 8, 256, 0, st>>>(f);
+    return cudaGetLastError();
+}
+
+}  // namespace vsa

@@ -1,0 +1,131 @@
+// topk.cu -- fixed-budget top-k key blocks plus sink and diagonal blocks,
+// emitted as a compact ascending index list per query block.
+//
+// "Adaptive tiling (SPADE)", The idea, step 4 (fixed per-row budget, static
+// sink and diagonal blocks), top_k_block_mask, and the recipe note (OR the
+// static blocks into the top-k mask).  Equal scores rank the lower block
+// index first, so the result is unique and bit-exact.
+//
+// One warp per row.  Scores map to order-preserving uint32 keys; a 4-pass
+// 8-bit radix select finds the k-th largest key T and how many keys equal to
+// T are taken (lowest indices first); a final ordered pass ranks the ties,
+// ORs in the static blocks and compacts the kept indices with ballots.
+#include "common.cuh"
+#include "internal.h"
+
+namespace vsa {
+
+namespace {
+
+constexpr int kWarps = 8;
+
+__device__ __forceinline__ uint32_t order_key(float f) {
+    uint32_t u = __float_as_uint(f);
+    if ((u & 0x7fffffffu) == 0u) u = 0u;              // -0 ranks equal to +0
+    return (u & 0x80000000u) ? ~u : (u | 0x80000000u);  // larger float -> larger key
+}
+
+__global__ void __launch_bounds__(kWarps * 32) topk_kernel(const float *__restrict__ scores, long long rows, int nb,
+                                                          int k, int n_sink, int diag_hw, int32_t *__restrict__ idx,
+                                                          int32_t *__restrict__ cnt, int cap) {
+    __shared__ uint32_t hist[kWarps][256];
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    uint32_t *h = hist[warp];
+    for (long long row = static_cast<long long>(blockIdx.x) * kWarps + warp; row < rows;
+         row += static_cast<long long>(gridDim.x) * kWarps) {
+        const float *s = scores + row * nb;
+        const int i = static_cast<int>(row % nb);  // query block of this row
+        uint32_t prefix = 0u, pmask = 0u;
+        int need = k;  // rank of the threshold among the keys still matching the prefix
+        #pragma unroll 1
+        for (int pass = 0; pass < 4; ++pass) {
+            const int shift = 24 - 8 * pass;
+            for (int b = lane; b < 256; b += 32) h[b] = 0u;
+            __syncwarp();
+            for (int j0 = 0; j0 < nb; j0 += 32) {
+                const int j = j0 + lane;
+                const bool in = j < nb;
+                const uint32_t key = in ? order_key(__ldg(s + j)) : 0u;
+                const bool match = in && (key & pmask) == prefix;
+                const uint32_t digit = (key >> shift) & 255u;
+                const uint32_t active = __ballot_sync(0xffffffffu, match);
+                if (match) {
+                    const uint32_t same = __match_any_sync(active, digit);
+                    if (lane == __ffs(same) - 1) atomicAdd(&h[digit], __popc(same));
+                }
+            }
+            __syncwarp();
+            // lane L owns digits 255-8L .. 248-8L (highest digits first)
+            uint32_t local[8];
+            uint32_t tot = 0;
+            #pragma unroll
+            for (int e = 0; e < 8; ++e) {
+                local[e] = h[255 - 8 * lane - e];
+                tot += local[e];
+            }
+            uint32_t incl = tot;
+            #pragma unroll
+            for (int off = 1; off < 32; off <<= 1) {
+                const uint32_t v = __shfl_up_sync(0xffffffffu, incl, off);
+                if (lane >= off) incl += v;
+            }
+            const uint32_t excl = incl - tot;
+            const bool mine = excl < static_cast<uint32_t>(need) && static_cast<uint32_t>(need) <= incl;
+            const uint32_t owner = __ballot_sync(0xffffffffu, mine);
+            const int src = __ffs(owner) - 1;
+            uint32_t digit = 0, above = 0;
+            if (lane == src) {
+                uint32_t run = excl;
+                #pragma unroll
+                for (int e = 0; e < 8; ++e) {
+                    if (run + local[e] >= static_cast<uint32_t>(need)) {
+                        digit = 255u - 8u * lane - e;
+                        above = run;
+                        break;
+                    }
+                    run += local[e];
+                }
+            }
+            digit = __shfl_sync(0xffffffffu, digit, src);
+            above = __shfl_sync(0xffffffffu, above, src);
+            need -= static_cast<int>(above);
+            prefix |= digit << shift;
+            pmask |= 255u << shift;
+            __syncwarp();
+        }
+        // prefix = the k-th largest key; take every larger key and the first
+        // `need` keys equal to it, then OR in the static blocks.
+        int32_t *out = idx + row * cap;
+        int taken_eq = 0, written = 0;
+        for (int j0 = 0; j0 < nb; j0 += 32) {
+            const int j = j0 + lane;
+            const bool in = j < nb;
+            const uint32_t key = in ? order_key(__ldg(s + j)) : 0u;
+            const bool eq = in && key == prefix;
+            const uint32_t eqm = __ballot_sync(0xffffffffu, eq);
+            const int rank = taken_eq + __popc(eqm & ((1u << lane) - 1u));
+            const int dd = j > i ? j - i : i - j;
+            const bool keep = in && (key > prefix || (eq && rank < need) || j < n_sink || dd <= diag_hw);
+            const uint32_t km = __ballot_sync(0xffffffffu, keep);
+            const int pos = written + __popc(km & ((1u << lane) - 1u));
+            if (keep && pos < cap) out[pos] = j;
+            taken_eq += __popc(eqm);
+            written += __popc(km);
+        }
+        for (int p = written + lane; p < cap; p += 32) out[p] = -1;
+        if (lane == 0) cnt[row] = written;
+    }
+}
+
+}  // namespace
+
+cudaError_t launch_topk(const float *scores, int BH, int nb, int k, int n_sink, int diag_hw, int32_t *idx,
+                        int32_t *cnt, int cap, cudaStream_t st) {
+    const long long rows = static_cast<long long>(BH) * nb;
+    long long blocks = (rows + kWarps - 1) / kWarps;
+    if (blocks > 148LL * 16) blocks = 148LL * 16;
+    topk_kernel<<<static_cast<int>(blocks), kWarps * 32, 0, st>>>(scores, rows, nb, k, n_sink, diag_hw, idx, cnt, cap);
+    return cudaGetLastError();
+}
+
+}  // namespace vsa

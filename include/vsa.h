@@ -1,0 +1,241 @@
+/*
+ * vsa.h -- C ABI of libvsa: structured and input-adaptive block-sparse
+ * self-attention over a video DiT's T-major spatiotemporal token sequence,
+ * for NVIDIA B200 (sm_100a).
+ *
+ * Conventions shared by every call
+ * --------------------------------
+ * - Token order is T-major: token (t, h, w) of a (T, Hg, Wg) latent grid is
+ *   at index (t*Hg + h)*Wg + w, S = T*Hg*Wg ("ADR-0001: Sparse-attention
+ *   roadmap for video DiTs", Conventions).
+ * - Tensors are dense row-major device arrays.  Q/K/V/O are [B, n_heads, S, D];
+ *   (b, h) pairs are flattened as bh = b*n_heads + h.
+ * - Every pointer argument is a DEVICE pointer unless stated, 16-byte aligned.
+ *   The caller owns every buffer; the library allocates no device memory.
+ * - `stream` is a cudaStream_t (NULL = the legacy default stream).  Every
+ *   call only enqueues work on it and returns without synchronising.
+ * - Argument errors are detected on the host before anything is launched
+ *   and return VSA_ERR_INVALID_ARGUMENT (the pages raise ValueError for
+ *   these, "ADR-0001", Conventions: Validation).  Violations that only the
+ *   device can see (a block index out of range, an empty key set) set a
+ *   device status word that vsa_device_status() returns (the pages'
+ *   RuntimeError).  A CUDA launch failure returns VSA_ERR_CUDA.
+ * - vsa_last_error() gives a readable message for the last non-OK status
+ *   returned on the calling host thread.
+ */
+#ifndef VSA_H
+#define VSA_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    VSA_OK = 0,
+    VSA_ERR_INVALID_ARGUMENT = 1, /* bad shape, size or option (ValueError)      */
+    VSA_ERR_RUNTIME = 2,          /* violated invariant seen on the device        */
+    VSA_ERR_CUDA = 3,             /* CUDA runtime / launch failure                */
+    VSA_ERR_UNSUPPORTED = 4,      /* valid request this build does not implement  */
+    VSA_ERR_TIMEOUT = 5           /* a bounded on-device wait gave up             */
+} vsa_status;
+
+typedef enum { VSA_BF16 = 0, VSA_F32 = 1 } vsa_dtype;
+
+/* A (t, h, w) triple: a latent grid (T, Hg, Wg), a tile (tt, th, tw) or a
+ * neighbourhood radius (rt, rh, rw).                                        */
+typedef struct { int32_t t, h, w; } vsa_dims3;
+
+typedef enum {
+    VSA_MASK_SPATIAL = 0,      /* same frame: tile (1, Hg, Wg), radius 0      */
+    VSA_MASK_TEMPORAL = 1,     /* same (h, w): tile (T, 1, 1), radius 0       */
+    VSA_MASK_SLIDING_TILE = 2  /* tiles whose coordinates differ by <= radius */
+} vsa_mask_kind;
+
+/* Message for the last non-OK status returned on this host thread ("" if none). */
+const char *vsa_last_error(void);
+
+/* Synchronises `stream`, then returns and clears the device status word of
+ * the current device: VSA_OK, VSA_ERR_RUNTIME (a device-side check failed)
+ * or VSA_ERR_TIMEOUT (a bounded wait inside a kernel gave up).  Meant for
+ * tests and debugging; the compute calls never synchronise.               */
+vsa_status vsa_device_status(void *stream);
+
+/* ------------------------------------------------------------------------ */
+/* Adaptive tiling: per-(b, head) choice of the most cohesive tiling.
+ * "Adaptive tiling (SPADE)", The idea, step 1, and the function table
+ * (block_self_similarity, select_tiling), "Deviations and notes" (selection
+ * statistic; divisible grids only).
+ *
+ * For every (b, head) and candidate c, the cohesion is the mean over the
+ * tiles of tiling c of the tile's SICS: the mean cosine similarity over the
+ * distinct pairs of its non-zero-norm queries, computed as
+ * (|sum of unit queries|^2 - m) / (m (m - 1)) (a tile with m < 2 scores 0).
+ * choice[bh] = argmax_c cohesion, ties to the lower c.
+ *
+ *   q        [B, n_heads, S, D] in `dtype` (VSA_BF16 or VSA_F32)
+ *   grid     (T, Hg, Wg) with T*Hg*Wg == S; every tile must divide it
+ *   tiles    HOST array of n_tiles candidate tiles (1 <= n_tiles <= 8)
+ *   choice   [B*n_heads] int32 output
+ *   sics     [B*n_heads, n_tiles] fp32 output, or NULL
+ *   workspace, workspace_bytes: device scratch of at least
+ *            vsa_select_tiling_workspace_size(...) bytes, 16-byte aligned;
+ *            its contents need not be initialised and are overwritten.
+ * Limits: D in {64, 128}; the lcm of the candidate tiles (per axis) may
+ * hold at most 256 cells of gcd-tile size (VSA_ERR_UNSUPPORTED otherwise).
+ * Cohesion is accumulated in fp32: candidates whose cohesion differs by
+ * less than about 1e-5 may be ranked either way.                          */
+size_t vsa_select_tiling_workspace_size(int B, int n_heads, vsa_dims3 grid,
+                                        const vsa_dims3 *tiles, int n_tiles);
+vsa_status vsa_select_tiling(const void *q, vsa_dtype dtype, int B, int n_heads,
+                             int S, int D, vsa_dims3 grid, const vsa_dims3 *tiles,
+                             int n_tiles, int32_t *choice, float *sics,
+                             void *workspace, size_t workspace_bytes, void *stream);
+
+/* ------------------------------------------------------------------------ */
+/* Tile-contiguous permutation and its inverse.
+ * "ADR-0001", step 6 (block_contiguous_permutation, invert_permutation);
+ * "Adaptive tiling (SPADE)", The idea, step 2, and the Recipe (argsort of
+ * tile_labels; take(..., argsort(order)) to return to T-major order).
+ *
+ * perm_c lists the tiles of tiling c in row-major tile order and, inside a
+ * tile, its tokens in T-major order (a stable argsort of the tile labels).
+ *   vsa_permute:   y[bh, p, :] = x[bh, perm_{c(bh)}[p], :]
+ *   vsa_unpermute: x[bh, perm_{c(bh)}[p], :] = y[bh, p, :]
+ * where c(bh) = choice[bh] (device int32 [B*n_heads]), or 0 if choice is NULL.
+ * x and y are [B, n_heads, S, D] in `dtype` and must not overlap.
+ * tiles is a HOST array of n_tiles (1..8) tiles that divide grid; a device
+ * choice outside [0, n_tiles) sets VSA_ERR_RUNTIME and that head is left
+ * unwritten.  The copy is exact (bit for bit).                            */
+vsa_status vsa_permute(const void *x, void *y, vsa_dtype dtype, int B, int n_heads,
+                       int S, int D, vsa_dims3 grid, const vsa_dims3 *tiles,
+                       int n_tiles, const int32_t *choice, void *stream);
+vsa_status vsa_unpermute(const void *y, void *x, vsa_dtype dtype, int B, int n_heads,
+                         int S, int D, vsa_dims3 grid, const vsa_dims3 *tiles,
+                         int n_tiles, const int32_t *choice, void *stream);
+
+/* ------------------------------------------------------------------------ */
+/* Per-block element-wise summaries.  "Adaptive tiling (SPADE)", The idea,
+ * step 3 (element-wise max/min summaries).
+ *   x_max[bh, i, d] = max_{r < block} x_perm[bh, i*block + r, d], x_min likewise.
+ * x_perm [B, n_heads, S, D]; x_max, x_min [B, n_heads, S/block, D], all in
+ * `dtype`.  block in {16, 32, 64, 128, 256}, S % block == 0, D in {64, 128}.
+ * The result is an exact selection of input values.                       */
+vsa_status vsa_block_summaries(const void *x_perm, vsa_dtype dtype, int B, int n_heads,
+                               int S, int D, int block, void *x_max, void *x_min,
+                               void *stream);
+
+/* ------------------------------------------------------------------------ */
+/* Block scores.  "Adaptive tiling (SPADE)", The idea, step 3, and the
+ * function table (minmax_block_scores).
+ *   scores[bh, i, j] = max((q_max_i + q_min_i) . k_max_j, (q_max_i + q_min_i) . k_min_j)
+ * unscaled, accumulated in fp32 as q_max.k + q_min.k, so every product of
+ * bf16 inputs is exact; on small-integer-valued inputs the scores are exact.
+ * Summaries are [B, n_heads, nb, D] in `dtype`; scores [B, n_heads, nb, nb]
+ * fp32.  D in {64, 128}, 1 <= nb.                                          */
+vsa_status vsa_block_scores(const void *q_max, const void *q_min, const void *k_max,
+                            const void *k_min, vsa_dtype dtype, int B, int n_heads,
+                            int nb, int D, float *scores, void *stream);
+
+/* ------------------------------------------------------------------------ */
+/* Top-k key blocks plus static sink and diagonal blocks, as a compact list.
+ * "Adaptive tiling (SPADE)", The idea, step 4 (fixed per-row budget plus
+ * static sink and diagonal blocks), function table (top_k_block_mask), the
+ * Recipe (k = max(1, floor(budget * n_blocks))) and the recipe note (OR the
+ * sink and diagonal blocks into the top-k mask).
+ *
+ * Row i of every (b, head) keeps the k highest scores (equal scores: lower
+ * block index first), then adds the blocks j < n_sink_blocks and
+ * |j - i| <= diag_halfwidth (diag_halfwidth = -1: none).  The kept block
+ * indices are written in ascending order to idx[bh, i, 0 .. cnt[bh, i]),
+ * the remaining slots get -1.
+ *   scores [B, n_heads, nb, nb] fp32 (NaN not allowed; -0 equals +0)
+ *   idx    [B, n_heads, nb, cap] int32,  cnt [B, n_heads, nb] int32
+ * 1 <= k <= nb, 0 <= n_sink_blocks <= nb, cap >= min(nb, k + n_sink_blocks
+ * + 2*diag_halfwidth + 1).  Integer output: bit-exact by construction.   */
+vsa_status vsa_topk_block_mask(const float *scores, int B, int n_heads, int nb, int k,
+                               int n_sink_blocks, int diag_halfwidth, int32_t *idx,
+                               int32_t *cnt, int cap, void *stream);
+
+/* ------------------------------------------------------------------------ */
+/* Structured static masks as block lists.  "ADR-0001", step 1
+ * (spatial_only_mask, temporal_only_mask, sliding_tile_block_mask).
+ *
+ * The mask is a tile neighbourhood: token i sees token j iff the coordinates
+ * of their tiles differ by at most the radius along (t, h, w), clipped at the
+ * grid border.  SPATIAL uses tile (1, Hg, Wg) and radius 0 (same frame);
+ * TEMPORAL uses tile (T, 1, 1) and radius 0 (same (h, w)); SLIDING_TILE uses
+ * the given tile and radius.  `tile` and `radius` are ignored for SPATIAL
+ * and TEMPORAL.  The list is expressed in the tile-contiguous order of that
+ * tile (use vsa_permute with the same tile):
+ *   - tile volume a multiple of block: query block i lists every block of
+ *     every neighbouring tile, ascending; *group_size_out = 0;
+ *   - block a multiple of the tile volume and radius 0: query block i lists
+ *     itself and a key is visible iff it lies in the query's group of
+ *     tile-volume tokens; *group_size_out = tile volume.
+ * idx [S/block, cap] int32 (-1 padded), cnt [S/block] int32 (the same list
+ * serves every batch entry and head); group_size_out is a HOST int.       */
+vsa_status vsa_structured_block_list(vsa_mask_kind kind, vsa_dims3 grid, vsa_dims3 tile,
+                                     vsa_dims3 radius, int block, int32_t *idx,
+                                     int32_t *cnt, int cap, int *group_size_out,
+                                     void *stream);
+
+/* ------------------------------------------------------------------------ */
+/* Block-sparse attention on tcgen05 tensor cores.  "Adaptive tiling (SPADE)",
+ * Recipe and recipe note (skipped blocks are dropped: the block mask is
+ * expanded to tokens and softmax attention runs over the kept keys).
+ *
+ * For query row p of query block i = p / block (tile-contiguous order):
+ *   o[p] = sum_j softmax_j(scale * q[p] . k[j]) v[j]
+ * over the keys j of the blocks idx[.., i, 0 .. cnt[.., i]) that are also in
+ * p's group of group_size tokens when group_size > 0.  QK^T and PV run in
+ * bf16 with fp32 accumulation, the online softmax in fp32.
+ *   q, k, v  [B, n_heads, S, D] bf16;  o [B, n_heads, S, D] in out_dtype
+ *   idx/cnt  [B, n_heads, nb, cap] / [B, n_heads, nb] if list_per_head,
+ *            else [nb, cap] / [nb] shared by every (b, head)
+ *   scale    softmax scale; <= 0 selects 1/sqrt(D) (_default_scale)
+ * block in {32, 64, 128}, S % block == 0, D in {64, 128}.  Each list must be
+ * strictly ascending with entries in [0, nb) and 1 <= cnt <= cap; rows whose
+ * list breaks this are written as zeros and set VSA_ERR_RUNTIME.          */
+vsa_status vsa_block_sparse_attention(const void *q, const void *k, const void *v,
+                                      void *o, vsa_dtype out_dtype, int B, int n_heads,
+                                      int S, int D, int block, const int32_t *idx,
+                                      const int32_t *cnt, int cap, int list_per_head,
+                                      int group_size, float scale, void *stream);
+
+/* ------------------------------------------------------------------------ */
+/* Symmetric sliding-window attention with global sinks.
+ * "fastvideo/mlx_runtime/windowed_attention.py": module docstring (Window
+ * policy), windowed_attention, _key_ranges_for_block, _default_scale.
+ *
+ * Key j is visible to query i iff j < sink or |i - j| <= window / 2; when
+ * window >= S every key is visible (dense attention, as the page does).
+ * Work is restricted to the 128x128 tiles that meet the window or the sinks.
+ *   q, k, v [B, n_heads, S, D] bf16 (any S >= 1); o in out_dtype
+ *   window >= 1, 0 <= sink <= S, scale <= 0 selects 1/sqrt(D)
+ *   chunk    the page's query chunk size; results do not depend on it.
+ *            0 selects min(window, 512); otherwise it must be >= 1.
+ * D in {64, 128}.                                                          */
+vsa_status vsa_window_attention(const void *q, const void *k, const void *v, void *o,
+                                vsa_dtype out_dtype, int B, int n_heads, int S, int D,
+                                int window, int sink, float scale, int chunk,
+                                void *stream);
+
+/* ------------------------------------------------------------------------ */
+/* Round-to-nearest-even fp32 -> bf16 conversion of n elements (x, y device).
+ * Used to feed fp32 tensors to the bf16 attention calls.                  */
+vsa_status vsa_cast_f32_to_bf16(const float *x, void *y, int64_t n, void *stream);
+
+/* Test hook for the bounded-wait machinery: launches one tiny kernel that
+ * waits on an mbarrier nothing will complete, gives up after timeout_ns of
+ * device time, records VSA_ERR_TIMEOUT in the device status word and
+ * returns.  vsa_device_status() then reports VSA_ERR_TIMEOUT.             */
+vsa_status vsa_debug_wait_timeout(int64_t timeout_ns, void *stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* VSA_H */

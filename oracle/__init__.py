@@ -188,7 +188,8 @@ def tile_neighbourhood_list(grid, tile, radius, block: int, cap: Optional[int] =
     T, H, W = grid
     S = T * H * W
     nb = S // block
-    if cap is None:
+    trim = cap is None
+    if trim:
         cap = nb
     idx = np.empty((nb, cap), np.int32)
     cnt = np.empty(nb, np.int32)
@@ -197,8 +198,9 @@ def tile_neighbourhood_list(grid, tile, radius, block: int, cap: Optional[int] =
                                            _ptr(idx), _ptr(cnt), ctypes.byref(g))
     if rc != 0:
         raise ValueError(f"unsupported tile/radius/block combination (rc={rc})")
-    used = int(cnt.max())
-    return idx[:, :used].copy() if cap == nb else idx, cnt, int(g.value)
+    if trim:
+        idx = idx[:, :int(cnt.max())].copy()
+    return idx, cnt, int(g.value)
 
 
 # --------------------------------------------------------------------------

@@ -1,0 +1,127 @@
+"""The C ABI without a GPU: libvsa.so loads, exports every function that
+include/vsa.h declares, and rejects invalid arguments on the host before any
+launch (the pages raise ValueError for these: "ADR-0001", Conventions;
+windowed_attention's and _validate_qkv's checks)."""
+
+import ctypes
+
+import pytest
+
+import block_sparse_self_b200 as vsa
+from block_sparse_self_b200 import Dims3
+
+FAKE = ctypes.c_void_p(0x10000)      # 16-byte aligned, never dereferenced
+NULL = ctypes.c_void_p(0)
+MIS = ctypes.c_void_p(0x10004)       # misaligned
+
+
+@pytest.fixture(scope="module")
+def L():
+    return vsa.lib()
+
+
+def test_every_declared_symbol_is_exported(L):
+    names = vsa.declared_functions()
+    assert len(names) >= 14
+    for n in names:
+        assert hasattr(L, n), n
+
+
+def _tiles(*ts):
+    arr = (Dims3 * len(ts))(*[Dims3(*t) for t in ts])
+    return arr, len(ts)
+
+
+def test_window_attention_argument_errors(L):
+    def call(**kw):
+        a = dict(q=FAKE, k=FAKE, v=ctypes.c_void_p(0x20000), o=ctypes.c_void_p(0x40000), out=vsa.BF16, B=1, H=2,
+                 S=256, D=64, window=64, sink=16, scale=0.0, chunk=0)
+        a.update(kw)
+        return L.vsa_window_attention(a["q"], a["k"], a["v"], a["o"], a["out"], a["B"], a["H"], a["S"], a["D"],
+                                      a["window"], a["sink"], a["scale"], a["chunk"], NULL)
+    assert call(window=0) == vsa.ERR_INVALID_ARGUMENT
+    assert "window must be >= 1" in vsa.last_error()
+    assert call(sink=-1) == vsa.ERR_INVALID_ARGUMENT
+    assert call(sink=257) == vsa.ERR_INVALID_ARGUMENT
+    assert "cannot exceed sequence length" in vsa.last_error()
+    assert call(chunk=-3) == vsa.ERR_INVALID_ARGUMENT
+    assert call(S=0) == vsa.ERR_INVALID_ARGUMENT
+    assert call(D=0) == vsa.ERR_INVALID_ARGUMENT
+    assert call(D=96) == vsa.ERR_UNSUPPORTED
+    assert call(q=NULL) == vsa.ERR_INVALID_ARGUMENT
+    assert call(k=MIS) == vsa.ERR_INVALID_ARGUMENT
+    assert call(out=7) == vsa.ERR_INVALID_ARGUMENT
+    assert call(o=FAKE) == vsa.ERR_INVALID_ARGUMENT  # output aliases q
+    assert call(scale=float("nan")) == vsa.ERR_INVALID_ARGUMENT
+
+
+def test_block_sparse_attention_argument_errors(L):
+    def call(**kw):
+        a = dict(B=1, H=2, S=256, D=64, block=32, cap=4, group=0)
+        a.update(kw)
+        return L.vsa_block_sparse_attention(FAKE, ctypes.c_void_p(0x20000), ctypes.c_void_p(0x30000),
+                                            ctypes.c_void_p(0x40000), vsa.F32, a["B"], a["H"], a["S"], a["D"],
+                                            a["block"], FAKE, FAKE, a["cap"], 1, a["group"], 0.0, NULL)
+    assert call(block=48) == vsa.ERR_INVALID_ARGUMENT
+    assert call(S=250) == vsa.ERR_INVALID_ARGUMENT
+    assert call(cap=0) == vsa.ERR_INVALID_ARGUMENT
+    assert call(group=-1) == vsa.ERR_INVALID_ARGUMENT
+    assert call(B=0) == vsa.ERR_INVALID_ARGUMENT
+
+
+def test_topk_argument_errors(L):
+    def call(nb=8, k=2, sink=1, dw=0, cap=4):
+        return L.vsa_topk_block_mask(FAKE, 1, 2, nb, k, sink, dw, ctypes.c_void_p(0x20000),
+                                     ctypes.c_void_p(0x30000), cap, NULL)
+    assert call(k=0) == vsa.ERR_INVALID_ARGUMENT
+    assert call(k=9) == vsa.ERR_INVALID_ARGUMENT
+    assert call(sink=-1) == vsa.ERR_INVALID_ARGUMENT
+    assert call(dw=-2) == vsa.ERR_INVALID_ARGUMENT
+    assert call(cap=3) == vsa.ERR_INVALID_ARGUMENT       # needs k + sink + 1 = 4
+    assert "cap" in vsa.last_error()
+    assert call(nb=0) == vsa.ERR_INVALID_ARGUMENT
+
+
+def test_permute_and_select_tiling_argument_errors(L):
+    arr, n = _tiles((2, 4, 4))
+    g = Dims3(4, 8, 8)
+    y = ctypes.c_void_p(0x100000)
+    assert L.vsa_permute(FAKE, y, vsa.F32, 1, 2, 256, 64, Dims3(4, 8, 4), arr, n, NULL, NULL) == \
+        vsa.ERR_INVALID_ARGUMENT  # grid product != S
+    bad, nb_ = _tiles((3, 4, 4))
+    assert L.vsa_permute(FAKE, y, vsa.F32, 1, 2, 256, 64, g, bad, nb_, NULL, NULL) == vsa.ERR_INVALID_ARGUMENT
+    assert "does not divide" in vsa.last_error()
+    assert L.vsa_permute(FAKE, FAKE, vsa.F32, 1, 2, 256, 64, g, arr, n, NULL, NULL) == vsa.ERR_INVALID_ARGUMENT
+    assert L.vsa_permute(FAKE, y, vsa.F32, 1, 2, 256, 64, g, arr, 0, NULL, NULL) == vsa.ERR_INVALID_ARGUMENT
+    # select_tiling: workspace size, then a too-small workspace
+    t3, n3 = _tiles((1, 8, 16), (2, 8, 8), (4, 4, 8))
+    ws = L.vsa_select_tiling_workspace_size(1, 24, Dims3(32, 48, 80), t3, n3)
+    assert ws == 24 * 240 * 3 * 4
+    assert L.vsa_select_tiling(FAKE, vsa.BF16, 1, 24, 122880, 128, Dims3(32, 48, 80), t3, n3, FAKE, NULL,
+                               y, ws - 256, NULL) == vsa.ERR_INVALID_ARGUMENT
+    # an lcm region of too many gcd cells is reported as unsupported
+    big, nbig = _tiles((1, 1, 7), (1, 1, 9), (1, 5, 1), (3, 1, 1))
+    assert L.vsa_select_tiling(FAKE, vsa.BF16, 1, 1, 3 * 5 * 63, 128, Dims3(3, 5, 63), big, nbig, FAKE, NULL,
+                               y, 1 << 20, NULL) == vsa.ERR_UNSUPPORTED
+
+
+def test_structured_list_argument_errors(L):
+    g = ctypes.c_int(0)
+    grid = Dims3(32, 48, 80)
+    idx, cnt = FAKE, ctypes.c_void_p(0x20000)
+    # sliding tile whose volume is neither a multiple nor a divisor of the block
+    assert L.vsa_structured_block_list(vsa.MASK_SLIDING_TILE, grid, Dims3(2, 3, 4), Dims3(1, 1, 1), 128, idx, cnt,
+                                       960, ctypes.byref(g), NULL) == vsa.ERR_UNSUPPORTED
+    assert L.vsa_structured_block_list(vsa.MASK_SLIDING_TILE, grid, Dims3(4, 8, 8), Dims3(1, 1, 1), 128, idx, cnt,
+                                       50, ctypes.byref(g), NULL) == vsa.ERR_INVALID_ARGUMENT  # longest list is 54
+    assert L.vsa_structured_block_list(7, grid, Dims3(4, 8, 8), Dims3(1, 1, 1), 128, idx, cnt, 960,
+                                       ctypes.byref(g), NULL) == vsa.ERR_INVALID_ARGUMENT
+
+
+def test_python_binding_rejects_cpu_tensors():
+    import torch
+    q = torch.zeros(1, 1, 128, 64)
+    with pytest.raises(ValueError):
+        vsa.window_attention(q, q, q, window=8)
+    with pytest.raises(ValueError):
+        vsa.permute(q, (2, 8, 8), [(1, 8, 8)])

@@ -1,0 +1,378 @@
+"""Parity of the CUDA path (through the C ABI) against the fp64 oracle.
+
+Integer and index outputs (permutations, summaries, block lists, tiling
+choices with a clear margin) must match bit for bit; attention outputs must be
+within max-abs 1e-2 and relative-L2 2e-3 of the fp64 oracle (bf16 inputs,
+fp32 accumulation).  Inputs come from the seeded generators in `workloads`.
+"""
+
+import numpy as np
+import pytest
+import torch
+
+import block_sparse_self_b200 as vsa
+import oracle
+from workloads import WORKLOADS, integer_grid, make_qkv, random_scores, smooth_qkv
+
+pytestmark = pytest.mark.gpu
+
+MAX_ABS, REL_L2 = 1e-2, 2e-3
+DEV = "cuda"
+
+
+@pytest.fixture(autouse=True)
+def _no_device_errors():
+    yield
+    vsa.device_status()  # raises if any kernel of the test recorded a failure
+
+
+def _np(t):
+    return t.detach().float().cpu().numpy()
+
+
+def assert_attn_close(got, want, what=""):
+    g = np.asarray(got, np.float64)
+    w = np.asarray(want, np.float64)
+    err = np.abs(g - w).max()
+    rl2 = np.linalg.norm(g - w) / max(np.linalg.norm(w), 1e-30)
+    assert np.isfinite(g).all(), what
+    assert err <= MAX_ABS and rl2 <= REL_L2, f"{what}: max-abs {err:.3e}, rel-L2 {rl2:.3e}"
+
+
+# --------------------------------------------------------------------------
+# permutation
+# --------------------------------------------------------------------------
+
+@pytest.mark.parametrize("dtype,D", [(torch.float32, 64), (torch.bfloat16, 128), (torch.bfloat16, 64),
+                                     (torch.float32, 128)])
+def test_permute_matches_oracle_permutation(dtype, D):
+    grid, tiles = (4, 8, 16), [(1, 8, 16), (2, 8, 8), (4, 4, 8)]
+    x = integer_grid((2, 3, 512, D), 11, dtype, DEV)
+    choice = torch.tensor([2, 0, 1, 1, 2, 0], dtype=torch.int32, device=DEV)
+    y = vsa.permute(x, grid, tiles, choice)
+    xb = x.cpu()
+    for bh, c in enumerate(choice.tolist()):
+        perm = torch.as_tensor(oracle.tile_permutation(grid, tiles[c]))
+        assert torch.equal(y.cpu().view(6, 512, D)[bh], xb.view(6, 512, D)[bh][perm])
+    assert torch.equal(vsa.unpermute(y, grid, tiles, choice), x)
+
+
+def test_permute_without_choice_and_ragged_rows():
+    grid, tile = (3, 4, 6), (1, 2, 3)   # S = 72: fewer rows than one work item
+    x = integer_grid((1, 2, 72, 64), 12, torch.bfloat16, DEV)
+    y = vsa.permute(x, grid, [tile])
+    perm = torch.as_tensor(oracle.tile_permutation(grid, tile))
+    assert torch.equal(y.cpu(), x.cpu()[:, :, perm])
+    assert torch.equal(vsa.unpermute(y, grid, [tile]), x)
+
+
+def test_permute_bad_choice_sets_runtime_status():
+    grid, tiles = (2, 8, 8), [(1, 8, 8), (2, 4, 4)]
+    x = integer_grid((1, 2, 128, 64), 13, torch.bfloat16, DEV)
+    choice = torch.tensor([0, 5], dtype=torch.int32, device=DEV)
+    vsa.permute(x, grid, tiles, choice)
+    with pytest.raises(RuntimeError):
+        vsa.device_status()
+
+
+# --------------------------------------------------------------------------
+# summaries, scores, top-k
+# --------------------------------------------------------------------------
+
+@pytest.mark.parametrize("dtype,D,block", [(torch.bfloat16, 128, 128), (torch.bfloat16, 64, 16),
+                                           (torch.float32, 64, 32), (torch.float32, 128, 256)])
+def test_block_summaries_bit_exact(dtype, D, block):
+    S = 1024
+    x = torch.randn(2, 2, S, D, generator=torch.Generator(DEV).manual_seed(3), device=DEV).to(dtype)
+    mx, mn = vsa.block_summaries(x, block)
+    for bh in range(4):
+        omx, omn = oracle.block_minmax(_np(x.view(4, S, D)[bh]), block)
+        assert np.array_equal(_np(mx.view(4, -1, D)[bh]), omx)
+        assert np.array_equal(_np(mn.view(4, -1, D)[bh]), omn)
+
+
+@pytest.mark.parametrize("dtype,D,nb", [(torch.bfloat16, 128, 40), (torch.float32, 64, 70), (torch.bfloat16, 64, 1)])
+def test_block_scores_exact_on_integer_grid(dtype, D, nb):
+    summ = [integer_grid((1, 2, nb, D), 20 + i, dtype, DEV) for i in range(4)]
+    s = vsa.block_scores(*summ)
+    for h in range(2):
+        want = oracle.block_scores(*(_np(t[0, h]) for t in summ))
+        assert np.array_equal(_np(s[0, h]).astype(np.float64), want)
+
+
+def test_block_scores_smooth_within_fp32_bound():
+    q, k, _ = smooth_qkv(1, 2, (4, 16, 32), 128, seed=5, device=DEV)
+    qp, kp = (vsa.permute(t, (4, 16, 32), [(1, 8, 16)]) for t in (q, k))
+    qmax, qmin = vsa.block_summaries(qp, 128)
+    kmax, kmin = vsa.block_summaries(kp, 128)
+    s = vsa.block_scores(qmax, qmin, kmax, kmin)
+    for h in range(2):
+        a = [_np(t[0, h]).astype(np.float64) for t in (qmax, qmin, kmax, kmin)]
+        want = oracle.block_scores(*a)
+        bound = 4 * np.finfo(np.float32).eps * (np.abs(a[0] + a[1]) @ np.maximum(np.abs(a[2]), np.abs(a[3])).T)
+        assert (np.abs(_np(s[0, h]) - want) <= bound + 1e-30).all()
+
+
+@pytest.mark.parametrize("nb,levels", [(1, 3), (5, 2), (33, 3), (240, 4), (240, 0), (960, 6)])
+def test_topk_lists_bit_exact(nb, levels):
+    sc = random_scores((2, 2, nb, nb), seed=nb + levels, levels=levels, device=DEV)
+    if levels == 0:
+        sc[0, 0, :, 3] = -0.0   # -0 and +0 must rank as equal
+        sc[0, 0, :, 4] = 0.0
+    settings = [(max(1, nb // 6), 1, 0), (1, 0, -1), (nb, 1, 0), (max(1, nb // 10), 3, 2)]
+    for k, n_sink, dw in settings:
+        idx, cnt = vsa.topk_block_mask(sc, k, n_sink, dw)
+        for bh in range(4):
+            oi, oc = oracle.topk_block_list(_np(sc.view(4, nb, nb)[bh]).astype(np.float64), k, n_sink, dw,
+                                            cap=idx.shape[-1])
+            assert np.array_equal(idx.view(4, nb, -1)[bh].cpu().numpy(), oi), (nb, k, n_sink, dw, bh)
+            assert np.array_equal(cnt.view(4, nb)[bh].cpu().numpy(), oc)
+
+
+# --------------------------------------------------------------------------
+# structured lists
+# --------------------------------------------------------------------------
+
+@pytest.mark.parametrize("grid,block,tile", [((32, 48, 80), 128, (4, 8, 8)), ((8, 4, 8), 32, (2, 2, 8)),
+                                             ((6, 12, 16), 64, (2, 4, 8))])
+def test_structured_lists_match_oracle(grid, block, tile):
+    for kind in ("spatial", "temporal", "sliding_tile"):
+        try:
+            idx, cnt, g = vsa.structured_block_list(kind, grid, block, tile=tile, radius=(1, 1, 1))
+        except NotImplementedError:   # e.g. temporal groups of 6 tokens in blocks of 64
+            t, r = oracle.structured_tile(kind, grid, tile, (1, 1, 1))
+            with pytest.raises(ValueError):
+                oracle.tile_neighbourhood_list(grid, t, r, block)
+            continue
+        t, r = oracle.structured_tile(kind, grid, tile, (1, 1, 1))
+        oi, oc, og = oracle.tile_neighbourhood_list(grid, t, r, block, cap=idx.shape[1])
+        assert g == og
+        assert np.array_equal(cnt.cpu().numpy(), oc)
+        assert np.array_equal(idx.cpu().numpy(), oi)
+
+
+# --------------------------------------------------------------------------
+# adaptive tiling choice
+# --------------------------------------------------------------------------
+
+@pytest.mark.parametrize("dtype,D", [(torch.bfloat16, 128), (torch.float32, 64)])
+def test_select_tiling_matches_oracle(dtype, D):
+    grid, tiles = (8, 16, 32), [(1, 8, 16), (2, 8, 8), (4, 4, 8)]
+    kinds = ["spatial", "temporal", "generic", "spatial", "temporal", "generic"]
+    q, _, _ = smooth_qkv(1, 6, grid, D, seed=9, kinds=kinds, dtype=dtype, device=DEV)
+    choice, sics = vsa.select_tiling(q, grid, tiles, return_sics=True)
+    flips = 0
+    for h in range(6):
+        oc, osc = oracle.select_tiling(_np(q[0, h]), grid, tiles)
+        np.testing.assert_allclose(_np(sics[h]), osc, atol=2e-5, rtol=0)
+        margin = np.sort(osc)[-1] - np.sort(osc)[-2]
+        if margin > 1e-4:
+            assert int(choice[h]) == oc, (h, osc)
+        else:
+            flips += 1
+    assert flips <= 1
+
+
+# --------------------------------------------------------------------------
+# attention
+# --------------------------------------------------------------------------
+
+def _random_lists(nb, cap, bh, seed, full_row=True):
+    rng = np.random.default_rng(seed)
+    idx = np.full((bh, nb, cap), -1, np.int32)
+    cnt = np.zeros((bh, nb), np.int32)
+    for b in range(bh):
+        for i in range(nb):
+            n = int(rng.integers(1, cap + 1))
+            if full_row and i == nb - 1:
+                n = cap
+            sel = np.sort(rng.choice(nb, n, replace=False))
+            idx[b, i, :n] = sel
+            cnt[b, i] = n
+    return idx, cnt
+
+
+@pytest.mark.parametrize("D,block,values,out", [(64, 32, "integer", torch.float32), (128, 64, "smooth", torch.bfloat16),
+                                                (128, 128, "smooth", torch.float32), (64, 128, "integer", torch.bfloat16),
+                                                (128, 32, "smooth", torch.bfloat16), (64, 64, "smooth", torch.float32)])
+def test_block_sparse_attention_random_lists(D, block, values, out):
+    B, H, S = 1, 2, 768
+    nb = S // block
+    if values == "integer":
+        q, k, v = (integer_grid((B, H, S, D), 40 + i, torch.bfloat16, DEV) for i in range(3))
+    else:
+        q, k, v = smooth_qkv(B, H, (3, 16, 16), D, seed=41, device=DEV)
+    idx, cnt = _random_lists(nb, min(nb, 5), B * H, seed=block + D)
+    ti = torch.as_tensor(idx, device=DEV).view(B, H, nb, -1)
+    tc = torch.as_tensor(cnt, device=DEV).view(B, H, nb)
+    o = vsa.block_sparse_attention(q, k, v, ti, tc, block, out_dtype=out)
+    for h in range(H):
+        want = oracle.block_sparse_attention(_np(q[0, h]), _np(k[0, h]), _np(v[0, h]), idx[h], cnt[h], block)
+        assert_attn_close(_np(o[0, h]), want, f"head {h}")
+
+
+def test_block_sparse_attention_group_mask_and_shared_list():
+    """temporal_only: tile (T,1,1) with T=8 inside blocks of 32 -> group mask."""
+    grid, block = (8, 8, 8), 32
+    q, k, v = smooth_qkv(2, 2, grid, 64, seed=44, device=DEV)
+    o = vsa.structured_attention(q, k, v, "temporal", grid, block, out_dtype=torch.float32)
+    t, r = oracle.structured_tile("temporal", grid)
+    idx, cnt, g = oracle.tile_neighbourhood_list(grid, t, r, block)
+    assert g == 8
+    perm = oracle.tile_permutation(grid, t)
+    for b in range(2):
+        for h in range(2):
+            qp, kp, vp = (oracle.permute_rows(_np(x[b, h]), perm) for x in (q, k, v))
+            op = oracle.block_sparse_attention(qp, kp, vp, idx, cnt, block, g)
+            want = np.empty_like(op)
+            want[perm] = op
+            assert_attn_close(_np(o[b, h]), want, f"b{b} h{h}")
+
+
+def test_block_sparse_attention_invalid_lists_write_zeros_and_set_status():
+    B, H, S, D, block = 1, 1, 512, 64, 128
+    q, k, v = (integer_grid((B, H, S, D), 50 + i, torch.bfloat16, DEV) for i in range(3))
+    idx = torch.tensor([[[0, 1], [1, 0], [2, 9], [3, -1]]], dtype=torch.int32, device=DEV).view(1, 1, 4, 2)
+    cnt = torch.tensor([2, 2, 2, 0], dtype=torch.int32, device=DEV).view(1, 1, 4)
+    o = vsa.block_sparse_attention(q, k, v, idx, cnt, block, out_dtype=torch.float32)
+    with pytest.raises(RuntimeError):
+        vsa.device_status()
+    oo = o.cpu()
+    assert (oo[0, 0, 128:] == 0).all()          # descending, out of range, empty
+    want = oracle.block_sparse_attention(_np(q[0, 0]), _np(k[0, 0]), _np(v[0, 0]), np.array([[0, 1]], np.int32),
+                                         np.array([2], np.int32), block, rows=np.arange(128))
+    assert_attn_close(_np(oo[0, 0, :128]), want)
+
+
+@pytest.mark.parametrize("S,D,window,sink", [(256, 64, 64, 16), (300, 128, 100, 7), (1000, 64, 2000, 0),
+                                             (384, 128, 1, 0), (640, 64, 257, 300), (1280, 128, 300, 128),
+                                             (129, 64, 128, 1)])
+def test_window_attention_matches_oracle(S, D, window, sink):
+    q, k, v = (integer_grid((1, 2, S, D), 60 + i, torch.bfloat16, DEV) for i in range(3))
+    o = vsa.window_attention(q, k, v, window, sink, out_dtype=torch.float32)
+    for h in range(2):
+        want = oracle.window_attention(_np(q[0, h]), _np(k[0, h]), _np(v[0, h]), window, sink)
+        assert_attn_close(_np(o[0, h]), want, f"head {h}")
+    # the page's query chunk size groups the work but never changes the result
+    o2 = vsa.window_attention(q, k, v, window, sink, chunk_size=7, out_dtype=torch.float32)
+    assert torch.equal(o, o2)
+
+
+def test_wait_timeout_is_reported():
+    vsa.debug_wait_timeout(2_000_000)  # 2 ms
+    with pytest.raises(RuntimeError, match="timeout"):
+        vsa.device_status()
+
+
+# --------------------------------------------------------------------------
+# end to end on the tiny workload, then sampled checks at full size
+# --------------------------------------------------------------------------
+
+def test_tiny_workload_end_to_end():
+    w = WORKLOADS["tiny_s256"]
+    q, k, v = make_qkv(w, device=DEV)                  # fp32 values on the {-4..4}/4 grid
+    o, mid = vsa.spade_attention(q, k, v, w.grid, list(w.tiles), topk=w.k, n_sink_blocks=1, diag_halfwidth=0,
+                                 out_dtype=torch.float32, return_intermediates=True)
+    ow = vsa.window_attention(q, k, v, w.window, w.sink, out_dtype=torch.float32)
+    for h in range(w.heads):
+        res = oracle.spade_head(_np(q[0, h]), _np(k[0, h]), _np(v[0, h]), w.grid, list(w.tiles), w.k)
+        assert np.array_equal(mid["idx"][0, h].cpu().numpy(), res["idx"])
+        assert np.array_equal(mid["cnt"][0, h].cpu().numpy(), res["cnt"])
+        assert np.array_equal(_np(mid["scores"][0, h]).astype(np.float64), res["score"])
+        assert_attn_close(_np(o[0, h]), res["out"], f"spade head {h}")
+        want = oracle.window_attention(_np(q[0, h]), _np(k[0, h]), _np(v[0, h]), w.window, w.sink)
+        assert_attn_close(_np(ow[0, h]), want, f"window head {h}")
+
+
+def _sample_blocks(nb, seed, n=16):
+    rng = np.random.default_rng(seed)
+    mid = rng.choice(np.arange(1, nb - 1), n - 2, replace=False)
+    return sorted({0, nb - 1, *mid.tolist()})
+
+
+def test_spade_fixed_full_size_sampled():
+    """40 heads, S = 30720, tile (1,8,16), k = 40: integer-grid values make
+    the block scores exact, so whole lists must match bit for bit."""
+    w = WORKLOADS["spade_fixed_s30720"]
+    q, k, v = make_qkv(w, device=DEV, values="integer")
+    o, mid = vsa.spade_attention(q, k, v, w.grid, list(w.tiles), topk=w.k, return_intermediates=True)
+    for h in (0, 23, 39):
+        blocks = _sample_blocks(w.nb, h)
+        res = oracle.spade_head(_np(q[0, h]), _np(k[0, h]), _np(v[0, h]), w.grid, list(w.tiles), w.k,
+                                query_blocks=blocks)
+        assert np.array_equal(mid["idx"][0, h].cpu().numpy(), res["idx"])
+        assert np.array_equal(mid["cnt"][0, h].cpu().numpy(), res["cnt"])
+        got = _np(mid["out_perm"][0, h])[res["rows"]]
+        assert_attn_close(got, res["out_perm"], f"head {h}")
+    # the unpermuted output is the permuted one scattered back
+    perm = torch.as_tensor(oracle.tile_permutation(w.grid, w.tiles[0]), device=DEV)
+    assert torch.equal(o[0, 5][perm], mid["out_perm"][0, 5])
+
+
+def test_spade_adaptive_full_size_sampled():
+    """24 heads, S = 122880, three candidate tilings, k = 96, smooth fields:
+    tiling choices must match the oracle wherever its margin is clear; the
+    lists must be valid top-k sets under the oracle's scores (fp32 rounding
+    may reorder near-ties), and rows whose lists match are compared."""
+    w = WORKLOADS["spade_adaptive_s122880"]
+    q, k, v = make_qkv(w, device=DEV)
+    o, mid = vsa.spade_attention(q, k, v, w.grid, list(w.tiles), topk=w.k, return_intermediates=True)
+    choice = mid["choice"].cpu().numpy()
+    picked = set()
+    for h in range(w.heads):
+        oc, osc = oracle.select_tiling(_np(q[0, h]), w.grid, list(w.tiles))
+        margin = np.sort(osc)[-1] - np.sort(osc)[-2]
+        if margin > 1e-4:
+            assert choice[h] == oc, (h, osc)
+        picked.add(int(choice[h]))
+    assert len(picked) >= 2   # the heads do not all pick one tiling
+    for h in (0, 13):
+        tile = w.tiles[int(choice[h])]
+        blocks = _sample_blocks(w.nb, 100 + h)
+        res = oracle.spade_head(_np(q[0, h]), _np(k[0, h]), _np(v[0, h]), w.grid, [tile], w.k, query_blocks=blocks)
+        gi = mid["idx"][0, h].cpu().numpy()
+        gc = mid["cnt"][0, h].cpu().numpy()
+        s = res["score"]
+        same = 0
+        for i in range(w.nb):
+            sel = set(gi[i, :gc[i]].tolist())
+            forced = {0, i}
+            assert forced <= sel and w.k <= len(sel) <= w.k + len(forced)
+            kth = np.sort(s[i])[::-1][w.k - 1]
+            tol = 1e-5 * max(1.0, float(np.abs(s[i]).max()))
+            assert all(s[i, j] >= kth - tol for j in sel - forced), (h, i)
+            assert all(s[i, j] <= kth + tol for j in set(range(w.nb)) - sel), (h, i)
+            same += int(np.array_equal(gi[i], res["idx"][i]))
+        assert same >= 0.9 * w.nb
+        got = _np(mid["out_perm"][0, h])
+        for bi, b in enumerate(blocks):
+            if np.array_equal(gi[b], res["idx"][b]):
+                assert_attn_close(got[b * 128:(b + 1) * 128], res["out_perm"][bi * 128:(bi + 1) * 128],
+                                  f"head {h} block {b}")
+
+
+def test_window_full_size_sampled():
+    w = WORKLOADS["window_s30720"]
+    q, k, v = make_qkv(w, device=DEV)
+    o = vsa.window_attention(q, k, v, w.window, w.sink, chunk_size=w.chunk)
+    for h in (0, 17):
+        rows = np.concatenate([np.arange(b * 128, (b + 1) * 128) for b in _sample_blocks(w.S // 128, h)])
+        want = oracle.window_attention(_np(q[0, h]), _np(k[0, h]), _np(v[0, h]), w.window, w.sink, rows=rows)
+        assert_attn_close(_np(o[0, h])[rows], want, f"head {h}")
+
+
+@pytest.mark.parametrize("kind", ["spatial", "temporal", "sliding_tile"])
+def test_structured_full_size_sampled(kind):
+    w = WORKLOADS["structured_s122880"]
+    q, k, v = make_qkv(w, device=DEV, B=2, heads=2)
+    o = vsa.structured_attention(q, k, v, kind, w.grid, 128, tile=w.sliding_tile, radius=w.sliding_radius)
+    t, r = oracle.structured_tile(kind, w.grid, w.sliding_tile, w.sliding_radius)
+    idx, cnt, g = oracle.tile_neighbourhood_list(w.grid, t, r, 128)
+    perm = oracle.tile_permutation(w.grid, t)
+    b, h = 1, 1
+    qp, kp, vp = (oracle.permute_rows(_np(x[b, h]), perm) for x in (q, k, v))
+    blocks = _sample_blocks(w.nb, 7)
+    rows = np.concatenate([np.arange(bb * 128, (bb + 1) * 128) for bb in blocks])
+    want = oracle.block_sparse_attention(qp, kp, vp, idx, cnt, 128, g, rows=rows)
+    got = _np(o[b, h])[perm[rows]]
+    assert_attn_close(got, want, kind)
