@@ -103,9 +103,10 @@ vsa_status check_d(int D) {
     return VSA_OK;
 }
 
-bool overlaps(const void *a, const void *b, size_t n) {
+// [a, a + na) and [b, b + nb) share a byte
+bool overlaps(const void *a, size_t na, const void *b, size_t nb) {
     const uintptr_t x = reinterpret_cast<uintptr_t>(a), y = reinterpret_cast<uintptr_t>(b);
-    return x < y + n && y < x + n;
+    return x < y + nb && y < x + na;
 }
 
 #define VSA_TRY(expr)                     \
@@ -181,7 +182,7 @@ static vsa_status permute_common(const void *src, void *dst, vsa_dtype dtype, in
     VSA_TRY(check_d(D));
     VSA_REQUIRE(aligned16(src) && aligned16(dst), "x and y must be non-NULL 16-byte aligned device pointers");
     const size_t bytes = static_cast<size_t>(B) * n_heads * S * D * esize_of(dtype);
-    VSA_REQUIRE(!overlaps(src, dst, bytes), "x and y must not overlap");
+    VSA_REQUIRE(!overlaps(src, bytes, dst, bytes), "x and y must not overlap");
     VSA_REQUIRE(choice == nullptr || aligned4(choice), "choice must be NULL or 4-byte aligned");
     VSA_TRY(check_grid(grid, S));
     TileSet ts;
@@ -305,8 +306,7 @@ static vsa_status check_attention_common(const void *q, const void *k, const voi
                 "q, k, v and o must be non-NULL 16-byte aligned device pointers");
     const size_t obytes = static_cast<size_t>(B) * n_heads * S * D * esize_of(out_dtype);
     const size_t ibytes = static_cast<size_t>(B) * n_heads * S * D * 2;
-    VSA_REQUIRE(!overlaps(o, q, obytes > ibytes ? obytes : ibytes) && !overlaps(o, k, obytes > ibytes ? obytes : ibytes) &&
-                    !overlaps(o, v, obytes > ibytes ? obytes : ibytes),
+    VSA_REQUIRE(!overlaps(o, obytes, q, ibytes) && !overlaps(o, obytes, k, ibytes) && !overlaps(o, obytes, v, ibytes),
                 "o must not overlap q, k or v");
     VSA_REQUIRE(scale == scale && scale < 3.0e38f, "scale must be finite");
     return VSA_OK;

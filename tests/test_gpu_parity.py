@@ -1,9 +1,13 @@
 """Parity of the CUDA path (through the C ABI) against the fp64 oracle.
 
 Integer and index outputs (permutations, summaries, block lists, tiling
-choices with a clear margin) must match bit for bit; attention outputs must be
-within max-abs 1e-2 and relative-L2 2e-3 of the fp64 oracle (bf16 inputs,
-fp32 accumulation).  Inputs come from the seeded generators in `workloads`.
+choices with a clear margin) must match bit for bit.  Attention outputs, with
+bf16 inputs and fp32 accumulation, must be within max-abs 1e-2 and relative-L2
+2e-3 of the fp64 oracle; that bar is applied to the kernel's fp32-output mode.
+A bf16 output is that fp32 result rounded once to nearest-even (checked bit
+for bit): bf16's unit roundoff 2^-8 alone puts about 1.6e-3 of relative-L2
+error on any bf16 output.  Inputs come from the seeded generators in
+`workloads`.
 """
 
 import numpy as np
@@ -119,7 +123,7 @@ def test_topk_lists_bit_exact(nb, levels):
     if levels == 0:
         sc[0, 0, :, 3] = -0.0   # -0 and +0 must rank as equal
         sc[0, 0, :, 4] = 0.0
-    settings = [(max(1, nb // 6), 1, 0), (1, 0, -1), (nb, 1, 0), (max(1, nb // 10), 3, 2)]
+    settings = [(max(1, nb // 6), 1, 0), (1, 0, -1), (nb, 1, 0), (max(1, nb // 10), min(3, nb), 2)]
     for k, n_sink, dw in settings:
         idx, cnt = vsa.topk_block_mask(sc, k, n_sink, dw)
         for bh in range(4):
@@ -192,10 +196,9 @@ def _random_lists(nb, cap, bh, seed, full_row=True):
     return idx, cnt
 
 
-@pytest.mark.parametrize("D,block,values,out", [(64, 32, "integer", torch.float32), (128, 64, "smooth", torch.bfloat16),
-                                                (128, 128, "smooth", torch.float32), (64, 128, "integer", torch.bfloat16),
-                                                (128, 32, "smooth", torch.bfloat16), (64, 64, "smooth", torch.float32)])
-def test_block_sparse_attention_random_lists(D, block, values, out):
+@pytest.mark.parametrize("D,block,values", [(64, 32, "integer"), (128, 64, "smooth"), (128, 128, "smooth"),
+                                            (64, 128, "integer"), (128, 32, "smooth"), (64, 64, "smooth")])
+def test_block_sparse_attention_random_lists(D, block, values):
     B, H, S = 1, 2, 768
     nb = S // block
     if values == "integer":
@@ -205,7 +208,9 @@ def test_block_sparse_attention_random_lists(D, block, values, out):
     idx, cnt = _random_lists(nb, min(nb, 5), B * H, seed=block + D)
     ti = torch.as_tensor(idx, device=DEV).view(B, H, nb, -1)
     tc = torch.as_tensor(cnt, device=DEV).view(B, H, nb)
-    o = vsa.block_sparse_attention(q, k, v, ti, tc, block, out_dtype=out)
+    o = vsa.block_sparse_attention(q, k, v, ti, tc, block, out_dtype=torch.float32)
+    ob = vsa.block_sparse_attention(q, k, v, ti, tc, block, out_dtype=torch.bfloat16)
+    assert torch.equal(ob, o.to(torch.bfloat16))
     for h in range(H):
         want = oracle.block_sparse_attention(_np(q[0, h]), _np(k[0, h]), _np(v[0, h]), idx[h], cnt[h], block)
         assert_attn_close(_np(o[0, h]), want, f"head {h}")
@@ -250,6 +255,7 @@ def test_block_sparse_attention_invalid_lists_write_zeros_and_set_status():
 def test_window_attention_matches_oracle(S, D, window, sink):
     q, k, v = (integer_grid((1, 2, S, D), 60 + i, torch.bfloat16, DEV) for i in range(3))
     o = vsa.window_attention(q, k, v, window, sink, out_dtype=torch.float32)
+    assert torch.equal(vsa.window_attention(q, k, v, window, sink), o.to(torch.bfloat16))
     for h in range(2):
         want = oracle.window_attention(_np(q[0, h]), _np(k[0, h]), _np(v[0, h]), window, sink)
         assert_attn_close(_np(o[0, h]), want, f"head {h}")
@@ -295,7 +301,8 @@ def test_spade_fixed_full_size_sampled():
     the block scores exact, so whole lists must match bit for bit."""
     w = WORKLOADS["spade_fixed_s30720"]
     q, k, v = make_qkv(w, device=DEV, values="integer")
-    o, mid = vsa.spade_attention(q, k, v, w.grid, list(w.tiles), topk=w.k, return_intermediates=True)
+    o, mid = vsa.spade_attention(q, k, v, w.grid, list(w.tiles), topk=w.k, out_dtype=torch.float32,
+                                 return_intermediates=True)
     for h in (0, 23, 39):
         blocks = _sample_blocks(w.nb, h)
         res = oracle.spade_head(_np(q[0, h]), _np(k[0, h]), _np(v[0, h]), w.grid, list(w.tiles), w.k,
@@ -316,7 +323,8 @@ def test_spade_adaptive_full_size_sampled():
     may reorder near-ties), and rows whose lists match are compared."""
     w = WORKLOADS["spade_adaptive_s122880"]
     q, k, v = make_qkv(w, device=DEV)
-    o, mid = vsa.spade_attention(q, k, v, w.grid, list(w.tiles), topk=w.k, return_intermediates=True)
+    o, mid = vsa.spade_attention(q, k, v, w.grid, list(w.tiles), topk=w.k, out_dtype=torch.float32,
+                                 return_intermediates=True)
     choice = mid["choice"].cpu().numpy()
     picked = set()
     for h in range(w.heads):
@@ -354,7 +362,7 @@ def test_spade_adaptive_full_size_sampled():
 def test_window_full_size_sampled():
     w = WORKLOADS["window_s30720"]
     q, k, v = make_qkv(w, device=DEV)
-    o = vsa.window_attention(q, k, v, w.window, w.sink, chunk_size=w.chunk)
+    o = vsa.window_attention(q, k, v, w.window, w.sink, chunk_size=w.chunk, out_dtype=torch.float32)
     for h in (0, 17):
         rows = np.concatenate([np.arange(b * 128, (b + 1) * 128) for b in _sample_blocks(w.S // 128, h)])
         want = oracle.window_attention(_np(q[0, h]), _np(k[0, h]), _np(v[0, h]), w.window, w.sink, rows=rows)
@@ -365,7 +373,8 @@ def test_window_full_size_sampled():
 def test_structured_full_size_sampled(kind):
     w = WORKLOADS["structured_s122880"]
     q, k, v = make_qkv(w, device=DEV, B=2, heads=2)
-    o = vsa.structured_attention(q, k, v, kind, w.grid, 128, tile=w.sliding_tile, radius=w.sliding_radius)
+    o = vsa.structured_attention(q, k, v, kind, w.grid, 128, tile=w.sliding_tile, radius=w.sliding_radius,
+                                 out_dtype=torch.float32)
     t, r = oracle.structured_tile(kind, w.grid, w.sliding_tile, w.sliding_radius)
     idx, cnt, g = oracle.tile_neighbourhood_list(w.grid, t, r, 128)
     perm = oracle.tile_permutation(w.grid, t)
