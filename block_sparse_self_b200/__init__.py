@@ -53,6 +53,7 @@ def lib() -> ctypes.CDLL:
         "vsa_device_status": ([P], I),
         "vsa_select_tiling_workspace_size": ([I, I, D3, P, I], SZ),
         "vsa_select_tiling": ([P, I, I, I, I, I, D3, P, I, P, P, P, SZ, P], I),
+        "vsa_select_tiling_noalloc": ([P, I, I, I, I, I, D3, P, I, P, P, P], I),
         "vsa_permute": ([P, P, I, I, I, I, I, D3, P, I, P, P], I),
         "vsa_unpermute": ([P, P, I, I, I, I, I, D3, P, I, P, P], I),
         "vsa_block_summaries": ([P, I, I, I, I, I, I, P, P, P], I),
@@ -153,6 +154,21 @@ def select_tiling(q: torch.Tensor, grid, tiles, return_sics: bool = False):
     ws = torch.empty(max(ws_bytes, 256) // 4, dtype=torch.float32, device=q.device)
     _check(lib().vsa_select_tiling(_ptr(q), _dtype_code(q, "q"), B, H, S, D, g, arr, n, _ptr(choice),
                                    _ptr(sics), _ptr(ws), ws.numel() * 4, _stream(q.device)))
+    return (choice, sics) if return_sics else choice
+
+
+def select_tiling_noalloc(q: torch.Tensor, grid, tiles, return_sics: bool = False):
+    """select_tiling for callers that cannot allocate device scratch: the
+    library's own fixed scratch array is used (see vsa_select_tiling_noalloc
+    in include/vsa.h for its size limit, and note that overlapping calls on
+    one GPU race on it).  Only the outputs are allocated here."""
+    _cuda(q, "q")
+    B, H, S, D = _bhsd(q, "q")
+    arr, n = _tiles_arg(tiles)
+    choice = torch.empty(B * H, dtype=torch.int32, device=q.device)
+    sics = torch.empty(B * H, n, dtype=torch.float32, device=q.device) if return_sics else None
+    _check(lib().vsa_select_tiling_noalloc(_ptr(q), _dtype_code(q, "q"), B, H, S, D, Dims3(*grid), arr, n,
+                                           _ptr(choice), _ptr(sics), _stream(q.device)))
     return (choice, sics) if return_sics else choice
 
 

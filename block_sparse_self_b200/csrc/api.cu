@@ -174,6 +174,36 @@ vsa_status vsa_select_tiling(const void *q, vsa_dtype dtype, int B, int n_heads,
                       "select_tiling launch");
 }
 
+vsa_status vsa_select_tiling_noalloc(const void *q, vsa_dtype dtype, int B, int n_heads, int S, int D,
+                                     vsa_dims3 grid, const vsa_dims3 *tiles, int n_tiles, int32_t *choice,
+                                     float *sics, void *stream) {
+    VSA_REQUIRE(esize_of(dtype) != 0, "dtype must be VSA_BF16 or VSA_F32");
+    VSA_TRY(check_bhsd(B, n_heads, S, D));
+    VSA_TRY(check_d(D));
+    VSA_REQUIRE(aligned16(q), "q must be a non-NULL 16-byte aligned device pointer");
+    VSA_REQUIRE(aligned4(choice), "choice must be a non-NULL 4-byte aligned device pointer");
+    VSA_REQUIRE(sics == nullptr || aligned4(sics), "sics must be NULL or 4-byte aligned");
+    VSA_TRY(check_grid(grid, S));
+    TileSet ts;
+    VSA_TRY(check_tiles(grid, tiles, n_tiles, &ts));
+    SelectGeom g;
+    if (!select_geometry(grid.t, grid.h, grid.w, ts, &g))
+        return fail(VSA_ERR_UNSUPPORTED,
+                    "the candidate tiles' lcm region holds %d cells of their gcd tile (at most 256 supported)",
+                    g.cells);
+    const size_t need = vsa_select_tiling_workspace_size(B, n_heads, grid, tiles, n_tiles);
+    VSA_REQUIRE(need <= VSA_SELECT_TILING_NOALLOC_MAX_BYTES,
+                "this call needs %zu bytes of scratch; the allocation-free variant holds at most %d bytes "
+                "(use vsa_select_tiling with a workspace instead)",
+                need, VSA_SELECT_TILING_NOALLOC_MAX_BYTES);
+    float *scratch = nullptr;
+    size_t scratch_bytes = 0;
+    VSA_TRY(select_static_scratch(&scratch, &scratch_bytes));
+    return check_cuda(launch_select_tiling(q, esize_of(dtype), B * n_heads, S, D, grid.t, grid.h, grid.w, ts, g,
+                                           choice, sics, scratch, status_or_null(), as_stream(stream)),
+                      "select_tiling (no-alloc) launch");
+}
+
 static vsa_status permute_common(const void *src, void *dst, vsa_dtype dtype, int B, int n_heads, int S, int D,
                                  vsa_dims3 grid, const vsa_dims3 *tiles, int n_tiles, const int32_t *choice,
                                  bool inverse, void *stream) {

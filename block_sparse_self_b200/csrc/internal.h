@@ -64,4 +64,8 @@ vsa_status launch_attention(const AttnLaunch &a, int *status, cudaStream_t st);
 
 cudaError_t launch_wait_timeout(uint64_t limit_ns, int *status, cudaStream_t st);
 
+// Address and size of the file-scope scratch array that
+// vsa_select_tiling_noalloc uses (looked up once per device).
+vsa_status select_static_scratch(float **ptr, size_t *bytes);
+
 }  // namespace vsa

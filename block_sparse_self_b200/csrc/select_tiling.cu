@@ -14,6 +14,8 @@
 // and turns the norm into the tile's SICS; it writes per-candidate sums of
 // tile SICS for its region.  Pass 2: one warp per bh adds the regions in a
 // fixed order, divides by the tile count and takes the argmax.
+#include <mutex>
+
 #include "common.cuh"
 #include "internal.h"
 
@@ -261,3 +263,40 @@ cudaError_t launch_select_tiling(const void *q, int esize, int BH, int S, int D,
 }
 
 }  // namespace vsa
+
+// ---------------------------------------------------------------------------
+// Scratch for vsa_select_tiling_noalloc: a file-scope device array, so that
+// callers who cannot allocate device memory need not pass a workspace.  Every
+// GPU that loads the library holds it until the process exits.
+// ---------------------------------------------------------------------------
+namespace {
+constexpr size_t kStaticScratchBytes = VSA_SELECT_TILING_NOALLOC_MAX_BYTES;
+static __device__ __align__(256) float g_select_scratch[kStaticScratchBytes / sizeof(float)];
+}  // namespace
+
+namespace vsa {
+
+// Device address of g_select_scratch on the current device.  In host code the
+// array's name is only a host-side stand-in, so the address is looked up with
+// cudaGetSymbolAddress once per device (with that device current) and cached.
+vsa_status select_static_scratch(float **ptr, size_t *bytes) {
+    static std::mutex mu;
+    static float *addr[128] = {};
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return check_cuda(e, "cudaGetDevice");
+    if (dev < 0 || dev >= 128) return fail(VSA_ERR_UNSUPPORTED, "device ordinal %d out of range", dev);
+    std::lock_guard<std::mutex> lock(mu);
+    if (!addr[dev]) {
+        void *p = nullptr;
+        e = cudaGetSymbolAddress(&p, g_select_scratch);
+        if (e != cudaSuccess) return check_cuda(e, "cudaGetSymbolAddress(select_tiling scratch)");
+        addr[dev] = static_cast<float *>(p);
+    }
+    *ptr = addr[dev];
+    *bytes = kStaticScratchBytes;
+    return VSA_OK;
+}
+
+}  // namespace vsa
+

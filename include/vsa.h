@@ -94,6 +94,32 @@ vsa_status vsa_select_tiling(const void *q, vsa_dtype dtype, int B, int n_heads,
                              int n_tiles, int32_t *choice, float *sics,
                              void *workspace, size_t workspace_bytes, void *stream);
 
+/* Allocation-free variant of vsa_select_tiling.  The pages have no
+ * counterpart: this entry point exists for callers that cannot allocate
+ * device memory, or pass a workspace, at the point where they choose the
+ * tilings -- for example code that runs inside a memory pool or allocator,
+ * a process whose device memory is entirely reserved by another framework's
+ * pool, or a plugin interface that hands over inputs and outputs but no
+ * allocator and no workspace argument.
+ *
+ * Same arguments and results as vsa_select_tiling, without the workspace.
+ * The scratch lives in a file-scope device array of
+ * VSA_SELECT_TILING_NOALLOC_MAX_BYTES bytes that every GPU loading the
+ * library holds until the process exits; a request whose scratch
+ * (vsa_select_tiling_workspace_size) exceeds it returns
+ * VSA_ERR_INVALID_ARGUMENT without launching anything.  The call allocates
+ * nothing.  The first call on a device looks the array's device address up
+ * (cudaGetSymbolAddress, with that device current) and caches it; make that
+ * first call before any stream capture.  All calls share the one array:
+ * every scratch entry a call reads is written earlier in the same call, so
+ * nothing has to start at zero, but calls whose work overlaps on the GPU
+ * (different streams, or different host threads on one device) race on it
+ * and must be serialised by the caller.                                   */
+#define VSA_SELECT_TILING_NOALLOC_MAX_BYTES (1 << 20)
+vsa_status vsa_select_tiling_noalloc(const void *q, vsa_dtype dtype, int B, int n_heads,
+                                     int S, int D, vsa_dims3 grid, const vsa_dims3 *tiles,
+                                     int n_tiles, int32_t *choice, float *sics, void *stream);
+
 /* ------------------------------------------------------------------------ */
 /* Tile-contiguous permutation and its inverse.
  * "ADR-0001", step 6 (block_contiguous_permutation, invert_permutation);
