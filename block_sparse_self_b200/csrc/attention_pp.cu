@@ -1,0 +1,580 @@
+// attention_pp.cu -- block-sparse and sliding-window attention on tcgen05 tensor
+// cores, two query tiles per CTA ("ping-pong") for 128-token blocks.
+//
+// Semantics are those of attention.cu ("Adaptive tiling (SPADE)", Recipe and
+// recipe note; "fastvideo/mlx_runtime/windowed_attention.py", Window policy
+// and _key_ranges_for_block).  This variant keeps the tensor pipe busy while a
+// softmax runs: each CTA owns two 128-row query tiles A and B, and while one
+// tile's softmax warpgroup turns S into P, the MMA warp runs the other tile's
+// QK^T and PV.
+//
+// Warps: 0-3 softmax/epilogue of tile A, 4-7 of tile B (thread = query row =
+// TMEM lane), 8 TMA producer, 9 MMA issuer and TMEM owner.  Three warps share
+// some SM sub-partitions, so a thread has at most 168 registers: the softmax
+// keeps one block's 128 scores in registers and rescales O in 8-column steps.
+// Tensor memory (512 columns): S_A, S_B (128 fp32 columns each), O_A, O_B
+// (D columns each).  P (bf16, 64 columns) is written over the first half of
+// its tile's S and is the TMEM operand of the PV MMA, so shared memory only
+// holds Q_A, Q_B, a ring of K tiles and a ring of V tiles.  The producer loads
+// and the MMA warp issues in one fixed program order:
+//   QK_A(0) QK_B(0) | PV_A(j) QK_A(j+1) PV_B(j) QK_B(j+1) | j = 0, 1, ...
+// An MMA only orders behind an earlier one with the same accumulator, so
+// QK_t(j+1), which overwrites the P_t(j) that PV_t(j) reads, first waits for
+// PV_t(j) to complete.
+//
+// The softmax takes 2^x for 5 of every 8 pairs of columns on the MUFU and for
+// the rest on the FMA pipe: Cody-Waite range reduction x = n + f with
+// n = rint(x), f in [-1/2, 1/2], and a degree-3 polynomial for 2^f whose
+// coefficients were fitted here by a Remez exchange on the relative error
+// (max relative error 7.5e-5, far below bf16's 2^-8 rounding of P).
+#include <math.h>
+
+#include "common.cuh"
+#include "internal.h"
+
+namespace vsa {
+
+namespace {
+
+struct PPArgs {
+    int S, nq;
+    const int32_t *idx, *cnt;
+    int cap, list_per_head, group, nb;
+    int half, sink, dense;
+    float scale_log2;
+    void *out;
+    int out_f32;
+    int *status;
+};
+
+template <int D>
+struct PPCfg {
+    static constexpr int KSLABS = D / 64;
+    static constexpr int SLAB = 128 * 128;         // 128 rows x 128 bytes
+    static constexpr int TILE_BYTES = SLAB * KSLABS;  // Q, K or V tile of 128 rows
+    static constexpr int NK = D == 128 ? 3 : 4;    // K ring depth
+    static constexpr int NV = D == 128 ? 2 : 4;    // V ring depth
+    static constexpr int O_COL = 256;              // O_A at 256, O_B at 256 + D
+    static constexpr int N_BARS = 1 + 2 * NK + 2 * NV + 2 + 2 + 2 + 1;
+    static constexpr int SMEM = 1024 + (2 + NK + NV) * TILE_BYTES + N_BARS * 8 + 64;
+    static_assert(SMEM <= 232448, "shared memory");
+};
+
+constexpr int kThreads = 320;
+constexpr float kRescale = 8.0f;     // rescale O only when the max grows by > 2^8
+constexpr float kRound = 12582912.f;  // 1.5 * 2^23
+constexpr float kC0 = 0.9999280571937561f, kC1 = 0.6932609677314758f, kC2 = 0.2426111251115799f,
+                kC3 = 0.0551716685295105f;
+
+__device__ __forceinline__ uint64_t f2pack(float lo, float hi) {
+    uint64_t r;
+    asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
+    return r;
+}
+__device__ __forceinline__ void f2unpack(uint64_t v, float &lo, float &hi) {
+    asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(v));
+}
+__device__ __forceinline__ uint64_t ffma2(uint64_t a, uint64_t b, uint64_t c) {
+    uint64_t d;
+    asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
+    return d;
+}
+__device__ __forceinline__ uint64_t fadd2(uint64_t a, uint64_t b) {
+    uint64_t d;
+    asm("add.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+    return d;
+}
+__device__ __forceinline__ uint64_t fsub2(uint64_t a, uint64_t b) {
+    uint64_t d;
+    asm("sub.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+    return d;
+}
+__device__ __forceinline__ float fmax3(float a, float b, float c) {
+    float d;
+    asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+    return d;
+}
+
+// 2^x for a pair on the FMA pipe (see the file comment).  x is clamped at
+// -125 so that every result stays a normal number (2^-125 ~ 2.4e-38).
+__device__ __forceinline__ uint64_t exp2_poly2(uint64_t x) {
+    float a, b;
+    f2unpack(x, a, b);
+    x = f2pack(fmaxf(a, -125.f), fmaxf(b, -125.f));
+    const uint64_t r2 = f2pack(kRound, kRound);
+    const uint64_t t = fadd2(x, r2);      // n sits in the low mantissa bits
+    const uint64_t n = fsub2(t, r2);      // rint(x)
+    const uint64_t f = fsub2(x, n);       // in [-1/2, 1/2]
+    uint64_t p = ffma2(f, f2pack(kC3, kC3), f2pack(kC2, kC2));
+    p = ffma2(p, f, f2pack(kC1, kC1));
+    p = ffma2(p, f, f2pack(kC0, kC0));
+    float plo, phi, tlo, thi;
+    f2unpack(p, plo, phi);
+    f2unpack(t, tlo, thi);
+    const float lo = __int_as_float(__float_as_int(plo) + (__float_as_int(tlo) << 23));
+    const float hi = __int_as_float(__float_as_int(phi) + (__float_as_int(thi) << 23));
+    return f2pack(lo, hi);
+}
+
+// D[tmem] (+)= A[tmem] * B[smem desc]^T (A = P, bf16, K-major in TMEM).
+__device__ __forceinline__ void umma_bf16_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc, uint32_t idesc,
+                                             uint32_t accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
+        "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate)
+        : "memory");
+}
+
+struct TileSched {
+    int qt;       // query tile index, -1 if this CTA has no such tile
+    int n;        // key blocks
+    int r0_len, r1_start;
+    const int32_t *list;
+};
+
+template <bool WINDOW>
+__device__ __forceinline__ TileSched make_sched(const PPArgs &a, int qt, int bh) {
+    TileSched t{};
+    t.qt = qt;
+    if (qt < 0 || qt >= a.nq) {
+        t.qt = -1;
+        return t;
+    }
+    const int S = a.S, BN = 128;
+    if constexpr (WINDOW) {
+        const int q0 = qt * BN;
+        if (a.dense) {
+            t.r0_len = (S + BN - 1) / BN;
+            t.n = t.r0_len;
+        } else {
+            const int qe = min(q0 + BN, S);
+            const int lo = max(0, q0 - a.half), hi = min(S, qe + a.half);
+            const int lb0 = lo / BN, lb1 = (hi + BN - 1) / BN;
+            const int sb = (a.sink + BN - 1) / BN;
+            if (sb == 0) {
+                t.r0_len = 0; t.r1_start = lb0; t.n = lb1 - lb0;
+            } else if (lb0 <= sb) {
+                t.r0_len = max(lb1, sb); t.n = t.r0_len;
+            } else {
+                t.r0_len = sb; t.r1_start = lb0; t.n = sb + (lb1 - lb0);
+            }
+        }
+    } else {
+        const size_t lrow = (a.list_per_head ? static_cast<size_t>(bh) * a.nb : 0) + qt;
+        t.list = a.idx + lrow * a.cap;
+        t.n = __ldg(a.cnt + lrow);
+    }
+    return t;
+}
+
+template <bool WINDOW>
+__device__ __forceinline__ int kblock_of(const TileSched &t, int j) {
+    if constexpr (WINDOW) return j < t.r0_len ? j : t.r1_start + (j - t.r0_len);
+    else return __ldg(t.list + j);
+}
+
+template <int D, bool WINDOW>
+__global__ void __launch_bounds__(kThreads, 1)
+attn_pp_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
+               const __grid_constant__ CUtensorMap tmV, const PPArgs a) {
+    using C = PPCfg<D>;
+    constexpr int BN = 128;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *base = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    uint8_t *sQ = base;                                  // [2][TILE]
+    uint8_t *sK = sQ + 2 * C::TILE_BYTES;                // [NK][TILE]
+    uint8_t *sV = sK + C::NK * C::TILE_BYTES;            // [NV][TILE]
+    uint64_t *q_full = reinterpret_cast<uint64_t *>(sV + C::NV * C::TILE_BYTES);
+    uint64_t *k_full = q_full + 1;
+    uint64_t *k_empty = k_full + C::NK;
+    uint64_t *v_full = k_empty + C::NK;
+    uint64_t *v_empty = v_full + C::NV;
+    uint64_t *s_full = v_empty + C::NV;   // [2]
+    uint64_t *p_full = s_full + 2;        // [2]
+    uint64_t *pv_done = p_full + 2;       // [2]
+    uint64_t *mma_done = pv_done + 2;
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(mma_done + 1);
+    volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
+    int *list_ok = reinterpret_cast<int *>(tmem_slot + 2);  // [2]
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int bh = blockIdx.y;
+    const int S = a.S;
+    TileSched ts[2] = {make_sched<WINDOW>(a, 2 * blockIdx.x, bh), make_sched<WINDOW>(a, 2 * blockIdx.x + 1, bh)};
+
+    if (threadIdx.x == 0) {
+        mbar_init(q_full, 1);
+        for (int s = 0; s < C::NK; ++s) {
+            mbar_init(&k_full[s], 1);
+            mbar_init(&k_empty[s], 1);
+        }
+        for (int s = 0; s < C::NV; ++s) {
+            mbar_init(&v_full[s], 1);
+            mbar_init(&v_empty[s], 1);
+        }
+        for (int t = 0; t < 2; ++t) {
+            mbar_init(&s_full[t], 1);
+            mbar_init(&p_full[t], 4);
+            mbar_init(&pv_done[t], 1);
+        }
+        mbar_init(mma_done, 1);
+        *abort_flag = 0;
+        list_ok[0] = list_ok[1] = 1;
+        fence_mbar_init();
+    }
+    if constexpr (!WINDOW) {
+        if (warp < 2) {  // warp t validates tile t's list
+            const TileSched &t = ts[warp];
+            if (t.qt >= 0) {
+                bool ok = t.n >= 1 && t.n <= a.cap;
+                if (ok) {
+                    for (int j = lane; j < t.n; j += 32) {
+                        const int v = __ldg(t.list + j);
+                        ok = ok && v >= 0 && v < a.nb && (j == 0 || __ldg(t.list + j - 1) < v);
+                    }
+                }
+                ok = __all_sync(0xffffffffu, ok);
+                if (lane == 0 && !ok) list_ok[warp] = 0;
+            }
+        }
+    }
+    if (warp == 9) {
+        tmem_alloc(tmem_slot, 512);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+    bool bad[2] = {false, false};
+    for (int t = 0; t < 2; ++t) {
+        if (ts[t].qt < 0) ts[t].n = 0;
+        if constexpr (!WINDOW) {
+            if (ts[t].qt >= 0 && !list_ok[t]) {
+                bad[t] = true;
+                ts[t].n = 0;
+                if (threadIdx.x == 0) report(a.status, DEV_RUNTIME);
+            }
+        }
+    }
+    const int nA = ts[0].n, nB = ts[1].n;
+    const int nmax = max(nA, nB);
+
+
+    if (warp == 8) {
+        // ================= TMA producer =================
+        if (lane == 0 && nmax > 0) {
+            tma_prefetch_desc(&tmQ);
+            tma_prefetch_desc(&tmK);
+            tma_prefetch_desc(&tmV);
+            const int nq_loaded = (nA > 0) + (nB > 0);
+            mbar_arrive_expect_tx(q_full, nq_loaded * C::TILE_BYTES);
+            for (int t = 0; t < 2; ++t)
+                if (ts[t].n > 0)
+                    for (int s = 0; s < C::KSLABS; ++s)
+                        tma_load_3d(sQ + t * C::TILE_BYTES + s * C::SLAB, &tmQ, q_full, s * 64, ts[t].qt * BN, bh);
+            uint32_t kc = 0, vc = 0;
+            bool ok = true;
+            auto load = [&](bool is_k, int t, int j) -> bool {
+                uint32_t &c = is_k ? kc : vc;
+                const int depth = is_k ? C::NK : C::NV;
+                const int slot = c % depth;
+                uint64_t *full = is_k ? &k_full[slot] : &v_full[slot];
+                uint64_t *empty = is_k ? &k_empty[slot] : &v_empty[slot];
+                if (c >= static_cast<uint32_t>(depth) && !mbar_wait(empty, ((c / depth) - 1) & 1, abort_flag))
+                    return false;
+                uint8_t *dst = (is_k ? sK : sV) + slot * C::TILE_BYTES;
+                const int kb = kblock_of<WINDOW>(ts[t], j);
+                mbar_arrive_expect_tx(full, C::TILE_BYTES);
+                for (int s = 0; s < C::KSLABS; ++s)
+                    tma_load_3d(dst + s * C::SLAB, is_k ? &tmK : &tmV, full, s * 64, kb * BN, bh);
+                ++c;
+                return true;
+            };
+            if (nA > 0) ok = ok && load(true, 0, 0);
+            if (nB > 0) ok = ok && load(true, 1, 0);
+            for (int j = 0; ok && j < nmax; ++j)
+                for (int t = 0; ok && t < 2; ++t)
+                    if (j < ts[t].n) {
+                        ok = load(false, t, j);
+                        if (ok && j + 1 < ts[t].n) ok = load(true, t, j + 1);
+                    }
+            if (!ok) {
+                if (!*abort_flag) { report(a.status, DEV_TIMEOUT); *abort_flag = 1; }
+                // let the loads already issued land before the CTA exits
+                mbar_wait(q_full, 0, nullptr);
+                for (uint32_t c = kc > static_cast<uint32_t>(C::NK) ? kc - C::NK : 0; c < kc; ++c)
+                    mbar_wait(&k_full[c % C::NK], (c / C::NK) & 1, nullptr);
+                for (uint32_t c = vc > static_cast<uint32_t>(C::NV) ? vc - C::NV : 0; c < vc; ++c)
+                    mbar_wait(&v_full[c % C::NV], (c / C::NV) & 1, nullptr);
+            }
+        }
+        __syncwarp();
+    } else if (warp == 9) {
+        // ================= MMA issuer =================
+        if (lane == 0) {
+            constexpr uint32_t idesc_qk = idesc_bf16_f32(128, BN, false);
+            constexpr uint32_t idesc_pv = idesc_bf16_f32(128, D, true);
+            const uint32_t aQ = smem_u32(sQ), aK = smem_u32(sK), aV = smem_u32(sV);
+            uint32_t kc = 0, vc = 0;
+            bool ok = true;
+            auto qk = [&](int t, int j) -> bool {
+                const int slot = kc % C::NK;
+                if (!mbar_wait(&k_full[slot], (kc / C::NK) & 1, abort_flag)) return false;
+                if (j > 0 && !mbar_wait(&pv_done[t], (j - 1) & 1, abort_flag)) return false;
+                tc_fence_after();
+                #pragma unroll
+                for (int kk = 0; kk < D / 16; ++kk) {
+                    const uint32_t off = (kk >> 2) * C::SLAB + (kk & 3) * 32;
+                    umma_bf16(tmem + t * 128, sdesc_sw128(aQ + t * C::TILE_BYTES + off, 16, 1024),
+                              sdesc_sw128(aK + slot * C::TILE_BYTES + off, 16, 1024), idesc_qk, kk > 0 ? 1u : 0u);
+                }
+                umma_commit(&s_full[t]);
+                umma_commit(&k_empty[slot]);
+                ++kc;
+                return true;
+            };
+            auto pv = [&](int t, int j) -> bool {
+                const int slot = vc % C::NV;
+                if (!mbar_wait(&p_full[t], j & 1, abort_flag)) return false;
+                if (!mbar_wait(&v_full[slot], (vc / C::NV) & 1, abort_flag)) return false;
+                tc_fence_after();
+                #pragma unroll
+                for (int kk = 0; kk < BN / 16; ++kk)
+                    umma_bf16_ts(tmem + C::O_COL + t * D, tmem + t * 128 + kk * 8,
+                                 sdesc_sw128(aV + slot * C::TILE_BYTES + kk * 2048, C::SLAB, 1024), idesc_pv,
+                                 (j > 0 || kk > 0) ? 1u : 0u);
+                umma_commit(&pv_done[t]);
+                umma_commit(&v_empty[slot]);
+                ++vc;
+                return true;
+            };
+            if (nmax > 0) {
+                ok = mbar_wait(q_full, 0, abort_flag);
+                if (ok && nA > 0) ok = qk(0, 0);
+                if (ok && nB > 0) ok = qk(1, 0);
+                for (int j = 0; ok && j < nmax; ++j)
+                    for (int t = 0; ok && t < 2; ++t)
+                        if (j < ts[t].n) {
+                            ok = pv(t, j);
+                            if (ok && j + 1 < ts[t].n) ok = qk(t, j + 1);
+                        }
+                if (!ok && !*abort_flag) { report(a.status, DEV_TIMEOUT); *abort_flag = 1; }
+            }
+            umma_commit(mma_done);
+            mbar_wait(mma_done, 0, nullptr);
+        }
+        __syncwarp();
+    } else {
+        // ================= softmax + epilogue (warps 0-7) =================
+        const int t = warp >> 2;                  // tile
+        const int wq = warp & 3;                  // TMEM lane quadrant
+        const int row = wq * 32 + lane;           // row of the tile
+        const TileSched &sc = ts[t];
+        const int n = sc.n;
+        const int q0 = (sc.qt < 0 ? 0 : sc.qt) * BN;
+        const int rg = q0 + row;
+        const bool row_valid = sc.qt >= 0 && rg < S;
+        const uint32_t t_lane = tmem + (static_cast<uint32_t>(wq * 32) << 16);
+        const uint32_t s_col = t * 128, o_col = C::O_COL + t * D;
+        const float sl2 = a.scale_log2;
+        const uint64_t sl2x2 = f2pack(sl2, sl2);
+        float m_ref = -INFINITY, l_sum = 0.f;
+        bool ok = true;
+        for (int j = 0; j < n; ++j) {
+            if (!mbar_wait(&s_full[t], j & 1, abort_flag)) { ok = false; break; }
+            tc_fence_after();
+            uint32_t x[BN];
+            #pragma unroll
+            for (int c = 0; c < BN / 32; ++c)
+                tmem_ld32(t_lane + s_col + 32 * c, *reinterpret_cast<uint32_t(*)[32]>(&x[32 * c]));
+            tmem_ld_wait();
+            const int kb = kblock_of<WINDOW>(sc, j);
+            const int ks = kb * BN;
+            bool full;
+            if constexpr (WINDOW) {
+                const int qe = min(q0 + BN, S);
+                full = (ks + BN <= S) && (a.dense || ks + BN <= a.sink || max(qe - 1 - ks, ks + BN - 1 - q0) <= a.half);
+                if (!full) {
+                    #pragma unroll
+                    for (int c = 0; c < BN; ++c) {
+                        const int kc2 = ks + c;
+                        const int dd = rg > kc2 ? rg - kc2 : kc2 - rg;
+                        if (!(kc2 < S && (a.dense || kc2 < a.sink || dd <= a.half))) x[c] = __float_as_uint(-INFINITY);
+                    }
+                }
+            } else {
+                full = a.group <= 0;
+                if (!full) {
+                    const int gq = rg / a.group;
+                    #pragma unroll
+                    for (int c = 0; c < BN; ++c)
+                        if ((ks + c) / a.group != gq) x[c] = __float_as_uint(-INFINITY);
+                }
+            }
+            // row max: four independent chains of 3-input max
+            float m4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+            #pragma unroll
+            for (int c = 0; c < BN; c += 8) {
+                #pragma unroll
+                for (int u = 0; u < 4; ++u)
+                    m4[u] = fmax3(m4[u], __uint_as_float(x[c + 2 * u]), __uint_as_float(x[c + 2 * u + 1]));
+            }
+            const float mb = fmaxf(fmaxf(m4[0], m4[1]), fmaxf(m4[2], m4[3])) * sl2;
+            const float m_new = fmaxf(m_ref, mb);
+            const bool need = m_new > m_ref + kRescale;
+            if (__any_sync(0xffffffffu, need)) {
+                if (j > 0) {
+                    if (!mbar_wait(&pv_done[t], (j - 1) & 1, abort_flag)) {
+                        ok = false;
+                    } else {
+                        tc_fence_after();
+                        const float alpha = (need && m_ref != -INFINITY) ? ex2_approx(m_ref - m_new) : 1.f;
+                        #pragma unroll 1
+                        for (int c = 0; c < D / 8; ++c) {
+                            uint32_t o[8];
+                            tmem_ld8(t_lane + o_col + 8 * c, o);
+                            tmem_ld_wait();
+                            #pragma unroll
+                            for (int e = 0; e < 8; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * alpha);
+                            tmem_st8(t_lane + o_col + 8 * c, o);
+                        }
+                        tmem_st_wait();
+                        l_sum *= alpha;
+                    }
+                }
+                if (need) m_ref = m_new;
+            }
+            if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
+            const float m_use = m_ref == -INFINITY ? 0.f : m_ref;
+            const uint64_t negm = f2pack(-m_use, -m_use);
+            uint64_t acc[4] = {0ull, 0ull, 0ull, 0ull};
+            #pragma unroll
+            for (int q = 0; q < BN / 2; ++q) {
+                uint64_t v = ffma2(f2pack(__uint_as_float(x[2 * q]), __uint_as_float(x[2 * q + 1])), sl2x2, negm);
+                if ((q & 7) >= 5) {
+                    v = exp2_poly2(v);
+                } else {
+                    float lo, hi;
+                    f2unpack(v, lo, hi);
+                    v = f2pack(ex2_approx(lo), ex2_approx(hi));
+                }
+                acc[q & 3] = fadd2(acc[q & 3], v);
+                float lo, hi;
+                f2unpack(v, lo, hi);
+                x[q] = pack_bf16x2(lo, hi);   // P, packed in place (q <= 2q)
+            }
+            {
+                float a0, a1, b0, b1, c0, c1, d0, d1;
+                f2unpack(acc[0], a0, a1);
+                f2unpack(acc[1], b0, b1);
+                f2unpack(acc[2], c0, c1);
+                f2unpack(acc[3], d0, d1);
+                l_sum += ((a0 + a1) + (b0 + b1)) + ((c0 + c1) + (d0 + d1));
+            }
+            // P over the first 64 columns of this tile's S
+            tmem_st32(t_lane + s_col, *reinterpret_cast<const uint32_t(*)[32]>(&x[0]));
+            tmem_st32(t_lane + s_col + 32, *reinterpret_cast<const uint32_t(*)[32]>(&x[32]));
+            tmem_st_wait();
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&p_full[t]);
+        }
+        if (!ok && !*abort_flag) { report(a.status, DEV_TIMEOUT); *abort_flag = 1; }
+
+        // ---- epilogue: O / l -> global ----
+        const size_t orow = static_cast<size_t>(bh) * S + rg;
+        bool have_o = ok && n > 0;
+        if (have_o && !mbar_wait(&pv_done[t], (n - 1) & 1, abort_flag)) {
+            have_o = false;
+            if (!*abort_flag) { report(a.status, DEV_TIMEOUT); *abort_flag = 1; }
+        }
+        if (have_o) {
+            tc_fence_after();
+            const float inv = l_sum > 0.f ? 1.f / l_sum : 0.f;
+            #pragma unroll
+            for (int c = 0; c < D / 32; ++c) {
+                uint32_t o[32];
+                tmem_ld32(t_lane + o_col + 32 * c, o);
+                tmem_ld_wait();
+                if (row_valid) {
+                    if (a.out_f32) {
+                        float4 *dst = reinterpret_cast<float4 *>(static_cast<float *>(a.out) + orow * D + 32 * c);
+                        #pragma unroll
+                        for (int e = 0; e < 8; ++e)
+                            dst[e] = make_float4(__uint_as_float(o[4 * e]) * inv, __uint_as_float(o[4 * e + 1]) * inv,
+                                                 __uint_as_float(o[4 * e + 2]) * inv, __uint_as_float(o[4 * e + 3]) * inv);
+                    } else {
+                        uint4 *dst = reinterpret_cast<uint4 *>(static_cast<__nv_bfloat16 *>(a.out) + orow * D + 32 * c);
+                        #pragma unroll
+                        for (int e = 0; e < 4; ++e) {
+                            const uint32_t *u = &o[8 * e];
+                            dst[e] = make_uint4(pack_bf16x2(__uint_as_float(u[0]) * inv, __uint_as_float(u[1]) * inv),
+                                                pack_bf16x2(__uint_as_float(u[2]) * inv, __uint_as_float(u[3]) * inv),
+                                                pack_bf16x2(__uint_as_float(u[4]) * inv, __uint_as_float(u[5]) * inv),
+                                                pack_bf16x2(__uint_as_float(u[6]) * inv, __uint_as_float(u[7]) * inv));
+                        }
+                    }
+                }
+            }
+            if (row_valid && l_sum <= 0.f) report(a.status, DEV_RUNTIME);
+        } else if (row_valid && bad[t]) {
+            if (a.out_f32) {
+                float4 *dst = reinterpret_cast<float4 *>(static_cast<float *>(a.out) + orow * D);
+                for (int e = 0; e < D / 4; ++e) dst[e] = make_float4(0.f, 0.f, 0.f, 0.f);
+            } else {
+                uint4 *dst = reinterpret_cast<uint4 *>(static_cast<__nv_bfloat16 *>(a.out) + orow * D);
+                for (int e = 0; e < D / 8; ++e) dst[e] = make_uint4(0u, 0u, 0u, 0u);
+            }
+        }
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 9) {
+        tc_fence_after();
+        tmem_dealloc(tmem, 512);
+    }
+}
+
+template <int D, bool WINDOW>
+vsa_status run_pp(const AttnLaunch &L, int *status, cudaStream_t st) {
+    using C = PPCfg<D>;
+    CUtensorMap mq, mk, mv;
+    if (!make_tile_map(&mq, L.q, D, L.S, L.BH, 128) || !make_tile_map(&mk, L.k, D, L.S, L.BH, 128) ||
+        !make_tile_map(&mv, L.v, D, L.S, L.BH, 128))
+        return fail(VSA_ERR_CUDA, "cuTensorMapEncodeTiled failed (driver entry point or arguments)");
+    auto kern = attn_pp_kernel<D, WINDOW>;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
+    if (e != cudaSuccess) return check_cuda(e, "cudaFuncSetAttribute(attention, two tiles)");
+    PPArgs a;
+    a.S = L.S;
+    a.nq = (L.S + 127) / 128;
+    a.idx = L.idx;
+    a.cnt = L.cnt;
+    a.cap = L.cap;
+    a.list_per_head = L.list_per_head;
+    a.group = L.group;
+    a.nb = L.nb;
+    a.half = L.half;
+    a.sink = L.sink;
+    a.dense = L.dense;
+    a.scale_log2 = L.scale * 1.4426950408889634f;
+    a.out = L.o;
+    a.out_f32 = L.out_f32;
+    a.status = status;
+    dim3 grid((a.nq + 1) / 2, L.BH);
+    kern<<<grid, kThreads, C::SMEM, st>>>(mq, mk, mv, a);
+    return check_cuda(cudaGetLastError(), "attention launch (two tiles)");
+}
+
+}  // namespace
+
+vsa_status launch_attention_pp(const AttnLaunch &L, int *status, cudaStream_t st) {
+    if (L.window) return L.D == 128 ? run_pp<128, true>(L, status, st) : run_pp<64, true>(L, status, st);
+    return L.D == 128 ? run_pp<128, false>(L, status, st) : run_pp<64, false>(L, status, st);
+}
+
+}  // namespace vsa

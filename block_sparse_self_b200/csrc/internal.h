@@ -61,6 +61,10 @@ struct AttnLaunch {
     float scale;
 };
 vsa_status launch_attention(const AttnLaunch &a, int *status, cudaStream_t st);
+// Two query tiles per CTA (128-token blocks only); launch_attention routes to it.
+vsa_status launch_attention_pp(const AttnLaunch &a, int *status, cudaStream_t st);
+// [BH, S, D] bf16 as a 3-D TMA tensor map (D, S, BH), box (64, rows, 1), 128-byte swizzle.
+bool make_tile_map(CUtensorMap *m, const void *ptr, int D, int S, int BH, int rows);
 
 cudaError_t launch_wait_timeout(uint64_t limit_ns, int *status, cudaStream_t st);
 
