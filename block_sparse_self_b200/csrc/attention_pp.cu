@@ -22,11 +22,10 @@
 // QK_t(j+1), which overwrites the P_t(j) that PV_t(j) reads, first waits for
 // PV_t(j) to complete.
 //
-// The softmax takes 2^x for 5 of every 8 pairs of columns on the MUFU and for
-// the rest on the FMA pipe: Cody-Waite range reduction x = n + f with
-// n = rint(x), f in [-1/2, 1/2], and a degree-3 polynomial for 2^f whose
-// coefficients were fitted here by a Remez exchange on the relative error
-// (max relative error 7.5e-5, far below bf16's 2^-8 rounding of P).
+// Softmax: after a row's first visible block the exponentials use the running
+// row max without taking the block's max at all; only if the block's P would
+// sum above 2^24 (the max grew, rare) is the running max raised, O and l
+// rescaled and the block redone from S, which is still intact in TMEM.
 #include <math.h>
 
 #include "common.cuh"
@@ -61,71 +60,11 @@ struct PPCfg {
 };
 
 constexpr int kThreads = 320;
-constexpr float kRescale = 8.0f;     // rescale O only when the max grows by > 2^8
-constexpr float kRound = 12582912.f;  // 1.5 * 2^23
-constexpr float kC0 = 0.9999280571937561f, kC1 = 0.6932609677314758f, kC2 = 0.2426111251115799f,
-                kC3 = 0.0551716685295105f;
+// The running row max is only raised when a block's P would sum above 2^24:
+// every P then stays in (0, 2^24] (bf16 has the range) and O, l stay far below
+// fp32 overflow for any key count a list can name, while redos are rare.
+constexpr float kMaxRowSum = 16777216.0f;
 
-__device__ __forceinline__ uint64_t f2pack(float lo, float hi) {
-    uint64_t r;
-    asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
-    return r;
-}
-__device__ __forceinline__ void f2unpack(uint64_t v, float &lo, float &hi) {
-    asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(v));
-}
-__device__ __forceinline__ uint64_t ffma2(uint64_t a, uint64_t b, uint64_t c) {
-    uint64_t d;
-    asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
-    return d;
-}
-__device__ __forceinline__ uint64_t fadd2(uint64_t a, uint64_t b) {
-    uint64_t d;
-    asm("add.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
-    return d;
-}
-__device__ __forceinline__ uint64_t fsub2(uint64_t a, uint64_t b) {
-    uint64_t d;
-    asm("sub.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
-    return d;
-}
-__device__ __forceinline__ float fmax3(float a, float b, float c) {
-    float d;
-    asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
-    return d;
-}
-
-// 2^x for a pair on the FMA pipe (see the file comment).  x is clamped at
-// -125 so that every result stays a normal number (2^-125 ~ 2.4e-38).
-__device__ __forceinline__ uint64_t exp2_poly2(uint64_t x) {
-    float a, b;
-    f2unpack(x, a, b);
-    x = f2pack(fmaxf(a, -125.f), fmaxf(b, -125.f));
-    const uint64_t r2 = f2pack(kRound, kRound);
-    const uint64_t t = fadd2(x, r2);      // n sits in the low mantissa bits
-    const uint64_t n = fsub2(t, r2);      // rint(x)
-    const uint64_t f = fsub2(x, n);       // in [-1/2, 1/2]
-    uint64_t p = ffma2(f, f2pack(kC3, kC3), f2pack(kC2, kC2));
-    p = ffma2(p, f, f2pack(kC1, kC1));
-    p = ffma2(p, f, f2pack(kC0, kC0));
-    float plo, phi, tlo, thi;
-    f2unpack(p, plo, phi);
-    f2unpack(t, tlo, thi);
-    const float lo = __int_as_float(__float_as_int(plo) + (__float_as_int(tlo) << 23));
-    const float hi = __int_as_float(__float_as_int(phi) + (__float_as_int(thi) << 23));
-    return f2pack(lo, hi);
-}
-
-// D[tmem] (+)= A[tmem] * B[smem desc]^T (A = P, bf16, K-major in TMEM).
-__device__ __forceinline__ void umma_bf16_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc, uint32_t idesc,
-                                             uint32_t accumulate) {
-    asm volatile(
-        "{\n\t.reg .pred p;\n\t"
-        "setp.ne.b32 p, %4, 0;\n\t"
-        "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
-        "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate)
-        : "memory");
-}
 
 struct TileSched {
     int qt;       // query tile index, -1 if this CTA has no such tile
@@ -317,7 +256,14 @@ attn_pp_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
         if (lane == 0) {
             constexpr uint32_t idesc_qk = idesc_bf16_f32(128, BN, false);
             constexpr uint32_t idesc_pv = idesc_bf16_f32(128, D, true);
-            const uint32_t aQ = smem_u32(sQ), aK = smem_u32(sK), aV = smem_u32(sV);
+            // Descriptor bases, built once.  The start-address field holds
+            // addr >> 4 in 14 bits and every shared address here is < 256 KB,
+            // so advancing a descriptor by a byte offset is a plain add of
+            // offset >> 4 with no carry out of the field.
+            const uint64_t dQ = sdesc_sw128(smem_u32(sQ), 16, 1024);
+            const uint64_t dK = sdesc_sw128(smem_u32(sK), 16, 1024);
+            const uint64_t dV = sdesc_sw128(smem_u32(sV), C::SLAB, 1024);
+            constexpr uint64_t kTile16 = C::TILE_BYTES >> 4;
             uint32_t kc = 0, vc = 0;
             bool ok = true;
             auto qk = [&](int t, int j) -> bool {
@@ -325,11 +271,12 @@ attn_pp_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
                 if (!mbar_wait(&k_full[slot], (kc / C::NK) & 1, abort_flag)) return false;
                 if (j > 0 && !mbar_wait(&pv_done[t], (j - 1) & 1, abort_flag)) return false;
                 tc_fence_after();
+                const uint64_t q0 = dQ + t * kTile16, k0 = dK + slot * kTile16;
+                const uint32_t d = tmem + t * 128;
                 #pragma unroll
                 for (int kk = 0; kk < D / 16; ++kk) {
-                    const uint32_t off = (kk >> 2) * C::SLAB + (kk & 3) * 32;
-                    umma_bf16(tmem + t * 128, sdesc_sw128(aQ + t * C::TILE_BYTES + off, 16, 1024),
-                              sdesc_sw128(aK + slot * C::TILE_BYTES + off, 16, 1024), idesc_qk, kk > 0 ? 1u : 0u);
+                    const uint64_t off = static_cast<uint64_t>(((kk >> 2) * C::SLAB + (kk & 3) * 32) >> 4);
+                    umma_bf16(d, q0 + off, k0 + off, idesc_qk, kk > 0 ? 1u : 0u);
                 }
                 umma_commit(&s_full[t]);
                 umma_commit(&k_empty[slot]);
@@ -341,11 +288,13 @@ attn_pp_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
                 if (!mbar_wait(&p_full[t], j & 1, abort_flag)) return false;
                 if (!mbar_wait(&v_full[slot], (vc / C::NV) & 1, abort_flag)) return false;
                 tc_fence_after();
+                const uint64_t v0 = dV + slot * kTile16;
+                const uint32_t d = tmem + C::O_COL + t * D, pa = tmem + t * 128;
+                const uint32_t acc0 = j > 0 ? 1u : 0u;
                 #pragma unroll
                 for (int kk = 0; kk < BN / 16; ++kk)
-                    umma_bf16_ts(tmem + C::O_COL + t * D, tmem + t * 128 + kk * 8,
-                                 sdesc_sw128(aV + slot * C::TILE_BYTES + kk * 2048, C::SLAB, 1024), idesc_pv,
-                                 (j > 0 || kk > 0) ? 1u : 0u);
+                    umma_bf16_ts(d, pa + kk * 8, v0 + static_cast<uint64_t>((kk * 2048) >> 4), idesc_pv,
+                                 kk > 0 ? 1u : acc0);
                 umma_commit(&pv_done[t]);
                 umma_commit(&v_empty[slot]);
                 ++vc;
@@ -380,7 +329,6 @@ attn_pp_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
         const uint32_t t_lane = tmem + (static_cast<uint32_t>(wq * 32) << 16);
         const uint32_t s_col = t * 128, o_col = C::O_COL + t * D;
         const float sl2 = a.scale_log2;
-        const uint64_t sl2x2 = f2pack(sl2, sl2);
         float m_ref = -INFINITY, l_sum = 0.f;
         bool ok = true;
         for (int j = 0; j < n; ++j) {
@@ -391,47 +339,79 @@ attn_pp_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
             for (int c = 0; c < BN / 32; ++c)
                 tmem_ld32(t_lane + s_col + 32 * c, *reinterpret_cast<uint32_t(*)[32]>(&x[32 * c]));
             tmem_ld_wait();
-            const int kb = kblock_of<WINDOW>(sc, j);
-            const int ks = kb * BN;
-            bool full;
-            if constexpr (WINDOW) {
-                const int qe = min(q0 + BN, S);
-                full = (ks + BN <= S) && (a.dense || ks + BN <= a.sink || max(qe - 1 - ks, ks + BN - 1 - q0) <= a.half);
-                if (!full) {
-                    #pragma unroll
-                    for (int c = 0; c < BN; ++c) {
-                        const int kc2 = ks + c;
-                        const int dd = rg > kc2 ? rg - kc2 : kc2 - rg;
-                        if (!(kc2 < S && (a.dense || kc2 < a.sink || dd <= a.half))) x[c] = __float_as_uint(-INFINITY);
+            auto apply_mask = [&]() {
+                if constexpr (WINDOW) {
+                    const int ks = kblock_of<WINDOW>(sc, j) * BN;
+                    const int qe = min(q0 + BN, S);
+                    const bool full = (ks + BN <= S) &&
+                                      (a.dense || ks + BN <= a.sink || max(qe - 1 - ks, ks + BN - 1 - q0) <= a.half);
+                    if (!full) {
+                        #pragma unroll
+                        for (int c = 0; c < BN; ++c) {
+                            const int kc2 = ks + c;
+                            const int dd = rg > kc2 ? rg - kc2 : kc2 - rg;
+                            if (!(kc2 < S && (a.dense || kc2 < a.sink || dd <= a.half)))
+                                x[c] = __float_as_uint(-INFINITY);
+                        }
+                    }
+                } else {
+                    if (a.group > 0) {
+                        const int ks = kblock_of<WINDOW>(sc, j) * BN;
+                        const int gq = rg / a.group;
+                        #pragma unroll
+                        for (int c = 0; c < BN; ++c)
+                            if ((ks + c) / a.group != gq) x[c] = __float_as_uint(-INFINITY);
                     }
                 }
-            } else {
-                full = a.group <= 0;
-                if (!full) {
-                    const int gq = rg / a.group;
-                    #pragma unroll
-                    for (int c = 0; c < BN; ++c)
-                        if ((ks + c) / a.group != gq) x[c] = __float_as_uint(-INFINITY);
-                }
-            }
-            // row max: four independent chains of 3-input max
-            float m4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
-            #pragma unroll
-            for (int c = 0; c < BN; c += 8) {
+            };
+            apply_mask();
+            // P = 2^(scale*log2e*S - m_use) in place (bf16 pairs), returns the row sum
+            auto exp_pass = [&](float m_use) -> float {
+                const float nm = -m_use;
+                float acc[4] = {0.f, 0.f, 0.f, 0.f};
                 #pragma unroll
-                for (int u = 0; u < 4; ++u)
-                    m4[u] = fmax3(m4[u], __uint_as_float(x[c + 2 * u]), __uint_as_float(x[c + 2 * u + 1]));
-            }
-            const float mb = fmaxf(fmaxf(m4[0], m4[1]), fmaxf(m4[2], m4[3])) * sl2;
-            const float m_new = fmaxf(m_ref, mb);
-            const bool need = m_new > m_ref + kRescale;
-            if (__any_sync(0xffffffffu, need)) {
+                for (int q = 0; q < BN / 2; ++q) {
+                    const float p0 = ex2_approx(fmaf(__uint_as_float(x[2 * q]), sl2, nm));
+                    const float p1 = ex2_approx(fmaf(__uint_as_float(x[2 * q + 1]), sl2, nm));
+                    acc[q & 3] += p0;
+                    acc[q & 3] += p1;
+                    x[q] = pack_bf16x2(p0, p1);   // P, packed in place (q <= 2q)
+                }
+                return (acc[0] + acc[1]) + (acc[2] + acc[3]);
+            };
+            auto raw_max = [&]() -> float {
+                float m4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+                #pragma unroll
+                for (int c = 0; c < BN; c += 8) {
+                    #pragma unroll
+                    for (int u = 0; u < 4; ++u)
+                        m4[u] = fmax3(m4[u], __uint_as_float(x[c + 2 * u]), __uint_as_float(x[c + 2 * u + 1]));
+                }
+                return fmaxf(fmaxf(m4[0], m4[1]), fmaxf(m4[2], m4[3]));
+            };
+            // first visible keys of this row: take the block max before the exponentials
+            if (m_ref == -INFINITY) m_ref = raw_max() * sl2;  // may stay -inf
+            // The running max is lazy: every P is at most the row sum, so a sum
+            // above kMaxRowSum (or inf) means the row's max grew; then O and l are
+            // rescaled and the block is redone from S, still intact in TMEM.
+            float rs = 0.f;
+            #pragma unroll 1
+            for (int pass = 0; pass < 2; ++pass) {
+                rs = exp_pass(m_ref == -INFINITY ? 0.f : m_ref);
+                const bool need = !(rs <= kMaxRowSum);
+                if (pass == 1 || !__any_sync(0xffffffffu, need)) break;
+                #pragma unroll
+                for (int c = 0; c < BN / 32; ++c)
+                    tmem_ld32(t_lane + s_col + 32 * c, *reinterpret_cast<uint32_t(*)[32]>(&x[32 * c]));
+                tmem_ld_wait();
+                apply_mask();
+                const float m_new = need ? fmaxf(m_ref, raw_max() * sl2) : m_ref;
                 if (j > 0) {
                     if (!mbar_wait(&pv_done[t], (j - 1) & 1, abort_flag)) {
                         ok = false;
                     } else {
                         tc_fence_after();
-                        const float alpha = (need && m_ref != -INFINITY) ? ex2_approx(m_ref - m_new) : 1.f;
+                        const float alpha = (m_new > m_ref && m_ref != -INFINITY) ? ex2_approx(m_ref - m_new) : 1.f;
                         #pragma unroll 1
                         for (int c = 0; c < D / 8; ++c) {
                             uint32_t o[8];
@@ -445,35 +425,11 @@ attn_pp_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
                         l_sum *= alpha;
                     }
                 }
-                if (need) m_ref = m_new;
+                if (!__all_sync(0xffffffffu, ok)) break;
+                m_ref = m_new;
             }
             if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
-            const float m_use = m_ref == -INFINITY ? 0.f : m_ref;
-            const uint64_t negm = f2pack(-m_use, -m_use);
-            uint64_t acc[4] = {0ull, 0ull, 0ull, 0ull};
-            #pragma unroll
-            for (int q = 0; q < BN / 2; ++q) {
-                uint64_t v = ffma2(f2pack(__uint_as_float(x[2 * q]), __uint_as_float(x[2 * q + 1])), sl2x2, negm);
-                if ((q & 7) >= 5) {
-                    v = exp2_poly2(v);
-                } else {
-                    float lo, hi;
-                    f2unpack(v, lo, hi);
-                    v = f2pack(ex2_approx(lo), ex2_approx(hi));
-                }
-                acc[q & 3] = fadd2(acc[q & 3], v);
-                float lo, hi;
-                f2unpack(v, lo, hi);
-                x[q] = pack_bf16x2(lo, hi);   // P, packed in place (q <= 2q)
-            }
-            {
-                float a0, a1, b0, b1, c0, c1, d0, d1;
-                f2unpack(acc[0], a0, a1);
-                f2unpack(acc[1], b0, b1);
-                f2unpack(acc[2], c0, c1);
-                f2unpack(acc[3], d0, d1);
-                l_sum += ((a0 + a1) + (b0 + b1)) + ((c0 + c1) + (d0 + d1));
-            }
+            l_sum += rs;
             // P over the first 64 columns of this tile's S
             tmem_st32(t_lane + s_col, *reinterpret_cast<const uint32_t(*)[32]>(&x[0]));
             tmem_st32(t_lane + s_col + 32, *reinterpret_cast<const uint32_t(*)[32]>(&x[32]));
