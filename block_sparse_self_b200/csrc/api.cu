@@ -256,6 +256,10 @@ vsa_status vsa_block_scores(const void *q_max, const void *q_min, const void *k_
                 "summaries must be non-NULL 16-byte aligned device pointers");
     VSA_REQUIRE(aligned4(scores), "scores must be a non-NULL 4-byte aligned device pointer");
     VSA_REQUIRE(static_cast<long long>(nb) <= 65535LL * 64, "nb too large");
+    if (dtype == VSA_BF16)  // tensor cores: exact bf16 products, fp32 accumulation
+        return check_cuda(launch_scores_tc(q_max, q_min, k_max, k_min, B * n_heads, nb, D, scores, status_or_null(),
+                                           as_stream(stream)),
+                          "block_scores launch");
     return check_cuda(launch_scores(q_max, q_min, k_max, k_min, esize_of(dtype), B * n_heads, nb, D, scores,
                                     as_stream(stream)),
                       "block_scores launch");

@@ -108,6 +108,34 @@ __device__ __forceinline__ void tma_load_3d(void *dst, const CUtensorMap *map, u
         : "memory");
 }
 
+// 5-D tile load; coordinates innermost first.
+__device__ __forceinline__ void tma_load_5d(void *dst, const CUtensorMap *map, uint64_t *bar, int c0, int c1, int c2,
+                                            int c3, int c4) {
+    asm volatile(
+        "cp.async.bulk.tensor.5d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
+        " [%0], [%1, {%3, %4, %5, %6, %7}], [%2];" ::"r"(smem_u32(dst)),
+        "l"(reinterpret_cast<uint64_t>(map)), "r"(smem_u32(bar)), "r"(c0), "r"(c1), "r"(c2), "r"(c3), "r"(c4)
+        : "memory");
+}
+
+// ---------------------------------------------------------------------------
+// Tile-contiguous order ("ADR-0001", step 6; "Adaptive tiling (SPADE)",
+// Recipe): position p holds the T-major token tile_token(p).  Tiles come in
+// row-major tile order, the tokens of a tile in T-major order.
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ int tile_token(int p, int H, int W, int tt, int th, int tw) {
+    const int vol = tt * th * tw;
+    const int tile = p / vol, r = p - tile * vol;
+    const int nth = H / th, ntw = W / tw;
+    const int ct = tile / (nth * ntw);
+    const int rem = tile - ct * (nth * ntw);
+    const int ch = rem / ntw, cw = rem - ch * ntw;
+    const int dt = r / (th * tw);
+    const int r2 = r - dt * (th * tw);
+    const int dh = r2 / tw, dw = r2 - dh * tw;
+    return ((ct * tt + dt) * H + ch * th + dh) * W + cw * tw + dw;
+}
+
 // ---------------------------------------------------------------------------
 // tcgen05: tensor memory allocation, MMA, commit, loads and stores
 // ---------------------------------------------------------------------------

@@ -16,9 +16,10 @@ vsa_status check_cuda(cudaError_t e, const char *what);
 // Device address of the status word of the current device.
 int *device_status_word();
 
+constexpr int kMaxTiles = 8;
 struct TileSet {
     int n;
-    int t[8], h[8], w[8];
+    int t[kMaxTiles], h[kMaxTiles], w[kMaxTiles];
 };
 
 // Launchers (arguments already validated by the C ABI layer).
@@ -28,8 +29,15 @@ cudaError_t launch_permute(const void *src, void *dst, int esize, int BH, int S,
 cudaError_t launch_cast_f32_bf16(const float *x, void *y, int64_t n, cudaStream_t st);
 cudaError_t launch_summaries(const void *x, int esize, int BH, int S, int D, int block, void *xmax, void *xmin,
                              cudaStream_t st);
+// Summaries of the tiles of a T-major x in each head's tile-contiguous order.
+cudaError_t launch_summaries_tiled(const void *x, int esize, int BH, int S, int D, int T, int H, int W,
+                                   const TileSet &tiles, const int32_t *choice, void *xmax, void *xmin, int *status,
+                                   cudaStream_t st);
 cudaError_t launch_scores(const void *qmax, const void *qmin, const void *kmax, const void *kmin, int esize, int BH,
                           int nb, int D, float *scores, cudaStream_t st);
+// bf16 summaries on tcgen05 (D in {64, 128})
+cudaError_t launch_scores_tc(const void *qmax, const void *qmin, const void *kmax, const void *kmin, int BH, int nb,
+                             int D, float *scores, int *status, cudaStream_t st);
 cudaError_t launch_topk(const float *scores, int BH, int nb, int k, int n_sink, int diag_hw, int32_t *idx,
                         int32_t *cnt, int cap, cudaStream_t st);
 cudaError_t launch_structured(int T, int H, int W, int tt, int th, int tw, int rt, int rh, int rw, int block,
@@ -59,12 +67,22 @@ struct AttnLaunch {
     // window mode
     int half, sink, dense;
     float scale;
+    // tiled mode: q, k, v, o in T-major order; each (b, head) uses its chosen
+    // tiling and the kernel permutes through its TMA boxes and epilogue
+    bool tiled;
+    int T, Hg, Wg;
+    TileSet tiles;
+    const int32_t *choice;
 };
 vsa_status launch_attention(const AttnLaunch &a, int *status, cudaStream_t st);
 // Two query tiles per CTA (128-token blocks only); launch_attention routes to it.
 vsa_status launch_attention_pp(const AttnLaunch &a, int *status, cudaStream_t st);
 // [BH, S, D] bf16 as a 3-D TMA tensor map (D, S, BH), box (64, rows, 1), 128-byte swizzle.
 bool make_tile_map(CUtensorMap *m, const void *ptr, int D, int S, int BH, int rows);
+// [BH, T, H, W, D] bf16 as a 5-D TMA tensor map (D, W, H, T, BH), box
+// (64, bw, bh, bt, 1), 128-byte swizzle: a (bt, bh, bw) token box lands as
+// rows of 128 bytes in (t, h, w) row-major order.
+bool make_box_map(CUtensorMap *m, const void *ptr, int D, int T, int H, int W, int BH, int bt, int bh, int bw);
 
 cudaError_t launch_wait_timeout(uint64_t limit_ns, int *status, cudaStream_t st);
 

@@ -28,20 +28,6 @@ struct PermArgs {
 constexpr int kRowsPerItem = 128;  // permuted rows handled per work item
 constexpr int kThreads = 256;
 
-// Token index (T-major) of position p in the tile-contiguous order.
-__device__ __forceinline__ int perm_token(int p, int H, int W, int tt, int th, int tw) {
-    const int vol = tt * th * tw;
-    const int tile = p / vol, r = p - tile * vol;
-    const int nth = H / th, ntw = W / tw;
-    const int ct = tile / (nth * ntw);
-    const int rem = tile - ct * (nth * ntw);
-    const int ch = rem / ntw, cw = rem - ch * ntw;
-    const int dt = r / (th * tw);
-    const int r2 = r - dt * (th * tw);
-    const int dh = r2 / tw, dw = r2 - dh * tw;
-    return ((ct * tt + dt) * H + ch * th + dh) * W + cw * tw + dw;
-}
-
 // CPR = 16-byte chunks per row.  Each work item is (bh, 128 consecutive
 // permuted positions); lanes move 16-byte chunks, 4 rows in flight per lane.
 template <int CPR>
@@ -77,7 +63,7 @@ __global__ void __launch_bounds__(kThreads) permute_kernel(const PermArgs a) {
                 const int p = p0 + r0 + u * RPP + rsub;
                 ok[u] = (r0 + u * RPP + rsub) < kRowsPerItem && p < a.S;
                 if (ok[u]) {
-                    const int tok = perm_token(p, a.H, a.W, tt, th, tw);
+                    const int tok = tile_token(p, a.H, a.W, tt, th, tw);
                     const size_t srow = head + (a.inverse ? p : tok);
                     drow[u] = head + (a.inverse ? tok : p);
                     v[u] = __ldcs(src + srow * CPR + chunk);

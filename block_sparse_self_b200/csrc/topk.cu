@@ -9,7 +9,10 @@
 // One warp per row.  Scores map to order-preserving uint32 keys; a 4-pass
 // 8-bit radix select finds the k-th largest key T and how many keys equal to
 // T are taken (lowest indices first); a final ordered pass ranks the ties,
-// ORs in the static blocks and compacts the kept indices with ballots.
+// ORs in the static blocks and compacts the kept indices with ballots.  Rows
+// of up to 1024 blocks keep their keys in registers and find the threshold by
+// bisection instead (below); longer rows use the radix select, re-reading the
+// row (from L1/L2) on each pass.
 #include "common.cuh"
 #include "internal.h"
 
@@ -117,6 +120,70 @@ __global__ void __launch_bounds__(kWarps * 32) topk_kernel(const float *__restri
     }
 }
 
+// Rows of up to 32 * NPL blocks: the keys stay in registers (block j in lane
+// j % 32, slot j / 32) and the k-th largest key T is found by bisection on
+// its bits: T is the largest value with count(key >= T) >= k, each count a
+// per-lane compare-and-add plus a warp sum.  No shared memory, no atomics.
+template <int NPL>
+__device__ __forceinline__ int count_ge(const uint32_t (&key)[NPL], uint32_t t) {
+    int c0 = 0, c1 = 0;
+    #pragma unroll
+    for (int i = 0; i < NPL; i += 2) {
+        c0 += key[i] >= t;
+        if (i + 1 < NPL) c1 += key[i + 1] >= t;
+    }
+    int c = c0 + c1;
+    #pragma unroll
+    for (int off = 16; off > 0; off >>= 1) c += __shfl_xor_sync(0xffffffffu, c, off);
+    return c;
+}
+
+template <int NPL>
+__global__ void __launch_bounds__(kWarps * 32) topk_reg_kernel(const float *__restrict__ scores, long long rows,
+                                                              int nb, int k, int n_sink, int diag_hw,
+                                                              int32_t *__restrict__ idx, int32_t *__restrict__ cnt,
+                                                              int cap) {
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    for (long long row = static_cast<long long>(blockIdx.x) * kWarps + warp; row < rows;
+         row += static_cast<long long>(gridDim.x) * kWarps) {
+        const float *s = scores + row * nb;
+        const int i = static_cast<int>(row % nb);
+        uint32_t key[NPL];  // 0 marks a slot past the row (every finite score maps above 0)
+        #pragma unroll
+        for (int t = 0; t < NPL; ++t) {
+            const int j = lane + 32 * t;
+            key[t] = j < nb ? order_key(__ldg(s + j)) : 0u;
+        }
+        uint32_t thr = 0u;
+        #pragma unroll 1
+        for (int bit = 31; bit >= 0; --bit) {
+            const uint32_t cand = thr | (1u << bit);
+            if (count_ge<NPL>(key, cand) >= k) thr = cand;
+        }
+        // thr = the k-th largest key; `need` keys equal to it are taken, lowest index first
+        const int need = k - (thr == 0xffffffffu ? 0 : count_ge<NPL>(key, thr + 1u));
+        int32_t *out = idx + row * cap;
+        int taken_eq = 0, written = 0;
+        #pragma unroll
+        for (int t = 0; t < NPL; ++t) {
+            const int j = lane + 32 * t;
+            const bool in = j < nb;
+            const bool eq = in && key[t] == thr;
+            const uint32_t eqm = __ballot_sync(0xffffffffu, eq);
+            const int rank = taken_eq + __popc(eqm & ((1u << lane) - 1u));
+            const int dd = j > i ? j - i : i - j;
+            const bool keep = in && (key[t] > thr || (eq && rank < need) || j < n_sink || dd <= diag_hw);
+            const uint32_t km = __ballot_sync(0xffffffffu, keep);
+            const int pos = written + __popc(km & ((1u << lane) - 1u));
+            if (keep && pos < cap) out[pos] = j;
+            taken_eq += __popc(eqm);
+            written += __popc(km);
+        }
+        for (int p = written + lane; p < cap; p += 32) out[p] = -1;
+        if (lane == 0) cnt[row] = written;
+    }
+}
+
 }  // namespace
 
 cudaError_t launch_topk(const float *scores, int BH, int nb, int k, int n_sink, int diag_hw, int32_t *idx,
@@ -124,7 +191,17 @@ cudaError_t launch_topk(const float *scores, int BH, int nb, int k, int n_sink, 
     const long long rows = static_cast<long long>(BH) * nb;
     long long blocks = (rows + kWarps - 1) / kWarps;
     if (blocks > 148LL * 16) blocks = 148LL * 16;
-    topk_kernel<<<static_cast<int>(blocks), kWarps * 32, 0, st>>>(scores, rows, nb, k, n_sink, diag_hw, idx, cnt, cap);
+    const int grid = static_cast<int>(blocks);
+    const int npl = (nb + 31) / 32;
+#define VSA_TOPK_REG(N) topk_reg_kernel<N><<<grid, kWarps * 32, 0, st>>>(scores, rows, nb, k, n_sink, diag_hw, idx, cnt, cap)
+    if (npl <= 1) VSA_TOPK_REG(1);
+    else if (npl <= 2) VSA_TOPK_REG(2);
+    else if (npl <= 4) VSA_TOPK_REG(4);
+    else if (npl <= 8) VSA_TOPK_REG(8);
+    else if (npl <= 16) VSA_TOPK_REG(16);
+    else if (npl <= 32) VSA_TOPK_REG(32);
+    else topk_kernel<<<grid, kWarps * 32, 0, st>>>(scores, rows, nb, k, n_sink, diag_hw, idx, cnt, cap);
+#undef VSA_TOPK_REG
     return cudaGetLastError();
 }
 

@@ -95,7 +95,8 @@ def test_block_summaries_bit_exact(dtype, D, block):
         assert np.array_equal(_np(mn.view(4, -1, D)[bh]), omn)
 
 
-@pytest.mark.parametrize("dtype,D,nb", [(torch.bfloat16, 128, 40), (torch.float32, 64, 70), (torch.bfloat16, 64, 1)])
+@pytest.mark.parametrize("dtype,D,nb", [(torch.bfloat16, 128, 40), (torch.float32, 64, 70), (torch.bfloat16, 64, 1),
+                                        (torch.bfloat16, 128, 300), (torch.bfloat16, 64, 129)])
 def test_block_scores_exact_on_integer_grid(dtype, D, nb):
     summ = [integer_grid((1, 2, nb, D), 20 + i, dtype, DEV) for i in range(4)]
     s = vsa.block_scores(*summ)
@@ -113,7 +114,8 @@ def test_block_scores_smooth_within_fp32_bound():
     for h in range(2):
         a = [_np(t[0, h]).astype(np.float64) for t in (qmax, qmin, kmax, kmin)]
         want = oracle.block_scores(*a)
-        bound = 4 * np.finfo(np.float32).eps * (np.abs(a[0] + a[1]) @ np.maximum(np.abs(a[2]), np.abs(a[3])).T)
+        # fp32 accumulation of q_max.k + q_min.k over 2D exact products
+        bound = 4 * np.finfo(np.float32).eps * ((np.abs(a[0]) + np.abs(a[1])) @ np.maximum(np.abs(a[2]), np.abs(a[3])).T)
         assert (np.abs(_np(s[0, h]) - want) <= bound + 1e-30).all()
 
 
