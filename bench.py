@@ -4,8 +4,11 @@
 One step = one pass of the whole hot path over one batch of synthetic input,
 on the SPADE adaptive workload (1 x 24 heads, grid 32x48x80, S = 122880,
 D = 128, bf16, candidate tiles (1,8,16), (2,8,8), (4,4,8), 10 % top-k budget):
-per-head tiling choice -> permute Q, K, V -> block summaries -> block scores ->
-top-k + sink + diagonal lists -> block-sparse attention -> inverse permute.
+per-head tiling choice -> block summaries -> block scores -> top-k + sink +
+diagonal lists -> block-sparse attention.  The permutation to each head's
+tile-contiguous order and back is done inside the summaries and attention
+kernels (TMA boxes in, token rows out); the explicit permute -> ... ->
+unpermute composition is timed beside it as a secondary line.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
 
@@ -52,7 +55,7 @@ def load_peaks():
 
 def kernel_source_hash() -> str:
     h = hashlib.sha256()
-    for f in ("attention.cu", "common.cuh"):
+    for f in ("attention_pp.cu", "common.cuh"):
         h.update(open(os.path.join(ROOT, "block_sparse_self_b200", "csrc", f), "rb").read())
     return h.hexdigest()[:16]
 
@@ -122,52 +125,76 @@ class ClockSampler:
 # --------------------------------------------------------------------------
 
 PHASES = ("select_tiling", "permute", "summaries", "scores", "topk", "attention", "unpermute")
+TILED_PHASES = ("select_tiling", "summaries", "scores", "topk", "attention")
 
 
 class SpadeStep:
-    """The SPADE path on preallocated device buffers (inputs resident in HBM)."""
+    """The SPADE path on preallocated device buffers (inputs resident in HBM).
 
-    def __init__(self, w, q, k, v):
+    tiled=True: summaries and attention read T-major Q/K/V through each head's
+    tiling and attention writes T-major O (no permuted copies); tiled=False:
+    explicit permute / unpermute around the same kernels."""
+
+    def __init__(self, w, q, k, v, tiled: bool = True):
         import block_sparse_self_b200 as vsa
         self.vsa, self.w = vsa, w
         self.q, self.k, self.v = q, k, v
         self.tiles = list(w.tiles)
         self.block = w.tiles[0][0] * w.tiles[0][1] * w.tiles[0][2]
         self.kk = w.k
+        self.tiled = tiled and self.block == 128 and vsa.tiled_supported(self.tiles)
+        self.phases = TILED_PHASES if self.tiled else PHASES
         self.events = []
 
     def launches(self) -> int:
-        return (2 if len(self.tiles) > 1 else 0) + 3 + 2 + 1 + 1 + 1 + 1
+        sel = 2 if len(self.tiles) > 1 else 0
+        if self.tiled:
+            return sel + 2 + 1 + 1 + 1
+        return sel + 3 + 2 + 1 + 1 + 1 + 1
 
     def __call__(self, record: bool):
         vsa, w = self.vsa, self.w
-        ev = [torch.cuda.Event(enable_timing=True) for _ in range(len(PHASES) + 1)] if record else None
-        mark = (lambda i: ev[i].record()) if record else (lambda i: None)
-        mark(0)
+        ev = [torch.cuda.Event(enable_timing=True) for _ in range(len(self.phases) + 1)] if record else None
+        n = [0]
+
+        def mark():
+            if record:
+                ev[n[0]].record()
+            n[0] += 1
+
+        mark()
         choice = vsa.select_tiling(self.q, w.grid, self.tiles) if len(self.tiles) > 1 else None
-        mark(1)
-        qp, kp, vp = (vsa.permute(x, w.grid, self.tiles, choice) for x in (self.q, self.k, self.v))
-        mark(2)
-        qmax, qmin = vsa.block_summaries(qp, self.block)
-        kmax, kmin = vsa.block_summaries(kp, self.block)
-        mark(3)
+        mark()
+        if self.tiled:
+            qmax, qmin = vsa.block_summaries_tiled(self.q, w.grid, self.tiles, choice, self.block)
+            kmax, kmin = vsa.block_summaries_tiled(self.k, w.grid, self.tiles, choice, self.block)
+        else:
+            qp, kp, vp = (vsa.permute(x, w.grid, self.tiles, choice) for x in (self.q, self.k, self.v))
+            mark()
+            qmax, qmin = vsa.block_summaries(qp, self.block)
+            kmax, kmin = vsa.block_summaries(kp, self.block)
+        mark()
         scores = vsa.block_scores(qmax, qmin, kmax, kmin)
-        mark(4)
+        mark()
         idx, cnt = vsa.topk_block_mask(scores, self.kk, w.n_sink_blocks, w.diag_halfwidth)
-        mark(5)
-        op = vsa.block_sparse_attention(qp, kp, vp, idx, cnt, self.block)
-        mark(6)
-        o = vsa.unpermute(op, w.grid, self.tiles, choice)
-        mark(7)
+        mark()
+        if self.tiled:
+            o = vsa.block_sparse_attention_tiled(self.q, self.k, self.v, w.grid, self.tiles, choice, idx, cnt)
+            mark()
+        else:
+            op = vsa.block_sparse_attention(qp, kp, vp, idx, cnt, self.block)
+            mark()
+            o = vsa.unpermute(op, w.grid, self.tiles, choice)
+            mark()
         if record:
             self.events.append(ev)
         self.last = dict(cnt=cnt, o=o, scores=scores, idx=idx)
         return o
 
     def phase_ms(self):
-        out = {p: [] for p in PHASES}
+        out = {p: [] for p in self.phases}
         for ev in self.events:
-            for i, p in enumerate(PHASES):
+            for i, p in enumerate(self.phases):
                 out[p].append(ev[i].elapsed_time(ev[i + 1]))
         return {p: float(np.mean(v)) for p, v in out.items() if v}
 
@@ -384,18 +411,34 @@ def extra_workloads(steps: int):
                    "attn_tflops": fl / ph["attention"] / 1e9, "phase_ms": ph}
     del q, k, v, st
 
-    # structured masks on a CFG pair
+    # structured masks on a CFG pair.  The attention kernel runs in the mode
+    # structured_attention picks: T-major directly for whole-frame tiles
+    # (spatial), through TMA boxes for sliding tiles, on permuted copies
+    # with a group mask for the temporal tile.
     w = WORKLOADS["structured_s122880"]
     q, k, v = make_qkv(w, device="cuda")
     res = {}
     for kind in w.structured:
         stile = vsa.structured_tile(kind, w.grid, w.sliding_tile)
         idx, cnt, g = vsa.structured_block_list(kind, w.grid, 128, w.sliding_tile, w.sliding_radius)
-        qp, kp, vp = (vsa.permute(x, w.grid, [stile]) for x in (q, k, v))
-        ms = timed(lambda: vsa.block_sparse_attention(qp, kp, vp, idx, cnt, 128, g), n=max(2, steps // 2))
+        if stile[1] == w.grid[1] and stile[2] == w.grid[2]:
+            mode = "t-major"
+            fn = lambda: vsa.block_sparse_attention(q, k, v, idx, cnt, 128, g)  # noqa: E731
+        elif g == 0 and vsa.tiled_supported([stile]):
+            mode = "tiled"
+            fn = lambda: vsa.block_sparse_attention_tiled(q, k, v, w.grid, [stile], None, idx, cnt)  # noqa: E731
+        else:
+            mode = "permuted copies"
+            qp, kp, vp = (vsa.permute(x, w.grid, [stile]) for x in (q, k, v))
+            fn = lambda: vsa.block_sparse_attention(qp, kp, vp, idx, cnt, 128, g)  # noqa: E731
+        ms = timed(fn, n=max(2, steps // 2))
+        call_ms = timed(lambda: vsa.structured_attention(q, k, v, kind, w.grid, 128, tile=w.sliding_tile,
+                                                         radius=w.sliding_radius), n=max(2, steps // 2))
         fl = float(cnt.to(torch.int64).sum().item()) * 4.0 * 128 * 128 * w.D * w.B * w.heads
-        res[kind] = {"attn_ms": ms, "tflops": fl / ms / 1e9, "group_size": g}
-        del qp, kp, vp
+        res[kind] = {"attn_ms": ms, "tflops": fl / ms / 1e9, "group_size": g, "mode": mode,
+                     "structured_attention_call_ms": call_ms}
+        fn = None
+        qp = kp = vp = None
     out[w.name] = res
     return out
 
@@ -440,7 +483,9 @@ def run_ours(args, w):
     mask_ms = ph["summaries"] + ph["scores"] + ph["topk"]
     mask_gbs = mask_pipeline_bytes(w, BH) / mask_ms / 1e6
     hbm = peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"])
-    roofline = {"bound": "tensor", "kernel": "vsa attn_kernel<128,128> (block-sparse)",
+    kname = ("attn_pp_kernel<128,false,true> (block-sparse, tiled)" if step.tiled
+             else "attn_pp_kernel<128,false,false> (block-sparse)")
+    roofline = {"bound": "tensor", "kernel": kname,
                 "achieved": achieved, "peak": peak, "unit": "TFLOP/s", "frac": achieved / peak,
                 "peak_kind": f"bf16_tflops_sustained ({peak_src})", "frac_of_burst": achieved / burst,
                 "traffic": profiled_traffic(w.name), "attn_ms_per_call": attn_ms,
@@ -458,6 +503,12 @@ def run_ours(args, w):
     extra = None
     if rank == 0 and world == 1 and not args.no_extra:
         extra = extra_workloads(max(3, args.steps // 2))
+        if step.tiled:  # the same step with explicit permuted copies, for comparison
+            ex = SpadeStep(wr, q, k, v, tiled=False)
+            ex_ms = time_steps(ex, max(3, args.steps // 2), 3, False)
+            extra["explicit_permute_" + w.name] = {"ms_per_step": ex_ms, "phase_ms": ex.phase_ms(),
+                                                   "same_output": bool(torch.equal(ex.last["o"], step.last["o"]))}
+            del ex
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:

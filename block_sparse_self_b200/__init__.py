@@ -57,10 +57,12 @@ def lib() -> ctypes.CDLL:
         "vsa_permute": ([P, P, I, I, I, I, I, D3, P, I, P, P], I),
         "vsa_unpermute": ([P, P, I, I, I, I, I, D3, P, I, P, P], I),
         "vsa_block_summaries": ([P, I, I, I, I, I, I, P, P, P], I),
+        "vsa_block_summaries_tiled": ([P, I, I, I, I, I, D3, P, I, P, I, P, P, P], I),
         "vsa_block_scores": ([P, P, P, P, I, I, I, I, I, P, P], I),
         "vsa_topk_block_mask": ([P, I, I, I, I, I, I, P, P, I, P], I),
         "vsa_structured_block_list": ([I, D3, D3, D3, I, P, P, I, P, P], I),
         "vsa_block_sparse_attention": ([P, P, P, P, I, I, I, I, I, I, P, P, I, I, I, F, P], I),
+        "vsa_block_sparse_attention_tiled": ([P, P, P, P, I, I, I, I, I, D3, P, I, P, P, P, I, I, F, P], I),
         "vsa_window_attention": ([P, P, P, P, I, I, I, I, I, I, I, F, I, P], I),
         "vsa_cast_f32_to_bf16": ([P, P, I64, P], I),
         "vsa_debug_wait_timeout": ([I64, P], I),
@@ -210,6 +212,29 @@ def block_summaries(x_perm: torch.Tensor, block: int):
     return xmax, xmin
 
 
+def _choice_arg(choice, BH):
+    if choice is not None:
+        _cuda(choice, "choice")
+        if choice.dtype != torch.int32 or choice.numel() != BH:
+            raise ValueError("choice must be int32 with B*H entries")
+    return _ptr(choice)
+
+
+def block_summaries_tiled(x: torch.Tensor, grid, tiles, choice: Optional[torch.Tensor], block: int):
+    """block_summaries(permute(x, grid, tiles, choice), block) read straight from T-major x."""
+    _cuda(x, "x")
+    B, H, S, D = _bhsd(x, "x")
+    if block <= 0 or S % block:
+        raise ValueError(f"block ({block}) must divide S ({S})")
+    arr, n = _tiles_arg(tiles)
+    xmax = torch.empty(B, H, S // block, D, dtype=x.dtype, device=x.device)
+    xmin = torch.empty_like(xmax)
+    _check(lib().vsa_block_summaries_tiled(_ptr(x), _dtype_code(x, "x"), B, H, S, D, Dims3(*grid), arr, n,
+                                           _choice_arg(choice, B * H), int(block), _ptr(xmax), _ptr(xmin),
+                                           _stream(x.device)))
+    return xmax, xmin
+
+
 def block_scores(q_max, q_min, k_max, k_min) -> torch.Tensor:
     """fp32 [B, H, nb, nb]: max((q_max+q_min).k_max, (q_max+q_min).k_min)."""
     for t, nm in ((q_max, "q_max"), (q_min, "q_min"), (k_max, "k_max"), (k_min, "k_min")):
@@ -312,6 +337,41 @@ def block_sparse_attention(q, k, v, idx, cnt, block: int, group_size: int = 0, s
     return o
 
 
+def block_sparse_attention_tiled(q, k, v, grid, tiles, choice, idx, cnt, scale: Optional[float] = None,
+                                 out_dtype=None) -> torch.Tensor:
+    """unpermute(block_sparse_attention(permute(q), permute(k), permute(v), idx, cnt, 128)) in one
+    kernel: q, k, v and the result stay in T-major order; lists number 128-token blocks of
+    each head's tile-contiguous order."""
+    B, H, S, D = _bhsd(q, "q")
+    if tuple(k.shape) != (B, H, S, D) or tuple(v.shape) != (B, H, S, D):
+        raise ValueError(f"q/k/v shapes must match exactly; got q={tuple(q.shape)}, k={tuple(k.shape)}, "
+                         f"v={tuple(v.shape)}")
+    odt = _out_dtype(out_dtype, q)
+    qb, kb, vb = _bf16(q, "q"), _bf16(k, "k"), _bf16(v, "v")
+    _cuda(idx, "idx")
+    _cuda(cnt, "cnt")
+    if idx.dtype != torch.int32 or cnt.dtype != torch.int32:
+        raise ValueError("idx and cnt must be int32")
+    arr, n = _tiles_arg(tiles)
+    o = torch.empty(B, H, S, D, dtype=odt, device=q.device)
+    _check(lib().vsa_block_sparse_attention_tiled(
+        _ptr(qb), _ptr(kb), _ptr(vb), _ptr(o), BF16 if odt == torch.bfloat16 else F32, B, H, S, D, Dims3(*grid),
+        arr, n, _choice_arg(choice, B * H), _ptr(idx), _ptr(cnt), int(idx.shape[-1]), 1 if idx.dim() == 4 else 0,
+        0.0 if scale is None else float(scale), _stream(q.device)))
+    return o
+
+
+def tiled_supported(tiles) -> bool:
+    """Whether every candidate tiling can run through the T-major (tiled) attention:
+    one common volume V, a multiple of 128, and each tile.t divisible by V/128."""
+    tiles = [tuple(t) for t in tiles]
+    vols = {t[0] * t[1] * t[2] for t in tiles}
+    if len(vols) != 1:
+        return False
+    vol = vols.pop()
+    return vol % 128 == 0 and all(t[0] % (vol // 128) == 0 for t in tiles)
+
+
 def window_attention(q, k, v, window: int, sink: int = 0, scale: Optional[float] = None,
                      chunk_size: Optional[int] = None, out_dtype=None) -> torch.Tensor:
     """Symmetric sliding-window attention with `sink` global keys (dense when window >= S)."""
@@ -352,12 +412,18 @@ def topk_budget(nb: int, budget: float) -> int:
 
 def spade_attention(q, k, v, grid, tiles, budget: Optional[float] = None, topk: Optional[int] = None,
                     n_sink_blocks: int = 1, diag_halfwidth: int = 0, scale: Optional[float] = None,
-                    out_dtype=None, return_intermediates: bool = False):
+                    out_dtype=None, return_intermediates: bool = False, tiled: Optional[bool] = None):
     """Adaptive tiling -> permutation -> min/max block scores -> top-k + sink +
     diagonal -> block-sparse attention -> inverse permutation, all on the GPU.
 
     Every candidate tile must have the same volume (the block size).  With a
     single candidate the tiling choice is skipped (choice 0 for every head).
+
+    tiled=True runs the permutation inside the summaries and attention kernels
+    (no permuted copies; block size 128, see tiled_supported); tiled=False
+    runs the explicit permute / unpermute steps; None picks tiled when it is
+    supported.  Both give identical results.  In tiled mode the permuted
+    tensors in the intermediates are computed afterwards, for inspection only.
     """
     tiles = [tuple(t) for t in tiles]
     vols = {t[0] * t[1] * t[2] for t in tiles}
@@ -367,14 +433,29 @@ def spade_attention(q, k, v, grid, tiles, budget: Optional[float] = None, topk: 
     B, H, S, D = _bhsd(q, "q")
     nb = S // block
     kk = topk if topk is not None else topk_budget(nb, budget if budget is not None else 0.17)
+    can_tile = block == 128 and tiled_supported(tiles)
+    if tiled is None:
+        tiled = can_tile
+    elif tiled and not can_tile:
+        raise ValueError("tiled mode needs 128-token blocks whose tiles satisfy tiled_supported()")
     choice = select_tiling(q, grid, tiles) if len(tiles) > 1 else None
-    qp, kp, vp = (permute(x, grid, tiles, choice) for x in (q, k, v))
-    qmax, qmin = block_summaries(qp, block)
-    kmax, kmin = block_summaries(kp, block)
-    scores = block_scores(qmax, qmin, kmax, kmin)
-    idx, cnt = topk_block_mask(scores, kk, n_sink_blocks, diag_halfwidth)
-    op = block_sparse_attention(qp, kp, vp, idx, cnt, block, 0, scale, out_dtype)
-    o = unpermute(op, grid, tiles, choice)
+    if tiled:
+        qb, kb, vb = _bf16(q, "q"), _bf16(k, "k"), _bf16(v, "v")
+        qmax, qmin = block_summaries_tiled(q, grid, tiles, choice, block)
+        kmax, kmin = block_summaries_tiled(k, grid, tiles, choice, block)
+        scores = block_scores(qmax, qmin, kmax, kmin)
+        idx, cnt = topk_block_mask(scores, kk, n_sink_blocks, diag_halfwidth)
+        o = block_sparse_attention_tiled(qb, kb, vb, grid, tiles, choice, idx, cnt, scale, out_dtype)
+        if return_intermediates:
+            qp, kp, vp, op = (permute(x, grid, tiles, choice) for x in (q, k, v, o))
+    else:
+        qp, kp, vp = (permute(x, grid, tiles, choice) for x in (q, k, v))
+        qmax, qmin = block_summaries(qp, block)
+        kmax, kmin = block_summaries(kp, block)
+        scores = block_scores(qmax, qmin, kmax, kmin)
+        idx, cnt = topk_block_mask(scores, kk, n_sink_blocks, diag_halfwidth)
+        op = block_sparse_attention(qp, kp, vp, idx, cnt, block, 0, scale, out_dtype)
+        o = unpermute(op, grid, tiles, choice)
     if return_intermediates:
         return o, dict(choice=choice, qp=qp, kp=kp, vp=vp, qmax=qmax, qmin=qmin, kmax=kmax, kmin=kmin,
                        scores=scores, idx=idx, cnt=cnt, out_perm=op, block=block, k=kk)
@@ -386,6 +467,10 @@ def structured_attention(q, k, v, kind: str, grid, block: int = 128, tile=(4, 8,
     """A structured static mask as block-sparse attention, in and out in T-major order."""
     st = structured_tile(kind, grid, tile)
     idx, cnt, g = structured_block_list(kind, grid, block, tile, radius, device=q.device)
+    if st[1] == grid[1] and st[2] == grid[2]:  # whole frames: the tile-contiguous order is T-major itself
+        return block_sparse_attention(q, k, v, idx, cnt, block, g, scale, out_dtype)
+    if g == 0 and block == 128 and tiled_supported([st]):
+        return block_sparse_attention_tiled(q, k, v, grid, [st], None, idx, cnt, scale, out_dtype)
     qp, kp, vp = (permute(x, grid, [st]) for x in (q, k, v))
     op = block_sparse_attention(qp, kp, vp, idx, cnt, block, g, scale, out_dtype)
     return unpermute(op, grid, [st])

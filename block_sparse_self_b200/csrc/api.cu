@@ -247,6 +247,26 @@ vsa_status vsa_block_summaries(const void *x_perm, vsa_dtype dtype, int B, int n
                       "block_summaries launch");
 }
 
+vsa_status vsa_block_summaries_tiled(const void *x, vsa_dtype dtype, int B, int n_heads, int S, int D,
+                                     vsa_dims3 grid, const vsa_dims3 *tiles, int n_tiles, const int32_t *choice,
+                                     int block, void *x_max, void *x_min, void *stream) {
+    VSA_REQUIRE(esize_of(dtype) != 0, "dtype must be VSA_BF16 or VSA_F32");
+    VSA_TRY(check_bhsd(B, n_heads, S, D));
+    VSA_TRY(check_d(D));
+    VSA_REQUIRE(block == 16 || block == 32 || block == 64 || block == 128 || block == 256,
+                "block must be one of 16, 32, 64, 128, 256, got %d", block);
+    VSA_REQUIRE(S % block == 0, "block (%d) must divide S (%d)", block, S);
+    VSA_REQUIRE(aligned16(x) && aligned16(x_max) && aligned16(x_min),
+                "x, x_max and x_min must be non-NULL 16-byte aligned device pointers");
+    VSA_REQUIRE(choice == nullptr || aligned4(choice), "choice must be NULL or 4-byte aligned");
+    VSA_TRY(check_grid(grid, S));
+    TileSet ts;
+    VSA_TRY(check_tiles(grid, tiles, n_tiles, &ts));
+    return check_cuda(launch_summaries_tiled(x, esize_of(dtype), B * n_heads, S, D, grid.t, grid.h, grid.w, ts,
+                                             choice, x_max, x_min, status_or_null(), as_stream(stream), block),
+                      "block_summaries_tiled launch");
+}
+
 vsa_status vsa_block_scores(const void *q_max, const void *q_min, const void *k_max, const void *k_min,
                             vsa_dtype dtype, int B, int n_heads, int nb, int D, float *scores, void *stream) {
     VSA_REQUIRE(esize_of(dtype) != 0, "dtype must be VSA_BF16 or VSA_F32");
@@ -365,6 +385,44 @@ vsa_status vsa_block_sparse_attention(const void *q, const void *k, const void *
     L.idx = idx; L.cnt = cnt; L.cap = cap; L.list_per_head = list_per_head ? 1 : 0;
     L.group = group_size; L.nb = S / block;
     L.scale = scale > 0.f ? scale : 1.0f / sqrtf(static_cast<float>(D));
+    return launch_attention(L, status_or_null(), as_stream(stream));
+}
+
+vsa_status vsa_block_sparse_attention_tiled(const void *q, const void *k, const void *v, void *o,
+                                            vsa_dtype out_dtype, int B, int n_heads, int S, int D, vsa_dims3 grid,
+                                            const vsa_dims3 *tiles, int n_tiles, const int32_t *choice,
+                                            const int32_t *idx, const int32_t *cnt, int cap, int list_per_head,
+                                            float scale, void *stream) {
+    VSA_TRY(check_attention_common(q, k, v, o, out_dtype, B, n_heads, S, D, scale));
+    VSA_REQUIRE(aligned4(idx) && aligned4(cnt), "idx and cnt must be non-NULL 4-byte aligned device pointers");
+    VSA_REQUIRE(cap >= 1, "cap must be >= 1, got %d", cap);
+    VSA_REQUIRE(choice == nullptr || aligned4(choice), "choice must be NULL or 4-byte aligned");
+    VSA_TRY(check_grid(grid, S));
+    TileSet ts;
+    VSA_TRY(check_tiles(grid, tiles, n_tiles, &ts));
+    const int vol = ts.t[0] * ts.h[0] * ts.w[0];
+    VSA_REQUIRE(vol % 128 == 0, "tile volume (%d) must be a multiple of 128", vol);
+    for (int c = 0; c < n_tiles; ++c) {
+        VSA_REQUIRE(ts.t[c] * ts.h[c] * ts.w[c] == vol, "every tile must have the volume of tile 0 (%d); tile %d has %d",
+                    vol, c, ts.t[c] * ts.h[c] * ts.w[c]);
+        VSA_REQUIRE(ts.t[c] % (vol / 128) == 0,
+                    "tile %d: tile.t (%d) must be divisible by volume / 128 (%d) so each 128-token block is whole "
+                    "(h, w) planes",
+                    c, ts.t[c], vol / 128);
+    }
+    AttnLaunch L{};
+    L.q = q; L.k = k; L.v = v; L.o = o;
+    L.out_f32 = out_dtype == VSA_F32;
+    L.BH = B * n_heads; L.S = S; L.D = D;
+    L.block = 128;
+    L.window = false;
+    L.idx = idx; L.cnt = cnt; L.cap = cap; L.list_per_head = list_per_head ? 1 : 0;
+    L.group = 0; L.nb = S / 128;
+    L.scale = scale > 0.f ? scale : 1.0f / sqrtf(static_cast<float>(D));
+    L.tiled = true;
+    L.T = grid.t; L.Hg = grid.h; L.Wg = grid.w;
+    L.tiles = ts;
+    L.choice = choice;
     return launch_attention(L, status_or_null(), as_stream(stream));
 }
 

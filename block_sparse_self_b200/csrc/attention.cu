@@ -498,8 +498,23 @@ bool make_tile_map(CUtensorMap *m, const void *ptr, int D, int S, int BH, int ro
 }
 
 
+bool make_box_map(CUtensorMap *m, const void *ptr, int D, int T, int H, int W, int BH, int bt, int bh, int bw) {
+    EncodeTiledFn enc = encode_fn();
+    if (!enc) return false;
+    const cuuint64_t e = 2;  // bf16
+    cuuint64_t dims[5] = {static_cast<cuuint64_t>(D), static_cast<cuuint64_t>(W), static_cast<cuuint64_t>(H),
+                          static_cast<cuuint64_t>(T), static_cast<cuuint64_t>(BH)};
+    cuuint64_t strides[4] = {static_cast<cuuint64_t>(D) * e, static_cast<cuuint64_t>(W) * D * e,
+                             static_cast<cuuint64_t>(H) * W * D * e, static_cast<cuuint64_t>(T) * H * W * D * e};
+    cuuint32_t box[5] = {64, static_cast<cuuint32_t>(bw), static_cast<cuuint32_t>(bh), static_cast<cuuint32_t>(bt), 1};
+    cuuint32_t estr[5] = {1, 1, 1, 1, 1};
+    return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 5, const_cast<void *>(ptr), dims, strides, box, estr,
+               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 vsa_status launch_attention(const AttnLaunch &L, int *status, cudaStream_t st) {
-    if (L.block == 128) return launch_attention_pp(L, status, st);  // two query tiles per CTA
+    if (L.block == 128 || L.tiled) return launch_attention_pp(L, status, st);  // two query tiles per CTA
     if (L.window) {
         if (L.D == 128) return run<128, 128, true>(L, status, st);
         return run<64, 128, true>(L, status, st);

@@ -44,7 +44,31 @@ struct PPArgs {
     void *out;
     int out_f32;
     int *status;
+    // tiled mode: T-major tensors, per-head tiling (all of volume 128 * m)
+    int H, W;
+    TileSet tiles;
+    const int32_t *choice;
 };
+
+// Tensor maps: slot 0 only, or one per candidate tiling in tiled mode.
+struct MapSet {
+    CUtensorMap q[kMaxTiles], k[kMaxTiles], v[kMaxTiles];
+};
+
+// In tiled mode, block b of a head whose tiling is (tt, th, tw) is the
+// 128-token box (tt/m, th, tw) at part b % m of tile b / m (m = volume/128):
+// its TMA coordinates in the (D, W, H, T, BH) tensor.
+struct BoxCoord {
+    int w, h, t;
+};
+__device__ __forceinline__ BoxCoord box_of(int b, int H, int W, int tt, int th, int tw) {
+    const int m = (tt * th * tw) / 128;
+    const int tile = b / m, part = b - tile * m;
+    const int nth = H / th, ntw = W / tw;
+    const int ct = tile / (nth * ntw), rem = tile - ct * (nth * ntw);
+    const int ch = rem / ntw, cw = rem - ch * ntw;
+    return BoxCoord{cw * tw, ch * th, ct * tt + part * (tt / m)};
+}
 
 template <int D>
 struct PPCfg {
@@ -114,10 +138,9 @@ __device__ __forceinline__ int kblock_of(const TileSched &t, int j) {
     else return __ldg(t.list + j);
 }
 
-template <int D, bool WINDOW>
+template <int D, bool WINDOW, bool TILED>
 __global__ void __launch_bounds__(kThreads, 1)
-attn_pp_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
-               const __grid_constant__ CUtensorMap tmV, const PPArgs a) {
+attn_pp_kernel(const __grid_constant__ MapSet maps, const PPArgs a) {
     using C = PPCfg<D>;
     constexpr int BN = 128;
     extern __shared__ uint8_t smem_raw[];
@@ -198,6 +221,27 @@ attn_pp_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
             }
         }
     }
+    int tc = 0;  // tiled mode: this head's tiling
+    if constexpr (TILED) {
+        if (a.choice) tc = __ldg(a.choice + bh);
+        if (tc < 0 || tc >= a.tiles.n) {  // the head is left unwritten
+            if (threadIdx.x == 0) report(a.status, DEV_RUNTIME);
+            ts[0].n = ts[1].n = 0;
+            ts[0].qt = ts[1].qt = -1;
+            tc = 0;
+        }
+    }
+    const int tt = a.tiles.t[tc], th = a.tiles.h[tc], tw = a.tiles.w[tc];
+    const CUtensorMap *tmQ = &maps.q[tc], *tmK = &maps.k[tc], *tmV = &maps.v[tc];
+    // one 128-row tile of Q, K or V: block b of this head
+    auto load_tile = [&](uint8_t *dst, const CUtensorMap *map, uint64_t *bar, int b) {
+        if constexpr (TILED) {
+            const BoxCoord c = box_of(b, a.H, a.W, tt, th, tw);
+            for (int s = 0; s < C::KSLABS; ++s) tma_load_5d(dst + s * C::SLAB, map, bar, s * 64, c.w, c.h, c.t, bh);
+        } else {
+            for (int s = 0; s < C::KSLABS; ++s) tma_load_3d(dst + s * C::SLAB, map, bar, s * 64, b * BN, bh);
+        }
+    };
     const int nA = ts[0].n, nB = ts[1].n;
     const int nmax = max(nA, nB);
 
@@ -205,15 +249,13 @@ attn_pp_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
     if (warp == 8) {
         // ================= TMA producer =================
         if (lane == 0 && nmax > 0) {
-            tma_prefetch_desc(&tmQ);
-            tma_prefetch_desc(&tmK);
-            tma_prefetch_desc(&tmV);
+            tma_prefetch_desc(tmQ);
+            tma_prefetch_desc(tmK);
+            tma_prefetch_desc(tmV);
             const int nq_loaded = (nA > 0) + (nB > 0);
             mbar_arrive_expect_tx(q_full, nq_loaded * C::TILE_BYTES);
             for (int t = 0; t < 2; ++t)
-                if (ts[t].n > 0)
-                    for (int s = 0; s < C::KSLABS; ++s)
-                        tma_load_3d(sQ + t * C::TILE_BYTES + s * C::SLAB, &tmQ, q_full, s * 64, ts[t].qt * BN, bh);
+                if (ts[t].n > 0) load_tile(sQ + t * C::TILE_BYTES, tmQ, q_full, ts[t].qt);
             uint32_t kc = 0, vc = 0;
             bool ok = true;
             auto load = [&](bool is_k, int t, int j) -> bool {
@@ -227,8 +269,7 @@ attn_pp_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
                 uint8_t *dst = (is_k ? sK : sV) + slot * C::TILE_BYTES;
                 const int kb = kblock_of<WINDOW>(ts[t], j);
                 mbar_arrive_expect_tx(full, C::TILE_BYTES);
-                for (int s = 0; s < C::KSLABS; ++s)
-                    tma_load_3d(dst + s * C::SLAB, is_k ? &tmK : &tmV, full, s * 64, kb * BN, bh);
+                load_tile(dst, is_k ? tmK : tmV, full, kb);
                 ++c;
                 return true;
             };
@@ -441,7 +482,8 @@ attn_pp_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
         if (!ok && !*abort_flag) { report(a.status, DEV_TIMEOUT); *abort_flag = 1; }
 
         // ---- epilogue: O / l -> global ----
-        const size_t orow = static_cast<size_t>(bh) * S + rg;
+        // output row: the permuted position itself, or its T-major token in tiled mode
+        const size_t orow = static_cast<size_t>(bh) * S + (TILED ? tile_token(rg, a.H, a.W, tt, th, tw) : rg);
         bool have_o = ok && n > 0;
         if (have_o && !mbar_wait(&pv_done[t], (n - 1) & 1, abort_flag)) {
             have_o = false;
@@ -495,14 +537,25 @@ attn_pp_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
     }
 }
 
-template <int D, bool WINDOW>
+template <int D, bool WINDOW, bool TILED>
 vsa_status run_pp(const AttnLaunch &L, int *status, cudaStream_t st) {
     using C = PPCfg<D>;
-    CUtensorMap mq, mk, mv;
-    if (!make_tile_map(&mq, L.q, D, L.S, L.BH, 128) || !make_tile_map(&mk, L.k, D, L.S, L.BH, 128) ||
-        !make_tile_map(&mv, L.v, D, L.S, L.BH, 128))
-        return fail(VSA_ERR_CUDA, "cuTensorMapEncodeTiled failed (driver entry point or arguments)");
-    auto kern = attn_pp_kernel<D, WINDOW>;
+    MapSet maps = {};  // copied into the launch parameters
+    bool ok = true;
+    if constexpr (TILED) {
+        for (int c = 0; c < L.tiles.n; ++c) {
+            const int m = L.tiles.t[c] * L.tiles.h[c] * L.tiles.w[c] / 128;
+            const int bt = L.tiles.t[c] / m, bhh = L.tiles.h[c], bw = L.tiles.w[c];
+            ok = ok && make_box_map(&maps.q[c], L.q, D, L.T, L.Hg, L.Wg, L.BH, bt, bhh, bw) &&
+                 make_box_map(&maps.k[c], L.k, D, L.T, L.Hg, L.Wg, L.BH, bt, bhh, bw) &&
+                 make_box_map(&maps.v[c], L.v, D, L.T, L.Hg, L.Wg, L.BH, bt, bhh, bw);
+        }
+    } else {
+        ok = make_tile_map(&maps.q[0], L.q, D, L.S, L.BH, 128) && make_tile_map(&maps.k[0], L.k, D, L.S, L.BH, 128) &&
+             make_tile_map(&maps.v[0], L.v, D, L.S, L.BH, 128);
+    }
+    if (!ok) return fail(VSA_ERR_CUDA, "cuTensorMapEncodeTiled failed (driver entry point or arguments)");
+    auto kern = attn_pp_kernel<D, WINDOW, TILED>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
     if (e != cudaSuccess) return check_cuda(e, "cudaFuncSetAttribute(attention, two tiles)");
     PPArgs a;
@@ -521,16 +574,22 @@ vsa_status run_pp(const AttnLaunch &L, int *status, cudaStream_t st) {
     a.out = L.o;
     a.out_f32 = L.out_f32;
     a.status = status;
+    a.H = L.Hg;
+    a.W = L.Wg;
+    a.tiles = L.tiles;
+    a.choice = L.choice;
+    if (!TILED) a.tiles.n = 1;
     dim3 grid((a.nq + 1) / 2, L.BH);
-    kern<<<grid, kThreads, C::SMEM, st>>>(mq, mk, mv, a);
+    kern<<<grid, kThreads, C::SMEM, st>>>(maps, a);
     return check_cuda(cudaGetLastError(), "attention launch (two tiles)");
 }
 
 }  // namespace
 
 vsa_status launch_attention_pp(const AttnLaunch &L, int *status, cudaStream_t st) {
-    if (L.window) return L.D == 128 ? run_pp<128, true>(L, status, st) : run_pp<64, true>(L, status, st);
-    return L.D == 128 ? run_pp<128, false>(L, status, st) : run_pp<64, false>(L, status, st);
+    if (L.window) return L.D == 128 ? run_pp<128, true, false>(L, status, st) : run_pp<64, true, false>(L, status, st);
+    if (L.tiled) return L.D == 128 ? run_pp<128, false, true>(L, status, st) : run_pp<64, false, true>(L, status, st);
+    return L.D == 128 ? run_pp<128, false, false>(L, status, st) : run_pp<64, false, false>(L, status, st);
 }
 
 }  // namespace vsa

@@ -29,10 +29,10 @@ cudaError_t launch_permute(const void *src, void *dst, int esize, int BH, int S,
 cudaError_t launch_cast_f32_bf16(const float *x, void *y, int64_t n, cudaStream_t st);
 cudaError_t launch_summaries(const void *x, int esize, int BH, int S, int D, int block, void *xmax, void *xmin,
                              cudaStream_t st);
-// Summaries of the tiles of a T-major x in each head's tile-contiguous order.
+// Summaries of the blocks of a T-major x taken in each head's tile-contiguous order.
 cudaError_t launch_summaries_tiled(const void *x, int esize, int BH, int S, int D, int T, int H, int W,
                                    const TileSet &tiles, const int32_t *choice, void *xmax, void *xmin, int *status,
-                                   cudaStream_t st);
+                                   cudaStream_t st, int block);
 cudaError_t launch_scores(const void *qmax, const void *qmin, const void *kmax, const void *kmin, int esize, int BH,
                           int nb, int D, float *scores, cudaStream_t st);
 // bf16 summaries on tcgen05 (D in {64, 128})

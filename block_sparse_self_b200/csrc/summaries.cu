@@ -6,6 +6,11 @@
 //
 // One CTA per (bh, block).  Lanes own 16-byte column chunks; row groups walk
 // the block's rows with 128-bit loads, then reduce through shared memory.
+//
+// Tiled variant: x stays in T-major token order and the block's rows are read
+// where the head's chosen tiling puts them (position p of the tile-contiguous
+// order is token tile_token(p)), which gives the same result as permuting
+// first without writing the permuted copy.
 #include "common.cuh"
 #include "internal.h"
 
@@ -56,23 +61,47 @@ struct Vec<float> {
     }
 };
 
-template <typename T, int CPR>
+struct TiledArgs {
+    int H, W;
+    TileSet tiles;
+    const int32_t *choice;
+    int *status;
+};
+
+template <typename T, int CPR, bool TILED>
 __global__ void __launch_bounds__(kThreads) summaries_kernel(const uint8_t *__restrict__ x, int S, int block, int nb,
-                                                             uint8_t *__restrict__ xmax, uint8_t *__restrict__ xmin) {
+                                                             uint8_t *__restrict__ xmax, uint8_t *__restrict__ xmin,
+                                                             const TiledArgs ta) {
     constexpr int RG = kThreads / CPR;  // row groups
     __shared__ uint4 smax[RG][CPR];
     __shared__ uint4 smin[RG][CPR];
     const int blk = blockIdx.x, bh = blockIdx.y;
     const int chunk = threadIdx.x % CPR, rg = threadIdx.x / CPR;
-    const size_t row0 = static_cast<size_t>(bh) * S + static_cast<size_t>(blk) * block;
-    const uint8_t *base = x + row0 * CPR * 16 + chunk * 16;
+    const size_t head = static_cast<size_t>(bh) * S;
+    int tt = 1, th = 1, tw = 1;
+    if constexpr (TILED) {
+        const int c = ta.choice ? __ldg(ta.choice + bh) : 0;
+        if (c < 0 || c >= ta.tiles.n) {  // the head's summaries are left unwritten
+            if (threadIdx.x == 0) report(ta.status, DEV_RUNTIME);
+            return;
+        }
+        tt = ta.tiles.t[c];
+        th = ta.tiles.h[c];
+        tw = ta.tiles.w[c];
+    }
+    // byte address of chunk `chunk` of the block's r-th row
+    auto row_ptr = [&](int r) -> const uint8_t * {
+        const int p = blk * block + r;
+        const int tok = TILED ? tile_token(p, ta.H, ta.W, tt, th, tw) : p;
+        return x + (head + tok) * CPR * 16 + chunk * 16;
+    };
     Vec<T> mx, mn;
     if (rg < block) {
-        mx = Vec<T>::load(base + static_cast<size_t>(rg) * CPR * 16);
+        mx = Vec<T>::load(row_ptr(rg));
         mn = mx;
         #pragma unroll 4
         for (int r = rg + RG; r < block; r += RG) {
-            const Vec<T> v = Vec<T>::load(base + static_cast<size_t>(r) * CPR * 16);
+            const Vec<T> v = Vec<T>::load(row_ptr(r));
             mx.vmax(v);
             mn.vmin(v);
         }
@@ -92,23 +121,43 @@ __global__ void __launch_bounds__(kThreads) summaries_kernel(const uint8_t *__re
     }
 }
 
-}  // namespace
-
-cudaError_t launch_summaries(const void *x, int esize, int BH, int S, int D, int block, void *xmax, void *xmin,
-                             cudaStream_t st) {
+template <bool TILED>
+cudaError_t run_summaries(const void *x, int esize, int BH, int S, int D, int block, void *xmax, void *xmin,
+                          const TiledArgs &ta, cudaStream_t st) {
     const int nb = S / block;
     const int cpr = D * esize / 16;
     dim3 grid(nb, BH);
     const uint8_t *xi = static_cast<const uint8_t *>(x);
     uint8_t *mx = static_cast<uint8_t *>(xmax), *mn = static_cast<uint8_t *>(xmin);
     if (esize == 2) {
-        if (cpr == 8) summaries_kernel<__nv_bfloat16, 8><<<grid, kThreads, 0, st>>>(xi, S, block, nb, mx, mn);
-        else summaries_kernel<__nv_bfloat16, 16><<<grid, kThreads, 0, st>>>(xi, S, block, nb, mx, mn);
+        if (cpr == 8) summaries_kernel<__nv_bfloat16, 8, TILED><<<grid, kThreads, 0, st>>>(xi, S, block, nb, mx, mn, ta);
+        else summaries_kernel<__nv_bfloat16, 16, TILED><<<grid, kThreads, 0, st>>>(xi, S, block, nb, mx, mn, ta);
     } else {
-        if (cpr == 16) summaries_kernel<float, 16><<<grid, kThreads, 0, st>>>(xi, S, block, nb, mx, mn);
-        else summaries_kernel<float, 32><<<grid, kThreads, 0, st>>>(xi, S, block, nb, mx, mn);
+        if (cpr == 16) summaries_kernel<float, 16, TILED><<<grid, kThreads, 0, st>>>(xi, S, block, nb, mx, mn, ta);
+        else summaries_kernel<float, 32, TILED><<<grid, kThreads, 0, st>>>(xi, S, block, nb, mx, mn, ta);
     }
     return cudaGetLastError();
+}
+
+}  // namespace
+
+cudaError_t launch_summaries(const void *x, int esize, int BH, int S, int D, int block, void *xmax, void *xmin,
+                             cudaStream_t st) {
+    TiledArgs ta{};
+    return run_summaries<false>(x, esize, BH, S, D, block, xmax, xmin, ta, st);
+}
+
+cudaError_t launch_summaries_tiled(const void *x, int esize, int BH, int S, int D, int T, int H, int W,
+                                   const TileSet &tiles, const int32_t *choice, void *xmax, void *xmin, int *status,
+                                   cudaStream_t st, int block) {
+    (void)T;
+    TiledArgs ta;
+    ta.H = H;
+    ta.W = W;
+    ta.tiles = tiles;
+    ta.choice = choice;
+    ta.status = status;
+    return run_summaries<true>(x, esize, BH, S, D, block, xmax, xmin, ta, st);
 }
 
 }  // namespace vsa

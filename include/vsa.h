@@ -153,6 +153,21 @@ vsa_status vsa_block_summaries(const void *x_perm, vsa_dtype dtype, int B, int n
                                int S, int D, int block, void *x_max, void *x_min,
                                void *stream);
 
+/* The same summaries read from a T-major x, with no permuted copy: block i of
+ * (b, head) covers positions [i*block, (i+1)*block) of that head's
+ * tile-contiguous order under tiles[choice[bh]] (the order vsa_permute
+ * writes).  The result equals vsa_permute followed by vsa_block_summaries,
+ * bit for bit.
+ *   x      [B, n_heads, S, D] in `dtype`, T-major (S = grid.t*grid.h*grid.w)
+ *   tiles, n_tiles, choice  as for vsa_permute (choice NULL: tile 0)
+ *   x_max, x_min  [B, n_heads, S/block, D] in `dtype`
+ * A choice outside [0, n_tiles) leaves that head's summaries unwritten and
+ * sets VSA_ERR_RUNTIME (read with vsa_device_status).                      */
+vsa_status vsa_block_summaries_tiled(const void *x, vsa_dtype dtype, int B, int n_heads,
+                                     int S, int D, vsa_dims3 grid, const vsa_dims3 *tiles,
+                                     int n_tiles, const int32_t *choice, int block,
+                                     void *x_max, void *x_min, void *stream);
+
 /* ------------------------------------------------------------------------ */
 /* Block scores.  "Adaptive tiling (SPADE)", The idea, step 3, and the
  * function table (minmax_block_scores).
@@ -230,6 +245,29 @@ vsa_status vsa_block_sparse_attention(const void *q, const void *k, const void *
                                       int S, int D, int block, const int32_t *idx,
                                       const int32_t *cnt, int cap, int list_per_head,
                                       int group_size, float scale, void *stream);
+
+/* Block-sparse attention on T-major q, k, v and o, with each (b, head) in its
+ * own tiling and no permuted copies ("Adaptive tiling (SPADE)", Recipe: the
+ * permutation, attention and inverse permutation in one pass).  Block i of
+ * (b, head) is positions [128 i, 128 i + 128) of the head's tile-contiguous
+ * order under tiles[choice[bh]]; idx/cnt list blocks in that numbering, as
+ * vsa_topk_block_mask writes them.  The result equals vsa_permute of q, k and
+ * v, vsa_block_sparse_attention with block 128 and group_size 0, then
+ * vsa_unpermute of o, bit for bit.
+ *   q, k, v  [B, n_heads, S, D] bf16, o [B, n_heads, S, D] in out_dtype, T-major
+ *   tiles    every candidate of the same volume V, a multiple of 128, with
+ *            tile.t divisible by V/128 (a 128-token block is tile.t*128/V
+ *            whole (h, w) planes of the tile)
+ *   choice   [B, n_heads] int32 or NULL (tile 0 for every head)
+ * Lists are checked as for vsa_block_sparse_attention; a choice outside
+ * [0, n_tiles) leaves the head unwritten and sets VSA_ERR_RUNTIME.         */
+vsa_status vsa_block_sparse_attention_tiled(const void *q, const void *k, const void *v,
+                                            void *o, vsa_dtype out_dtype, int B,
+                                            int n_heads, int S, int D, vsa_dims3 grid,
+                                            const vsa_dims3 *tiles, int n_tiles,
+                                            const int32_t *choice, const int32_t *idx,
+                                            const int32_t *cnt, int cap, int list_per_head,
+                                            float scale, void *stream);
 
 /* ------------------------------------------------------------------------ */
 /* Symmetric sliding-window attention with global sinks.

@@ -95,6 +95,36 @@ def test_block_summaries_bit_exact(dtype, D, block):
         assert np.array_equal(_np(mn.view(4, -1, D)[bh]), omn)
 
 
+@pytest.mark.parametrize("dtype,D,block", [(torch.bfloat16, 128, 128), (torch.float32, 64, 32),
+                                           (torch.bfloat16, 64, 256), (torch.float32, 128, 16)])
+def test_block_summaries_tiled_matches_oracle_and_permuted_path(dtype, D, block):
+    """Summaries read from T-major x through each head's tiling equal those of
+    the permuted copy, bit for bit, and the oracle's."""
+    grid, tiles = (4, 8, 16), [(1, 8, 16), (2, 8, 8), (4, 4, 8)]
+    S = 512
+    x = torch.randn(2, 3, S, D, generator=torch.Generator(DEV).manual_seed(71), device=DEV).to(dtype)
+    choice = torch.tensor([2, 0, 1, 1, 2, 0], dtype=torch.int32, device=DEV)
+    mx, mn = vsa.block_summaries_tiled(x, grid, tiles, choice, block)
+    wmx, wmn = vsa.block_summaries(vsa.permute(x, grid, tiles, choice), block)
+    assert torch.equal(mx, wmx) and torch.equal(mn, wmn)
+    for bh, c in enumerate(choice.tolist()):
+        xp = oracle.permute_rows(_np(x.view(6, S, D)[bh]), oracle.tile_permutation(grid, tiles[c]))
+        omx, omn = oracle.block_minmax(xp, block)
+        assert np.array_equal(_np(mx.view(6, -1, D)[bh]), omx)
+        assert np.array_equal(_np(mn.view(6, -1, D)[bh]), omn)
+    # no choice: tile 0 for every head
+    mx0, _ = vsa.block_summaries_tiled(x, grid, tiles, None, block)
+    assert torch.equal(mx0, vsa.block_summaries(vsa.permute(x, grid, tiles[:1]), block)[0])
+
+
+def test_block_summaries_tiled_bad_choice_sets_runtime_status():
+    grid, tiles = (2, 8, 8), [(1, 8, 8), (2, 4, 4)]
+    x = integer_grid((1, 2, 128, 64), 72, torch.bfloat16, DEV)
+    vsa.block_summaries_tiled(x, grid, tiles, torch.tensor([1, -1], dtype=torch.int32, device=DEV), 64)
+    with pytest.raises(RuntimeError):
+        vsa.device_status()
+
+
 @pytest.mark.parametrize("dtype,D,nb", [(torch.bfloat16, 128, 40), (torch.float32, 64, 70), (torch.bfloat16, 64, 1),
                                         (torch.bfloat16, 128, 300), (torch.bfloat16, 64, 129)])
 def test_block_scores_exact_on_integer_grid(dtype, D, nb):
@@ -218,6 +248,61 @@ def test_block_sparse_attention_random_lists(D, block, values):
         assert_attn_close(_np(o[0, h]), want, f"head {h}")
 
 
+@pytest.mark.parametrize("D,grid,tiles,values", [
+    (128, (4, 8, 16), [(1, 8, 16), (2, 8, 8), (4, 4, 8)], "smooth"),   # volume 128: one block per tile
+    (64, (4, 8, 16), [(2, 8, 16), (4, 8, 8)], "integer"),               # volume 256: two blocks per tile
+    (128, (8, 8, 8), [(4, 8, 8), (8, 4, 8)], "smooth"),                 # volume 256, every tile.t even
+])
+def test_block_sparse_attention_tiled_matches_oracle_and_permuted_path(D, grid, tiles, values):
+    """T-major attention through each head's tiling (TMA boxes in, token rows
+    out) equals permute -> attention -> unpermute bit for bit, and the oracle."""
+    B, H = 2, 2
+    S = grid[0] * grid[1] * grid[2]
+    nb = S // 128
+    if values == "integer":
+        q, k, v = (integer_grid((B, H, S, D), 73 + i, torch.bfloat16, DEV) for i in range(3))
+    else:
+        q, k, v = smooth_qkv(B, H, grid, D, seed=74, device=DEV)
+    choice = torch.tensor([(i * 5 + 1) % len(tiles) for i in range(B * H)], dtype=torch.int32, device=DEV)
+    idx, cnt = _random_lists(nb, min(nb, 3), B * H, seed=D + nb)
+    ti = torch.as_tensor(idx, device=DEV).view(B, H, nb, -1)
+    tc = torch.as_tensor(cnt, device=DEV).view(B, H, nb)
+    o = vsa.block_sparse_attention_tiled(q, k, v, grid, tiles, choice, ti, tc, out_dtype=torch.float32)
+    ob = vsa.block_sparse_attention_tiled(q, k, v, grid, tiles, choice, ti, tc, out_dtype=torch.bfloat16)
+    assert torch.equal(ob, o.to(torch.bfloat16))
+    qp, kp, vp = (vsa.permute(x, grid, tiles, choice) for x in (q, k, v))
+    op = vsa.block_sparse_attention(qp, kp, vp, ti, tc, 128, out_dtype=torch.float32)
+    assert torch.equal(o, vsa.unpermute(op, grid, tiles, choice))
+    for bh, c in enumerate(choice.tolist()):
+        b, h = divmod(bh, H)
+        perm = oracle.tile_permutation(grid, tiles[c])
+        qo, ko, vo = (oracle.permute_rows(_np(x[b, h]), perm) for x in (q, k, v))
+        want = oracle.block_sparse_attention(qo, ko, vo, idx[bh], cnt[bh], 128)
+        assert_attn_close(_np(o[b, h])[perm], want, f"b{b} h{h}")
+
+
+def test_block_sparse_attention_tiled_bad_choice_and_lists():
+    grid, tiles = (2, 8, 16), [(1, 8, 16), (2, 8, 8)]
+    q, k, v = (integer_grid((1, 2, 256, 64), 75 + i, torch.bfloat16, DEV) for i in range(3))
+    idx = torch.tensor([[0, 1], [0, 1], [1, 0], [0, 1]], dtype=torch.int32, device=DEV).view(1, 2, 2, 2)
+    cnt = torch.full((1, 2, 2), 2, dtype=torch.int32, device=DEV)
+    o = vsa.block_sparse_attention_tiled(q, k, v, grid, tiles, torch.tensor([0, 1], dtype=torch.int32, device=DEV),
+                                         idx, cnt, out_dtype=torch.float32)
+    with pytest.raises(RuntimeError):   # head 1's first list is descending
+        vsa.device_status()
+    perm1 = torch.as_tensor(oracle.tile_permutation(grid, tiles[1]), device=DEV)
+    assert (o[0, 1][perm1[:128]] == 0).all()
+    o2 = vsa.block_sparse_attention_tiled(q, k, v, grid, tiles, torch.tensor([0, 2], dtype=torch.int32, device=DEV),
+                                          idx[:, :1].expand(1, 2, 2, 2).contiguous(), cnt, out_dtype=torch.float32)
+    with pytest.raises(RuntimeError):   # choice 2 is out of range
+        vsa.device_status()
+    assert torch.isfinite(o2[0, 0]).all()
+    with pytest.raises(ValueError):     # mixed volumes
+        vsa.block_sparse_attention_tiled(q, k, v, grid, [(1, 8, 16), (1, 8, 8)], None, idx, cnt)
+    with pytest.raises(ValueError):     # volume 256 with tile.t = 1: a block is not whole planes
+        vsa.block_sparse_attention_tiled(q, k, v, (1, 16, 16), [(1, 16, 16)], None, idx, cnt)
+
+
 def test_block_sparse_attention_group_mask_and_shared_list():
     """temporal_only: tile (T,1,1) with T=8 inside blocks of 32 -> group mask."""
     grid, block = (8, 8, 8), 32
@@ -316,6 +401,9 @@ def test_spade_fixed_full_size_sampled():
     # the unpermuted output is the permuted one scattered back
     perm = torch.as_tensor(oracle.tile_permutation(w.grid, w.tiles[0]), device=DEV)
     assert torch.equal(o[0, 5][perm], mid["out_perm"][0, 5])
+    # tiled (in-kernel permutation) and explicit permute paths agree bit for bit
+    assert torch.equal(o, vsa.spade_attention(q, k, v, w.grid, list(w.tiles), topk=w.k, out_dtype=torch.float32,
+                                              tiled=False))
 
 
 def test_spade_adaptive_full_size_sampled():
@@ -336,6 +424,9 @@ def test_spade_adaptive_full_size_sampled():
             assert choice[h] == oc, (h, osc)
         picked.add(int(choice[h]))
     assert len(picked) >= 2   # the heads do not all pick one tiling
+    # tiled (in-kernel permutation) and explicit permute paths agree bit for bit
+    assert torch.equal(o, vsa.spade_attention(q, k, v, w.grid, list(w.tiles), topk=w.k, out_dtype=torch.float32,
+                                              tiled=False))
     for h in (0, 13):
         tile = w.tiles[int(choice[h])]
         blocks = _sample_blocks(w.nb, 100 + h)
