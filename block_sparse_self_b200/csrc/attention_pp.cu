@@ -48,12 +48,17 @@ struct PPArgs {
     int H, W;
     TileSet tiles;
     const int32_t *choice;
+    struct BoxGeom {
+        FastDiv m, nthw, ntw;  // m = volume / 128, tiles per frame, tiles per tile row
+        int bt;                // frames of one 128-token box: tile.t / m
+    } geom[kMaxTiles];
 };
 
 // Tensor maps: slot 0 only, or one per candidate tiling in tiled mode.
 struct MapSet {
     CUtensorMap q[kMaxTiles], k[kMaxTiles], v[kMaxTiles];
 };
+static_assert(sizeof(MapSet) + sizeof(PPArgs) <= 4096, "kernel parameters");
 
 // In tiled mode, block b of a head whose tiling is (tt, th, tw) is the
 // 128-token box (tt/m, th, tw) at part b % m of tile b / m (m = volume/128):
@@ -61,13 +66,12 @@ struct MapSet {
 struct BoxCoord {
     int w, h, t;
 };
-__device__ __forceinline__ BoxCoord box_of(int b, int H, int W, int tt, int th, int tw) {
-    const int m = (tt * th * tw) / 128;
-    const int tile = b / m, part = b - tile * m;
-    const int nth = H / th, ntw = W / tw;
-    const int ct = tile / (nth * ntw), rem = tile - ct * (nth * ntw);
-    const int ch = rem / ntw, cw = rem - ch * ntw;
-    return BoxCoord{cw * tw, ch * th, ct * tt + part * (tt / m)};
+__device__ __forceinline__ BoxCoord box_of(uint32_t b, const PPArgs::BoxGeom &g, int th, int tw) {
+    const uint32_t tile = fdiv(b, g.m), part = b - tile * g.m.d;
+    const uint32_t ct = fdiv(tile, g.nthw), rem = tile - ct * g.nthw.d;
+    const uint32_t ch = fdiv(rem, g.ntw), cw = rem - ch * g.ntw.d;
+    return BoxCoord{static_cast<int>(cw) * tw, static_cast<int>(ch) * th,
+                    static_cast<int>(ct * g.m.d + part) * g.bt};
 }
 
 template <int D>
@@ -78,7 +82,7 @@ struct PPCfg {
     static constexpr int NK = D == 128 ? 3 : 4;    // K ring depth
     static constexpr int NV = D == 128 ? 2 : 4;    // V ring depth
     static constexpr int O_COL = 256;              // O_A at 256, O_B at 256 + D
-    static constexpr int N_BARS = 1 + 2 * NK + 2 * NV + 2 + 2 + 2 + 1;
+    static constexpr int N_BARS = 1 + 2 * NK + 2 * NV + 2 + 2 + 2 + 1 + 8;
     static constexpr int SMEM = 1024 + (2 + NK + NV) * TILE_BYTES + N_BARS * 8 + 64;
     static_assert(SMEM <= 232448, "shared memory");
 };
@@ -157,7 +161,8 @@ attn_pp_kernel(const __grid_constant__ MapSet maps, const PPArgs a) {
     uint64_t *p_full = s_full + 2;        // [2]
     uint64_t *pv_done = p_full + 2;       // [2]
     uint64_t *mma_done = pv_done + 2;
-    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(mma_done + 1);
+    uint64_t *turn = mma_done + 1;        // [2][4]: turn[4 t + q] is waited on by tile t's warp q
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(turn + 8);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
     int *list_ok = reinterpret_cast<int *>(tmem_slot + 2);  // [2]
 
@@ -182,8 +187,8 @@ attn_pp_kernel(const __grid_constant__ MapSet maps, const PPArgs a) {
             mbar_init(&pv_done[t], 1);
         }
         mbar_init(mma_done, 1);
+        for (int i = 0; i < 8; ++i) mbar_init(&turn[i], 1);
         *abort_flag = 0;
-        list_ok[0] = list_ok[1] = 1;
         fence_mbar_init();
     }
     if constexpr (!WINDOW) {
@@ -198,7 +203,9 @@ attn_pp_kernel(const __grid_constant__ MapSet maps, const PPArgs a) {
                     }
                 }
                 ok = __all_sync(0xffffffffu, ok);
-                if (lane == 0 && !ok) list_ok[warp] = 0;
+                // written only here (read after the barrier below): an initial
+                // value set by another thread could land after this store
+                if (lane == 0) list_ok[warp] = ok ? 1 : 0;
             }
         }
     }
@@ -236,7 +243,7 @@ attn_pp_kernel(const __grid_constant__ MapSet maps, const PPArgs a) {
     // one 128-row tile of Q, K or V: block b of this head
     auto load_tile = [&](uint8_t *dst, const CUtensorMap *map, uint64_t *bar, int b) {
         if constexpr (TILED) {
-            const BoxCoord c = box_of(b, a.H, a.W, tt, th, tw);
+            const BoxCoord c = box_of(static_cast<uint32_t>(b), a.geom[tc], th, tw);
             for (int s = 0; s < C::KSLABS; ++s) tma_load_5d(dst + s * C::SLAB, map, bar, s * 64, c.w, c.h, c.t, bh);
         } else {
             for (int s = 0; s < C::KSLABS; ++s) tma_load_3d(dst + s * C::SLAB, map, bar, s * 64, b * BN, bh);
@@ -367,6 +374,8 @@ attn_pp_kernel(const __grid_constant__ MapSet maps, const PPArgs a) {
         const int q0 = (sc.qt < 0 ? 0 : sc.qt) * BN;
         const int rg = q0 + row;
         const bool row_valid = sc.qt >= 0 && rg < S;
+        // output row: the permuted position itself, or its T-major token in tiled mode
+        const uint32_t orow_in_head = TILED ? tile_token(rg, a.H, a.W, tt, th, tw) : rg;
         const uint32_t t_lane = tmem + (static_cast<uint32_t>(wq * 32) << 16);
         const uint32_t s_col = t * 128, o_col = C::O_COL + t * D;
         const float sl2 = a.scale_log2;
@@ -432,6 +441,18 @@ attn_pp_kernel(const __grid_constant__ MapSet maps, const PPArgs a) {
             };
             // first visible keys of this row: take the block max before the exponentials
             if (m_ref == -INFINITY) m_ref = raw_max() * sl2;  // may stay -inf
+            // The two tiles' warps on one SM sub-partition share its exponential
+            // unit, so they take turns at their exponential passes: tile 0 takes
+            // block 0 first, then each hands the turn to the other while its own
+            // MMAs run.  Without this the two tiles fall into step, exponentiate
+            // together at half rate and then both wait for the tensor core.
+            const int n_other = ts[t ^ 1].n;
+            const bool wait_turn = t == 0 ? (j >= 1 && j - 1 < n_other) : (j < n_other);
+            if (wait_turn &&
+                !__all_sync(0xffffffffu, mbar_wait(&turn[4 * t + wq], (t == 0 ? j - 1 : j) & 1, abort_flag))) {
+                ok = false;
+                break;
+            }
             // The running max is lazy: every P is at most the row sum, so a sum
             // above kMaxRowSum (or inf) means the row's max grew; then O and l are
             // rescaled and the block is redone from S, still intact in TMEM.
@@ -469,6 +490,9 @@ attn_pp_kernel(const __grid_constant__ MapSet maps, const PPArgs a) {
                 if (!__all_sync(0xffffffffu, ok)) break;
                 m_ref = m_new;
             }
+            const bool hand_over = t == 0 ? (j < n_other) : (j + 1 < n_other);
+            __syncwarp();
+            if (hand_over && lane == 0) mbar_arrive(&turn[4 * (t ^ 1) + wq]);
             if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
             l_sum += rs;
             // P over the first 64 columns of this tile's S
@@ -482,8 +506,7 @@ attn_pp_kernel(const __grid_constant__ MapSet maps, const PPArgs a) {
         if (!ok && !*abort_flag) { report(a.status, DEV_TIMEOUT); *abort_flag = 1; }
 
         // ---- epilogue: O / l -> global ----
-        // output row: the permuted position itself, or its T-major token in tiled mode
-        const size_t orow = static_cast<size_t>(bh) * S + (TILED ? tile_token(rg, a.H, a.W, tt, th, tw) : rg);
+        const size_t orow = static_cast<size_t>(bh) * S + orow_in_head;
         bool have_o = ok && n > 0;
         if (have_o && !mbar_wait(&pv_done[t], (n - 1) & 1, abort_flag)) {
             have_o = false;
@@ -579,6 +602,20 @@ vsa_status run_pp(const AttnLaunch &L, int *status, cudaStream_t st) {
     a.tiles = L.tiles;
     a.choice = L.choice;
     if (!TILED) a.tiles.n = 1;
+    for (int c = 0; c < kMaxTiles; ++c) {
+        auto &g = a.geom[c];
+        if (TILED && c < L.tiles.n) {
+            const int tt = L.tiles.t[c], th = L.tiles.h[c], tw = L.tiles.w[c];
+            const int m = tt * th * tw / 128;
+            g.m = make_fastdiv(m);
+            g.nthw = make_fastdiv((L.Hg / th) * (L.Wg / tw));
+            g.ntw = make_fastdiv(L.Wg / tw);
+            g.bt = tt / m;
+        } else {
+            g.m = g.nthw = g.ntw = make_fastdiv(1);
+            g.bt = 1;
+        }
+    }
     dim3 grid((a.nq + 1) / 2, L.BH);
     kern<<<grid, kThreads, C::SMEM, st>>>(maps, a);
     return check_cuda(cudaGetLastError(), "attention launch (two tiles)");

@@ -119,6 +119,29 @@ __device__ __forceinline__ void tma_load_5d(void *dst, const CUtensorMap *map, u
 }
 
 // ---------------------------------------------------------------------------
+// Division by a divisor fixed before the launch, as a multiply-high, an add
+// and a shift (Granlund and Montgomery, "Division by invariant integers using
+// multiplication", 1994): with l = ceil(log2 d) and
+// mul = floor(2^32 (2^l - d) / d) + 1, n / d = (umulhi(mul, n) + n) >> l for
+// every 32-bit n (the sum is taken in 64 bits).  Runtime divisions otherwise
+// go through the reciprocal unit, which the softmax keeps busy.
+// ---------------------------------------------------------------------------
+struct FastDiv {
+    uint32_t d, mul, shift;
+};
+
+inline FastDiv make_fastdiv(uint32_t d) {
+    uint32_t l = 0;
+    while ((uint64_t{1} << l) < d) ++l;
+    const uint64_t mul = ((uint64_t{1} << 32) * ((uint64_t{1} << l) - d)) / d + 1;
+    return FastDiv{d, static_cast<uint32_t>(mul), l};
+}
+
+__device__ __forceinline__ uint32_t fdiv(uint32_t n, const FastDiv &f) {
+    return static_cast<uint32_t>((static_cast<uint64_t>(__umulhi(f.mul, n)) + n) >> f.shift);
+}
+
+// ---------------------------------------------------------------------------
 // Tile-contiguous order ("ADR-0001", step 6; "Adaptive tiling (SPADE)",
 // Recipe): position p holds the T-major token tile_token(p).  Tiles come in
 // row-major tile order, the tokens of a tile in T-major order.

@@ -63,7 +63,7 @@ __global__ void __launch_bounds__(kThreads) sics_partial_kernel(const SelArgs a)
         #pragma unroll
         for (int e = 0; e < EPL; ++e) acc[e] = 0.f;
         float m = 0.f;
-        #pragma unroll 2
+        #pragma unroll 8
         for (int tok0 = 0; tok0 < cvol; tok0 += TPI) {  // uniform trip count: shuffles below
             const int tok = tok0 + lane / LPT;
             const bool valid = tok < cvol;

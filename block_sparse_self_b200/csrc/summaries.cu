@@ -78,21 +78,20 @@ __global__ void __launch_bounds__(kThreads) summaries_kernel(const uint8_t *__re
     const int blk = blockIdx.x, bh = blockIdx.y;
     const int chunk = threadIdx.x % CPR, rg = threadIdx.x / CPR;
     const size_t head = static_cast<size_t>(bh) * S;
-    int tt = 1, th = 1, tw = 1;
+    __shared__ int row_tok[256];  // tiled mode: T-major token of each of the block's rows
     if constexpr (TILED) {
         const int c = ta.choice ? __ldg(ta.choice + bh) : 0;
-        if (c < 0 || c >= ta.tiles.n) {  // the head's summaries are left unwritten
+        if (c < 0 || c >= ta.tiles.n) {  // the head's summaries are left unwritten (uniform over the CTA)
             if (threadIdx.x == 0) report(ta.status, DEV_RUNTIME);
             return;
         }
-        tt = ta.tiles.t[c];
-        th = ta.tiles.h[c];
-        tw = ta.tiles.w[c];
+        for (int r = threadIdx.x; r < block; r += kThreads)
+            row_tok[r] = tile_token(blk * block + r, ta.H, ta.W, ta.tiles.t[c], ta.tiles.h[c], ta.tiles.w[c]);
+        __syncthreads();
     }
     // byte address of chunk `chunk` of the block's r-th row
     auto row_ptr = [&](int r) -> const uint8_t * {
-        const int p = blk * block + r;
-        const int tok = TILED ? tile_token(p, ta.H, ta.W, tt, th, tw) : p;
+        const int tok = TILED ? row_tok[r] : blk * block + r;
         return x + (head + tok) * CPR * 16 + chunk * 16;
     };
     Vec<T> mx, mn;
