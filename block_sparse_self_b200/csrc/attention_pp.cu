@@ -82,7 +82,7 @@ struct PPCfg {
     static constexpr int NK = D == 128 ? 3 : 4;    // K ring depth
     static constexpr int NV = D == 128 ? 2 : 4;    // V ring depth
     static constexpr int O_COL = 256;              // O_A at 256, O_B at 256 + D
-    static constexpr int N_BARS = 1 + 2 * NK + 2 * NV + 2 + 2 + 2 + 1 + 8;
+    static constexpr int N_BARS = 1 + 2 * NK + 2 * NV + 2 + 2 + 2 + 1;
     static constexpr int SMEM = 1024 + (2 + NK + NV) * TILE_BYTES + N_BARS * 8 + 64;
     static_assert(SMEM <= 232448, "shared memory");
 };
@@ -161,8 +161,7 @@ attn_pp_kernel(const __grid_constant__ MapSet maps, const PPArgs a) {
     uint64_t *p_full = s_full + 2;        // [2]
     uint64_t *pv_done = p_full + 2;       // [2]
     uint64_t *mma_done = pv_done + 2;
-    uint64_t *turn = mma_done + 1;        // [2][4]: turn[4 t + q] is waited on by tile t's warp q
-    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(turn + 8);
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(mma_done + 1);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
     int *list_ok = reinterpret_cast<int *>(tmem_slot + 2);  // [2]
 
@@ -187,7 +186,6 @@ attn_pp_kernel(const __grid_constant__ MapSet maps, const PPArgs a) {
             mbar_init(&pv_done[t], 1);
         }
         mbar_init(mma_done, 1);
-        for (int i = 0; i < 8; ++i) mbar_init(&turn[i], 1);
         *abort_flag = 0;
         fence_mbar_init();
     }
@@ -382,7 +380,7 @@ attn_pp_kernel(const __grid_constant__ MapSet maps, const PPArgs a) {
         float m_ref = -INFINITY, l_sum = 0.f;
         bool ok = true;
         for (int j = 0; j < n; ++j) {
-            if (!mbar_wait(&s_full[t], j & 1, abort_flag)) { ok = false; break; }
+            if (!__all_sync(0xffffffffu, mbar_wait(&s_full[t], j & 1, abort_flag))) { ok = false; break; }
             tc_fence_after();
             uint32_t x[BN];
             #pragma unroll
@@ -441,18 +439,6 @@ attn_pp_kernel(const __grid_constant__ MapSet maps, const PPArgs a) {
             };
             // first visible keys of this row: take the block max before the exponentials
             if (m_ref == -INFINITY) m_ref = raw_max() * sl2;  // may stay -inf
-            // The two tiles' warps on one SM sub-partition share its exponential
-            // unit, so they take turns at their exponential passes: tile 0 takes
-            // block 0 first, then each hands the turn to the other while its own
-            // MMAs run.  Without this the two tiles fall into step, exponentiate
-            // together at half rate and then both wait for the tensor core.
-            const int n_other = ts[t ^ 1].n;
-            const bool wait_turn = t == 0 ? (j >= 1 && j - 1 < n_other) : (j < n_other);
-            if (wait_turn &&
-                !__all_sync(0xffffffffu, mbar_wait(&turn[4 * t + wq], (t == 0 ? j - 1 : j) & 1, abort_flag))) {
-                ok = false;
-                break;
-            }
             // The running max is lazy: every P is at most the row sum, so a sum
             // above kMaxRowSum (or inf) means the row's max grew; then O and l are
             // rescaled and the block is redone from S, still intact in TMEM.
@@ -469,7 +455,7 @@ attn_pp_kernel(const __grid_constant__ MapSet maps, const PPArgs a) {
                 apply_mask();
                 const float m_new = need ? fmaxf(m_ref, raw_max() * sl2) : m_ref;
                 if (j > 0) {
-                    if (!mbar_wait(&pv_done[t], (j - 1) & 1, abort_flag)) {
+                    if (!__all_sync(0xffffffffu, mbar_wait(&pv_done[t], (j - 1) & 1, abort_flag))) {
                         ok = false;
                     } else {
                         tc_fence_after();
@@ -490,9 +476,6 @@ attn_pp_kernel(const __grid_constant__ MapSet maps, const PPArgs a) {
                 if (!__all_sync(0xffffffffu, ok)) break;
                 m_ref = m_new;
             }
-            const bool hand_over = t == 0 ? (j < n_other) : (j + 1 < n_other);
-            __syncwarp();
-            if (hand_over && lane == 0) mbar_arrive(&turn[4 * (t ^ 1) + wq]);
             if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
             l_sum += rs;
             // P over the first 64 columns of this tile's S
@@ -508,7 +491,7 @@ attn_pp_kernel(const __grid_constant__ MapSet maps, const PPArgs a) {
         // ---- epilogue: O / l -> global ----
         const size_t orow = static_cast<size_t>(bh) * S + orow_in_head;
         bool have_o = ok && n > 0;
-        if (have_o && !mbar_wait(&pv_done[t], (n - 1) & 1, abort_flag)) {
+        if (have_o && !__all_sync(0xffffffffu, mbar_wait(&pv_done[t], (n - 1) & 1, abort_flag))) {
             have_o = false;
             if (!*abort_flag) { report(a.status, DEV_TIMEOUT); *abort_flag = 1; }
         }
