@@ -159,6 +159,36 @@ __device__ __forceinline__ int tile_token(int p, int H, int W, int tt, int th, i
     return ((ct * tt + dt) * H + ch * th + dh) * W + cw * tw + dw;
 }
 
+// tile_token with every division by a per-tiling constant done as a
+// multiply-shift (FastDiv); the divisors come from make_tile_divs on the host.
+struct TileDivs {
+    FastDiv vol, nthw, ntw, thw, tw;  // tile volume, tiles per frame, tiles per tile row, th*tw, tw
+    int tt, th, H, W;
+};
+
+inline TileDivs make_tile_divs(int H, int W, int tt, int th, int tw) {
+    TileDivs d;
+    d.vol = make_fastdiv(static_cast<uint32_t>(tt * th * tw));
+    d.nthw = make_fastdiv(static_cast<uint32_t>((H / th) * (W / tw)));
+    d.ntw = make_fastdiv(static_cast<uint32_t>(W / tw));
+    d.thw = make_fastdiv(static_cast<uint32_t>(th * tw));
+    d.tw = make_fastdiv(static_cast<uint32_t>(tw));
+    d.tt = tt;
+    d.th = th;
+    d.H = H;
+    d.W = W;
+    return d;
+}
+
+__device__ __forceinline__ uint32_t tile_token_fast(uint32_t p, const TileDivs &d) {
+    const uint32_t tile = fdiv(p, d.vol), r = p - tile * d.vol.d;
+    const uint32_t ct = fdiv(tile, d.nthw), rem = tile - ct * d.nthw.d;
+    const uint32_t ch = fdiv(rem, d.ntw), cw = rem - ch * d.ntw.d;
+    const uint32_t dt = fdiv(r, d.thw), r2 = r - dt * d.thw.d;
+    const uint32_t dh = fdiv(r2, d.tw), dw = r2 - dh * d.tw.d;
+    return ((ct * d.tt + dt) * d.H + ch * d.th + dh) * d.W + cw * d.tw.d + dw;
+}
+
 // ---------------------------------------------------------------------------
 // tcgen05: tensor memory allocation, MMA, commit, loads and stores
 // ---------------------------------------------------------------------------

@@ -20,6 +20,7 @@ struct PermArgs {
     uint8_t *dst;
     int S, T, H, W, BH;
     TileSet tiles;
+    TileDivs divs[kMaxTiles];  // per candidate tiling
     const int32_t *choice;
     int inverse;
     int *status;
@@ -49,7 +50,7 @@ __global__ void __launch_bounds__(kThreads) permute_kernel(const PermArgs a) {
                 continue;
             }
         }
-        const int tt = a.tiles.t[c], th = a.tiles.h[c], tw = a.tiles.w[c];
+        const TileDivs dv = a.divs[c];
         const size_t head = static_cast<size_t>(bh) * a.S;
         const uint4 *src = reinterpret_cast<const uint4 *>(a.src);
         uint4 *dst = reinterpret_cast<uint4 *>(a.dst);
@@ -63,7 +64,7 @@ __global__ void __launch_bounds__(kThreads) permute_kernel(const PermArgs a) {
                 const int p = p0 + r0 + u * RPP + rsub;
                 ok[u] = (r0 + u * RPP + rsub) < kRowsPerItem && p < a.S;
                 if (ok[u]) {
-                    const int tok = tile_token(p, a.H, a.W, tt, th, tw);
+                    const int tok = static_cast<int>(tile_token_fast(static_cast<uint32_t>(p), dv));
                     const size_t srow = head + (a.inverse ? p : tok);
                     drow[u] = head + (a.inverse ? tok : p);
                     v[u] = __ldcs(src + srow * CPR + chunk);
@@ -117,6 +118,8 @@ cudaError_t launch_permute(const void *src, void *dst, int esize, int BH, int S,
     a.dst = static_cast<uint8_t *>(dst);
     a.S = S; a.T = T; a.H = H; a.W = W; a.BH = BH;
     a.tiles = tiles;
+    for (int c = 0; c < kMaxTiles; ++c)
+        a.divs[c] = c < tiles.n ? make_tile_divs(H, W, tiles.t[c], tiles.h[c], tiles.w[c]) : make_tile_divs(1, 1, 1, 1, 1);
     a.choice = choice;
     a.inverse = inverse ? 1 : 0;
     a.status = status;

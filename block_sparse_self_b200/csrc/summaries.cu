@@ -62,8 +62,8 @@ struct Vec<float> {
 };
 
 struct TiledArgs {
-    int H, W;
     TileSet tiles;
+    TileDivs divs[kMaxTiles];  // per candidate tiling
     const int32_t *choice;
     int *status;
 };
@@ -78,20 +78,38 @@ __global__ void __launch_bounds__(kThreads) summaries_kernel(const uint8_t *__re
     const int blk = blockIdx.x, bh = blockIdx.y;
     const int chunk = threadIdx.x % CPR, rg = threadIdx.x / CPR;
     const size_t head = static_cast<size_t>(bh) * S;
-    __shared__ int row_tok[256];  // tiled mode: T-major token of each of the block's rows
+    int c = 0;
+    uint32_t origin = 0, rr0 = 0;  // tiled mode, block within one tile: the tile's first token, block offset
+    bool one_tile = false;
     if constexpr (TILED) {
-        const int c = ta.choice ? __ldg(ta.choice + bh) : 0;
+        c = ta.choice ? __ldg(ta.choice + bh) : 0;
         if (c < 0 || c >= ta.tiles.n) {  // the head's summaries are left unwritten (uniform over the CTA)
             if (threadIdx.x == 0) report(ta.status, DEV_RUNTIME);
             return;
         }
-        for (int r = threadIdx.x; r < block; r += kThreads)
-            row_tok[r] = tile_token(blk * block + r, ta.H, ta.W, ta.tiles.t[c], ta.tiles.h[c], ta.tiles.w[c]);
-        __syncthreads();
+        const TileDivs &d = ta.divs[c];
+        const uint32_t p0 = static_cast<uint32_t>(blk * block);
+        one_tile = static_cast<uint32_t>(block) <= d.vol.d;  // then block divides the volume
+        if (one_tile) {
+            const uint32_t tile = fdiv(p0, d.vol);
+            rr0 = p0 - tile * d.vol.d;
+            origin = tile_token_fast(tile * d.vol.d, d);
+        }
     }
     // byte address of chunk `chunk` of the block's r-th row
     auto row_ptr = [&](int r) -> const uint8_t * {
-        const int tok = TILED ? row_tok[r] : blk * block + r;
+        uint32_t tok = static_cast<uint32_t>(blk * block + r);
+        if constexpr (TILED) {
+            const TileDivs &d = ta.divs[c];
+            if (one_tile) {
+                const uint32_t rr = rr0 + static_cast<uint32_t>(r);
+                const uint32_t dt = fdiv(rr, d.thw), r2 = rr - dt * d.thw.d;
+                const uint32_t dh = fdiv(r2, d.tw), dw = r2 - dh * d.tw.d;
+                tok = origin + (dt * d.H + dh) * d.W + dw;
+            } else {
+                tok = tile_token_fast(tok, d);
+            }
+        }
         return x + (head + tok) * CPR * 16 + chunk * 16;
     };
     Vec<T> mx, mn;
@@ -151,9 +169,9 @@ cudaError_t launch_summaries_tiled(const void *x, int esize, int BH, int S, int 
                                    cudaStream_t st, int block) {
     (void)T;
     TiledArgs ta;
-    ta.H = H;
-    ta.W = W;
     ta.tiles = tiles;
+    for (int c = 0; c < kMaxTiles; ++c)
+        ta.divs[c] = c < tiles.n ? make_tile_divs(H, W, tiles.t[c], tiles.h[c], tiles.w[c]) : make_tile_divs(1, 1, 1, 1, 1);
     ta.choice = choice;
     ta.status = status;
     return run_summaries<true>(x, esize, BH, S, D, block, xmax, xmin, ta, st);
