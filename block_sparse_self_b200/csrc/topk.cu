@@ -126,16 +126,10 @@ __global__ void __launch_bounds__(kWarps * 32) topk_kernel(const float *__restri
 // per-lane compare-and-add plus a warp sum.  No shared memory, no atomics.
 template <int NPL>
 __device__ __forceinline__ int count_ge(const uint32_t (&key)[NPL], uint32_t t) {
-    int c0 = 0, c1 = 0;
+    uint32_t c[4] = {0u, 0u, 0u, 0u};
     #pragma unroll
-    for (int i = 0; i < NPL; i += 2) {
-        c0 += key[i] >= t;
-        if (i + 1 < NPL) c1 += key[i + 1] >= t;
-    }
-    int c = c0 + c1;
-    #pragma unroll
-    for (int off = 16; off > 0; off >>= 1) c += __shfl_xor_sync(0xffffffffu, c, off);
-    return c;
+    for (int i = 0; i < NPL; ++i) c[i & 3] += key[i] >= t ? 1u : 0u;
+    return static_cast<int>(__reduce_add_sync(0xffffffffu, (c[0] + c[1]) + (c[2] + c[3])));
 }
 
 template <int NPL>
