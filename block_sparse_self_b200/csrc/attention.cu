@@ -304,10 +304,11 @@ attn_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUt
                 } else {
                     full = a.group <= 0;
                     if (!full) {
-                        const int gq = rg / a.group;
+                        // key ks + c is in the row's group iff it lies in [g0, g0 + group)
+                        const int g0 = (rg / a.group) * a.group - ks;
                         #pragma unroll
                         for (int c = 0; c < BN; ++c)
-                            if ((ks + c) / a.group != gq) x[c] = -INFINITY;
+                            if (c < g0 || c >= g0 + a.group) x[c] = -INFINITY;
                     }
                 }
                 float mb = -INFINITY;
@@ -497,6 +498,18 @@ bool make_tile_map(CUtensorMap *m, const void *ptr, int D, int S, int BH, int ro
                CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+
+bool make_scores_store_map(CUtensorMap *m, float *ptr, int nb, int BH) {
+    EncodeTiledFn enc = encode_fn();
+    if (!enc) return false;
+    cuuint64_t dims[3] = {static_cast<cuuint64_t>(nb), static_cast<cuuint64_t>(nb), static_cast<cuuint64_t>(BH)};
+    cuuint64_t strides[2] = {static_cast<cuuint64_t>(nb) * 4, static_cast<cuuint64_t>(nb) * nb * 4};
+    cuuint32_t box[3] = {32, 128, 1};
+    cuuint32_t estr[3] = {1, 1, 1};
+    return enc(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 3, ptr, dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+               CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_NONE,
+               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
 
 bool make_box_map(CUtensorMap *m, const void *ptr, int D, int T, int H, int W, int BH, int bt, int bh, int bw) {
     EncodeTiledFn enc = encode_fn();

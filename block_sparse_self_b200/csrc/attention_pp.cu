@@ -405,10 +405,11 @@ attn_pp_kernel(const __grid_constant__ MapSet maps, const PPArgs a) {
                 } else {
                     if (a.group > 0) {
                         const int ks = kblock_of<WINDOW>(sc, j) * BN;
-                        const int gq = rg / a.group;
+                        // key ks + c is in the row's group iff it lies in [g0, g0 + group)
+                        const int g0 = (rg / a.group) * a.group - ks;
                         #pragma unroll
                         for (int c = 0; c < BN; ++c)
-                            if ((ks + c) / a.group != gq) x[c] = __float_as_uint(-INFINITY);
+                            if (c < g0 || c >= g0 + a.group) x[c] = __float_as_uint(-INFINITY);
                     }
                 }
             };

@@ -83,6 +83,9 @@ bool make_tile_map(CUtensorMap *m, const void *ptr, int D, int S, int BH, int ro
 // (64, bw, bh, bt, 1), 128-byte swizzle: a (bt, bh, bw) token box lands as
 // rows of 128 bytes in (t, h, w) row-major order.
 bool make_box_map(CUtensorMap *m, const void *ptr, int D, int T, int H, int W, int BH, int bt, int bh, int bw);
+// [BH, nb, nb] fp32 scores as a 3-D tensor (nb, nb, BH), box (32, 128, 1), 128-byte swizzle, for TMA stores
+// (needs nb % 4 == 0 and a 16-byte aligned base).
+bool make_scores_store_map(CUtensorMap *m, float *ptr, int nb, int BH);
 
 cudaError_t launch_wait_timeout(uint64_t limit_ns, int *status, cudaStream_t st);
 
