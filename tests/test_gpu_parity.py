@@ -165,6 +165,33 @@ def test_topk_lists_bit_exact(nb, levels):
             assert np.array_equal(cnt.view(4, nb)[bh].cpu().numpy(), oc)
 
 
+@pytest.mark.parametrize("nb", [200, 960, 1000])
+@pytest.mark.parametrize("kind", ["negative", "narrow", "wide_ties", "spread"])
+def test_topk_threshold_search_paths(nb, kind):
+    """Score rows that drive the threshold search down each of its paths: all
+    negative (padded slots share the threshold's prefix), values within a few
+    ulps of each other (many keys share every prefix), exact ties wider than
+    the candidate buffer, and magnitudes spread over many octaves."""
+    g = torch.Generator(DEV).manual_seed(nb + len(kind))
+    x = torch.randn(2, 1, nb, nb, generator=g, device=DEV)
+    if kind == "negative":
+        sc = -x.abs() - 100.0
+    elif kind == "narrow":
+        sc = 1.0 + x * 1e-6
+    elif kind == "wide_ties":
+        sc = torch.where(x > -0.5, torch.full_like(x, 2.5), x)  # ~70% of each row ties at the top
+    else:
+        sc = torch.sign(x) * torch.exp2(x * 20.0)
+    sc = sc.contiguous()
+    for k, n_sink, dw in [(max(1, nb // 10), 1, 0), (max(1, nb // 3), 0, -1)]:
+        idx, cnt = vsa.topk_block_mask(sc, k, n_sink, dw)
+        for bh in range(2):
+            oi, oc = oracle.topk_block_list(_np(sc.view(2, nb, nb)[bh]).astype(np.float64), k, n_sink, dw,
+                                            cap=idx.shape[-1])
+            assert np.array_equal(idx.view(2, nb, -1)[bh].cpu().numpy(), oi), (kind, nb, k, bh)
+            assert np.array_equal(cnt.view(2, nb)[bh].cpu().numpy(), oc)
+
+
 # --------------------------------------------------------------------------
 # structured lists
 # --------------------------------------------------------------------------
