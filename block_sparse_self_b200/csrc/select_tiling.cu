@@ -36,8 +36,12 @@ struct SelArgs {
     TileSet tiles;
     int Rt, Rh, Rw, Ct, Ch, Cw;
     int nrt, nrh, nrw;  // regions per axis
-    int cells;
+    int cells, items;
     FastDiv cell_hw, cell_w;  // Ch * Cw and Cw: token of a cell -> (dt, dh, dw)
+    int nch, ncw;             // cells of a region along h and w
+    int tpr_t[kMaxTiles], tpr_h[kMaxTiles], tpr_w[kMaxTiles];  // candidate c: its tiles per region axis
+    int cpt_t[kMaxTiles], cpt_h[kMaxTiles], cpt_w[kMaxTiles];  // candidate c: cells per tile axis
+    int item_first[kMaxTiles + 1];                             // candidate c's first item in a region
     float *partial;     // [BH][n_regions][tiles.n]
 };
 
@@ -49,10 +53,12 @@ __global__ void __launch_bounds__(kThreads) sics_partial_kernel(const SelArgs a)
     constexpr int EPC = 16 / sizeof(T);  // elements per chunk
     constexpr int EPL = EPC * CPL;       // elements per lane
     constexpr int TPI = 32 / LPT;        // query rows per warp pass
+    constexpr int CPR = LPT * CPL;       // 16-byte chunks per query row
     extern __shared__ float sm[];
     float *cell_sum = sm;                               // [cells][D]
     float *cell_cnt = cell_sum + a.cells * a.D;         // [cells]
     float *tile_val = cell_cnt + a.cells;               // [items]
+    int *cell_off = reinterpret_cast<int *>(tile_val + a.items);  // [cvol]: token offset inside a cell
     const int region = blockIdx.x, bh = blockIdx.y;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int lt = lane % LPT;
@@ -61,6 +67,15 @@ __global__ void __launch_bounds__(kThreads) sics_partial_kernel(const SelArgs a)
     const int nch = a.Rh / a.Ch, ncw = a.Rw / a.Cw;
     const int cvol = a.Ct * a.Ch * a.Cw;
     const size_t head = static_cast<size_t>(bh) * a.S;
+    // every cell has the same shape: offsets of its tokens from its first one, once per CTA
+    for (int tk = threadIdx.x; tk < cvol; tk += kThreads) {
+        const int dt = static_cast<int>(fdiv(static_cast<uint32_t>(tk), a.cell_hw));
+        const int r2 = tk - dt * (a.Ch * a.Cw);
+        const int dh = static_cast<int>(fdiv(static_cast<uint32_t>(r2), a.cell_w)), dw = r2 - dh * a.Cw;
+        cell_off[tk] = (dt * a.H + dh) * a.W + dw;
+    }
+    __syncthreads();
+    const uint4 *q4 = reinterpret_cast<const uint4 *>(a.q);
 
     for (int cell = warp; cell < a.cells; cell += kWarps) {
         const int ct = cell / (nch * ncw), ch = (cell / ncw) % nch, cw = cell % ncw;
@@ -69,45 +84,52 @@ __global__ void __launch_bounds__(kThreads) sics_partial_kernel(const SelArgs a)
         #pragma unroll
         for (int e = 0; e < EPL; ++e) acc[e] = 0.f;
         float m = 0.f;
-        #pragma unroll 2
-        for (int tok0 = 0; tok0 < cvol; tok0 += TPI) {  // uniform trip count: shuffles below
-            const int tok = tok0 + lane / LPT;
-            const bool valid = tok < cvol;
-            const int dt = static_cast<int>(fdiv(static_cast<uint32_t>(tok), a.cell_hw));
-            const int r2 = tok - dt * (a.Ch * a.Cw);
-            const int dh = static_cast<int>(fdiv(static_cast<uint32_t>(r2), a.cell_w)), dw = r2 - dh * a.Cw;
-            const size_t token = static_cast<size_t>((tb + dt) * a.H + hb + dh) * a.W + wb + dw;
-            const uint4 *row = reinterpret_cast<const uint4 *>(a.q + ((head + token) * a.D) * sizeof(T));
-            uint4 raw[CPL];
+        // chunk lt of the cell's first token; each token adds cell_off * CPR chunks
+        const uint4 *cell_q = q4 + (head + static_cast<size_t>((tb * a.H + hb) * a.W + wb)) * CPR + lt;
+        // NB passes' loads are issued before any of them is used
+        constexpr int NB = sizeof(T) == 2 ? 4 : 2;
+        #pragma unroll 1
+        for (int tok_b = 0; tok_b < cvol; tok_b += NB * TPI) {  // uniform trip count: shuffles below
+            uint4 raw[NB][CPL];
             #pragma unroll
-            for (int u = 0; u < CPL; ++u) raw[u] = valid ? __ldcs(row + lt + LPT * u) : make_uint4(0u, 0u, 0u, 0u);
-            float x[EPL];
-            #pragma unroll
-            for (int u = 0; u < CPL; ++u) {
-                if constexpr (sizeof(T) == 2) {
-                    const __nv_bfloat162 *hv = reinterpret_cast<const __nv_bfloat162 *>(&raw[u]);
-                    #pragma unroll
-                    for (int e = 0; e < EPC / 2; ++e) {
-                        const float2 f = __bfloat1622float2(hv[e]);
-                        x[u * EPC + 2 * e] = f.x;
-                        x[u * EPC + 2 * e + 1] = f.y;
-                    }
-                } else {
-                    const float *fv = reinterpret_cast<const float *>(&raw[u]);
-                    #pragma unroll
-                    for (int e = 0; e < EPC; ++e) x[u * EPC + e] = fv[e];
-                }
-            }
-            float ss = 0.f;
-            #pragma unroll
-            for (int e = 0; e < EPL; ++e) ss = fmaf(x[e], x[e], ss);
-            #pragma unroll
-            for (int off = LPT / 2; off > 0; off >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, off);
-            if (ss > 0.f) {
-                const float inv = rsqrtf(ss);
+            for (int pb = 0; pb < NB; ++pb) {
+                const int tok = tok_b + pb * TPI + lane / LPT;
+                const bool valid = tok < cvol;
+                const uint4 *row = cell_q + static_cast<size_t>(cell_off[valid ? tok : 0]) * CPR;
                 #pragma unroll
-                for (int e = 0; e < EPL; ++e) acc[e] = fmaf(x[e], inv, acc[e]);
-                m += 1.f;
+                for (int u = 0; u < CPL; ++u)
+                    raw[pb][u] = valid ? __ldcs(row + LPT * u) : make_uint4(0u, 0u, 0u, 0u);
+            }
+            #pragma unroll
+            for (int pb = 0; pb < NB; ++pb) {
+                float x[EPL];
+                #pragma unroll
+                for (int u = 0; u < CPL; ++u) {
+                    if constexpr (sizeof(T) == 2) {
+                        // bf16 -> fp32 is the bf16 bits in the high half of the word
+                        const uint32_t w[4] = {raw[pb][u].x, raw[pb][u].y, raw[pb][u].z, raw[pb][u].w};
+                        #pragma unroll
+                        for (int e = 0; e < 4; ++e) {
+                            x[u * EPC + 2 * e] = __uint_as_float(w[e] << 16);
+                            x[u * EPC + 2 * e + 1] = __uint_as_float(w[e] & 0xffff0000u);
+                        }
+                    } else {
+                        const float *fv = reinterpret_cast<const float *>(&raw[pb][u]);
+                        #pragma unroll
+                        for (int e = 0; e < EPC; ++e) x[u * EPC + e] = fv[e];
+                    }
+                }
+                float ss = 0.f;
+                #pragma unroll
+                for (int e = 0; e < EPL; ++e) ss = fmaf(x[e], x[e], ss);
+                #pragma unroll
+                for (int off = LPT / 2; off > 0; off >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, off);
+                if (ss > 0.f) {
+                    const float inv = rsqrtf(ss);
+                    #pragma unroll
+                    for (int e = 0; e < EPL; ++e) acc[e] = fmaf(x[e], inv, acc[e]);
+                    m += 1.f;
+                }
             }
         }
         // add the rows of the warp's token slots (lanes with the same lt)
@@ -127,47 +149,49 @@ __global__ void __launch_bounds__(kThreads) sics_partial_kernel(const SelArgs a)
     }
     __syncthreads();
 
-    // candidate tiles inside this region: item -> (candidate c, tile index)
-    int items = 0;
-    for (int c = 0; c < a.tiles.n; ++c)
-        items += (a.Rt / a.tiles.t[c]) * (a.Rh / a.tiles.h[c]) * (a.Rw / a.tiles.w[c]);
-    for (int item = warp; item < items; item += kWarps) {
-        int c = 0, rem = item;
-        while (true) {
-            const int n = (a.Rt / a.tiles.t[c]) * (a.Rh / a.tiles.h[c]) * (a.Rw / a.tiles.w[c]);
-            if (rem < n) break;
-            rem -= n;
-            ++c;
-        }
-        const int tt = a.tiles.t[c], th = a.tiles.h[c], tw = a.tiles.w[c];
-        const int nth = a.Rh / th, ntw = a.Rw / tw;
-        const int at = rem / (nth * ntw), ah = (rem / ntw) % nth, aw = rem % ntw;
-        // cells of this tile, in cell coordinates
-        const int c0t = at * tt / a.Ct, c0h = ah * th / a.Ch, c0w = aw * tw / a.Cw;
-        const int kt = tt / a.Ct, kh = th / a.Ch, kw = tw / a.Cw;
-        float sq = 0.f, m = 0.f;
-        for (int d = lane; d < a.D; d += 32) {
-            float s = 0.f;
-            for (int x = 0; x < kt; ++x)
-                for (int y = 0; y < kh; ++y)
-                    for (int z = 0; z < kw; ++z)
-                        s += cell_sum[(((c0t + x) * nch + c0h + y) * ncw + c0w + z) * a.D + d];
-            sq = fmaf(s, s, sq);
-        }
-        for (int x = 0; x < kt; ++x)
-            for (int y = 0; y < kh; ++y)
-                for (int z = 0; z < kw; ++z) m += cell_cnt[((c0t + x) * nch + c0h + y) * ncw + c0w + z];
-        #pragma unroll
-        for (int off = 16; off > 0; off >>= 1) sq += __shfl_down_sync(0xffffffffu, sq, off);
-        if (lane == 0) tile_val[item] = m >= 2.f ? (sq - m) / (m * (m - 1.f)) : 0.f;
+    // candidate tiles inside this region, candidate by candidate (the same
+    // item layout in every region, precomputed on the host): sum the tile's
+    // cells, four channels per lane, and turn |sum|^2 into the tile's SICS
+    int item = 0;
+    for (int c = 0; c < a.tiles.n; ++c) {
+        const int kt = a.cpt_t[c], kh = a.cpt_h[c], kw = a.cpt_w[c];
+        for (int at = 0; at < a.tpr_t[c]; ++at)
+            for (int ah = 0; ah < a.tpr_h[c]; ++ah)
+                for (int aw = 0; aw < a.tpr_w[c]; ++aw, ++item) {
+                    if (item % kWarps != warp) continue;  // warp-uniform
+                    float sq = 0.f, m = 0.f;
+                    for (int d4 = lane; d4 < a.D / 4; d4 += 32) {
+                        float4 sum = make_float4(0.f, 0.f, 0.f, 0.f);
+                        for (int x = 0; x < kt; ++x)
+                            for (int y = 0; y < kh; ++y) {
+                                const int row = ((at * kt + x) * a.nch + ah * kh + y) * a.ncw + aw * kw;
+                                for (int z = 0; z < kw; ++z) {
+                                    const float4 v = reinterpret_cast<const float4 *>(cell_sum + (row + z) * a.D)[d4];
+                                    sum.x += v.x;
+                                    sum.y += v.y;
+                                    sum.z += v.z;
+                                    sum.w += v.w;
+                                }
+                            }
+                        sq = fmaf(sum.x, sum.x, sq);
+                        sq = fmaf(sum.y, sum.y, sq);
+                        sq = fmaf(sum.z, sum.z, sq);
+                        sq = fmaf(sum.w, sum.w, sq);
+                    }
+                    for (int x = 0; x < kt; ++x)
+                        for (int y = 0; y < kh; ++y) {
+                            const int row = ((at * kt + x) * a.nch + ah * kh + y) * a.ncw + aw * kw;
+                            for (int z = 0; z < kw; ++z) m += cell_cnt[row + z];
+                        }
+                    #pragma unroll
+                    for (int off = 16; off > 0; off >>= 1) sq += __shfl_down_sync(0xffffffffu, sq, off);
+                    if (lane == 0) tile_val[item] = m >= 2.f ? (sq - m) / (m * (m - 1.f)) : 0.f;
+                }
     }
     __syncthreads();
     if (threadIdx.x < a.tiles.n) {
         const int c = threadIdx.x;
-        int first = 0;
-        for (int cc = 0; cc < c; ++cc)
-            first += (a.Rt / a.tiles.t[cc]) * (a.Rh / a.tiles.h[cc]) * (a.Rw / a.tiles.w[cc]);
-        const int n = (a.Rt / a.tiles.t[c]) * (a.Rh / a.tiles.h[c]) * (a.Rw / a.tiles.w[c]);
+        const int first = a.item_first[c], n = a.item_first[c + 1] - first;
         float s = 0.f;
         for (int i = 0; i < n; ++i) s += tile_val[first + i];
         const int n_regions = a.nrt * a.nrh * a.nrw;
@@ -244,7 +268,22 @@ cudaError_t launch_select_tiling(const void *q, int esize, int BH, int S, int D,
     int items = 0;
     for (int c = 0; c < tiles.n; ++c)
         items += (g.Rt / tiles.t[c]) * (g.Rh / tiles.h[c]) * (g.Rw / tiles.w[c]);
-    const size_t smem = (static_cast<size_t>(g.cells) * D + g.cells + items) * sizeof(float);
+    a.items = items;
+    a.nch = g.Rh / g.Ch;
+    a.ncw = g.Rw / g.Cw;
+    a.item_first[0] = 0;
+    for (int c = 0; c < kMaxTiles; ++c) {
+        const bool on = c < tiles.n;
+        a.tpr_t[c] = on ? g.Rt / tiles.t[c] : 0;
+        a.tpr_h[c] = on ? g.Rh / tiles.h[c] : 0;
+        a.tpr_w[c] = on ? g.Rw / tiles.w[c] : 0;
+        a.cpt_t[c] = on ? tiles.t[c] / g.Ct : 0;
+        a.cpt_h[c] = on ? tiles.h[c] / g.Ch : 0;
+        a.cpt_w[c] = on ? tiles.w[c] / g.Cw : 0;
+        a.item_first[c + 1] = a.item_first[c] + a.tpr_t[c] * a.tpr_h[c] * a.tpr_w[c];
+    }
+    const size_t cvol = static_cast<size_t>(g.Ct) * g.Ch * g.Cw;
+    const size_t smem = (static_cast<size_t>(g.cells) * D + g.cells + items) * sizeof(float) + cvol * sizeof(int);
     dim3 grid(g.n_regions, BH);
     const int lpt = D * esize / 16;
     cudaError_t e = cudaSuccess;
