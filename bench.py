@@ -413,8 +413,8 @@ def extra_workloads(steps: int):
 
     # structured masks on a CFG pair.  The attention kernel runs in the mode
     # structured_attention picks: T-major directly for whole-frame tiles
-    # (spatial), through TMA boxes for sliding tiles, on permuted copies
-    # with a group mask for the temporal tile.
+    # (spatial), through TMA boxes for sliding tiles, and for the temporal
+    # tile through (T, 1, 128/T) boxes with a strided group mask.
     w = WORKLOADS["structured_s122880"]
     q, k, v = make_qkv(w, device="cuda")
     res = {}
@@ -427,6 +427,11 @@ def extra_workloads(steps: int):
         elif g == 0 and vsa.tiled_supported([stile]):
             mode = "tiled"
             fn = lambda: vsa.block_sparse_attention_tiled(q, k, v, w.grid, [stile], None, idx, cnt)  # noqa: E731
+        elif kind == "temporal" and 128 % w.grid[0] == 0 and w.grid[2] % (128 // w.grid[0]) == 0:
+            mode = "tiled, strided groups"
+            sg = 128 // w.grid[0]
+            fn = lambda: vsa.block_sparse_attention_tiled(q, k, v, w.grid, [(w.grid[0], 1, sg)], None, idx, cnt,  # noqa: E731
+                                                          group_stride=sg if sg > 1 else 0)
         else:
             mode = "permuted copies"
             qp, kp, vp = (vsa.permute(x, w.grid, [stile]) for x in (q, k, v))

@@ -62,7 +62,7 @@ def lib() -> ctypes.CDLL:
         "vsa_topk_block_mask": ([P, I, I, I, I, I, I, P, P, I, P], I),
         "vsa_structured_block_list": ([I, D3, D3, D3, I, P, P, I, P, P], I),
         "vsa_block_sparse_attention": ([P, P, P, P, I, I, I, I, I, I, P, P, I, I, I, F, P], I),
-        "vsa_block_sparse_attention_tiled": ([P, P, P, P, I, I, I, I, I, D3, P, I, P, P, P, I, I, F, P], I),
+        "vsa_block_sparse_attention_tiled": ([P, P, P, P, I, I, I, I, I, D3, P, I, P, P, P, I, I, I, F, P], I),
         "vsa_window_attention": ([P, P, P, P, I, I, I, I, I, I, I, F, I, P], I),
         "vsa_cast_f32_to_bf16": ([P, P, I64, P], I),
         "vsa_debug_wait_timeout": ([I64, P], I),
@@ -338,10 +338,11 @@ def block_sparse_attention(q, k, v, idx, cnt, block: int, group_size: int = 0, s
 
 
 def block_sparse_attention_tiled(q, k, v, grid, tiles, choice, idx, cnt, scale: Optional[float] = None,
-                                 out_dtype=None) -> torch.Tensor:
+                                 out_dtype=None, group_stride: int = 0) -> torch.Tensor:
     """unpermute(block_sparse_attention(permute(q), permute(k), permute(v), idx, cnt, 128)) in one
     kernel: q, k, v and the result stay in T-major order; lists number 128-token blocks of
-    each head's tile-contiguous order."""
+    each head's tile-contiguous order.  group_stride s > 0 restricts each query to keys
+    whose position differs from its own by a multiple of s (see include/vsa.h)."""
     B, H, S, D = _bhsd(q, "q")
     if tuple(k.shape) != (B, H, S, D) or tuple(v.shape) != (B, H, S, D):
         raise ValueError(f"q/k/v shapes must match exactly; got q={tuple(q.shape)}, k={tuple(k.shape)}, "
@@ -357,7 +358,7 @@ def block_sparse_attention_tiled(q, k, v, grid, tiles, choice, idx, cnt, scale: 
     _check(lib().vsa_block_sparse_attention_tiled(
         _ptr(qb), _ptr(kb), _ptr(vb), _ptr(o), BF16 if odt == torch.bfloat16 else F32, B, H, S, D, Dims3(*grid),
         arr, n, _choice_arg(choice, B * H), _ptr(idx), _ptr(cnt), int(idx.shape[-1]), 1 if idx.dim() == 4 else 0,
-        0.0 if scale is None else float(scale), _stream(q.device)))
+        int(group_stride), 0.0 if scale is None else float(scale), _stream(q.device)))
     return o
 
 
@@ -469,6 +470,14 @@ def structured_attention(q, k, v, kind: str, grid, block: int = 128, tile=(4, 8,
     idx, cnt, g = structured_block_list(kind, grid, block, tile, radius, device=q.device)
     if st[1] == grid[1] and st[2] == grid[2]:  # whole frames: the tile-contiguous order is T-major itself
         return block_sparse_attention(q, k, v, idx, cnt, block, g, scale, out_dtype)
+    T = grid[0]
+    if kind == "temporal" and block == 128 and T <= 128 and 128 % T == 0 and grid[2] % (128 // T) == 0:
+        # tile (T, 1, 128/T): a block is all frames of 128/T neighbouring columns, position
+        # t * s + w with s = 128/T, and the temporal mask is "same w", i.e. equal mod s;
+        # the diagonal list is the same as for tile (T, 1, 1)
+        s = 128 // T
+        return block_sparse_attention_tiled(q, k, v, grid, [(T, 1, s)], None, idx, cnt, scale, out_dtype,
+                                            group_stride=s if s > 1 else 0)
     if g == 0 and block == 128 and tiled_supported([st]):
         return block_sparse_attention_tiled(q, k, v, grid, [st], None, idx, cnt, scale, out_dtype)
     qp, kp, vp = (permute(x, grid, [st]) for x in (q, k, v))

@@ -392,8 +392,10 @@ vsa_status vsa_block_sparse_attention_tiled(const void *q, const void *k, const 
                                             vsa_dtype out_dtype, int B, int n_heads, int S, int D, vsa_dims3 grid,
                                             const vsa_dims3 *tiles, int n_tiles, const int32_t *choice,
                                             const int32_t *idx, const int32_t *cnt, int cap, int list_per_head,
-                                            float scale, void *stream) {
+                                            int group_stride, float scale, void *stream) {
     VSA_TRY(check_attention_common(q, k, v, o, out_dtype, B, n_heads, S, D, scale));
+    VSA_REQUIRE(group_stride == 0 || (group_stride >= 2 && group_stride <= 128 && (group_stride & (group_stride - 1)) == 0),
+                "group_stride must be 0 or a power of two in [2, 128], got %d", group_stride);
     VSA_REQUIRE(aligned4(idx) && aligned4(cnt), "idx and cnt must be non-NULL 4-byte aligned device pointers");
     VSA_REQUIRE(cap >= 1, "cap must be >= 1, got %d", cap);
     VSA_REQUIRE(choice == nullptr || aligned4(choice), "choice must be NULL or 4-byte aligned");
@@ -420,6 +422,7 @@ vsa_status vsa_block_sparse_attention_tiled(const void *q, const void *k, const 
     L.group = 0; L.nb = S / 128;
     L.scale = scale > 0.f ? scale : 1.0f / sqrtf(static_cast<float>(D));
     L.tiled = true;
+    L.gstride = group_stride;
     L.T = grid.t; L.Hg = grid.h; L.Wg = grid.w;
     L.tiles = ts;
     L.choice = choice;

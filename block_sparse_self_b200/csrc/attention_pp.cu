@@ -39,6 +39,7 @@ struct PPArgs {
     int S, nq;
     const int32_t *idx, *cnt;
     int cap, list_per_head, group, nb;
+    int gstride;  // > 1: keys share a row's group iff their positions agree with it mod gstride (a power of two)
     int half, sink, dense;
     float scale_log2;
     void *out;
@@ -410,6 +411,13 @@ attn_pp_kernel(const __grid_constant__ MapSet maps, const PPArgs a) {
                         #pragma unroll
                         for (int c = 0; c < BN; ++c)
                             if (c < g0 || c >= g0 + a.group) x[c] = __float_as_uint(-INFINITY);
+                    } else if (a.gstride > 1) {
+                        const int ks = kblock_of<WINDOW>(sc, j) * BN;
+                        // key ks + c is in the row's group iff (ks + c - rg) is a multiple of gstride
+                        const int r0 = (rg - ks) & (a.gstride - 1);
+                        #pragma unroll
+                        for (int c = 0; c < BN; ++c)
+                            if ((c & (a.gstride - 1)) != r0) x[c] = __float_as_uint(-INFINITY);
                     }
                 }
             };
@@ -573,6 +581,7 @@ vsa_status run_pp(const AttnLaunch &L, int *status, cudaStream_t st) {
     a.cap = L.cap;
     a.list_per_head = L.list_per_head;
     a.group = L.group;
+    a.gstride = L.gstride;
     a.nb = L.nb;
     a.half = L.half;
     a.sink = L.sink;

@@ -70,6 +70,7 @@ struct AttnLaunch {
     // tiled mode: q, k, v, o in T-major order; each (b, head) uses its chosen
     // tiling and the kernel permutes through its TMA boxes and epilogue
     bool tiled;
+    int gstride;  // tiled mode: strided groups (0 = none)
     int T, Hg, Wg;
     TileSet tiles;
     const int32_t *choice;

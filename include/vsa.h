@@ -259,6 +259,11 @@ vsa_status vsa_block_sparse_attention(const void *q, const void *k, const void *
  *            tile.t divisible by V/128 (a 128-token block is tile.t*128/V
  *            whole (h, w) planes of the tile)
  *   choice   [B, n_heads] int32 or NULL (tile 0 for every head)
+ *   group_stride  0, or a power of two s in [2, 128]: a key is then visible
+ *            to a query only if their positions (tile-contiguous order)
+ *            differ by a multiple of s.  With tile (T, 1, 128 / T) and the
+ *            diagonal list this is the temporal-only mask ("ADR-0001", step 1):
+ *            position t * s + w of a block holds frame t of column w.
  * Lists are checked as for vsa_block_sparse_attention; a choice outside
  * [0, n_tiles) leaves the head unwritten and sets VSA_ERR_RUNTIME.         */
 vsa_status vsa_block_sparse_attention_tiled(const void *q, const void *k, const void *v,
@@ -267,7 +272,7 @@ vsa_status vsa_block_sparse_attention_tiled(const void *q, const void *k, const 
                                             const vsa_dims3 *tiles, int n_tiles,
                                             const int32_t *choice, const int32_t *idx,
                                             const int32_t *cnt, int cap, int list_per_head,
-                                            float scale, void *stream);
+                                            int group_stride, float scale, void *stream);
 
 /* ------------------------------------------------------------------------ */
 /* Symmetric sliding-window attention with global sinks.

@@ -330,6 +330,29 @@ def test_block_sparse_attention_tiled_bad_choice_and_lists():
         vsa.block_sparse_attention_tiled(q, k, v, (1, 16, 16), [(1, 16, 16)], None, idx, cnt)
 
 
+@pytest.mark.parametrize("D,grid", [(64, (16, 4, 16)), (128, (32, 2, 8))])
+def test_temporal_attention_through_strided_groups(D, grid):
+    """temporal_only via tile (T, 1, 128/T) and a strided group mask, with no
+    permuted copies, against the oracle's same-(h, w) attention."""
+    q, k, v = smooth_qkv(1, 2, grid, D, seed=76, device=DEV)
+    o = vsa.structured_attention(q, k, v, "temporal", grid, 128, out_dtype=torch.float32)
+    t, r = oracle.structured_tile("temporal", grid)
+    idx, cnt, g = oracle.tile_neighbourhood_list(grid, t, r, 128)
+    perm = oracle.tile_permutation(grid, t)
+    for h in range(2):
+        qp, kp, vp = (oracle.permute_rows(_np(x[0, h]), perm) for x in (q, k, v))
+        op = oracle.block_sparse_attention(qp, kp, vp, idx, cnt, 128, g)
+        want = np.empty_like(op)
+        want[perm] = op
+        assert_attn_close(_np(o[0, h]), want, f"h{h}")
+    qb, kb, vb = (x.to(torch.bfloat16) for x in (q, k, v))
+    ti = torch.as_tensor(idx, device=DEV)
+    tc = torch.as_tensor(cnt, device=DEV)
+    with pytest.raises(ValueError):   # a stride must be a power of two
+        vsa.block_sparse_attention_tiled(qb, kb, vb, grid, [(grid[0], 1, 128 // grid[0])], None, ti, tc,
+                                         group_stride=3)
+
+
 def test_block_sparse_attention_group_mask_and_shared_list():
     """temporal_only: tile (T,1,1) with T=8 inside blocks of 32 -> group mask."""
     grid, block = (8, 8, 8), 32
