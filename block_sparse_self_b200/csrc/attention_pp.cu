@@ -423,18 +423,26 @@ attn_pp_kernel(const __grid_constant__ MapSet maps, const PPArgs a) {
             };
             apply_mask();
             // P = 2^(scale*log2e*S - m_use) in place (bf16 pairs), returns the row sum
+            // The arguments and the row sum use two-wide fp32 instructions: the
+            // exponentials are bound by the exponential unit, and fewer issue
+            // slots here leave more to the other tile's warp on the sub-partition.
             auto exp_pass = [&](float m_use) -> float {
-                const float nm = -m_use;
-                float acc[4] = {0.f, 0.f, 0.f, 0.f};
+                const uint64_t sl2x2 = f32x2(sl2, sl2), nmx2 = f32x2(-m_use, -m_use);
+                uint64_t acc[2] = {f32x2(0.f, 0.f), f32x2(0.f, 0.f)};
                 #pragma unroll
                 for (int q = 0; q < BN / 2; ++q) {
-                    const float p0 = ex2_approx(fmaf(__uint_as_float(x[2 * q]), sl2, nm));
-                    const float p1 = ex2_approx(fmaf(__uint_as_float(x[2 * q + 1]), sl2, nm));
-                    acc[q & 3] += p0;
-                    acc[q & 3] += p1;
+                    float a0, a1;
+                    f32x2_split(fma_f32x2(f32x2(__uint_as_float(x[2 * q]), __uint_as_float(x[2 * q + 1])), sl2x2, nmx2),
+                                a0, a1);
+                    const float p0 = ex2_approx(a0);
+                    const float p1 = ex2_approx(a1);
+                    acc[q & 1] = add_f32x2(acc[q & 1], f32x2(p0, p1));
                     x[q] = pack_bf16x2(p0, p1);   // P, packed in place (q <= 2q)
                 }
-                return (acc[0] + acc[1]) + (acc[2] + acc[3]);
+                float s0, s1, s2, s3;
+                f32x2_split(acc[0], s0, s1);
+                f32x2_split(acc[1], s2, s3);
+                return (s0 + s2) + (s1 + s3);
             };
             auto raw_max = [&]() -> float {
                 float m4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
