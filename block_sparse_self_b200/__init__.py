@@ -463,6 +463,62 @@ def spade_attention(q, k, v, grid, tiles, budget: Optional[float] = None, topk: 
     return o
 
 
+def spade_attention_host(q, k, v, grid, tiles, out: Optional[torch.Tensor] = None, chunks: int = 8,
+                         device=None, **kwargs) -> torch.Tensor:
+    """spade_attention for inputs and output in (pinned) host memory.
+
+    The B*H (batch, head) rows are taken in `chunks` groups.  Each group's
+    copy to the device, its attention and the copy of its output back run on
+    separate streams, so the copies of one group overlap the kernels of
+    another.  Every (batch, head) is independent of the others, so the result
+    equals spade_attention on the whole batch.  Returns `out` (allocated
+    pinned when not given) once the last copy back has finished.  Keyword
+    arguments go to spade_attention (budget, topk, n_sink_blocks, ...).
+    """
+    for t, nm in ((q, "q"), (k, "k"), (v, "v")):
+        if not isinstance(t, torch.Tensor) or t.is_cuda or not t.is_contiguous():
+            raise ValueError(f"{nm} must be a contiguous host tensor")
+    B, H, S, D = _bhsd(q, "q")
+    if tuple(k.shape) != (B, H, S, D) or tuple(v.shape) != (B, H, S, D):
+        raise ValueError("q/k/v shapes must match exactly")
+    odt = _out_dtype(kwargs.get("out_dtype"), q)
+    if out is None:
+        out = torch.empty(q.shape, dtype=odt, pin_memory=True)
+    elif out.shape != q.shape or out.dtype != odt or out.is_cuda or not out.is_contiguous():
+        raise ValueError("out must be a contiguous host tensor of q's shape and the output dtype")
+    dev = torch.device("cuda", torch.cuda.current_device()) if device is None else torch.device(device)
+    BH = B * H
+    n_chunks = max(1, min(int(chunks), BH))
+    bounds = [(BH * g // n_chunks, BH * (g + 1) // n_chunks) for g in range(n_chunks)]
+    rows = max(b - a for a, b in bounds)
+    flat = [x.view(BH, S, D) for x in (q, k, v)]
+    oflat = out.view(BH, S, D)
+    comp = torch.cuda.current_stream(dev)
+    h2d, d2h = torch.cuda.Stream(dev), torch.cuda.Stream(dev)
+    slots = [[torch.empty(rows, S, D, dtype=q.dtype, device=dev) for _ in range(3)] for _ in range(2)]
+    used = [None, None]  # per slot: event after the attention that last read it
+    for g, (a, b) in enumerate(bounds):
+        n, slot = b - a, g % 2
+        with torch.cuda.stream(h2d):
+            if used[slot] is not None:
+                h2d.wait_event(used[slot])
+            for src, dst in zip(flat, slots[slot]):
+                dst[:n].copy_(src[a:b], non_blocking=True)
+            ready = h2d.record_event()
+        comp.wait_event(ready)
+        qd, kd, vd = (x[:n].view(1, n, S, D) for x in slots[slot])
+        o = spade_attention(qd, kd, vd, grid, tiles, **kwargs)
+        used[slot] = comp.record_event()
+        with torch.cuda.stream(d2h):
+            d2h.wait_event(used[slot])
+            oflat[a:b].copy_(o.view(n, S, D), non_blocking=True)
+            o.record_stream(d2h)
+    for x in slots[0] + slots[1]:
+        x.record_stream(comp)
+    d2h.synchronize()
+    return out
+
+
 def structured_attention(q, k, v, kind: str, grid, block: int = 128, tile=(4, 8, 8), radius=(1, 1, 1),
                          scale: Optional[float] = None, out_dtype=None):
     """A structured static mask as block-sparse attention, in and out in T-major order."""

@@ -427,6 +427,18 @@ def test_tiny_workload_end_to_end():
         assert_attn_close(_np(ow[0, h]), want, f"window head {h}")
 
 
+@pytest.mark.parametrize("chunks", [1, 3, 8])
+def test_spade_attention_host_buffers_match_device(chunks):
+    """The host-buffer entry point (copies of one group of heads overlapping
+    the kernels of another) returns exactly the device result."""
+    grid, tiles = (4, 8, 16), [(1, 8, 16), (2, 8, 8), (4, 4, 8)]
+    q, k, v = smooth_qkv(2, 3, grid, 128, seed=77, device=DEV)
+    want = vsa.spade_attention(q, k, v, grid, tiles, topk=2, out_dtype=torch.float32)
+    qh, kh, vh = (x.cpu().pin_memory() for x in (q, k, v))
+    got = vsa.spade_attention_host(qh, kh, vh, grid, tiles, chunks=chunks, topk=2, out_dtype=torch.float32)
+    assert not got.is_cuda and torch.equal(got, want.cpu())
+
+
 def _sample_blocks(nb, seed, n=16):
     rng = np.random.default_rng(seed)
     mid = rng.choice(np.arange(1, nb - 1), n - 2, replace=False)
