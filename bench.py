@@ -213,6 +213,22 @@ def mask_pipeline_bytes(w, BH: int) -> float:
     return float(summ + scores + topk)
 
 
+def rank_workload(w, rank: int):
+    """Each rank's own batch of heads (weak scaling): the same shapes, its own
+    seeded inputs, no data exchanged between ranks."""
+    from dataclasses import replace
+    return replace(w, seed_base=w.seed_base + 100 * rank)
+
+
+def reduce_over_ranks(x: float, op: str, dist_on: bool, device) -> float:
+    """MAX (times) or SUM (work) of a per-rank number over all ranks."""
+    t = torch.tensor([float(x)], dtype=torch.float64, device=device)
+    if dist_on:
+        ops = {"max": torch.distributed.ReduceOp.MAX, "sum": torch.distributed.ReduceOp.SUM}
+        torch.distributed.all_reduce(t, op=ops[op])
+    return float(t.item())
+
+
 def time_steps(fn, steps: int, warmup: int, dist_on: bool):
     for _ in range(warmup):
         fn(False)
@@ -466,8 +482,7 @@ def run_ours(args, w):
     peaks, peak_src = load_peaks()
 
     # each rank: its own batch of heads (weak scaling, no data-path collective)
-    from dataclasses import replace
-    wr = replace(w, seed_base=w.seed_base + 100 * rank)
+    wr = rank_workload(w, rank)
     q, k, v = make_qkv(wr, device="cuda")
     step = SpadeStep(wr, q, k, v)
     BH = w.B * w.heads
@@ -479,11 +494,9 @@ def run_ours(args, w):
     flops = computed_flops(step.last["cnt"], step.block, w.D)
     vsa.device_status()
 
-    t = torch.tensor([ms], device="cuda")
-    if dist_on:
-        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-    ms_max = float(t.item())
-    value = world * flops / ms_max / 1e9  # TFLOP/s (ms -> 1e-3 s, 1e12)
+    ms_max = reduce_over_ranks(ms, "max", dist_on, "cuda")
+    total_flops = reduce_over_ranks(flops, "sum", dist_on, "cuda")  # every rank's computed blocks
+    value = total_flops / ms_max / 1e9  # TFLOP/s (ms -> 1e-3 s, 1e12)
 
     attn_ms = ph["attention"]
     achieved = flops / attn_ms / 1e9
@@ -503,10 +516,8 @@ def run_ours(args, w):
     e2e = None
     if not args.no_e2e:
         e_ms, h2d, d2h = run_e2e(w, step, q, k, v, max(2, args.steps // 2))
-        te = torch.tensor([e_ms], device="cuda")
-        if dist_on:
-            torch.distributed.all_reduce(te, op=torch.distributed.ReduceOp.MAX)
-        e2e = {"value": world * flops / float(te.item()) / 1e9, "unit": UNIT, "ms_per_step": float(te.item()),
+        e_max = reduce_over_ranks(e_ms, "max", dist_on, "cuda")
+        e2e = {"value": total_flops / e_max / 1e9, "unit": UNIT, "ms_per_step": e_max,
                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h}
 
     extra = None
