@@ -36,6 +36,8 @@ def lib():
         L.orc_permute_rows.argtypes = [P, i64, i32, P, P]
         L.orc_unpermute_rows.argtypes = [P, i64, i32, P, P]
         L.orc_tile_sics.argtypes = [P] + [i32] * 7 + [P]
+        L.orc_tile_counts.argtypes = [P] + [i32] * 7 + [P]
+        L.orc_pad_grid.argtypes = [P] + [i32] * 7 + [P]
         L.orc_select_tiling.argtypes = [P, i32, i32, i32, i32, P, i32, P]
         L.orc_select_tiling.restype = i32
         L.orc_block_minmax.argtypes = [P, i64, i32, i32, P, P]
@@ -45,7 +47,7 @@ def lib():
         L.orc_tile_neighbourhood_list.argtypes = [i32] * 11 + [P, P, P]
         L.orc_tile_neighbourhood_list.restype = i32
         L.orc_window_attention.argtypes = [P, P, P, i64, i32, i32, i32, dbl, i32, P, i64, P]
-        L.orc_block_sparse_attention.argtypes = [P, P, P, i64, i32, i32, P, P, i32, i32, dbl, P, i64, P]
+        L.orc_block_sparse_attention.argtypes = [P, P, P, i64, i32, i32, P, P, i32, i32, dbl, P, P, i64, P]
         L.orc_window_key_ranges.argtypes = [i64] * 5 + [P]
         L.orc_window_key_ranges.restype = i32
         _lib = L
@@ -106,6 +108,51 @@ def unpermute_rows(y, perm) -> np.ndarray:
 
 
 # --------------------------------------------------------------------------
+# grids the tiles do not divide ("Adaptive tiling (SPADE)", Deviations and
+# notes: pad with zero tokens, excluded from the cohesion; mask padded keys)
+# --------------------------------------------------------------------------
+
+def padded_grid(grid, tiles):
+    """Each axis rounded up to a multiple of every candidate's extent on it
+    (their least common multiple), so that every candidate tiles it."""
+    out = []
+    for ax in range(3):
+        l = 1
+        for t in tiles:
+            l = l * t[ax] // np.gcd(l, t[ax])
+        out.append(-(-grid[ax] // l) * l)
+    return tuple(int(x) for x in out)
+
+
+def pad_grid(x, grid, padded) -> np.ndarray:
+    """[T*H*W, D] T-major -> [Tp*Hp*Wp, D] with zero tokens outside (T, H, W)."""
+    x = _f32(x)
+    T, H, W = grid
+    Tp, Hp, Wp = padded
+    y = np.empty((Tp * Hp * Wp, x.shape[1]), np.float32)
+    lib().orc_pad_grid(_ptr(x), T, H, W, x.shape[1], Tp, Hp, Wp, _ptr(y))
+    return y
+
+
+def real_tokens(grid, padded) -> np.ndarray:
+    """Boolean mask over the padded grid's T-major tokens: inside (T, H, W)."""
+    T, H, W = grid
+    Tp, Hp, Wp = padded
+    t, h, w = np.meshgrid(np.arange(Tp), np.arange(Hp), np.arange(Wp), indexing="ij")
+    return ((t < T) & (h < H) & (w < W)).reshape(-1)
+
+
+def tile_counts(q, grid, tile) -> np.ndarray:
+    """Non-zero-norm queries per tile of one tiling."""
+    q = _f32(q)
+    T, H, W = grid
+    n = (T * H * W) // (tile[0] * tile[1] * tile[2])
+    out = np.empty(n, dtype=np.int64)
+    lib().orc_tile_counts(_ptr(q), T, H, W, q.shape[1], *tile, _ptr(out))
+    return out
+
+
+# --------------------------------------------------------------------------
 # tiling choice
 # --------------------------------------------------------------------------
 
@@ -152,7 +199,10 @@ def block_scores(qmax, qmin, kmax, kmin) -> np.ndarray:
 
 
 def list_cap(nb: int, k: int, n_sink: int, diag_halfwidth: int) -> int:
-    return min(nb, k + n_sink + 2 * diag_halfwidth + 1)
+    """Longest possible list: k top blocks, the sinks and the diagonal band
+    (2 dw + 1 blocks; none when diag_halfwidth is -1)."""
+    band = 2 * diag_halfwidth + 1 if diag_halfwidth >= 0 else 0
+    return min(nb, k + n_sink + band)
 
 
 def topk_block_list(score, k: int, n_sink: int = 1, diag_halfwidth: int = 0,
@@ -236,17 +286,20 @@ def dense_attention(q, k, v, scale=None, rows=None):
 
 
 def block_sparse_attention(qp, kp, vp, idx, cnt, block: int, group_size: int = 0,
-                           scale=None, rows=None):
-    """Block-list attention for one head in the permuted order."""
+                           scale=None, rows=None, key_ok=None):
+    """Block-list attention for one head in the permuted order; key_ok[p] == 0
+    masks key p (padding)."""
     qp, kp, vp = _f32(qp), _f32(kp), _f32(vp)
     S, D = qp.shape
     idx = np.ascontiguousarray(idx, np.int32)
     cnt = np.ascontiguousarray(cnt, np.int32)
     r = _rows(rows, S)
+    ok = None if key_ok is None else np.ascontiguousarray(key_ok, np.uint8)
     out = np.empty((len(r), D), np.float64)
     lib().orc_block_sparse_attention(_ptr(qp), _ptr(kp), _ptr(vp), S, D, block,
                                      _ptr(idx), _ptr(cnt), idx.shape[1], group_size,
-                                     default_scale(D, scale), _ptr(r), len(r), _ptr(out))
+                                     default_scale(D, scale), None if ok is None else _ptr(ok),
+                                     _ptr(r), len(r), _ptr(out))
     return out
 
 
@@ -265,30 +318,43 @@ def spade_head(q, k, v, grid, tiles, k_blocks: int, n_sink: int = 1,
     """Adaptive tiling -> permutation -> min/max scores -> top-k + sink +
     diagonal -> block-sparse attention -> inverse permutation, for one head.
 
+    A grid the candidates do not divide is first zero-padded to padded_grid()
+    (the pages' recipe); the zero tokens drop out of the cohesion by having
+    zero norm, take part in the summaries, and are masked as keys.  ``out``
+    then holds the real tokens only; ``perm`` and the blocks refer to the
+    padded grid.
+
     Returns a dict with every intermediate.  With ``query_blocks`` only those
     query blocks (in the permuted order) are attended; ``out_perm`` then holds
     just their rows and ``out`` is None.
     """
     q, k, v = _f32(q), _f32(k), _f32(v)
+    real_grid = tuple(grid)
+    grid = padded_grid(real_grid, tiles)
+    padded = grid != real_grid
+    if padded:  # zero tokens up to a grid every candidate tiles; padded keys masked below
+        q, k, v = (pad_grid(x, real_grid, grid) for x in (q, k, v))
     choice, cohesion = select_tiling(q, grid, tiles) if len(tiles) > 1 else (0, None)
     tile = tiles[choice]
     block = tile[0] * tile[1] * tile[2]
     perm = tile_permutation(grid, tile)
     qp, kp, vp = (permute_rows(x, perm) for x in (q, k, v))
+    key_ok = real_tokens(real_grid, grid)[perm].astype(np.uint8) if padded else None
     qmax, qmin = block_minmax(qp, block)
     kmax, kmin = block_minmax(kp, block)
     score = block_scores(qmax, qmin, kmax, kmin)
     idx, cnt = topk_block_list(score, k_blocks, n_sink, diag_halfwidth)
     res = dict(choice=choice, cohesion=cohesion, perm=perm, block=block,
                qmax=qmax, qmin=qmin, kmax=kmax, kmin=kmin, score=score,
-               idx=idx, cnt=cnt)
+               idx=idx, cnt=cnt, padded_grid=grid, key_ok=key_ok)
     if query_blocks is None:
-        op = block_sparse_attention(qp, kp, vp, idx, cnt, block, 0, scale)
+        op = block_sparse_attention(qp, kp, vp, idx, cnt, block, 0, scale, key_ok=key_ok)
         res["out_perm"] = op
-        res["out"] = _unpermute64(op, perm)
+        out = _unpermute64(op, perm)
+        res["out"] = out[real_tokens(real_grid, grid)] if padded else out
     else:
         rows = np.concatenate([np.arange(b * block, (b + 1) * block) for b in query_blocks])
-        res["out_perm"] = block_sparse_attention(qp, kp, vp, idx, cnt, block, 0, scale, rows)
+        res["out_perm"] = block_sparse_attention(qp, kp, vp, idx, cnt, block, 0, scale, rows, key_ok=key_ok)
         res["rows"] = rows
         res["out"] = None
     return res

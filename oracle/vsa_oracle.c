@@ -87,6 +87,24 @@ void orc_unpermute_rows(const float *y, int64_t S, int D, const int64_t *perm, f
 }
 
 /* ----------------------------------------------------------------------- */
+/* Grids the tiles do not divide  [SPADE "Deviations and notes": pad the     */
+/* grid to a multiple of the tiles with zero tokens, excluded from the       */
+/* cohesion, and mask the padded keys]                                      */
+/* ----------------------------------------------------------------------- */
+
+/* y = x zero-padded from the T-major grid (T, H, W) to (Tp, Hp, Wp): token
+ * (t, h, w) keeps its coordinates, every token outside (T, H, W) is zero.  */
+void orc_pad_grid(const float *x, int T, int H, int W, int D, int Tp, int Hp, int Wp, float *y)
+{
+    memset(y, 0, sizeof(float) * (size_t)((int64_t)Tp * Hp * Wp * D));
+    for (int t = 0; t < T; ++t)
+        for (int h = 0; h < H; ++h)
+            for (int w = 0; w < W; ++w)
+                memcpy(y + (((int64_t)t * Hp + h) * Wp + w) * D, x + (((int64_t)t * H + h) * W + w) * D,
+                       sizeof(float) * (size_t)D);
+}
+
+/* ----------------------------------------------------------------------- */
 /* Query cohesion (SICS) and the per-head tiling choice  [SPADE step 1;     */
 /* function table: block_self_similarity, select_tiling; "Deviations"]      */
 /* ----------------------------------------------------------------------- */
@@ -126,9 +144,28 @@ void orc_tile_sics(const float *q, int T, int H, int W, int D,
     free(label);
 }
 
-/* Cohesion of a tiling = mean of its tiles' SICS.  The choice is the
- * candidate with the largest cohesion; equal cohesion goes to the lower
- * candidate index.  scores[c] receives each candidate's cohesion.         */
+/* Number of non-zero-norm queries in every tile of one tiling.            */
+void orc_tile_counts(const float *q, int T, int H, int W, int D,
+                     int tt, int th, int tw, int64_t *m)
+{
+    int64_t S = (int64_t)T * H * W;
+    int64_t n_tiles = S / ((int64_t)tt * th * tw);
+    int64_t *label = (int64_t *)malloc(sizeof(int64_t) * S);
+    orc_tile_labels(T, H, W, tt, th, tw, label);
+    for (int64_t c = 0; c < n_tiles; ++c) m[c] = 0;
+    for (int64_t i = 0; i < S; ++i) {
+        int nz = 0;
+        for (int d = 0; d < D && !nz; ++d) nz = q[i * D + d] != 0.0f;
+        if (nz) m[label[i]] += 1;
+    }
+    free(label);
+}
+
+/* Cohesion of a tiling = mean of its tiles' SICS, over the tiles that hold
+ * at least one non-zero-norm query (a tile made only of zero padding is not
+ * a tile of the video; with no zero tokens every tile counts).  The choice
+ * is the candidate with the largest cohesion; equal cohesion goes to the
+ * lower candidate index.  scores[c] receives each candidate's cohesion.   */
 int orc_select_tiling(const float *q, int T, int H, int W, int D,
                       const int *tiles, int n_tiles, double *scores)
 {
@@ -137,10 +174,15 @@ int orc_select_tiling(const float *q, int T, int H, int W, int D,
         int tt = tiles[3 * c], th = tiles[3 * c + 1], tw = tiles[3 * c + 2];
         int64_t n = ((int64_t)T * H * W) / ((int64_t)tt * th * tw);
         double *ts = (double *)malloc(sizeof(double) * (size_t)n);
+        int64_t *m = (int64_t *)malloc(sizeof(int64_t) * (size_t)n);
         orc_tile_sics(q, T, H, W, D, tt, th, tw, ts);
+        orc_tile_counts(q, T, H, W, D, tt, th, tw, m);
         double acc = 0.0;
-        for (int64_t i = 0; i < n; ++i) acc += ts[i];
-        scores[c] = acc / (double)n;
+        int64_t used = 0;
+        for (int64_t i = 0; i < n; ++i)
+            if (m[i] >= 1) { acc += ts[i]; ++used; }
+        scores[c] = used > 0 ? acc / (double)used : 0.0;
+        free(m);
         free(ts);
         if (scores[c] > scores[best]) best = c;
     }
@@ -369,11 +411,12 @@ void orc_window_attention(const float *q, const float *k, const float *v,
 /* Block-sparse attention for one head in the permuted order: query row p of
  * query block i = p / block sees every key of every block listed for i
  * (idx[i*cap .. i*cap+cnt[i])), restricted to keys of the same group of
- * group_size tokens when group_size > 0.  rows[] selects output rows.      */
+ * group_size tokens when group_size > 0, and to keys with key_ok[t] != 0
+ * when key_ok is given (padded keys are masked).  rows[] selects output rows. */
 void orc_block_sparse_attention(const float *q, const float *k, const float *v,
                                 int64_t S, int D, int block,
                                 const int32_t *idx, const int32_t *cnt, int cap,
-                                int group_size, double scale,
+                                int group_size, double scale, const unsigned char *key_ok,
                                 const int64_t *rows, int64_t n_rows, double *out)
 {
     #pragma omp parallel
@@ -388,7 +431,7 @@ void orc_block_sparse_attention(const float *q, const float *k, const float *v,
             for (int c = 0; c < cnt[i]; ++c) {
                 int64_t j = idx[i * cap + c];
                 for (int64_t t = j * block; t < (j + 1) * block; ++t)
-                    if (group_size <= 0 || t / group_size == p / group_size) vis[t] = 1;
+                    if ((group_size <= 0 || t / group_size == p / group_size) && (!key_ok || key_ok[t])) vis[t] = 1;
             }
             orc_softmax_row(q, k, v, p, D, scale, vis, S, logit, out + r * D);
         }

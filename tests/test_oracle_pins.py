@@ -399,3 +399,69 @@ def test_sampled_rows_match_full_rows():
     full = oracle.spade_head(q, k, v, grid, [(2, 4, 4)], k_blocks=2)
     part = oracle.spade_head(q, k, v, grid, [(2, 4, 4)], k_blocks=2, query_blocks=[0, 5, 7])
     np.testing.assert_array_equal(part["out_perm"], full["out_perm"][part["rows"]])
+
+
+# --------------------------------------------------------------------------
+# grids the tiles do not divide ("Adaptive tiling (SPADE)", Deviations and
+# notes: pad to a multiple of the tiles with zero tokens, excluded from the
+# cohesion, and mask the padded keys)
+# --------------------------------------------------------------------------
+
+def test_padded_grid_is_the_per_axis_lcm_multiple():
+    tiles = [(1, 8, 16), (2, 8, 8), (4, 4, 8)]
+    assert oracle.padded_grid((16, 45, 80), tiles) == (16, 48, 80)   # Wan's 16 x 45 x 80
+    assert oracle.padded_grid((13, 45, 81), tiles) == (16, 48, 96)
+    assert oracle.padded_grid((32, 48, 80), tiles) == (32, 48, 80)   # divisible: unchanged
+    assert oracle.padded_grid((3, 5, 6), [(1, 2, 4), (2, 2, 2)]) == (4, 6, 8)
+
+
+def test_pad_grid_keeps_coordinates_and_zero_fills():
+    grid, padded = (3, 5, 6), (4, 6, 8)
+    x = np.arange(3 * 5 * 6 * 2, dtype=np.float32).reshape(-1, 2) + 1
+    y = oracle.pad_grid(x, grid, padded)
+    real = oracle.real_tokens(grid, padded)
+    assert real.sum() == 90 and np.array_equal(y[real], x)
+    assert (y[~real] == 0).all()
+    # token (t, h, w) of the real grid sits at (t, h, w) of the padded one
+    t, h, w = 2, 4, 5
+    assert np.array_equal(y[(t * 6 + h) * 8 + w], x[(t * 5 + h) * 6 + w])
+
+
+def test_padded_all_blocks_budget_equals_dense_attention_over_the_real_tokens():
+    """pad = mask: with every block kept, the padded composition must be dense
+    attention over the real tokens alone (the padding takes no part)."""
+    grid = (3, 5, 6)
+    tiles = [(1, 2, 4), (2, 2, 2)]
+    q, k, v = (integer_grid((90, 16), 90 + o, torch.float32).numpy() for o in range(3))
+    nb = 4 * 6 * 8 // 8
+    res = oracle.spade_head(q, k, v, grid, tiles, k_blocks=nb, n_sink=0, diag_halfwidth=-1)
+    assert res["padded_grid"] == (4, 6, 8) and (res["cnt"] == nb).all()
+    np.testing.assert_allclose(res["out"], _sdpa64(q, k, v, 16 ** -0.5), atol=1e-12, rtol=0)
+
+
+def test_padded_cohesion_by_brute_force():
+    """Cohesion on a padded grid: per tile the mean cosine over distinct pairs
+    of its non-zero queries, averaged over the tiles that hold any query; the
+    zero padding adds neither queries nor tiles."""
+    grid, tiles = (3, 5, 6), [(1, 2, 4), (2, 2, 2), (1, 2, 2)]
+    padded = oracle.padded_grid(grid, tiles)
+    q = integer_grid((90, 8), 95, torch.float32).numpy()
+    q[7] = 0.0                                   # one real zero-norm query too
+    qp = oracle.pad_grid(q, grid, padded)
+    _, got = oracle.select_tiling(qp, padded, tiles)
+    tp, hp, wp = _coords(padded)
+    for c, (tt, th, tw) in enumerate(tiles):
+        label = ((tp // tt) * (padded[1] // th) + hp // th) * (padded[2] // tw) + wp // tw
+        vals = []
+        for lab in np.unique(label):
+            rows = qp[label == lab]
+            rows = rows[np.linalg.norm(rows, axis=1) > 0].astype(np.float64)
+            if len(rows) == 0:
+                continue
+            n = rows / np.linalg.norm(rows, axis=1, keepdims=True)
+            if len(n) < 2:
+                vals.append(0.0)
+                continue
+            pairs = [n[i] @ n[j] for i in range(len(n)) for j in range(len(n)) if i != j]
+            vals.append(float(np.mean(pairs)))
+        assert abs(got[c] - np.mean(vals)) < 1e-12, (c, got[c], np.mean(vals))
