@@ -392,8 +392,9 @@ def window_tile_pairs(S: int, window: int, sink: int, bn: int = 128) -> int:
 
 
 def extra_workloads(steps: int):
-    """Secondary lines: window (S=30720), SPADE fixed tiling (S=30720),
-    structured masks on a CFG pair (S=122880), and dense SDPA context."""
+    """Secondary lines: window (S=30720), SPADE fixed tiling (S=30720), SPADE
+    adaptive on a padded 16 x 45 x 80 grid (S=57600), structured masks on a
+    CFG pair (S=122880), and dense SDPA context."""
     import block_sparse_self_b200 as vsa
     out = {}
 
@@ -429,6 +430,21 @@ def extra_workloads(steps: int):
     fl = computed_flops(st.last["cnt"], st.block, w.D)
     out[w.name] = {"ms_per_step": ms, "tflops_step": fl / ms / 1e9, "attn_ms": ph["attention"],
                    "attn_tflops": fl / ph["attention"] / 1e9, "phase_ms": ph}
+    del q, k, v, st
+
+    # SPADE with adaptive tiling on a grid the candidates do not divide
+    # (16 x 45 x 80, zero-padded to 16 x 48 x 80 inside the kernels; every
+    # 128-position query block of it holds real tokens, so the counted blocks
+    # are the computed ones)
+    w = WORKLOADS["spade_adaptive_pad_s57600"]
+    q, k, v = make_qkv(w, device="cuda")
+    st = SpadeStep(w, q, k, v)
+    ms = timed(lambda: st(True), n=steps)
+    ph = st.phase_ms()
+    fl = computed_flops(st.last["cnt"], st.block, w.D)
+    out[w.name] = {"ms_per_step": ms, "tflops_step": fl / ms / 1e9, "attn_ms": ph["attention"],
+                   "attn_tflops": fl / ph["attention"] / 1e9, "phase_ms": ph,
+                   "padded_grid": list(vsa.padded_grid(w.grid, w.tiles))}
     del q, k, v, st
 
     # structured masks on a CFG pair.  The attention kernel runs in the mode

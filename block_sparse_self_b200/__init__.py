@@ -51,6 +51,7 @@ def lib() -> ctypes.CDLL:
     sig = {
         "vsa_last_error": ([], ctypes.c_char_p),
         "vsa_device_status": ([P], I),
+        "vsa_padded_grid": ([D3, P, I, P], I),
         "vsa_select_tiling_workspace_size": ([I, I, D3, P, I], SZ),
         "vsa_select_tiling": ([P, I, I, I, I, I, D3, P, I, P, P, P, SZ, P], I),
         "vsa_select_tiling_noalloc": ([P, I, I, I, I, I, D3, P, I, P, P, P], I),
@@ -135,6 +136,20 @@ def _tiles_arg(tiles: Sequence[Sequence[int]]):
     return arr, len(tiles)
 
 
+def padded_grid(grid, tiles) -> Tuple[int, int, int]:
+    """The grid every candidate tiles: each axis rounded up to a multiple of the
+    candidates' lcm on it (equal to grid when they all divide it).  Positions,
+    tilings and block indices of the calls below refer to this grid."""
+    arr, n = _tiles_arg(tiles)
+    out = Dims3()
+    _check(lib().vsa_padded_grid(Dims3(*grid), arr, n, ctypes.byref(out)))
+    return (out.t, out.h, out.w)
+
+
+def _grid_tokens(grid) -> int:
+    return int(grid[0]) * int(grid[1]) * int(grid[2])
+
+
 def device_status(stream=None) -> None:
     """Synchronise the stream; raise if a kernel recorded a device-side failure."""
     _check(lib().vsa_device_status(_stream() if stream is None else stream))
@@ -176,13 +191,17 @@ def select_tiling_noalloc(q: torch.Tensor, grid, tiles, return_sics: bool = Fals
 
 def _permute(x, grid, tiles, choice, inverse):
     _cuda(x, "x")
-    B, H, S, D = _bhsd(x, "x")
+    B, H, rows, D = _bhsd(x, "x")
     if choice is not None:
         _cuda(choice, "choice")
         if choice.dtype != torch.int32 or choice.numel() != B * H:
             raise ValueError("choice must be int32 with B*H entries")
     arr, n = _tiles_arg(tiles)
-    y = torch.empty_like(x)
+    S, Sp = _grid_tokens(grid), _grid_tokens(padded_grid(grid, tiles))
+    if rows != (Sp if inverse else S):
+        raise ValueError(f"x has {rows} rows per head; expected {Sp if inverse else S} "
+                         f"({'padded' if inverse else 'real'} tokens of grid {tuple(grid)})")
+    y = torch.empty(B, H, S if inverse else Sp, D, dtype=x.dtype, device=x.device)
     fn = lib().vsa_unpermute if inverse else lib().vsa_permute
     _check(fn(_ptr(x), _ptr(y), _dtype_code(x, "x"), B, H, S, D, Dims3(*grid), arr, n, _ptr(choice),
               _stream(x.device)))
@@ -190,12 +209,14 @@ def _permute(x, grid, tiles, choice, inverse):
 
 
 def permute(x: torch.Tensor, grid, tiles, choice: Optional[torch.Tensor] = None) -> torch.Tensor:
-    """Tile-contiguous order: y[b, h, p] = x[b, h, perm_c(p)] (c = choice[b*H+h] or 0)."""
+    """Tile-contiguous order: y[b, h, p] = x[b, h, perm_c(p)] (c = choice[b*H+h] or 0).
+    On a grid the tiles do not divide, y covers padded_grid(grid, tiles), with
+    zero rows at padding positions."""
     return _permute(x, grid, tiles, choice, False)
 
 
 def unpermute(y: torch.Tensor, grid, tiles, choice: Optional[torch.Tensor] = None) -> torch.Tensor:
-    """Inverse of permute: back to T-major order."""
+    """Inverse of permute: back to T-major order (padding rows dropped)."""
     return _permute(y, grid, tiles, choice, True)
 
 
@@ -221,13 +242,15 @@ def _choice_arg(choice, BH):
 
 
 def block_summaries_tiled(x: torch.Tensor, grid, tiles, choice: Optional[torch.Tensor], block: int):
-    """block_summaries(permute(x, grid, tiles, choice), block) read straight from T-major x."""
+    """block_summaries(permute(x, grid, tiles, choice), block) read straight from T-major x
+    (blocks of padded_grid(grid, tiles); padding positions count as zero rows)."""
     _cuda(x, "x")
     B, H, S, D = _bhsd(x, "x")
-    if block <= 0 or S % block:
-        raise ValueError(f"block ({block}) must divide S ({S})")
+    Sp = _grid_tokens(padded_grid(grid, tiles))
+    if block <= 0 or Sp % block:
+        raise ValueError(f"block ({block}) must divide the padded token count ({Sp})")
     arr, n = _tiles_arg(tiles)
-    xmax = torch.empty(B, H, S // block, D, dtype=x.dtype, device=x.device)
+    xmax = torch.empty(B, H, Sp // block, D, dtype=x.dtype, device=x.device)
     xmin = torch.empty_like(xmax)
     _check(lib().vsa_block_summaries_tiled(_ptr(x), _dtype_code(x, "x"), B, H, S, D, Dims3(*grid), arr, n,
                                            _choice_arg(choice, B * H), int(block), _ptr(xmax), _ptr(xmin),
@@ -419,6 +442,10 @@ def spade_attention(q, k, v, grid, tiles, budget: Optional[float] = None, topk: 
 
     Every candidate tile must have the same volume (the block size).  With a
     single candidate the tiling choice is skipped (choice 0 for every head).
+    A grid the candidates do not divide is zero-padded (padded_grid): the
+    padding holds no query of the cohesion, takes part in the summaries as
+    zero tokens and is masked as keys; the result holds the real tokens only.
+    Padded grids run in tiled mode, which masks the padding keys.
 
     tiled=True runs the permutation inside the summaries and attention kernels
     (no permuted copies; block size 128, see tiled_supported); tiled=False
@@ -432,13 +459,17 @@ def spade_attention(q, k, v, grid, tiles, budget: Optional[float] = None, topk: 
         raise ValueError("candidate tiles must share one volume (the block size)")
     block = vols.pop()
     B, H, S, D = _bhsd(q, "q")
-    nb = S // block
+    pgrid = padded_grid(grid, tiles)
+    nb = _grid_tokens(pgrid) // block
     kk = topk if topk is not None else topk_budget(nb, budget if budget is not None else 0.17)
     can_tile = block == 128 and tiled_supported(tiles)
     if tiled is None:
         tiled = can_tile
     elif tiled and not can_tile:
         raise ValueError("tiled mode needs 128-token blocks whose tiles satisfy tiled_supported()")
+    if not tiled and tuple(pgrid) != tuple(grid):
+        raise NotImplementedError(f"grid {tuple(grid)} is padded to {pgrid}: its padding keys are masked in "
+                                  "tiled mode only (128-token blocks, see tiled_supported)")
     choice = select_tiling(q, grid, tiles) if len(tiles) > 1 else None
     if tiled:
         qb, kb, vb = _bf16(q, "q"), _bf16(k, "k"), _bf16(v, "v")
@@ -459,7 +490,7 @@ def spade_attention(q, k, v, grid, tiles, budget: Optional[float] = None, topk: 
         o = unpermute(op, grid, tiles, choice)
     if return_intermediates:
         return o, dict(choice=choice, qp=qp, kp=kp, vp=vp, qmax=qmax, qmin=qmin, kmax=kmax, kmin=kmin,
-                       scores=scores, idx=idx, cnt=cnt, out_perm=op, block=block, k=kk)
+                       scores=scores, idx=idx, cnt=cnt, out_perm=op, block=block, k=kk, padded_grid=pgrid)
     return o
 
 

@@ -3,8 +3,9 @@
 //
 // Validation follows the pages' rules ("fastvideo/mlx_runtime/
 // windowed_attention.py": _validate_qkv, windowed_attention argument checks,
-// _default_scale; "Adaptive tiling (SPADE)", Deviations: divisible grids
-// only) and the limits of this implementation.
+// _default_scale; "Adaptive tiling (SPADE)", Deviations and notes: a grid
+// the candidates do not divide is zero-padded) and the limits of this
+// implementation.
 #include <stdarg.h>
 #include <stdio.h>
 
@@ -72,23 +73,39 @@ vsa_status check_grid(vsa_dims3 grid, int S) {
     return VSA_OK;
 }
 
-vsa_status check_tiles(vsa_dims3 grid, const vsa_dims3 *tiles, int n_tiles, TileSet *ts) {
+long long lcm_ll(long long a, long long b) {
+    long long x = a, y = b;
+    while (y) { const long long r = x % y; x = y; y = r; }
+    return a / x * b;
+}
+
+// Candidate tiles need not divide the grid: the grid is then zero-padded on
+// each axis to the next multiple of the candidates' lcm ("Adaptive tiling
+// (SPADE)", Deviations and notes); *padded receives that grid.
+vsa_status check_tiles(vsa_dims3 grid, const vsa_dims3 *tiles, int n_tiles, TileSet *ts, vsa_dims3 *padded = nullptr) {
     VSA_REQUIRE(tiles != nullptr, "tiles must not be NULL");
     VSA_REQUIRE(n_tiles >= 1 && n_tiles <= 8, "n_tiles must be in [1, 8], got %d", n_tiles);
     ts->n = n_tiles;
+    long long l[3] = {1, 1, 1};
     for (int c = 0; c < n_tiles; ++c) {
         const vsa_dims3 t = tiles[c];
         VSA_REQUIRE(t.t > 0 && t.h > 0 && t.w > 0, "tile %d must be positive, got (%d, %d, %d)", c, t.t, t.h, t.w);
-        VSA_REQUIRE(grid.t % t.t == 0 && grid.h % t.h == 0 && grid.w % t.w == 0,
-                    "tile %d (%d, %d, %d) does not divide the grid (%d, %d, %d)", c, t.t, t.h, t.w, grid.t,
-                    grid.h, grid.w);
         ts->t[c] = t.t;
         ts->h[c] = t.h;
         ts->w[c] = t.w;
+        l[0] = lcm_ll(l[0], t.t);
+        l[1] = lcm_ll(l[1], t.h);
+        l[2] = lcm_ll(l[2], t.w);
+        VSA_REQUIRE(l[0] <= (1 << 20) && l[1] <= (1 << 20) && l[2] <= (1 << 20), "the candidate tiles' lcm is too large");
     }
     for (int c = n_tiles; c < 8; ++c) ts->t[c] = ts->h[c] = ts->w[c] = 1;
+    const long long pt = (grid.t + l[0] - 1) / l[0] * l[0], ph = (grid.h + l[1] - 1) / l[1] * l[1],
+                    pw = (grid.w + l[2] - 1) / l[2] * l[2];
+    VSA_REQUIRE(pt * ph * pw <= 0x7fffffffLL, "the padded grid (%lld, %lld, %lld) has too many tokens", pt, ph, pw);
+    if (padded) *padded = vsa_dims3{static_cast<int32_t>(pt), static_cast<int32_t>(ph), static_cast<int32_t>(pw)};
     return VSA_OK;
 }
+
 
 vsa_status check_bhsd(int B, int n_heads, int S, int D) {
     VSA_REQUIRE(B >= 1 && n_heads >= 1, "B and n_heads must be >= 1, got %d, %d", B, n_heads);
@@ -123,6 +140,14 @@ extern "C" {
 
 const char *vsa_last_error(void) { return g_last_error.c_str(); }
 
+vsa_status vsa_padded_grid(vsa_dims3 grid, const vsa_dims3 *tiles, int n_tiles, vsa_dims3 *padded) {
+    VSA_REQUIRE(grid.t > 0 && grid.h > 0 && grid.w > 0, "grid dimensions must be positive, got (%d, %d, %d)",
+                grid.t, grid.h, grid.w);
+    VSA_REQUIRE(padded != nullptr, "padded must not be NULL");
+    TileSet ts;
+    return check_tiles(grid, tiles, n_tiles, &ts, padded);
+}
+
 vsa_status vsa_device_status(void *stream) {
     cudaError_t e = cudaStreamSynchronize(as_stream(stream));
     if (e != cudaSuccess) return check_cuda(e, "cudaStreamSynchronize");
@@ -140,11 +165,13 @@ vsa_status vsa_device_status(void *stream) {
 
 size_t vsa_select_tiling_workspace_size(int B, int n_heads, vsa_dims3 grid, const vsa_dims3 *tiles, int n_tiles) {
     TileSet ts;
+    vsa_dims3 pg;
     if (B < 1 || n_heads < 1 || grid.t < 1 || grid.h < 1 || grid.w < 1) return 0;
-    if (check_tiles(grid, tiles, n_tiles, &ts) != VSA_OK) return 0;
+    if (check_tiles(grid, tiles, n_tiles, &ts, &pg) != VSA_OK) return 0;
     SelectGeom g;
-    if (!select_geometry(grid.t, grid.h, grid.w, ts, &g)) return 0;
-    const size_t bytes = static_cast<size_t>(B) * n_heads * g.n_regions * n_tiles * sizeof(float);
+    if (!select_geometry(pg.t, pg.h, pg.w, ts, &g)) return 0;
+    // per region and candidate: a SICS sum and a tile count
+    const size_t bytes = static_cast<size_t>(B) * n_heads * g.n_regions * 2 * n_tiles * sizeof(float);
     return (bytes + 255) & ~static_cast<size_t>(255);
 }
 
@@ -159,18 +186,19 @@ vsa_status vsa_select_tiling(const void *q, vsa_dtype dtype, int B, int n_heads,
     VSA_REQUIRE(sics == nullptr || aligned4(sics), "sics must be NULL or 4-byte aligned");
     VSA_TRY(check_grid(grid, S));
     TileSet ts;
-    VSA_TRY(check_tiles(grid, tiles, n_tiles, &ts));
+    vsa_dims3 pg;
+    VSA_TRY(check_tiles(grid, tiles, n_tiles, &ts, &pg));
     SelectGeom g;
-    if (!select_geometry(grid.t, grid.h, grid.w, ts, &g))
+    if (!select_geometry(pg.t, pg.h, pg.w, ts, &g))
         return fail(VSA_ERR_UNSUPPORTED,
                     "the candidate tiles' lcm region holds %d cells of their gcd tile (at most 256 supported)",
                     g.cells);
     const size_t need = vsa_select_tiling_workspace_size(B, n_heads, grid, tiles, n_tiles);
     VSA_REQUIRE(aligned16(workspace), "workspace must be a non-NULL 16-byte aligned device pointer");
     VSA_REQUIRE(workspace_bytes >= need, "workspace holds %zu bytes, %zu needed", workspace_bytes, need);
-    return check_cuda(launch_select_tiling(q, esize_of(dtype), B * n_heads, S, D, grid.t, grid.h, grid.w, ts, g,
-                                           choice, sics, static_cast<float *>(workspace), status_or_null(),
-                                           as_stream(stream)),
+    return check_cuda(launch_select_tiling(q, esize_of(dtype), B * n_heads, D, grid.t, grid.h, grid.w, pg.t, pg.h,
+                                           pg.w, ts, g, choice, sics, static_cast<float *>(workspace),
+                                           status_or_null(), as_stream(stream)),
                       "select_tiling launch");
 }
 
@@ -185,9 +213,10 @@ vsa_status vsa_select_tiling_noalloc(const void *q, vsa_dtype dtype, int B, int 
     VSA_REQUIRE(sics == nullptr || aligned4(sics), "sics must be NULL or 4-byte aligned");
     VSA_TRY(check_grid(grid, S));
     TileSet ts;
-    VSA_TRY(check_tiles(grid, tiles, n_tiles, &ts));
+    vsa_dims3 pg;
+    VSA_TRY(check_tiles(grid, tiles, n_tiles, &ts, &pg));
     SelectGeom g;
-    if (!select_geometry(grid.t, grid.h, grid.w, ts, &g))
+    if (!select_geometry(pg.t, pg.h, pg.w, ts, &g))
         return fail(VSA_ERR_UNSUPPORTED,
                     "the candidate tiles' lcm region holds %d cells of their gcd tile (at most 256 supported)",
                     g.cells);
@@ -199,8 +228,8 @@ vsa_status vsa_select_tiling_noalloc(const void *q, vsa_dtype dtype, int B, int 
     float *scratch = nullptr;
     size_t scratch_bytes = 0;
     VSA_TRY(select_static_scratch(&scratch, &scratch_bytes));
-    return check_cuda(launch_select_tiling(q, esize_of(dtype), B * n_heads, S, D, grid.t, grid.h, grid.w, ts, g,
-                                           choice, sics, scratch, status_or_null(), as_stream(stream)),
+    return check_cuda(launch_select_tiling(q, esize_of(dtype), B * n_heads, D, grid.t, grid.h, grid.w, pg.t, pg.h,
+                                           pg.w, ts, g, choice, sics, scratch, status_or_null(), as_stream(stream)),
                       "select_tiling (no-alloc) launch");
 }
 
@@ -211,14 +240,18 @@ static vsa_status permute_common(const void *src, void *dst, vsa_dtype dtype, in
     VSA_TRY(check_bhsd(B, n_heads, S, D));
     VSA_TRY(check_d(D));
     VSA_REQUIRE(aligned16(src) && aligned16(dst), "x and y must be non-NULL 16-byte aligned device pointers");
-    const size_t bytes = static_cast<size_t>(B) * n_heads * S * D * esize_of(dtype);
-    VSA_REQUIRE(!overlaps(src, bytes, dst, bytes), "x and y must not overlap");
     VSA_REQUIRE(choice == nullptr || aligned4(choice), "choice must be NULL or 4-byte aligned");
     VSA_TRY(check_grid(grid, S));
     TileSet ts;
-    VSA_TRY(check_tiles(grid, tiles, n_tiles, &ts));
-    return check_cuda(launch_permute(src, dst, esize_of(dtype), B * n_heads, S, D, grid.t, grid.h, grid.w, ts,
-                                     choice, inverse, status_or_null(), as_stream(stream)),
+    vsa_dims3 pg;
+    VSA_TRY(check_tiles(grid, tiles, n_tiles, &ts, &pg));
+    const long long Sp = static_cast<long long>(pg.t) * pg.h * pg.w;
+    VSA_REQUIRE(static_cast<long long>(B) * n_heads * Sp <= 0x7fffffffLL, "B * n_heads * padded tokens too large");
+    const size_t row = static_cast<size_t>(D) * esize_of(dtype);
+    const size_t tbytes = static_cast<size_t>(B) * n_heads * S * row, pbytes = static_cast<size_t>(B) * n_heads * Sp * row;
+    VSA_REQUIRE(!overlaps(src, inverse ? pbytes : tbytes, dst, inverse ? tbytes : pbytes), "x and y must not overlap");
+    return check_cuda(launch_permute(src, dst, esize_of(dtype), B * n_heads, D, grid.t, grid.h, grid.w, pg.t, pg.h,
+                                     pg.w, ts, choice, inverse, status_or_null(), as_stream(stream)),
                       inverse ? "unpermute launch" : "permute launch");
 }
 
@@ -255,15 +288,20 @@ vsa_status vsa_block_summaries_tiled(const void *x, vsa_dtype dtype, int B, int 
     VSA_TRY(check_d(D));
     VSA_REQUIRE(block == 16 || block == 32 || block == 64 || block == 128 || block == 256,
                 "block must be one of 16, 32, 64, 128, 256, got %d", block);
-    VSA_REQUIRE(S % block == 0, "block (%d) must divide S (%d)", block, S);
     VSA_REQUIRE(aligned16(x) && aligned16(x_max) && aligned16(x_min),
                 "x, x_max and x_min must be non-NULL 16-byte aligned device pointers");
     VSA_REQUIRE(choice == nullptr || aligned4(choice), "choice must be NULL or 4-byte aligned");
     VSA_TRY(check_grid(grid, S));
     TileSet ts;
-    VSA_TRY(check_tiles(grid, tiles, n_tiles, &ts));
-    return check_cuda(launch_summaries_tiled(x, esize_of(dtype), B * n_heads, S, D, grid.t, grid.h, grid.w, ts,
-                                             choice, x_max, x_min, status_or_null(), as_stream(stream), block),
+    vsa_dims3 pg;
+    VSA_TRY(check_tiles(grid, tiles, n_tiles, &ts, &pg));
+    const long long Sp = static_cast<long long>(pg.t) * pg.h * pg.w;
+    VSA_REQUIRE(Sp % block == 0, "block (%d) must divide the padded token count (%lld)", block, Sp);
+    VSA_REQUIRE(Sp / block <= 0x7fffffffLL && static_cast<long long>(B) * n_heads <= 65535,
+                "too many blocks or heads");
+    return check_cuda(launch_summaries_tiled(x, esize_of(dtype), B * n_heads, D, grid.t, grid.h, grid.w, pg.t, pg.h,
+                                             pg.w, ts, choice, x_max, x_min, status_or_null(), as_stream(stream),
+                                             block),
                       "block_summaries_tiled launch");
 }
 
@@ -401,7 +439,9 @@ vsa_status vsa_block_sparse_attention_tiled(const void *q, const void *k, const 
     VSA_REQUIRE(choice == nullptr || aligned4(choice), "choice must be NULL or 4-byte aligned");
     VSA_TRY(check_grid(grid, S));
     TileSet ts;
-    VSA_TRY(check_tiles(grid, tiles, n_tiles, &ts));
+    vsa_dims3 pg;
+    VSA_TRY(check_tiles(grid, tiles, n_tiles, &ts, &pg));
+    const long long Sp = static_cast<long long>(pg.t) * pg.h * pg.w;
     const int vol = ts.t[0] * ts.h[0] * ts.w[0];
     VSA_REQUIRE(vol % 128 == 0, "tile volume (%d) must be a multiple of 128", vol);
     for (int c = 0; c < n_tiles; ++c) {
@@ -411,6 +451,10 @@ vsa_status vsa_block_sparse_attention_tiled(const void *q, const void *k, const 
                     "tile %d: tile.t (%d) must be divisible by volume / 128 (%d) so each 128-token block is whole "
                     "(h, w) planes",
                     c, ts.t[c], vol / 128);
+        // a TMA box (one 128-token block) must fit inside the real tensor
+        if (ts.t[c] / (vol / 128) > grid.t || ts.h[c] > grid.h || ts.w[c] > grid.w)
+            return fail(VSA_ERR_UNSUPPORTED, "tile %d: its 128-token box (%d, %d, %d) is larger than the grid (%d, %d, %d)",
+                        c, ts.t[c] / (vol / 128), ts.h[c], ts.w[c], grid.t, grid.h, grid.w);
     }
     AttnLaunch L{};
     L.q = q; L.k = k; L.v = v; L.o = o;
@@ -419,11 +463,12 @@ vsa_status vsa_block_sparse_attention_tiled(const void *q, const void *k, const 
     L.block = 128;
     L.window = false;
     L.idx = idx; L.cnt = cnt; L.cap = cap; L.list_per_head = list_per_head ? 1 : 0;
-    L.group = 0; L.nb = S / 128;
+    L.group = 0; L.nb = static_cast<int>(Sp / 128);
     L.scale = scale > 0.f ? scale : 1.0f / sqrtf(static_cast<float>(D));
     L.tiled = true;
     L.gstride = group_stride;
     L.T = grid.t; L.Hg = grid.h; L.Wg = grid.w;
+    L.Tp = pg.t; L.Hp = pg.h; L.Wp = pg.w;
     L.tiles = ts;
     L.choice = choice;
     return launch_attention(L, status_or_null(), as_stream(stream));

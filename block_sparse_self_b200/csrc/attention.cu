@@ -343,16 +343,16 @@ attn_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUt
                 if (!__all_sync(0xffffffffu, ok)) ok = false;
                 if (!ok) break;
                 const float m_use = m_ref == -INFINITY ? 0.f : m_ref;
-                float rs = 0.f;
+                // the row sum adds the bf16-rounded P that the PV MMA multiplies
+                float s0 = 0.f, s1 = 0.f;
                 #pragma unroll
-                for (int c = 0; c < BN; ++c) {
-                    const float p = ex2_approx(fmaf(x[c], sl2, -m_use));
-                    x[c] = p;
-                    rs += p;
+                for (int c = 0; c < BN; c += 2) {
+                    const uint32_t pk = pack_bf16x2(ex2_approx(fmaf(x[c], sl2, -m_use)),
+                                                    ex2_approx(fmaf(x[c + 1], sl2, -m_use)));
+                    raw[c >> 1] = pk;
+                    add_bf16x2_f32(pk, s0, s1);
                 }
-                l_sum += rs;
-                #pragma unroll
-                for (int c = 0; c < BN; c += 2) raw[c >> 1] = pack_bf16x2(x[c], x[c + 1]);
+                l_sum += s0 + s1;
             } else {
                 #pragma unroll
                 for (int c = 0; c < BN / 2; ++c) raw[c] = 0u;

@@ -22,6 +22,12 @@
 // QK_t(j+1), which overwrites the P_t(j) that PV_t(j) reads, first waits for
 // PV_t(j) to complete.
 //
+// Tiled mode on a zero-padded grid ("Adaptive tiling (SPADE)", Deviations
+// and notes): block lists count blocks of the padded grid, the TMA boxes read
+// the real tensors and fill the part past their edge with zeros, keys there
+// are masked in the blocks that cross the edge, rows there are not written,
+// and query tiles wholly past the edge are skipped.
+//
 // Softmax: after a row's first visible block the exponentials use the running
 // row max without taking the block's max at all; only if the block's P would
 // sum above 2^24 (the max grew, rare) is the running max raised, O and l
@@ -36,7 +42,8 @@ namespace vsa {
 namespace {
 
 struct PPArgs {
-    int S, nq;
+    int S, nq;        // positions per head (tiled mode: of the padded grid), query tiles
+    int S_out;        // rows per head of o (tiled mode: real tokens)
     const int32_t *idx, *cnt;
     int cap, list_per_head, group, nb;
     int gstride;  // > 1: keys share a row's group iff their positions agree with it mod gstride (a power of two)
@@ -46,11 +53,14 @@ struct PPArgs {
     int out_f32;
     int *status;
     // tiled mode: T-major tensors, per-head tiling (all of volume 128 * m)
-    int H, W;
+    int H, W;         // the padded grid's frame (equal to the real one when nothing is padded)
+    int padded;
+    RealGrid real;
     TileSet tiles;
     const int32_t *choice;
     struct BoxGeom {
         FastDiv m, nthw, ntw;  // m = volume / 128, tiles per frame, tiles per tile row
+        FastDiv bhw, bw;       // box frame (th * tw) and row (tw): key column -> (dt, dh, dw)
         int bt;                // frames of one 128-token box: tile.t / m
     } geom[kMaxTiles];
 };
@@ -238,6 +248,18 @@ attn_pp_kernel(const __grid_constant__ MapSet maps, const PPArgs a) {
         }
     }
     const int tt = a.tiles.t[tc], th = a.tiles.h[tc], tw = a.tiles.w[tc];
+    if constexpr (TILED) {
+        if (a.padded) {  // a query box wholly in the padding has no row to write
+            for (int t = 0; t < 2; ++t) {
+                if (ts[t].qt < 0) continue;
+                const BoxCoord c = box_of(static_cast<uint32_t>(ts[t].qt), a.geom[tc], th, tw);
+                if (c.t >= a.real.T || c.h >= a.real.H || c.w >= a.real.W) {
+                    ts[t].qt = -1;
+                    ts[t].n = 0;
+                }
+            }
+        }
+    }
     const CUtensorMap *tmQ = &maps.q[tc], *tmK = &maps.k[tc], *tmV = &maps.v[tc];
     // one 128-row tile of Q, K or V: block b of this head
     auto load_tile = [&](uint8_t *dst, const CUtensorMap *map, uint64_t *bar, int b) {
@@ -372,9 +394,16 @@ attn_pp_kernel(const __grid_constant__ MapSet maps, const PPArgs a) {
         const int n = sc.n;
         const int q0 = (sc.qt < 0 ? 0 : sc.qt) * BN;
         const int rg = q0 + row;
-        const bool row_valid = sc.qt >= 0 && rg < S;
+        bool row_valid = sc.qt >= 0 && rg < S;
         // output row: the permuted position itself, or its T-major token in tiled mode
-        const uint32_t orow_in_head = TILED ? tile_token(rg, a.H, a.W, tt, th, tw) : rg;
+        uint32_t orow_in_head = rg;
+        if constexpr (TILED) {
+            int pt, ph, pw;
+            tile_coords(rg, a.H, a.W, tt, th, tw, pt, ph, pw);
+            const int tok = real_token(pt, ph, pw, a.real);
+            row_valid = row_valid && tok >= 0;
+            orow_in_head = tok < 0 ? 0u : static_cast<uint32_t>(tok);
+        }
         const uint32_t t_lane = tmem + (static_cast<uint32_t>(wq * 32) << 16);
         const uint32_t s_col = t * 128, o_col = C::O_COL + t * D;
         const float sl2 = a.scale_log2;
@@ -388,6 +417,28 @@ attn_pp_kernel(const __grid_constant__ MapSet maps, const PPArgs a) {
             for (int c = 0; c < BN / 32; ++c)
                 tmem_ld32(t_lane + s_col + 32 * c, *reinterpret_cast<uint32_t(*)[32]>(&x[32 * c]));
             tmem_ld_wait();
+            // padded grid: which of the key block's 128 columns are real tokens
+            // (column u * 32 + lane in bit lane of kv[u]); all ones off the edge
+            uint32_t kv[4] = {~0u, ~0u, ~0u, ~0u};
+            bool key_edge = false;
+            if constexpr (TILED) {
+                if (a.padded) {
+                    const PPArgs::BoxGeom &g = a.geom[tc];
+                    const BoxCoord c = box_of(static_cast<uint32_t>(kblock_of<WINDOW>(sc, j)), g, th, tw);
+                    key_edge = c.t + g.bt > a.real.T || c.h + th > a.real.H || c.w + tw > a.real.W;
+                    if (key_edge) {
+                        #pragma unroll
+                        for (int u = 0; u < 4; ++u) {
+                            const uint32_t col = static_cast<uint32_t>(u * 32 + lane);
+                            const uint32_t dt = fdiv(col, g.bhw), r2 = col - dt * g.bhw.d;
+                            const uint32_t dh = fdiv(r2, g.bw), dw = r2 - dh * g.bw.d;
+                            kv[u] = __ballot_sync(0xffffffffu, c.t + static_cast<int>(dt) < a.real.T &&
+                                                                   c.h + static_cast<int>(dh) < a.real.H &&
+                                                                   c.w + static_cast<int>(dw) < a.real.W);
+                        }
+                    }
+                }
+            }
             auto apply_mask = [&]() {
                 if constexpr (WINDOW) {
                     const int ks = kblock_of<WINDOW>(sc, j) * BN;
@@ -419,29 +470,35 @@ attn_pp_kernel(const __grid_constant__ MapSet maps, const PPArgs a) {
                         for (int c = 0; c < BN; ++c)
                             if ((c & (a.gstride - 1)) != r0) x[c] = __float_as_uint(-INFINITY);
                     }
+                    if (key_edge) {
+                        #pragma unroll
+                        for (int c = 0; c < BN; ++c)
+                            if (!((kv[c >> 5] >> (c & 31)) & 1u)) x[c] = __float_as_uint(-INFINITY);
+                    }
                 }
             };
             apply_mask();
             // P = 2^(scale*log2e*S - m_use) in place (bf16 pairs), returns the row sum
-            // The arguments and the row sum use two-wide fp32 instructions: the
-            // exponentials are bound by the exponential unit, and fewer issue
-            // slots here leave more to the other tile's warp on the sub-partition.
+            // The arguments use two-wide fp32 instructions: the exponentials are
+            // bound by the exponential unit, and fewer issue slots here leave more
+            // to the other tile's warp on the sub-partition.  The row sum adds the
+            // bf16-rounded P that the PV MMA multiplies, so O / l is a convex
+            // combination of V rows: a row held by a few keys then carries no
+            // rounding error in its weights' total (measured cost: about 2 % of
+            // the kernel's time, against 4.5 % for unpacking each pair first).
             auto exp_pass = [&](float m_use) -> float {
                 const uint64_t sl2x2 = f32x2(sl2, sl2), nmx2 = f32x2(-m_use, -m_use);
-                uint64_t acc[2] = {f32x2(0.f, 0.f), f32x2(0.f, 0.f)};
+                float s0 = 0.f, s1 = 0.f, s2 = 0.f, s3 = 0.f;
                 #pragma unroll
                 for (int q = 0; q < BN / 2; ++q) {
                     float a0, a1;
                     f32x2_split(fma_f32x2(f32x2(__uint_as_float(x[2 * q]), __uint_as_float(x[2 * q + 1])), sl2x2, nmx2),
                                 a0, a1);
-                    const float p0 = ex2_approx(a0);
-                    const float p1 = ex2_approx(a1);
-                    acc[q & 1] = add_f32x2(acc[q & 1], f32x2(p0, p1));
-                    x[q] = pack_bf16x2(p0, p1);   // P, packed in place (q <= 2q)
+                    const uint32_t pk = pack_bf16x2(ex2_approx(a0), ex2_approx(a1));
+                    if (q & 1) add_bf16x2_f32(pk, s2, s3);
+                    else add_bf16x2_f32(pk, s0, s1);
+                    x[q] = pk;   // P, packed in place (q <= 2q)
                 }
-                float s0, s1, s2, s3;
-                f32x2_split(acc[0], s0, s1);
-                f32x2_split(acc[1], s2, s3);
                 return (s0 + s2) + (s1 + s3);
             };
             auto raw_max = [&]() -> float {
@@ -506,7 +563,7 @@ attn_pp_kernel(const __grid_constant__ MapSet maps, const PPArgs a) {
         if (!ok && !*abort_flag) { report(a.status, DEV_TIMEOUT); *abort_flag = 1; }
 
         // ---- epilogue: O / l -> global ----
-        const size_t orow = static_cast<size_t>(bh) * S + orow_in_head;
+        const size_t orow = static_cast<size_t>(bh) * a.S_out + orow_in_head;
         bool have_o = ok && n > 0;
         if (have_o && !__all_sync(0xffffffffu, mbar_wait(&pv_done[t], (n - 1) & 1, abort_flag))) {
             have_o = false;
@@ -569,6 +626,7 @@ vsa_status run_pp(const AttnLaunch &L, int *status, cudaStream_t st) {
         for (int c = 0; c < L.tiles.n; ++c) {
             const int m = L.tiles.t[c] * L.tiles.h[c] * L.tiles.w[c] / 128;
             const int bt = L.tiles.t[c] / m, bhh = L.tiles.h[c], bw = L.tiles.w[c];
+            // the real tensors: boxes reaching past them read zeros
             ok = ok && make_box_map(&maps.q[c], L.q, D, L.T, L.Hg, L.Wg, L.BH, bt, bhh, bw) &&
                  make_box_map(&maps.k[c], L.k, D, L.T, L.Hg, L.Wg, L.BH, bt, bhh, bw) &&
                  make_box_map(&maps.v[c], L.v, D, L.T, L.Hg, L.Wg, L.BH, bt, bhh, bw);
@@ -582,8 +640,10 @@ vsa_status run_pp(const AttnLaunch &L, int *status, cudaStream_t st) {
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
     if (e != cudaSuccess) return check_cuda(e, "cudaFuncSetAttribute(attention, two tiles)");
     PPArgs a;
-    a.S = L.S;
-    a.nq = (L.S + 127) / 128;
+    const int positions = TILED ? L.Tp * L.Hp * L.Wp : L.S;
+    a.S = positions;
+    a.S_out = L.S;
+    a.nq = (positions + 127) / 128;
     a.idx = L.idx;
     a.cnt = L.cnt;
     a.cap = L.cap;
@@ -598,8 +658,10 @@ vsa_status run_pp(const AttnLaunch &L, int *status, cudaStream_t st) {
     a.out = L.o;
     a.out_f32 = L.out_f32;
     a.status = status;
-    a.H = L.Hg;
-    a.W = L.Wg;
+    a.H = TILED ? L.Hp : L.Hg;
+    a.W = TILED ? L.Wp : L.Wg;
+    a.padded = TILED && positions != L.S;
+    a.real = RealGrid{L.T, L.Hg, L.Wg};
     a.tiles = L.tiles;
     a.choice = L.choice;
     if (!TILED) a.tiles.n = 1;
@@ -609,11 +671,13 @@ vsa_status run_pp(const AttnLaunch &L, int *status, cudaStream_t st) {
             const int tt = L.tiles.t[c], th = L.tiles.h[c], tw = L.tiles.w[c];
             const int m = tt * th * tw / 128;
             g.m = make_fastdiv(m);
-            g.nthw = make_fastdiv((L.Hg / th) * (L.Wg / tw));
-            g.ntw = make_fastdiv(L.Wg / tw);
+            g.nthw = make_fastdiv((L.Hp / th) * (L.Wp / tw));
+            g.ntw = make_fastdiv(L.Wp / tw);
+            g.bhw = make_fastdiv(th * tw);
+            g.bw = make_fastdiv(tw);
             g.bt = tt / m;
         } else {
-            g.m = g.nthw = g.ntw = make_fastdiv(1);
+            g.m = g.nthw = g.ntw = g.bhw = g.bw = make_fastdiv(1);
             g.bt = 1;
         }
     }

@@ -160,7 +160,8 @@ __device__ __forceinline__ uint32_t fdiv(uint32_t n, const FastDiv &f) {
 // Recipe): position p holds the T-major token tile_token(p).  Tiles come in
 // row-major tile order, the tokens of a tile in T-major order.
 // ---------------------------------------------------------------------------
-__device__ __forceinline__ int tile_token(int p, int H, int W, int tt, int th, int tw) {
+// (t, h, w) of position p in a grid of H x W frames (every axis a multiple of the tile's)
+__device__ __forceinline__ void tile_coords(int p, int H, int W, int tt, int th, int tw, int &t, int &h, int &w) {
     const int vol = tt * th * tw;
     const int tile = p / vol, r = p - tile * vol;
     const int nth = H / th, ntw = W / tw;
@@ -170,7 +171,15 @@ __device__ __forceinline__ int tile_token(int p, int H, int W, int tt, int th, i
     const int dt = r / (th * tw);
     const int r2 = r - dt * (th * tw);
     const int dh = r2 / tw, dw = r2 - dh * tw;
-    return ((ct * tt + dt) * H + ch * th + dh) * W + cw * tw + dw;
+    t = ct * tt + dt;
+    h = ch * th + dh;
+    w = cw * tw + dw;
+}
+
+__device__ __forceinline__ int tile_token(int p, int H, int W, int tt, int th, int tw) {
+    int t, h, w;
+    tile_coords(p, H, W, tt, th, tw, t, h, w);
+    return (t * H + h) * W + w;
 }
 
 // tile_token with every division by a per-tiling constant done as a
@@ -194,13 +203,34 @@ inline TileDivs make_tile_divs(int H, int W, int tt, int th, int tw) {
     return d;
 }
 
-__device__ __forceinline__ uint32_t tile_token_fast(uint32_t p, const TileDivs &d) {
+__device__ __forceinline__ void tile_coords_fast(uint32_t p, const TileDivs &d, uint32_t &t, uint32_t &h,
+                                                 uint32_t &w) {
     const uint32_t tile = fdiv(p, d.vol), r = p - tile * d.vol.d;
     const uint32_t ct = fdiv(tile, d.nthw), rem = tile - ct * d.nthw.d;
     const uint32_t ch = fdiv(rem, d.ntw), cw = rem - ch * d.ntw.d;
     const uint32_t dt = fdiv(r, d.thw), r2 = r - dt * d.thw.d;
     const uint32_t dh = fdiv(r2, d.tw), dw = r2 - dh * d.tw.d;
-    return ((ct * d.tt + dt) * d.H + ch * d.th + dh) * d.W + cw * d.tw.d + dw;
+    t = ct * d.tt + dt;
+    h = ch * d.th + dh;
+    w = cw * d.tw.d + dw;
+}
+
+__device__ __forceinline__ uint32_t tile_token_fast(uint32_t p, const TileDivs &d) {
+    uint32_t t, h, w;
+    tile_coords_fast(p, d, t, h, w);
+    return (t * d.H + h) * d.W + w;
+}
+
+// A grid that the candidate tiles do not divide is zero-padded on each axis
+// ("Adaptive tiling (SPADE)", Deviations and notes): positions and tilings
+// refer to the padded grid (tile_coords over it), tensors hold only the real
+// (T, H, W) tokens.  The real token at padded coordinates, or -1 for padding.
+struct RealGrid {
+    int T, H, W;
+};
+__device__ __forceinline__ int real_token(uint32_t t, uint32_t h, uint32_t w, const RealGrid &g) {
+    if (t >= static_cast<uint32_t>(g.T) || h >= static_cast<uint32_t>(g.H) || w >= static_cast<uint32_t>(g.W)) return -1;
+    return static_cast<int>((t * g.H + h) * g.W + w);
 }
 
 // ---------------------------------------------------------------------------
@@ -365,6 +395,16 @@ __device__ __forceinline__ void named_barrier(int id, int count) {
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
     __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
     return *reinterpret_cast<uint32_t *>(&v);
+}
+
+// acc_lo += low bf16 of pk, acc_hi += high bf16 of pk: sm_100 mixed-precision
+// adds (the bf16 operand widens exactly, then one fp32 rounding), with no
+// separate unpacking of the pair.
+__device__ __forceinline__ void add_bf16x2_f32(uint32_t pk, float &acc_lo, float &acc_hi) {
+    asm("{\n\t.reg .b16 lo, hi;\n\tmov.b32 {lo, hi}, %2;\n\t"
+        "add.rn.f32.bf16 %0, lo, %0;\n\tadd.rn.f32.bf16 %1, hi, %1;\n\t}"
+        : "+f"(acc_lo), "+f"(acc_hi)
+        : "r"(pk));
 }
 
 }  // namespace vsa

@@ -23,16 +23,19 @@ struct TileSet {
 };
 
 // Launchers (arguments already validated by the C ABI layer).
-cudaError_t launch_permute(const void *src, void *dst, int esize, int BH, int S, int D, int T, int H, int W,
-                           const TileSet &tiles, const int32_t *choice, bool inverse, int *status,
+// (T, H, W): the real grid (T-major side); (Tp, Hp, Wp): the grid the tiles
+// cut, equal to it or zero-padded (permuted side).
+cudaError_t launch_permute(const void *src, void *dst, int esize, int BH, int D, int T, int H, int W, int Tp, int Hp,
+                           int Wp, const TileSet &tiles, const int32_t *choice, bool inverse, int *status,
                            cudaStream_t st);
 cudaError_t launch_cast_f32_bf16(const float *x, void *y, int64_t n, cudaStream_t st);
 cudaError_t launch_summaries(const void *x, int esize, int BH, int S, int D, int block, void *xmax, void *xmin,
                              cudaStream_t st);
 // Summaries of the blocks of a T-major x taken in each head's tile-contiguous order.
-cudaError_t launch_summaries_tiled(const void *x, int esize, int BH, int S, int D, int T, int H, int W,
-                                   const TileSet &tiles, const int32_t *choice, void *xmax, void *xmin, int *status,
-                                   cudaStream_t st, int block);
+// (T, H, W) real grid, (Tp, Hp, Wp) padded grid: padding rows are zero vectors.
+cudaError_t launch_summaries_tiled(const void *x, int esize, int BH, int D, int T, int H, int W, int Tp, int Hp,
+                                   int Wp, const TileSet &tiles, const int32_t *choice, void *xmax, void *xmin,
+                                   int *status, cudaStream_t st, int block);
 cudaError_t launch_scores(const void *qmax, const void *qmin, const void *kmax, const void *kmin, int esize, int BH,
                           int nb, int D, float *scores, cudaStream_t st);
 // bf16 summaries on tcgen05 (D in {64, 128})
@@ -46,11 +49,14 @@ cudaError_t launch_structured(int T, int H, int W, int tt, int th, int tw, int r
 struct SelectGeom {
     int Rt, Rh, Rw;   // region = per-axis lcm of the candidate tiles
     int Ct, Ch, Cw;   // cell = per-axis gcd of the candidate tiles
-    int n_regions;    // regions per (b, head)
+    int n_regions;    // regions per (b, head) of the padded grid
     int cells;        // cells per region
 };
-bool select_geometry(int T, int H, int W, const TileSet &tiles, SelectGeom *g);
-cudaError_t launch_select_tiling(const void *q, int esize, int BH, int S, int D, int T, int H, int W,
+// (Tp, Hp, Wp): the padded grid (every axis a multiple of the region's).
+bool select_geometry(int Tp, int Hp, int Wp, const TileSet &tiles, SelectGeom *g);
+// Per region and candidate: the sum of SICS over its tiles that hold a non-zero
+// query, and the number of such tiles (two floats each).
+cudaError_t launch_select_tiling(const void *q, int esize, int BH, int D, int T, int H, int W, int Tp, int Hp, int Wp,
                                  const TileSet &tiles, const SelectGeom &g, int32_t *choice, float *sics,
                                  float *partial, int *status, cudaStream_t st);
 
@@ -71,7 +77,8 @@ struct AttnLaunch {
     // tiling and the kernel permutes through its TMA boxes and epilogue
     bool tiled;
     int gstride;  // tiled mode: strided groups (0 = none)
-    int T, Hg, Wg;
+    int T, Hg, Wg;      // tiled mode: the real grid (S = T * Hg * Wg tokens in q, k, v, o)
+    int Tp, Hp, Wp;     // tiled mode: the padded grid the tiles cut (block lists over its positions)
     TileSet tiles;
     const int32_t *choice;
 };

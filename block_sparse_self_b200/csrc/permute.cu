@@ -7,7 +7,9 @@
 // Position p of the tile-contiguous order holds token perm(p): tiles in
 // row-major tile order, tokens of a tile in T-major order.  perm is computed
 // arithmetically from (grid, tile); the chosen tiling of each (b, head) is
-// read on the device.
+// read on the device.  On a zero-padded grid ("Adaptive tiling (SPADE)",
+// Deviations and notes) the permuted order covers the padded grid: padding
+// positions are written as zero rows, and going back writes real tokens only.
 #include "common.cuh"
 #include "internal.h"
 
@@ -18,9 +20,11 @@ namespace {
 struct PermArgs {
     const uint8_t *src;
     uint8_t *dst;
-    int S, T, H, W, BH;
+    int S, Sp, BH;             // tokens per head: real (T-major side), padded (permuted side)
+    RealGrid real;
+    int padded;                // Sp != S
     TileSet tiles;
-    TileDivs divs[kMaxTiles];  // per candidate tiling
+    TileDivs divs[kMaxTiles];  // per candidate tiling, over the padded grid
     const int32_t *choice;
     int inverse;
     int *status;
@@ -35,7 +39,7 @@ template <int CPR>
 __global__ void __launch_bounds__(kThreads) permute_kernel(const PermArgs a) {
     constexpr int RPP = kThreads / CPR;  // rows per pass
     constexpr int UNROLL = 4;
-    const int items_per_head = (a.S + kRowsPerItem - 1) / kRowsPerItem;
+    const int items_per_head = (a.Sp + kRowsPerItem - 1) / kRowsPerItem;
     const long long n_items = static_cast<long long>(items_per_head) * a.BH;
     const int chunk = threadIdx.x % CPR;
     const int rsub = threadIdx.x / CPR;
@@ -51,7 +55,7 @@ __global__ void __launch_bounds__(kThreads) permute_kernel(const PermArgs a) {
             }
         }
         const TileDivs dv = a.divs[c];
-        const size_t head = static_cast<size_t>(bh) * a.S;
+        const size_t head_t = static_cast<size_t>(bh) * a.S, head_p = static_cast<size_t>(bh) * a.Sp;
         const uint4 *src = reinterpret_cast<const uint4 *>(a.src);
         uint4 *dst = reinterpret_cast<uint4 *>(a.dst);
         #pragma unroll 1
@@ -62,12 +66,24 @@ __global__ void __launch_bounds__(kThreads) permute_kernel(const PermArgs a) {
             #pragma unroll
             for (int u = 0; u < UNROLL; ++u) {
                 const int p = p0 + r0 + u * RPP + rsub;
-                ok[u] = (r0 + u * RPP + rsub) < kRowsPerItem && p < a.S;
+                ok[u] = (r0 + u * RPP + rsub) < kRowsPerItem && p < a.Sp;
                 if (ok[u]) {
-                    const int tok = static_cast<int>(tile_token_fast(static_cast<uint32_t>(p), dv));
-                    const size_t srow = head + (a.inverse ? p : tok);
-                    drow[u] = head + (a.inverse ? tok : p);
-                    v[u] = __ldcs(src + srow * CPR + chunk);
+                    int tok;
+                    if (a.padded) {
+                        uint32_t t, h, w;
+                        tile_coords_fast(static_cast<uint32_t>(p), dv, t, h, w);
+                        tok = real_token(t, h, w, a.real);
+                    } else {
+                        tok = static_cast<int>(tile_token_fast(static_cast<uint32_t>(p), dv));
+                    }
+                    if (a.inverse) {  // padding positions have no token to go back to
+                        ok[u] = tok >= 0;
+                        drow[u] = head_t + tok;
+                        if (ok[u]) v[u] = __ldcs(src + (head_p + p) * CPR + chunk);
+                    } else {          // padding positions become zero rows
+                        drow[u] = head_p + p;
+                        v[u] = tok >= 0 ? __ldcs(src + (head_t + tok) * CPR + chunk) : make_uint4(0u, 0u, 0u, 0u);
+                    }
                 }
             }
             #pragma unroll
@@ -110,21 +126,25 @@ int sm_count() {
 
 }  // namespace
 
-cudaError_t launch_permute(const void *src, void *dst, int esize, int BH, int S, int D, int T, int H, int W,
-                           const TileSet &tiles, const int32_t *choice, bool inverse, int *status,
+cudaError_t launch_permute(const void *src, void *dst, int esize, int BH, int D, int T, int H, int W, int Tp, int Hp,
+                           int Wp, const TileSet &tiles, const int32_t *choice, bool inverse, int *status,
                            cudaStream_t st) {
     PermArgs a;
     a.src = static_cast<const uint8_t *>(src);
     a.dst = static_cast<uint8_t *>(dst);
-    a.S = S; a.T = T; a.H = H; a.W = W; a.BH = BH;
+    a.S = T * H * W;
+    a.Sp = Tp * Hp * Wp;
+    a.real = RealGrid{T, H, W};
+    a.padded = a.Sp != a.S;
+    a.BH = BH;
     a.tiles = tiles;
     for (int c = 0; c < kMaxTiles; ++c)
-        a.divs[c] = c < tiles.n ? make_tile_divs(H, W, tiles.t[c], tiles.h[c], tiles.w[c]) : make_tile_divs(1, 1, 1, 1, 1);
+        a.divs[c] = c < tiles.n ? make_tile_divs(Hp, Wp, tiles.t[c], tiles.h[c], tiles.w[c]) : make_tile_divs(1, 1, 1, 1, 1);
     a.choice = choice;
     a.inverse = inverse ? 1 : 0;
     a.status = status;
     const int cpr = D * esize / 16;
-    const long long items = static_cast<long long>((S + kRowsPerItem - 1) / kRowsPerItem) * BH;
+    const long long items = static_cast<long long>((a.Sp + kRowsPerItem - 1) / kRowsPerItem) * BH;
     const int grid = static_cast<int>(items < 16LL * sm_count() ? items : 16LL * sm_count());
     switch (cpr) {
         case 8: permute_kernel<8><<<grid, kThreads, 0, st>>>(a); break;

@@ -14,6 +14,13 @@
 // and turns the norm into the tile's SICS; it writes per-candidate sums of
 // tile SICS for its region.  Pass 2: one warp per bh adds the regions in a
 // fixed order, divides by the tile count and takes the argmax.
+//
+// A grid the candidates do not divide is zero-padded per axis to a multiple of
+// the region ("Adaptive tiling (SPADE)", Deviations and notes).  Padding
+// tokens have zero norm, so they are never loaded: cells past the real grid
+// are skipped and cells across its edge test each token.  The mean is taken
+// over the tiles that hold at least one non-zero query, so every region
+// reports its SICS sum and the number of such tiles.
 #include <mutex>
 
 #include "common.cuh"
@@ -32,17 +39,17 @@ int lcm(int a, int b) { return a / gcd(a, b) * b; }
 
 struct SelArgs {
     const uint8_t *q;
-    int S, H, W, D, esize;
+    int S, T, H, W, D, esize;  // S = T * H * W real tokens per head
     TileSet tiles;
     int Rt, Rh, Rw, Ct, Ch, Cw;
-    int nrt, nrh, nrw;  // regions per axis
+    int nrt, nrh, nrw;  // regions per axis of the padded grid
     int cells, items;
     FastDiv cell_hw, cell_w;  // Ch * Cw and Cw: token of a cell -> (dt, dh, dw)
     int nch, ncw;             // cells of a region along h and w
     int tpr_t[kMaxTiles], tpr_h[kMaxTiles], tpr_w[kMaxTiles];  // candidate c: its tiles per region axis
     int cpt_t[kMaxTiles], cpt_h[kMaxTiles], cpt_w[kMaxTiles];  // candidate c: cells per tile axis
     int item_first[kMaxTiles + 1];                             // candidate c's first item in a region
-    float *partial;     // [BH][n_regions][tiles.n]
+    float *partial;     // [BH][n_regions][2][tiles.n]: SICS sums, then counts of tiles with a query
 };
 
 // LPT lanes share a query row; each lane takes CPL of the row's 16-byte chunks,
@@ -58,7 +65,8 @@ __global__ void __launch_bounds__(kThreads) sics_partial_kernel(const SelArgs a)
     float *cell_sum = sm;                               // [cells][D]
     float *cell_cnt = cell_sum + a.cells * a.D;         // [cells]
     float *tile_val = cell_cnt + a.cells;               // [items]
-    int *cell_off = reinterpret_cast<int *>(tile_val + a.items);  // [cvol]: token offset inside a cell
+    float *tile_used = tile_val + a.items;              // [items]: 1 if the tile holds a non-zero query
+    int *cell_off = reinterpret_cast<int *>(tile_used + a.items);  // [cvol]: token offset inside a cell
     const int region = blockIdx.x, bh = blockIdx.y;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int lt = lane % LPT;
@@ -80,6 +88,11 @@ __global__ void __launch_bounds__(kThreads) sics_partial_kernel(const SelArgs a)
     for (int cell = warp; cell < a.cells; cell += kWarps) {
         const int ct = cell / (nch * ncw), ch = (cell / ncw) % nch, cw = cell % ncw;
         const int tb = t0 + ct * a.Ct, hb = h0 + ch * a.Ch, wb = w0 + cw * a.Cw;
+        // padded grids: a cell wholly past the real grid holds only zero tokens
+        // (no loads), one across its edge tests each token (warp-uniform flags)
+        const bool outside = tb >= a.T || hb >= a.H || wb >= a.W;
+        const bool interior = tb + a.Ct <= a.T && hb + a.Ch <= a.H && wb + a.Cw <= a.W;
+        const int n_tok = outside ? 0 : cvol;
         float acc[EPL];
         #pragma unroll
         for (int e = 0; e < EPL; ++e) acc[e] = 0.f;
@@ -89,12 +102,18 @@ __global__ void __launch_bounds__(kThreads) sics_partial_kernel(const SelArgs a)
         // NB passes' loads are issued before any of them is used
         constexpr int NB = sizeof(T) == 2 ? 4 : 2;
         #pragma unroll 1
-        for (int tok_b = 0; tok_b < cvol; tok_b += NB * TPI) {  // uniform trip count: shuffles below
+        for (int tok_b = 0; tok_b < n_tok; tok_b += NB * TPI) {  // uniform trip count: shuffles below
             uint4 raw[NB][CPL];
             #pragma unroll
             for (int pb = 0; pb < NB; ++pb) {
                 const int tok = tok_b + pb * TPI + lane / LPT;
-                const bool valid = tok < cvol;
+                bool valid = tok < cvol;
+                if (!interior && valid) {
+                    const int dt = static_cast<int>(fdiv(static_cast<uint32_t>(tok), a.cell_hw));
+                    const int r2 = tok - dt * (a.Ch * a.Cw);
+                    const int dh = static_cast<int>(fdiv(static_cast<uint32_t>(r2), a.cell_w)), dw = r2 - dh * a.Cw;
+                    valid = tb + dt < a.T && hb + dh < a.H && wb + dw < a.W;
+                }
                 const uint4 *row = cell_q + static_cast<size_t>(cell_off[valid ? tok : 0]) * CPR;
                 #pragma unroll
                 for (int u = 0; u < CPL; ++u)
@@ -185,24 +204,31 @@ __global__ void __launch_bounds__(kThreads) sics_partial_kernel(const SelArgs a)
                         }
                     #pragma unroll
                     for (int off = 16; off > 0; off >>= 1) sq += __shfl_down_sync(0xffffffffu, sq, off);
-                    if (lane == 0) tile_val[item] = m >= 2.f ? (sq - m) / (m * (m - 1.f)) : 0.f;
+                    if (lane == 0) {
+                        tile_val[item] = m >= 2.f ? (sq - m) / (m * (m - 1.f)) : 0.f;
+                        tile_used[item] = m >= 1.f ? 1.f : 0.f;
+                    }
                 }
     }
     __syncthreads();
     if (threadIdx.x < a.tiles.n) {
         const int c = threadIdx.x;
         const int first = a.item_first[c], n = a.item_first[c + 1] - first;
-        float s = 0.f;
-        for (int i = 0; i < n; ++i) s += tile_val[first + i];
+        float s = 0.f, used = 0.f;
+        for (int i = 0; i < n; ++i) {
+            s += tile_val[first + i];
+            used += tile_used[first + i];
+        }
         const int n_regions = a.nrt * a.nrh * a.nrw;
-        a.partial[(static_cast<size_t>(bh) * n_regions + region) * a.tiles.n + c] = s;
+        float *out = a.partial + (static_cast<size_t>(bh) * n_regions + region) * 2 * a.tiles.n;
+        out[c] = s;
+        out[a.tiles.n + c] = used;
     }
 }
 
 struct FinalArgs {
     const float *partial;
     int BH, n_regions, n_tiles;
-    float tiles_total[8];  // tiles of candidate c over the whole grid
     int32_t *choice;
     float *sics;
 };
@@ -214,13 +240,20 @@ __global__ void sics_final_kernel(const FinalArgs a) {
     float best = 0.f;
     int best_c = 0;
     for (int c = 0; c < a.n_tiles; ++c) {
-        float s = 0.f;
-        for (int r = lane; r < a.n_regions; r += 32)
-            s += a.partial[(static_cast<size_t>(bh) * a.n_regions + r) * a.n_tiles + c];
+        float s = 0.f, used = 0.f;  // tile counts are exact in fp32 (far below 2^24)
+        for (int r = lane; r < a.n_regions; r += 32) {
+            const float *p = a.partial + (static_cast<size_t>(bh) * a.n_regions + r) * 2 * a.n_tiles;
+            s += p[c];
+            used += p[a.n_tiles + c];
+        }
         #pragma unroll
-        for (int off = 16; off > 0; off >>= 1) s += __shfl_down_sync(0xffffffffu, s, off);
+        for (int off = 16; off > 0; off >>= 1) {
+            s += __shfl_down_sync(0xffffffffu, s, off);
+            used += __shfl_down_sync(0xffffffffu, used, off);
+        }
         s = __shfl_sync(0xffffffffu, s, 0);
-        const float mean = s / a.tiles_total[c];
+        used = __shfl_sync(0xffffffffu, used, 0);
+        const float mean = used > 0.f ? s / used : 0.f;
         if (c == 0 || mean > best) {
             best = mean;
             best_c = c;
@@ -232,7 +265,7 @@ __global__ void sics_final_kernel(const FinalArgs a) {
 
 }  // namespace
 
-bool select_geometry(int T, int H, int W, const TileSet &tiles, SelectGeom *g) {
+bool select_geometry(int Tp, int Hp, int Wp, const TileSet &tiles, SelectGeom *g) {
     int Rt = 1, Rh = 1, Rw = 1, Ct = tiles.t[0], Ch = tiles.h[0], Cw = tiles.w[0];
     for (int c = 0; c < tiles.n; ++c) {
         Rt = lcm(Rt, tiles.t[c]);
@@ -244,23 +277,23 @@ bool select_geometry(int T, int H, int W, const TileSet &tiles, SelectGeom *g) {
     }
     g->Rt = Rt; g->Rh = Rh; g->Rw = Rw;
     g->Ct = Ct; g->Ch = Ch; g->Cw = Cw;
-    if (T % Rt || H % Rh || W % Rw) return false;
-    g->n_regions = (T / Rt) * (H / Rh) * (W / Rw);
+    if (Tp % Rt || Hp % Rh || Wp % Rw) return false;
+    g->n_regions = (Tp / Rt) * (Hp / Rh) * (Wp / Rw);
     g->cells = (Rt / Ct) * (Rh / Ch) * (Rw / Cw);
     return g->cells <= kMaxCells;
 }
 
-cudaError_t launch_select_tiling(const void *q, int esize, int BH, int S, int D, int T, int H, int W,
+cudaError_t launch_select_tiling(const void *q, int esize, int BH, int D, int T, int H, int W, int Tp, int Hp, int Wp,
                                  const TileSet &tiles, const SelectGeom &g, int32_t *choice, float *sics,
                                  float *partial, int *status, cudaStream_t st) {
     (void)status;
     SelArgs a;
     a.q = static_cast<const uint8_t *>(q);
-    a.S = S; a.H = H; a.W = W; a.D = D; a.esize = esize;
+    a.S = T * H * W; a.T = T; a.H = H; a.W = W; a.D = D; a.esize = esize;
     a.tiles = tiles;
     a.Rt = g.Rt; a.Rh = g.Rh; a.Rw = g.Rw;
     a.Ct = g.Ct; a.Ch = g.Ch; a.Cw = g.Cw;
-    a.nrt = T / g.Rt; a.nrh = H / g.Rh; a.nrw = W / g.Rw;
+    a.nrt = Tp / g.Rt; a.nrh = Hp / g.Rh; a.nrw = Wp / g.Rw;
     a.cells = g.cells;
     a.cell_hw = make_fastdiv(static_cast<uint32_t>(g.Ch * g.Cw));
     a.cell_w = make_fastdiv(static_cast<uint32_t>(g.Cw));
@@ -283,7 +316,7 @@ cudaError_t launch_select_tiling(const void *q, int esize, int BH, int S, int D,
         a.item_first[c + 1] = a.item_first[c] + a.tpr_t[c] * a.tpr_h[c] * a.tpr_w[c];
     }
     const size_t cvol = static_cast<size_t>(g.Ct) * g.Ch * g.Cw;
-    const size_t smem = (static_cast<size_t>(g.cells) * D + g.cells + items) * sizeof(float) + cvol * sizeof(int);
+    const size_t smem = (static_cast<size_t>(g.cells) * D + g.cells + 2 * items) * sizeof(float) + cvol * sizeof(int);
     dim3 grid(g.n_regions, BH);
     const int lpt = D * esize / 16;
     cudaError_t e = cudaSuccess;
@@ -311,8 +344,6 @@ cudaError_t launch_select_tiling(const void *q, int esize, int BH, int S, int D,
     f.BH = BH;
     f.n_regions = g.n_regions;
     f.n_tiles = tiles.n;
-    for (int c = 0; c < 8; ++c)
-        f.tiles_total[c] = c < tiles.n ? static_cast<float>(S / (tiles.t[c] * tiles.h[c] * tiles.w[c])) : 1.f;
     f.choice = choice;
     f.sics = sics;
     sics_final_kernel<<<(BH + 7) / 8, 256, 0, st>>>(f);

@@ -10,7 +10,9 @@
 // Tiled variant: x stays in T-major token order and the block's rows are read
 // where the head's chosen tiling puts them (position p of the tile-contiguous
 // order is token tile_token(p)), which gives the same result as permuting
-// first without writing the permuted copy.
+// first without writing the permuted copy.  On a zero-padded grid ("Adaptive
+// tiling (SPADE)", Deviations and notes) the positions cover the padded grid
+// and a padding position counts as a zero row.
 #include "common.cuh"
 #include "internal.h"
 
@@ -63,12 +65,13 @@ struct Vec<float> {
 
 struct TiledArgs {
     TileSet tiles;
-    TileDivs divs[kMaxTiles];  // per candidate tiling
+    TileDivs divs[kMaxTiles];  // per candidate tiling, over the (padded) grid
+    RealGrid real;             // PAD: the real grid
     const int32_t *choice;
     int *status;
 };
 
-template <typename T, int CPR, bool TILED>
+template <typename T, int CPR, bool TILED, bool PAD>
 __global__ void __launch_bounds__(kThreads) summaries_kernel(const uint8_t *__restrict__ x, int S, int block, int nb,
                                                              uint8_t *__restrict__ xmax, uint8_t *__restrict__ xmin,
                                                              const TiledArgs ta) {
@@ -80,6 +83,7 @@ __global__ void __launch_bounds__(kThreads) summaries_kernel(const uint8_t *__re
     const size_t head = static_cast<size_t>(bh) * S;
     int c = 0;
     uint32_t origin = 0, rr0 = 0;  // tiled mode, block within one tile: the tile's first token, block offset
+    uint32_t ot = 0, oh = 0, ow = 0;  // PAD: the tile's first coordinates
     bool one_tile = false;
     if constexpr (TILED) {
         c = ta.choice ? __ldg(ta.choice + bh) : 0;
@@ -93,15 +97,31 @@ __global__ void __launch_bounds__(kThreads) summaries_kernel(const uint8_t *__re
         if (one_tile) {
             const uint32_t tile = fdiv(p0, d.vol);
             rr0 = p0 - tile * d.vol.d;
-            origin = tile_token_fast(tile * d.vol.d, d);
+            if constexpr (PAD) tile_coords_fast(tile * d.vol.d, d, ot, oh, ow);
+            else origin = tile_token_fast(tile * d.vol.d, d);
         }
     }
-    // byte address of chunk `chunk` of the block's r-th row
+    // byte address of chunk `chunk` of the block's r-th row (PAD: nullptr for padding)
     auto row_ptr = [&](int r) -> const uint8_t * {
         uint32_t tok = static_cast<uint32_t>(blk * block + r);
         if constexpr (TILED) {
             const TileDivs &d = ta.divs[c];
-            if (one_tile) {
+            if constexpr (PAD) {
+                uint32_t t, h, w;
+                if (one_tile) {
+                    const uint32_t rr = rr0 + static_cast<uint32_t>(r);
+                    const uint32_t dt = fdiv(rr, d.thw), r2 = rr - dt * d.thw.d;
+                    const uint32_t dh = fdiv(r2, d.tw), dw = r2 - dh * d.tw.d;
+                    t = ot + dt;
+                    h = oh + dh;
+                    w = ow + dw;
+                } else {
+                    tile_coords_fast(tok, d, t, h, w);
+                }
+                const int rt = real_token(t, h, w, ta.real);
+                if (rt < 0) return nullptr;
+                tok = static_cast<uint32_t>(rt);
+            } else if (one_tile) {
                 const uint32_t rr = rr0 + static_cast<uint32_t>(r);
                 const uint32_t dt = fdiv(rr, d.thw), r2 = rr - dt * d.thw.d;
                 const uint32_t dh = fdiv(r2, d.tw), dw = r2 - dh * d.tw.d;
@@ -112,13 +132,26 @@ __global__ void __launch_bounds__(kThreads) summaries_kernel(const uint8_t *__re
         }
         return x + (head + tok) * CPR * 16 + chunk * 16;
     };
+    auto load_row = [&](int r) -> Vec<T> {
+        if constexpr (PAD) {
+            const uint8_t *ptr = row_ptr(r);
+            if (!ptr) {
+                Vec<T> z;
+                *reinterpret_cast<uint4 *>(&z) = make_uint4(0u, 0u, 0u, 0u);  // +0.0 in every element
+                return z;
+            }
+            return Vec<T>::load(ptr);
+        } else {
+            return Vec<T>::load(row_ptr(r));
+        }
+    };
     Vec<T> mx, mn;
     if (rg < block) {
-        mx = Vec<T>::load(row_ptr(rg));
+        mx = load_row(rg);
         mn = mx;
         #pragma unroll 4
         for (int r = rg + RG; r < block; r += RG) {
-            const Vec<T> v = Vec<T>::load(row_ptr(r));
+            const Vec<T> v = load_row(r);
             mx.vmax(v);
             mn.vmin(v);
         }
@@ -138,20 +171,21 @@ __global__ void __launch_bounds__(kThreads) summaries_kernel(const uint8_t *__re
     }
 }
 
-template <bool TILED>
-cudaError_t run_summaries(const void *x, int esize, int BH, int S, int D, int block, void *xmax, void *xmin,
+// S: tokens per head of x; Sp: positions per head (the padded grid's tokens, or S)
+template <bool TILED, bool PAD>
+cudaError_t run_summaries(const void *x, int esize, int BH, int S, int Sp, int D, int block, void *xmax, void *xmin,
                           const TiledArgs &ta, cudaStream_t st) {
-    const int nb = S / block;
+    const int nb = Sp / block;
     const int cpr = D * esize / 16;
     dim3 grid(nb, BH);
     const uint8_t *xi = static_cast<const uint8_t *>(x);
     uint8_t *mx = static_cast<uint8_t *>(xmax), *mn = static_cast<uint8_t *>(xmin);
     if (esize == 2) {
-        if (cpr == 8) summaries_kernel<__nv_bfloat16, 8, TILED><<<grid, kThreads, 0, st>>>(xi, S, block, nb, mx, mn, ta);
-        else summaries_kernel<__nv_bfloat16, 16, TILED><<<grid, kThreads, 0, st>>>(xi, S, block, nb, mx, mn, ta);
+        if (cpr == 8) summaries_kernel<__nv_bfloat16, 8, TILED, PAD><<<grid, kThreads, 0, st>>>(xi, S, block, nb, mx, mn, ta);
+        else summaries_kernel<__nv_bfloat16, 16, TILED, PAD><<<grid, kThreads, 0, st>>>(xi, S, block, nb, mx, mn, ta);
     } else {
-        if (cpr == 16) summaries_kernel<float, 16, TILED><<<grid, kThreads, 0, st>>>(xi, S, block, nb, mx, mn, ta);
-        else summaries_kernel<float, 32, TILED><<<grid, kThreads, 0, st>>>(xi, S, block, nb, mx, mn, ta);
+        if (cpr == 16) summaries_kernel<float, 16, TILED, PAD><<<grid, kThreads, 0, st>>>(xi, S, block, nb, mx, mn, ta);
+        else summaries_kernel<float, 32, TILED, PAD><<<grid, kThreads, 0, st>>>(xi, S, block, nb, mx, mn, ta);
     }
     return cudaGetLastError();
 }
@@ -161,20 +195,22 @@ cudaError_t run_summaries(const void *x, int esize, int BH, int S, int D, int bl
 cudaError_t launch_summaries(const void *x, int esize, int BH, int S, int D, int block, void *xmax, void *xmin,
                              cudaStream_t st) {
     TiledArgs ta{};
-    return run_summaries<false>(x, esize, BH, S, D, block, xmax, xmin, ta, st);
+    return run_summaries<false, false>(x, esize, BH, S, S, D, block, xmax, xmin, ta, st);
 }
 
-cudaError_t launch_summaries_tiled(const void *x, int esize, int BH, int S, int D, int T, int H, int W,
-                                   const TileSet &tiles, const int32_t *choice, void *xmax, void *xmin, int *status,
-                                   cudaStream_t st, int block) {
-    (void)T;
+cudaError_t launch_summaries_tiled(const void *x, int esize, int BH, int D, int T, int H, int W, int Tp, int Hp,
+                                   int Wp, const TileSet &tiles, const int32_t *choice, void *xmax, void *xmin,
+                                   int *status, cudaStream_t st, int block) {
     TiledArgs ta;
     ta.tiles = tiles;
     for (int c = 0; c < kMaxTiles; ++c)
-        ta.divs[c] = c < tiles.n ? make_tile_divs(H, W, tiles.t[c], tiles.h[c], tiles.w[c]) : make_tile_divs(1, 1, 1, 1, 1);
+        ta.divs[c] = c < tiles.n ? make_tile_divs(Hp, Wp, tiles.t[c], tiles.h[c], tiles.w[c]) : make_tile_divs(1, 1, 1, 1, 1);
+    ta.real = RealGrid{T, H, W};
     ta.choice = choice;
     ta.status = status;
-    return run_summaries<true>(x, esize, BH, S, D, block, xmax, xmin, ta, st);
+    const int S = T * H * W, Sp = Tp * Hp * Wp;
+    if (Sp != S) return run_summaries<true, true>(x, esize, BH, S, Sp, D, block, xmax, xmin, ta, st);
+    return run_summaries<true, false>(x, esize, BH, S, S, D, block, xmax, xmin, ta, st);
 }
 
 }  // namespace vsa

@@ -64,19 +64,37 @@ const char *vsa_last_error(void);
 vsa_status vsa_device_status(void *stream);
 
 /* ------------------------------------------------------------------------ */
+/* Grids the candidate tiles do not divide.  "Adaptive tiling (SPADE)",
+ * Deviations and notes: the grid is padded with zero tokens until every
+ * candidate tiles it, the padding takes no part in the cohesion, and padded
+ * keys are masked.  Here each axis is rounded up to the next multiple of the
+ * least common multiple of the candidates' extents on that axis:
+ *   padded = (ceil(T / lt) lt, ceil(Hg / lh) lh, ceil(Wg / lw) lw).
+ * Every call that takes (grid, tiles) works on that padded grid: tilings,
+ * permuted positions and block indices refer to it (Sp = padded.t * padded.h
+ * * padded.w positions per head), while the T-major tensors it reads or
+ * writes hold the S = T*Hg*Wg real tokens only.  With a grid every
+ * candidate divides, padded == grid and Sp == S.
+ * Returns VSA_ERR_INVALID_ARGUMENT for a non-positive grid or tile, an lcm
+ * above 2^20 or a padded grid of 2^31 tokens or more.                      */
+vsa_status vsa_padded_grid(vsa_dims3 grid, const vsa_dims3 *tiles, int n_tiles,
+                           vsa_dims3 *padded);
+
+/* ------------------------------------------------------------------------ */
 /* Adaptive tiling: per-(b, head) choice of the most cohesive tiling.
  * "Adaptive tiling (SPADE)", The idea, step 1, and the function table
  * (block_self_similarity, select_tiling), "Deviations and notes" (selection
- * statistic; divisible grids only).
+ * statistic; zero-padded grids).
  *
  * For every (b, head) and candidate c, the cohesion is the mean over the
- * tiles of tiling c of the tile's SICS: the mean cosine similarity over the
- * distinct pairs of its non-zero-norm queries, computed as
- * (|sum of unit queries|^2 - m) / (m (m - 1)) (a tile with m < 2 scores 0).
- * choice[bh] = argmax_c cohesion, ties to the lower c.
+ * tiles of tiling c (of the padded grid, see vsa_padded_grid) that hold at
+ * least one non-zero-norm query of the tile's SICS: the mean cosine
+ * similarity over the distinct pairs of its non-zero-norm queries, computed
+ * as (|sum of unit queries|^2 - m) / (m (m - 1)) (a tile with m < 2 scores
+ * 0).  choice[bh] = argmax_c cohesion, ties to the lower c.
  *
  *   q        [B, n_heads, S, D] in `dtype` (VSA_BF16 or VSA_F32)
- *   grid     (T, Hg, Wg) with T*Hg*Wg == S; every tile must divide it
+ *   grid     (T, Hg, Wg) with T*Hg*Wg == S (padded as vsa_padded_grid says)
  *   tiles    HOST array of n_tiles candidate tiles (1 <= n_tiles <= 8)
  *   choice   [B*n_heads] int32 output
  *   sics     [B*n_heads, n_tiles] fp32 output, or NULL
@@ -131,10 +149,13 @@ vsa_status vsa_select_tiling_noalloc(const void *q, vsa_dtype dtype, int B, int 
  *   vsa_permute:   y[bh, p, :] = x[bh, perm_{c(bh)}[p], :]
  *   vsa_unpermute: x[bh, perm_{c(bh)}[p], :] = y[bh, p, :]
  * where c(bh) = choice[bh] (device int32 [B*n_heads]), or 0 if choice is NULL.
- * x and y are [B, n_heads, S, D] in `dtype` and must not overlap.
- * tiles is a HOST array of n_tiles (1..8) tiles that divide grid; a device
- * choice outside [0, n_tiles) sets VSA_ERR_RUNTIME and that head is left
- * unwritten.  The copy is exact (bit for bit).                            */
+ * x is [B, n_heads, S, D] (T-major, S = T*Hg*Wg) and y [B, n_heads, Sp, D]
+ * (Sp of vsa_padded_grid; Sp == S when the tiles divide grid), both in
+ * `dtype`, not overlapping.  On a padded grid perm runs over the padded
+ * grid's tokens: vsa_permute writes zero rows at padding positions and
+ * vsa_unpermute ignores them.  tiles is a HOST array of n_tiles (1..8)
+ * tiles; a device choice outside [0, n_tiles) sets VSA_ERR_RUNTIME and that
+ * head is left unwritten.  The copy is exact (bit for bit).               */
 vsa_status vsa_permute(const void *x, void *y, vsa_dtype dtype, int B, int n_heads,
                        int S, int D, vsa_dims3 grid, const vsa_dims3 *tiles,
                        int n_tiles, const int32_t *choice, void *stream);
@@ -160,7 +181,9 @@ vsa_status vsa_block_summaries(const void *x_perm, vsa_dtype dtype, int B, int n
  * bit for bit.
  *   x      [B, n_heads, S, D] in `dtype`, T-major (S = grid.t*grid.h*grid.w)
  *   tiles, n_tiles, choice  as for vsa_permute (choice NULL: tile 0)
- *   x_max, x_min  [B, n_heads, S/block, D] in `dtype`
+ *   x_max, x_min  [B, n_heads, Sp/block, D] in `dtype` (Sp of
+ *          vsa_padded_grid, a multiple of block); padding positions count
+ *          as zero rows, as in the output of vsa_permute
  * A choice outside [0, n_tiles) leaves that head's summaries unwritten and
  * sets VSA_ERR_RUNTIME (read with vsa_device_status).                      */
 vsa_status vsa_block_summaries_tiled(const void *x, vsa_dtype dtype, int B, int n_heads,
@@ -239,7 +262,9 @@ vsa_status vsa_structured_block_list(vsa_mask_kind kind, vsa_dims3 grid, vsa_dim
  *   scale    softmax scale; <= 0 selects 1/sqrt(D) (_default_scale)
  * block in {32, 64, 128}, S % block == 0, D in {64, 128}.  Each list must be
  * strictly ascending with entries in [0, nb) and 1 <= cnt <= cap; rows whose
- * list breaks this are written as zeros and set VSA_ERR_RUNTIME.          */
+ * list breaks this are written as zeros and set VSA_ERR_RUNTIME.  Every one
+ * of the S rows is a key here: for a zero-padded grid, whose padding keys
+ * must be masked, use vsa_block_sparse_attention_tiled.                   */
 vsa_status vsa_block_sparse_attention(const void *q, const void *k, const void *v,
                                       void *o, vsa_dtype out_dtype, int B, int n_heads,
                                       int S, int D, int block, const int32_t *idx,
@@ -253,7 +278,11 @@ vsa_status vsa_block_sparse_attention(const void *q, const void *k, const void *
  * order under tiles[choice[bh]]; idx/cnt list blocks in that numbering, as
  * vsa_topk_block_mask writes them.  The result equals vsa_permute of q, k and
  * v, vsa_block_sparse_attention with block 128 and group_size 0, then
- * vsa_unpermute of o, bit for bit.
+ * vsa_unpermute of o, bit for bit, when the tiles divide the grid.  On a
+ * grid they do not divide (vsa_padded_grid), positions and blocks refer to
+ * the padded grid (nb = Sp/128), keys at padding positions are masked out
+ * (the zero-padding recipe of "Adaptive tiling (SPADE)", Deviations and
+ * notes) and only the S real rows of o are written.
  *   q, k, v  [B, n_heads, S, D] bf16, o [B, n_heads, S, D] in out_dtype, T-major
  *   tiles    every candidate of the same volume V, a multiple of 128, with
  *            tile.t divisible by V/128 (a 128-token block is tile.t*128/V

@@ -88,21 +88,45 @@ def test_permute_and_select_tiling_argument_errors(L):
     y = ctypes.c_void_p(0x100000)
     assert L.vsa_permute(FAKE, y, vsa.F32, 1, 2, 256, 64, Dims3(4, 8, 4), arr, n, NULL, NULL) == \
         vsa.ERR_INVALID_ARGUMENT  # grid product != S
-    bad, nb_ = _tiles((3, 4, 4))
+    bad, nb_ = _tiles((0, 4, 4))
     assert L.vsa_permute(FAKE, y, vsa.F32, 1, 2, 256, 64, g, bad, nb_, NULL, NULL) == vsa.ERR_INVALID_ARGUMENT
-    assert "does not divide" in vsa.last_error()
+    assert "must be positive" in vsa.last_error()
     assert L.vsa_permute(FAKE, FAKE, vsa.F32, 1, 2, 256, 64, g, arr, n, NULL, NULL) == vsa.ERR_INVALID_ARGUMENT
     assert L.vsa_permute(FAKE, y, vsa.F32, 1, 2, 256, 64, g, arr, 0, NULL, NULL) == vsa.ERR_INVALID_ARGUMENT
     # select_tiling: workspace size, then a too-small workspace
     t3, n3 = _tiles((1, 8, 16), (2, 8, 8), (4, 4, 8))
     ws = L.vsa_select_tiling_workspace_size(1, 24, Dims3(32, 48, 80), t3, n3)
-    assert ws == 24 * 240 * 3 * 4
+    assert ws == 24 * 240 * 2 * 3 * 4   # per region and candidate: a SICS sum and a tile count
     assert L.vsa_select_tiling(FAKE, vsa.BF16, 1, 24, 122880, 128, Dims3(32, 48, 80), t3, n3, FAKE, NULL,
                                y, ws - 256, NULL) == vsa.ERR_INVALID_ARGUMENT
     # an lcm region of too many gcd cells is reported as unsupported
     big, nbig = _tiles((1, 1, 7), (1, 1, 9), (1, 5, 1), (3, 1, 1))
     assert L.vsa_select_tiling(FAKE, vsa.BF16, 1, 1, 3 * 5 * 63, 128, Dims3(3, 5, 63), big, nbig, FAKE, NULL,
                                y, 1 << 20, NULL) == vsa.ERR_UNSUPPORTED
+
+
+@pytest.mark.parametrize("grid,tiles", [
+    ((16, 45, 80), [(1, 8, 16), (2, 8, 8), (4, 4, 8)]),   # the height no candidate divides
+    ((21, 45, 80), [(1, 8, 16), (2, 8, 8), (4, 4, 8)]),
+    ((32, 48, 80), [(1, 8, 16), (2, 8, 8), (4, 4, 8)]),   # divisible: unchanged
+    ((3, 5, 13), [(2, 3, 4), (3, 2, 6)]),
+    ((1, 1, 1), [(4, 4, 8)]),
+])
+def test_padded_grid_matches_oracle(L, grid, tiles):
+    import oracle
+    assert vsa.padded_grid(grid, tiles) == oracle.padded_grid(grid, tiles)
+
+
+def test_padded_grid_argument_errors(L):
+    out = Dims3()
+    arr, n = _tiles((2, 4, 4))
+    assert L.vsa_padded_grid(Dims3(0, 8, 8), arr, n, ctypes.byref(out)) == vsa.ERR_INVALID_ARGUMENT
+    assert L.vsa_padded_grid(Dims3(4, 8, 8), arr, n, None) == vsa.ERR_INVALID_ARGUMENT
+    assert L.vsa_padded_grid(Dims3(4, 8, 8), arr, 9, ctypes.byref(out)) == vsa.ERR_INVALID_ARGUMENT
+    big, nbig = _tiles((1, 1, 1 << 15), (1, 1, (1 << 15) - 1))   # lcm above 2^20
+    assert L.vsa_padded_grid(Dims3(4, 8, 8), big, nbig, ctypes.byref(out)) == vsa.ERR_INVALID_ARGUMENT
+    huge, nh = _tiles((1, 1, 1))
+    assert L.vsa_padded_grid(Dims3(2048, 2048, 1024), huge, nh, ctypes.byref(out)) == vsa.ERR_INVALID_ARGUMENT
 
 
 def test_structured_list_argument_errors(L):

@@ -67,6 +67,8 @@ class Workload:
 
     @property
     def nb(self) -> int:
+        """Blocks of the grid itself (a grid the tiles do not divide has more
+        blocks once padded; its workloads give topk explicitly)."""
         return self.S // self.block
 
     @property
@@ -100,6 +102,14 @@ WORKLOADS = {
         name="spade_adaptive_s122880", B=1, heads=24, grid=(32, 48, 80),
         D=128, dtype=torch.bfloat16, values="smooth_adaptive", seed_base=3000,
         tiles=((1, 8, 16), (2, 8, 8), (4, 4, 8)), budget=0.10),
+    # SPADE with adaptive tiling on a grid the candidates do not divide: the
+    # 16 x 45 x 80 latent the pages name for it (no candidate's height divides
+    # 45).  S = 57600 real tokens; k = 48 is 10 % of the 480 blocks of the
+    # zero-padded 16 x 48 x 80 grid the candidates tile.
+    "spade_adaptive_pad_s57600": Workload(
+        name="spade_adaptive_pad_s57600", B=1, heads=24, grid=(16, 45, 80),
+        D=128, dtype=torch.bfloat16, values="smooth_adaptive", seed_base=5000,
+        tiles=((1, 8, 16), (2, 8, 8), (4, 4, 8)), topk=48),
     # Structured static masks on a CFG pair, S = 122880.
     "structured_s122880": Workload(
         name="structured_s122880", B=2, heads=24, grid=(32, 48, 80), D=128,
