@@ -521,8 +521,8 @@ def run_ours(args, w):
     mask_ms = ph["summaries"] + ph["scores"] + ph["topk"]
     mask_gbs = mask_pipeline_bytes(w, BH) / mask_ms / 1e6
     hbm = peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"])
-    kname = ("attn_pp_kernel<128,false,true> (block-sparse, tiled)" if step.tiled
-             else "attn_pp_kernel<128,false,false> (block-sparse)")
+    kname = ("attn_pp_kernel<128,false,true,false> (block-sparse, tiled)" if step.tiled
+             else "attn_pp_kernel<128,false,false,false> (block-sparse)")
     roofline = {"bound": "tensor", "kernel": kname,
                 "achieved": achieved, "peak": peak, "unit": "TFLOP/s", "frac": achieved / peak,
                 "peak_kind": f"bf16_tflops_sustained ({peak_src})", "frac_of_burst": achieved / burst,

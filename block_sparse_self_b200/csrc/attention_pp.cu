@@ -54,7 +54,6 @@ struct PPArgs {
     int *status;
     // tiled mode: T-major tensors, per-head tiling (all of volume 128 * m)
     int H, W;         // the padded grid's frame (equal to the real one when nothing is padded)
-    int padded;
     RealGrid real;
     TileSet tiles;
     const int32_t *choice;
@@ -153,7 +152,9 @@ __device__ __forceinline__ int kblock_of(const TileSched &t, int j) {
     else return __ldg(t.list + j);
 }
 
-template <int D, bool WINDOW, bool TILED>
+// PAD (tiled mode only): the grid is zero-padded, so padding rows and keys need
+// handling; a separate instantiation keeps that code out of the common case.
+template <int D, bool WINDOW, bool TILED, bool PAD>
 __global__ void __launch_bounds__(kThreads, 1)
 attn_pp_kernel(const __grid_constant__ MapSet maps, const PPArgs a) {
     using C = PPCfg<D>;
@@ -248,8 +249,8 @@ attn_pp_kernel(const __grid_constant__ MapSet maps, const PPArgs a) {
         }
     }
     const int tt = a.tiles.t[tc], th = a.tiles.h[tc], tw = a.tiles.w[tc];
-    if constexpr (TILED) {
-        if (a.padded) {  // a query box wholly in the padding has no row to write
+    if constexpr (PAD) {
+        {  // a query box wholly in the padding has no row to write
             for (int t = 0; t < 2; ++t) {
                 if (ts[t].qt < 0) continue;
                 const BoxCoord c = box_of(static_cast<uint32_t>(ts[t].qt), a.geom[tc], th, tw);
@@ -397,12 +398,14 @@ attn_pp_kernel(const __grid_constant__ MapSet maps, const PPArgs a) {
         bool row_valid = sc.qt >= 0 && rg < S;
         // output row: the permuted position itself, or its T-major token in tiled mode
         uint32_t orow_in_head = rg;
-        if constexpr (TILED) {
+        if constexpr (PAD) {
             int pt, ph, pw;
             tile_coords(rg, a.H, a.W, tt, th, tw, pt, ph, pw);
             const int tok = real_token(pt, ph, pw, a.real);
             row_valid = row_valid && tok >= 0;
             orow_in_head = tok < 0 ? 0u : static_cast<uint32_t>(tok);
+        } else if constexpr (TILED) {
+            orow_in_head = tile_token(rg, a.H, a.W, tt, th, tw);
         }
         const uint32_t t_lane = tmem + (static_cast<uint32_t>(wq * 32) << 16);
         const uint32_t s_col = t * 128, o_col = C::O_COL + t * D;
@@ -421,8 +424,8 @@ attn_pp_kernel(const __grid_constant__ MapSet maps, const PPArgs a) {
             // (column u * 32 + lane in bit lane of kv[u]); all ones off the edge
             uint32_t kv[4] = {~0u, ~0u, ~0u, ~0u};
             bool key_edge = false;
-            if constexpr (TILED) {
-                if (a.padded) {
+            if constexpr (PAD) {
+                {
                     const PPArgs::BoxGeom &g = a.geom[tc];
                     const BoxCoord c = box_of(static_cast<uint32_t>(kblock_of<WINDOW>(sc, j)), g, th, tw);
                     key_edge = c.t + g.bt > a.real.T || c.h + th > a.real.H || c.w + tw > a.real.W;
@@ -484,8 +487,9 @@ attn_pp_kernel(const __grid_constant__ MapSet maps, const PPArgs a) {
             // to the other tile's warp on the sub-partition.  The row sum adds the
             // bf16-rounded P that the PV MMA multiplies, so O / l is a convex
             // combination of V rows: a row held by a few keys then carries no
-            // rounding error in its weights' total (measured cost: about 2 % of
-            // the kernel's time, against 4.5 % for unpacking each pair first).
+            // rounding error in its weights' total.  The mixed-precision adds take
+            // each half of the packed pair as it is; unpacking the pair first for
+            // two-wide adds measured a few percent slower.
             auto exp_pass = [&](float m_use) -> float {
                 const uint64_t sl2x2 = f32x2(sl2, sl2), nmx2 = f32x2(-m_use, -m_use);
                 float s0 = 0.f, s1 = 0.f, s2 = 0.f, s3 = 0.f;
@@ -617,7 +621,7 @@ attn_pp_kernel(const __grid_constant__ MapSet maps, const PPArgs a) {
     }
 }
 
-template <int D, bool WINDOW, bool TILED>
+template <int D, bool WINDOW, bool TILED, bool PAD = false>
 vsa_status run_pp(const AttnLaunch &L, int *status, cudaStream_t st) {
     using C = PPCfg<D>;
     MapSet maps = {};  // copied into the launch parameters
@@ -636,7 +640,7 @@ vsa_status run_pp(const AttnLaunch &L, int *status, cudaStream_t st) {
              make_tile_map(&maps.v[0], L.v, D, L.S, L.BH, 128);
     }
     if (!ok) return fail(VSA_ERR_CUDA, "cuTensorMapEncodeTiled failed (driver entry point or arguments)");
-    auto kern = attn_pp_kernel<D, WINDOW, TILED>;
+    auto kern = attn_pp_kernel<D, WINDOW, TILED, PAD>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
     if (e != cudaSuccess) return check_cuda(e, "cudaFuncSetAttribute(attention, two tiles)");
     PPArgs a;
@@ -660,7 +664,6 @@ vsa_status run_pp(const AttnLaunch &L, int *status, cudaStream_t st) {
     a.status = status;
     a.H = TILED ? L.Hp : L.Hg;
     a.W = TILED ? L.Wp : L.Wg;
-    a.padded = TILED && positions != L.S;
     a.real = RealGrid{L.T, L.Hg, L.Wg};
     a.tiles = L.tiles;
     a.choice = L.choice;
@@ -690,7 +693,11 @@ vsa_status run_pp(const AttnLaunch &L, int *status, cudaStream_t st) {
 
 vsa_status launch_attention_pp(const AttnLaunch &L, int *status, cudaStream_t st) {
     if (L.window) return L.D == 128 ? run_pp<128, true, false>(L, status, st) : run_pp<64, true, false>(L, status, st);
-    if (L.tiled) return L.D == 128 ? run_pp<128, false, true>(L, status, st) : run_pp<64, false, true>(L, status, st);
+    if (L.tiled) {
+        if (L.Tp * L.Hp * L.Wp != L.S)  // a zero-padded grid
+            return L.D == 128 ? run_pp<128, false, true, true>(L, status, st) : run_pp<64, false, true, true>(L, status, st);
+        return L.D == 128 ? run_pp<128, false, true>(L, status, st) : run_pp<64, false, true>(L, status, st);
+    }
     return L.D == 128 ? run_pp<128, false, false>(L, status, st) : run_pp<64, false, false>(L, status, st);
 }
 
