@@ -117,12 +117,19 @@ def test_block_summaries_tiled_matches_oracle_and_permuted_path(dtype, D, block)
     assert torch.equal(mx0, vsa.block_summaries(vsa.permute(x, grid, tiles[:1]), block)[0])
 
 
-def test_block_summaries_tiled_bad_choice_sets_runtime_status():
-    grid, tiles = (2, 8, 8), [(1, 8, 8), (2, 4, 4)]
-    x = integer_grid((1, 2, 128, 64), 72, torch.bfloat16, DEV)
-    vsa.block_summaries_tiled(x, grid, tiles, torch.tensor([1, -1], dtype=torch.int32, device=DEV), 64)
+@pytest.mark.parametrize("grid,tiles,block", [((2, 8, 8), [(1, 8, 8), (2, 4, 4)], 64),
+                                              ((2, 8, 16), [(1, 8, 16), (2, 8, 8)], 128)])
+def test_block_summaries_tiled_bad_choice_sets_runtime_status(grid, tiles, block):
+    """A choice out of range leaves that head unwritten and sets the status, in
+    the row-gather kernel (64-token blocks) and the TMA one (128-token boxes);
+    the other head is still summarised."""
+    S = grid[0] * grid[1] * grid[2]
+    x = integer_grid((1, 2, S, 64), 72, torch.bfloat16, DEV)
+    mx, mn = vsa.block_summaries_tiled(x, grid, tiles, torch.tensor([1, -1], dtype=torch.int32, device=DEV), block)
     with pytest.raises(RuntimeError):
         vsa.device_status()
+    want = vsa.block_summaries(vsa.permute(x[:, :1], grid, tiles[1:]), block)
+    assert torch.equal(mx[:, :1], want[0]) and torch.equal(mn[:, :1], want[1])
 
 
 @pytest.mark.parametrize("dtype,D,nb", [(torch.bfloat16, 128, 40), (torch.float32, 64, 70), (torch.bfloat16, 64, 1),
