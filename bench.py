@@ -21,6 +21,7 @@ step, all ranks together (each rank runs its own batch: weak scaling).
 from __future__ import annotations
 
 import argparse
+import dataclasses
 import datetime
 import hashlib
 import json
@@ -583,10 +584,16 @@ def main():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-extra", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--heads", type=int, default=None,
+                    help="run the workload with this many heads (smaller cases for profilers; not a bench line)")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
     w = WORKLOADS[args.workload]
+    if args.heads is not None:
+        if args.heads < 1:
+            ap.error("--heads must be >= 1")
+        w = dataclasses.replace(w, heads=args.heads)
     if args.impl == "reference":
         run_reference(args, w)
     else:

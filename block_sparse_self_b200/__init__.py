@@ -362,10 +362,11 @@ def block_sparse_attention(q, k, v, idx, cnt, block: int, group_size: int = 0, s
 
 def block_sparse_attention_tiled(q, k, v, grid, tiles, choice, idx, cnt, scale: Optional[float] = None,
                                  out_dtype=None, group_stride: int = 0) -> torch.Tensor:
-    """unpermute(block_sparse_attention(permute(q), permute(k), permute(v), idx, cnt, 128)) in one
-    kernel: q, k, v and the result stay in T-major order; lists number 128-token blocks of
-    each head's tile-contiguous order.  group_stride s > 0 restricts each query to keys
-    whose position differs from its own by a multiple of s (see include/vsa.h)."""
+    """unpermute(block_sparse_attention(permute(q), permute(k), permute(v), idx, cnt, block)) in one
+    kernel: q, k, v and the result stay in T-major order; lists number the blocks of each
+    head's tile-contiguous order (block = the tile volume if 32 or 64, else 128 tokens).
+    group_stride s > 0 (128-token blocks) restricts each query to keys whose position
+    differs from its own by a multiple of s (see include/vsa.h)."""
     B, H, S, D = _bhsd(q, "q")
     if tuple(k.shape) != (B, H, S, D) or tuple(v.shape) != (B, H, S, D):
         raise ValueError(f"q/k/v shapes must match exactly; got q={tuple(q.shape)}, k={tuple(k.shape)}, "
@@ -387,12 +388,15 @@ def block_sparse_attention_tiled(q, k, v, grid, tiles, choice, idx, cnt, scale: 
 
 def tiled_supported(tiles) -> bool:
     """Whether every candidate tiling can run through the T-major (tiled) attention:
-    one common volume V, a multiple of 128, and each tile.t divisible by V/128."""
+    one common volume V, either 32 or 64 (a block is the tile) or a multiple of 128
+    (a block is 128 tokens: each tile.t divisible by V/128)."""
     tiles = [tuple(t) for t in tiles]
     vols = {t[0] * t[1] * t[2] for t in tiles}
     if len(vols) != 1:
         return False
     vol = vols.pop()
+    if vol in (32, 64):
+        return True
     return vol % 128 == 0 and all(t[0] % (vol // 128) == 0 for t in tiles)
 
 
@@ -448,7 +452,7 @@ def spade_attention(q, k, v, grid, tiles, budget: Optional[float] = None, topk: 
     Padded grids run in tiled mode, which masks the padding keys.
 
     tiled=True runs the permutation inside the summaries and attention kernels
-    (no permuted copies; block size 128, see tiled_supported); tiled=False
+    (no permuted copies; blocks of 32, 64 or 128 tokens, see tiled_supported); tiled=False
     runs the explicit permute / unpermute steps; None picks tiled when it is
     supported.  Both give identical results.  In tiled mode the permuted
     tensors in the intermediates are computed afterwards, for inspection only.
@@ -462,14 +466,14 @@ def spade_attention(q, k, v, grid, tiles, budget: Optional[float] = None, topk: 
     pgrid = padded_grid(grid, tiles)
     nb = _grid_tokens(pgrid) // block
     kk = topk if topk is not None else topk_budget(nb, budget if budget is not None else 0.17)
-    can_tile = block == 128 and tiled_supported(tiles)
+    can_tile = block in (32, 64, 128) and tiled_supported(tiles)
     if tiled is None:
         tiled = can_tile
     elif tiled and not can_tile:
-        raise ValueError("tiled mode needs 128-token blocks whose tiles satisfy tiled_supported()")
+        raise ValueError("tiled mode needs blocks of 32, 64 or 128 tokens whose tiles satisfy tiled_supported()")
     if not tiled and tuple(pgrid) != tuple(grid):
         raise NotImplementedError(f"grid {tuple(grid)} is padded to {pgrid}: its padding keys are masked in "
-                                  "tiled mode only (128-token blocks, see tiled_supported)")
+                                  "tiled mode only (see tiled_supported)")
     choice = select_tiling(q, grid, tiles) if len(tiles) > 1 else None
     if tiled:
         qb, kb, vb = _bf16(q, "q"), _bf16(k, "k"), _bf16(v, "v")

@@ -443,27 +443,31 @@ vsa_status vsa_block_sparse_attention_tiled(const void *q, const void *k, const 
     VSA_TRY(check_tiles(grid, tiles, n_tiles, &ts, &pg));
     const long long Sp = static_cast<long long>(pg.t) * pg.h * pg.w;
     const int vol = ts.t[0] * ts.h[0] * ts.w[0];
-    VSA_REQUIRE(vol % 128 == 0, "tile volume (%d) must be a multiple of 128", vol);
+    // blocks: the tile itself for volumes 32, 64 and 128, else 128-token parts of it
+    VSA_REQUIRE(vol == 32 || vol == 64 || vol % 128 == 0, "tile volume (%d) must be 32, 64 or a multiple of 128", vol);
+    const int blk = vol < 128 ? vol : 128;
+    if (group_stride != 0 && blk != 128)
+        return fail(VSA_ERR_UNSUPPORTED, "group_stride needs 128-token blocks; the tiles hold %d tokens", vol);
     for (int c = 0; c < n_tiles; ++c) {
         VSA_REQUIRE(ts.t[c] * ts.h[c] * ts.w[c] == vol, "every tile must have the volume of tile 0 (%d); tile %d has %d",
                     vol, c, ts.t[c] * ts.h[c] * ts.w[c]);
-        VSA_REQUIRE(ts.t[c] % (vol / 128) == 0,
-                    "tile %d: tile.t (%d) must be divisible by volume / 128 (%d) so each 128-token block is whole "
+        VSA_REQUIRE(ts.t[c] % (vol / blk) == 0,
+                    "tile %d: tile.t (%d) must be divisible by volume / %d (%d) so each %d-token block is whole "
                     "(h, w) planes",
-                    c, ts.t[c], vol / 128);
-        // a TMA box (one 128-token block) must fit inside the real tensor
-        if (ts.t[c] / (vol / 128) > grid.t || ts.h[c] > grid.h || ts.w[c] > grid.w)
-            return fail(VSA_ERR_UNSUPPORTED, "tile %d: its 128-token box (%d, %d, %d) is larger than the grid (%d, %d, %d)",
-                        c, ts.t[c] / (vol / 128), ts.h[c], ts.w[c], grid.t, grid.h, grid.w);
+                    c, ts.t[c], blk, vol / blk, blk);
+        // a TMA box (one block) must fit inside the real tensor
+        if (ts.t[c] / (vol / blk) > grid.t || ts.h[c] > grid.h || ts.w[c] > grid.w)
+            return fail(VSA_ERR_UNSUPPORTED, "tile %d: its %d-token box (%d, %d, %d) is larger than the grid (%d, %d, %d)",
+                        c, blk, ts.t[c] / (vol / blk), ts.h[c], ts.w[c], grid.t, grid.h, grid.w);
     }
     AttnLaunch L{};
     L.q = q; L.k = k; L.v = v; L.o = o;
     L.out_f32 = out_dtype == VSA_F32;
     L.BH = B * n_heads; L.S = S; L.D = D;
-    L.block = 128;
+    L.block = blk;
     L.window = false;
     L.idx = idx; L.cnt = cnt; L.cap = cap; L.list_per_head = list_per_head ? 1 : 0;
-    L.group = 0; L.nb = static_cast<int>(Sp / 128);
+    L.group = 0; L.nb = static_cast<int>(Sp / blk);
     L.scale = scale > 0.f ? scale : 1.0f / sqrtf(static_cast<float>(D));
     L.tiled = true;
     L.gstride = group_stride;

@@ -17,6 +17,15 @@
 // The running max m is only raised (and O, l rescaled) when a row's max grows
 // by more than 2^8; the final O / l is exact either way because O and l always
 // share the same reference.  All waits are bounded (see common.cuh).
+//
+// Tiled mode (TILED): Q, K, V and O stay in T-major order and each (b, head)
+// uses its chosen tiling; a block of BN tokens is one 5-D TMA box of whole
+// (h, w) planes of its tile, which lands in shared memory as BN rows in
+// tile-contiguous order, and the epilogue writes each row to its token.  On a
+// zero-padded grid (PAD; "Adaptive tiling (SPADE)", Deviations and notes) the
+// boxes read zeros past the real tensors, keys there are masked in the blocks
+// that cross the edge, rows there are not written and query blocks wholly in
+// the padding are skipped.
 #include <math.h>
 
 #include "common.cuh"
@@ -27,7 +36,8 @@ namespace vsa {
 namespace {
 
 struct AttnArgs {
-    int S, BH, nq;
+    int S, BH, nq;   // S: positions per head (tiled mode: of the padded grid)
+    int S_out;       // rows per head of o (tiled mode: real tokens)
     // block-list mode
     const int32_t *idx, *cnt;
     int cap, list_per_head, group, nb;
@@ -37,7 +47,34 @@ struct AttnArgs {
     void *out;
     int out_f32;
     int *status;
+    // tiled mode
+    int H, W;  // the padded grid's frame
+    RealGrid real;
+    TileSet tiles;
+    const int32_t *choice;
+    struct BoxGeom {
+        FastDiv m, nthw, ntw;  // m = volume / BN, tiles per frame, tiles per tile row
+        FastDiv bhw, bw;       // box frame (th * tw) and row (tw): key column -> (dt, dh, dw)
+        int bt;                // frames of one BN-token box
+    } geom[kMaxTiles];
 };
+
+// Tensor maps: slot 0 only, or one per candidate tiling in tiled mode.
+struct AttnMaps {
+    CUtensorMap q[kMaxTiles], k[kMaxTiles], v[kMaxTiles];
+};
+static_assert(sizeof(AttnMaps) + sizeof(AttnArgs) <= 4096, "kernel parameters");
+
+// Block b of a head in tiled mode: the TMA coordinates (w, h, t) of its box.
+struct BoxAt {
+    int w, h, t;
+};
+__device__ __forceinline__ BoxAt box_at(uint32_t b, const AttnArgs::BoxGeom &g, int th, int tw) {
+    const uint32_t tile = fdiv(b, g.m), part = b - tile * g.m.d;
+    const uint32_t ct = fdiv(tile, g.nthw), rem = tile - ct * g.nthw.d;
+    const uint32_t ch = fdiv(rem, g.ntw), cw = rem - ch * g.ntw.d;
+    return BoxAt{static_cast<int>(cw) * tw, static_cast<int>(ch) * th, static_cast<int>(ct * g.m.d + part) * g.bt};
+}
 
 template <int D, int BN>
 struct Cfg {
@@ -66,10 +103,9 @@ struct Cfg {
 
 constexpr float kRescaleLog2 = 8.0f;  // rescale O only when the max grows by > 2^8
 
-template <int D, int BN, bool WINDOW>
+template <int D, int BN, bool WINDOW, bool TILED, bool PAD>
 __global__ void __launch_bounds__(192, 1)
-attn_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
-            const __grid_constant__ CUtensorMap tmV, const AttnArgs a) {
+attn_kernel(const __grid_constant__ AttnMaps maps, const AttnArgs a) {
     using C = Cfg<D, BN>;
     extern __shared__ uint8_t smem_raw[];
     uint8_t *base = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -173,15 +209,44 @@ attn_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUt
             n_kb = 0;
         }
     }
+    int tc = 0;             // tiled mode: this head's tiling
+    bool q_skip = false;    // tiled mode: the query block has no row to write
+    if constexpr (TILED) {
+        if (a.choice) tc = __ldg(a.choice + bh);
+        if (tc < 0 || tc >= a.tiles.n) {  // the head is left unwritten
+            if (threadIdx.x == 0) report(a.status, DEV_RUNTIME);
+            tc = 0;
+            n_kb = 0;
+            q_skip = true;
+        }
+        if constexpr (PAD) {
+            const BoxAt qb = box_at(static_cast<uint32_t>(qt), a.geom[tc], a.tiles.h[tc], a.tiles.w[tc]);
+            if (qb.t >= a.real.T || qb.h >= a.real.H || qb.w >= a.real.W) {  // wholly in the padding
+                n_kb = 0;
+                q_skip = true;
+            }
+        }
+    }
+    const int th = a.tiles.h[tc], tw = a.tiles.w[tc];
+    const CUtensorMap *tmQ = &maps.q[tc], *tmK = &maps.k[tc], *tmV = &maps.v[tc];
+    // block b's BN rows of Q, K or V into dst (slabs of 64 columns, `slab` bytes apart)
+    auto load_block = [&](uint8_t *dst, int slab, const CUtensorMap *map, uint64_t *bar, int b) {
+        if constexpr (TILED) {
+            const BoxAt c = box_at(static_cast<uint32_t>(b), a.geom[tc], th, tw);
+            for (int s = 0; s < C::KSLABS; ++s) tma_load_5d(dst + s * slab, map, bar, s * 64, c.w, c.h, c.t, bh);
+        } else {
+            for (int s = 0; s < C::KSLABS; ++s) tma_load_3d(dst + s * slab, map, bar, s * 64, b * BN, bh);
+        }
+    };
 
     if (warp == 4) {
         // ================= TMA producer =================
         if (lane == 0 && n_kb > 0) {
-            tma_prefetch_desc(&tmQ);
-            tma_prefetch_desc(&tmK);
-            tma_prefetch_desc(&tmV);
+            tma_prefetch_desc(tmQ);
+            tma_prefetch_desc(tmK);
+            tma_prefetch_desc(tmV);
             mbar_arrive_expect_tx(q_full, BN * 128 * C::KSLABS);
-            for (int s = 0; s < C::KSLABS; ++s) tma_load_3d(sQ + s * C::SLAB_Q, &tmQ, q_full, s * 64, q_row0, bh);
+            load_block(sQ, C::SLAB_Q, tmQ, q_full, qt);
             int issued = 0;
             for (int j = 0; j < n_kb; ++j) {
                 const int st = j % C::NS;
@@ -191,11 +256,9 @@ attn_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUt
                 }
                 const int kb = kblock(j);
                 mbar_arrive_expect_tx(&k_full[st], C::K_BYTES);
-                for (int s = 0; s < C::KSLABS; ++s)
-                    tma_load_3d(sK + st * C::K_BYTES + s * BN * 128, &tmK, &k_full[st], s * 64, kb * BN, bh);
+                load_block(sK + st * C::K_BYTES, BN * 128, tmK, &k_full[st], kb);
                 mbar_arrive_expect_tx(&v_full[st], C::V_BYTES);
-                for (int s = 0; s < C::KSLABS; ++s)
-                    tma_load_3d(sV + st * C::V_BYTES + s * BN * 128, &tmV, &v_full[st], s * 64, kb * BN, bh);
+                load_block(sV + st * C::V_BYTES, BN * 128, tmV, &v_full[st], kb);
                 issued = j + 1;
             }
             if (*abort_flag) {
@@ -261,8 +324,21 @@ attn_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUt
         const int row = threadIdx.x;                 // 0..127: TMEM lane = query row in the tile
         const int rows_valid = BN;                   // rows of the tile that exist
         const bool warp_valid = warp * 32 < rows_valid;
-        const int rg = q_row0 + row;                 // token index in the head
-        const bool row_valid = warp_valid && row < rows_valid && rg < S;
+        const int rg = q_row0 + row;                 // position in the head
+        bool row_valid = warp_valid && row < rows_valid && rg < S && !q_skip;
+        // output row: the position itself, or its T-major token in tiled mode
+        int orow_in_head = rg;
+        if constexpr (TILED) {
+            int pt, ph, pw;
+            tile_coords(row_valid ? rg : 0, a.H, a.W, a.tiles.t[tc], th, tw, pt, ph, pw);
+            if constexpr (PAD) {
+                const int tok = real_token(pt, ph, pw, a.real);
+                row_valid = row_valid && tok >= 0;
+                orow_in_head = tok < 0 ? 0 : tok;
+            } else {
+                orow_in_head = (pt * a.H + ph) * a.W + pw;
+            }
+        }
         const uint32_t t_lane = tmem + (static_cast<uint32_t>(warp * 32) << 16);
         const float sl2 = a.scale_log2;
         float m_ref = -INFINITY, l_sum = 0.f;
@@ -309,6 +385,27 @@ attn_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUt
                         #pragma unroll
                         for (int c = 0; c < BN; ++c)
                             if (c < g0 || c >= g0 + a.group) x[c] = -INFINITY;
+                    }
+                    if constexpr (PAD) {
+                        // a key box crossing the real grid's edge: mask its padding columns
+                        // (column u * 32 + lane is bit lane of kv[u])
+                        const AttnArgs::BoxGeom &g = a.geom[tc];
+                        const BoxAt c = box_at(static_cast<uint32_t>(kb), g, th, tw);
+                        if (c.t + g.bt > a.real.T || c.h + th > a.real.H || c.w + tw > a.real.W) {
+                            uint32_t kv[BN / 32];
+                            #pragma unroll
+                            for (int u = 0; u < BN / 32; ++u) {
+                                const uint32_t col = static_cast<uint32_t>(u * 32 + lane);
+                                const uint32_t dt = fdiv(col, g.bhw), r2 = col - dt * g.bhw.d;
+                                const uint32_t dh = fdiv(r2, g.bw), dw = r2 - dh * g.bw.d;
+                                kv[u] = __ballot_sync(0xffffffffu, c.t + static_cast<int>(dt) < a.real.T &&
+                                                                       c.h + static_cast<int>(dh) < a.real.H &&
+                                                                       c.w + static_cast<int>(dw) < a.real.W);
+                            }
+                            #pragma unroll
+                            for (int cc = 0; cc < BN; ++cc)
+                                if (!((kv[cc >> 5] >> (cc & 31)) & 1u)) x[cc] = -INFINITY;
+                        }
                     }
                 }
                 float mb = -INFINITY;
@@ -375,7 +472,7 @@ attn_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUt
         if (!ok && !*abort_flag) { report(a.status, DEV_TIMEOUT); *abort_flag = 1; }
 
         // ---- epilogue: O / l -> global ----
-        const size_t orow = static_cast<size_t>(bh) * S + rg;
+        const size_t orow = static_cast<size_t>(bh) * a.S_out + orow_in_head;
         bool have_o = ok && n_kb > 0;
         if (have_o) {
             if (!mbar_wait(pv_done, (n_kb - 1) & 1, abort_flag)) {
@@ -432,20 +529,34 @@ attn_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUt
     }
 }
 
-template <int D, int BN, bool WINDOW>
+template <int D, int BN, bool WINDOW, bool TILED = false, bool PAD = false>
 vsa_status run(const AttnLaunch &L, int *status, cudaStream_t st) {
     using C = Cfg<D, BN>;
-    CUtensorMap mq, mk, mv;
-    if (!make_tile_map(&mq, L.q, D, L.S, L.BH, BN) || !make_tile_map(&mk, L.k, D, L.S, L.BH, BN) ||
-        !make_tile_map(&mv, L.v, D, L.S, L.BH, BN))
-        return fail(VSA_ERR_CUDA, "cuTensorMapEncodeTiled failed (driver entry point or arguments)");
-    auto kern = attn_kernel<D, BN, WINDOW>;
+    AttnMaps maps = {};  // copied into the launch parameters
+    bool ok = true;
+    if constexpr (TILED) {
+        for (int c = 0; c < L.tiles.n; ++c) {
+            const int m = L.tiles.t[c] * L.tiles.h[c] * L.tiles.w[c] / BN;
+            const int bt = L.tiles.t[c] / m, bhh = L.tiles.h[c], bw = L.tiles.w[c];
+            // the real tensors: boxes reaching past them read zeros
+            ok = ok && make_box_map(&maps.q[c], L.q, D, L.T, L.Hg, L.Wg, L.BH, bt, bhh, bw) &&
+                 make_box_map(&maps.k[c], L.k, D, L.T, L.Hg, L.Wg, L.BH, bt, bhh, bw) &&
+                 make_box_map(&maps.v[c], L.v, D, L.T, L.Hg, L.Wg, L.BH, bt, bhh, bw);
+        }
+    } else {
+        ok = make_tile_map(&maps.q[0], L.q, D, L.S, L.BH, BN) && make_tile_map(&maps.k[0], L.k, D, L.S, L.BH, BN) &&
+             make_tile_map(&maps.v[0], L.v, D, L.S, L.BH, BN);
+    }
+    if (!ok) return fail(VSA_ERR_CUDA, "cuTensorMapEncodeTiled failed (driver entry point or arguments)");
+    auto kern = attn_kernel<D, BN, WINDOW, TILED, PAD>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
     if (e != cudaSuccess) return check_cuda(e, "cudaFuncSetAttribute(attention)");
     AttnArgs a;
-    a.S = L.S;
+    const int positions = TILED ? L.Tp * L.Hp * L.Wp : L.S;
+    a.S = positions;
+    a.S_out = L.S;
     a.BH = L.BH;
-    a.nq = (L.S + BN - 1) / BN;
+    a.nq = (positions + BN - 1) / BN;
     a.idx = L.idx;
     a.cnt = L.cnt;
     a.cap = L.cap;
@@ -459,8 +570,30 @@ vsa_status run(const AttnLaunch &L, int *status, cudaStream_t st) {
     a.out = L.o;
     a.out_f32 = L.out_f32;
     a.status = status;
+    a.H = TILED ? L.Hp : L.Hg;
+    a.W = TILED ? L.Wp : L.Wg;
+    a.real = RealGrid{L.T, L.Hg, L.Wg};
+    a.tiles = L.tiles;
+    a.choice = L.choice;
+    if (!TILED) a.tiles.n = 1;
+    for (int c = 0; c < kMaxTiles; ++c) {
+        auto &g = a.geom[c];
+        if (TILED && c < L.tiles.n) {
+            const int tt = L.tiles.t[c], th = L.tiles.h[c], tw = L.tiles.w[c];
+            const int m = tt * th * tw / BN;
+            g.m = make_fastdiv(m);
+            g.nthw = make_fastdiv((L.Hp / th) * (L.Wp / tw));
+            g.ntw = make_fastdiv(L.Wp / tw);
+            g.bhw = make_fastdiv(th * tw);
+            g.bw = make_fastdiv(tw);
+            g.bt = tt / m;
+        } else {
+            g.m = g.nthw = g.ntw = g.bhw = g.bw = make_fastdiv(1);
+            g.bt = 1;
+        }
+    }
     dim3 grid(a.nq, L.BH);
-    kern<<<grid, 192, C::SMEM, st>>>(mq, mk, mv, a);
+    kern<<<grid, 192, C::SMEM, st>>>(maps, a);
     return check_cuda(cudaGetLastError(), "attention launch");
 }
 
@@ -527,7 +660,16 @@ bool make_box_map(CUtensorMap *m, const void *ptr, int D, int T, int H, int W, i
 }
 
 vsa_status launch_attention(const AttnLaunch &L, int *status, cudaStream_t st) {
-    if (L.block == 128 || L.tiled) return launch_attention_pp(L, status, st);  // two query tiles per CTA
+    if (L.block == 128) return launch_attention_pp(L, status, st);  // two query tiles per CTA
+    if (L.tiled) {
+        const bool pad = L.Tp * L.Hp * L.Wp != L.S;
+        if (L.D == 128) {
+            if (L.block == 64) return pad ? run<128, 64, false, true, true>(L, status, st) : run<128, 64, false, true>(L, status, st);
+            return pad ? run<128, 32, false, true, true>(L, status, st) : run<128, 32, false, true>(L, status, st);
+        }
+        if (L.block == 64) return pad ? run<64, 64, false, true, true>(L, status, st) : run<64, 64, false, true>(L, status, st);
+        return pad ? run<64, 32, false, true, true>(L, status, st) : run<64, 32, false, true>(L, status, st);
+    }
     if (L.window) {
         if (L.D == 128) return run<128, 128, true>(L, status, st);
         return run<64, 128, true>(L, status, st);

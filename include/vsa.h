@@ -284,11 +284,13 @@ vsa_status vsa_block_sparse_attention(const void *q, const void *k, const void *
  * (the zero-padding recipe of "Adaptive tiling (SPADE)", Deviations and
  * notes) and only the S real rows of o are written.
  *   q, k, v  [B, n_heads, S, D] bf16, o [B, n_heads, S, D] in out_dtype, T-major
- *   tiles    every candidate of the same volume V, a multiple of 128, with
- *            tile.t divisible by V/128 (a 128-token block is tile.t*128/V
- *            whole (h, w) planes of the tile)
+ *   tiles    every candidate of the same volume V: 32 or 64 (a block is the
+ *            tile), or a multiple of 128 with tile.t divisible by V/128 (a
+ *            128-token block is tile.t*128/V whole (h, w) planes of the tile);
+ *            a block's box must fit inside the real grid (VSA_ERR_UNSUPPORTED
+ *            otherwise).  Lists count blocks of min(V, 128) tokens.
  *   choice   [B, n_heads] int32 or NULL (tile 0 for every head)
- *   group_stride  0, or a power of two s in [2, 128]: a key is then visible
+ *   group_stride  0, or (128-token blocks only) a power of two s in [2, 128]: a key is then visible
  *            to a query only if their positions (tile-contiguous order)
  *            differ by a multiple of s.  With tile (T, 1, 128 / T) and the
  *            diagonal list this is the temporal-only mask ("ADR-0001", step 1):

@@ -261,3 +261,92 @@ def test_spade_padded_full_size_sampled():
             if keep.any():
                 assert_attn_close(got[rows][keep], res["out_perm"][bi * 128:(bi + 1) * 128][keep],
                                   f"head {h} block {b}")
+
+
+# --------------------------------------------------------------------------
+# SPADE's own 64-token candidates on grids they do not divide
+# --------------------------------------------------------------------------
+
+SPADE64 = [(1, 4, 16), (1, 8, 8)]
+
+
+@pytest.mark.parametrize("D,grid", [(64, (3, 13, 20)), (128, (5, 10, 18))])
+def test_tiled_attention_64_token_boxes_mask_padding_keys(D, grid):
+    B, H = 1, 2
+    S = grid[0] * grid[1] * grid[2]
+    pg = vsa.padded_grid(grid, SPADE64)
+    Sp = pg[0] * pg[1] * pg[2]
+    nb = Sp // 64
+    q, k, v = (integer_grid((B, H, S, D), 94 + i, torch.bfloat16, DEV) for i in range(3))
+    choice = torch.tensor([0, 1], dtype=torch.int32, device=DEV)
+    idx, cnt = _lists_with_diagonal(nb, min(nb, 5), B * H, seed=D + nb)
+    ti = torch.as_tensor(idx, device=DEV).view(B, H, nb, -1)
+    tc = torch.as_tensor(cnt, device=DEV).view(B, H, nb)
+    o = vsa.block_sparse_attention_tiled(q, k, v, grid, SPADE64, choice, ti, tc, out_dtype=torch.float32)
+    for h, c in enumerate(choice.tolist()):
+        _, perm, real = _padded(grid, SPADE64, SPADE64[c])
+        qo, ko, vo = (_oracle_perm_padded(_np(x[0, h]), grid, SPADE64, SPADE64[c]) for x in (q, k, v))
+        want_p = oracle.block_sparse_attention(qo, ko, vo, idx[h], cnt[h], 64, key_ok=real[perm].astype(np.uint8))
+        want = np.zeros((Sp, D))
+        want[perm] = want_p
+        assert_attn_close(_np(o[0, h]), want[real], f"head {h}")
+
+
+def test_spade_64_token_candidates_on_padded_grid():
+    """The pages' case in small: a height no 64-token candidate divides.  One
+    candidate, integer-grid values: lists bit-exact with the oracle's."""
+    grid, tiles = (3, 13, 20), [(1, 8, 8)]
+    S = grid[0] * grid[1] * grid[2]
+    q, k, v = (integer_grid((1, 2, S, 64), 97 + i, torch.bfloat16, DEV) for i in range(3))
+    o, mid = vsa.spade_attention(q, k, v, grid, tiles, topk=3, out_dtype=torch.float32, return_intermediates=True)
+    for h in range(2):
+        res = oracle.spade_head(_np(q[0, h]), _np(k[0, h]), _np(v[0, h]), grid, tiles, 3)
+        assert np.array_equal(mid["idx"][0, h].cpu().numpy(), res["idx"])
+        assert np.array_equal(mid["cnt"][0, h].cpu().numpy(), res["cnt"])
+        assert_attn_close(_np(o[0, h]), res["out"], f"head {h}")
+
+
+def test_spade_64_token_candidates_wan_grid_sampled():
+    """16 x 45 x 80 with SPADE's (1, 4, 16) and (1, 8, 8) candidates (padded to
+    16 x 48 x 80, 960 blocks of 64), 4 heads, k = 96: choices where clear, lists
+    valid top-k sets under the oracle's scores, sampled real rows compared."""
+    grid = (16, 45, 80)
+    kinds = ["spatial", "temporal", "spatial", "temporal"]
+    q, k, v = smooth_qkv(1, 4, grid, 128, seed=98, kinds=kinds, device=DEV)
+    kk = 96
+    o, mid = vsa.spade_attention(q, k, v, grid, SPADE64, topk=kk, out_dtype=torch.float32, return_intermediates=True)
+    pg = oracle.padded_grid(grid, SPADE64)
+    nb = pg[0] * pg[1] * pg[2] // 64
+    assert mid["idx"].shape[2] == nb
+    checked = 0
+    for h in range(4):
+        res = oracle.spade_head(_np(q[0, h]), _np(k[0, h]), _np(v[0, h]), grid, SPADE64, kk,
+                                query_blocks=_sample_blocks(nb, 300 + h))
+        margin = np.sort(res["cohesion"])[-1] - np.sort(res["cohesion"])[-2]
+        if margin <= 1e-4:
+            continue
+        assert int(mid["choice"][h]) == res["choice"]
+        gi, gc = mid["idx"][0, h].cpu().numpy(), mid["cnt"][0, h].cpu().numpy()
+        s = res["score"]
+        same = 0
+        for i in range(nb):
+            sel = set(gi[i, :gc[i]].tolist())
+            forced = {0, i}
+            assert forced <= sel and kk <= len(sel) <= kk + len(forced)
+            kth = np.sort(s[i])[::-1][kk - 1]
+            tol = 1e-5 * max(1.0, float(np.abs(s[i]).max()))
+            assert all(s[i, j] >= kth - tol for j in sel - forced), (h, i)
+            same += int(np.array_equal(gi[i], res["idx"][i]))
+        assert same >= 0.9 * nb
+        real_p = oracle.real_tokens(grid, pg)[res["perm"]]
+        got = _np(mid["out_perm"][0, h])
+        blocks = _sample_blocks(nb, 300 + h)
+        for bi, b in enumerate(blocks):
+            if not np.array_equal(gi[b], res["idx"][b]):
+                continue
+            rows = np.arange(b * 64, (b + 1) * 64)
+            keep = real_p[rows]
+            if keep.any():
+                assert_attn_close(got[rows][keep], res["out_perm"][bi * 64:(bi + 1) * 64][keep], f"head {h} block {b}")
+        checked += 1
+    assert checked >= 2

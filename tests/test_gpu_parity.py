@@ -547,3 +547,54 @@ def test_structured_full_size_sampled(kind):
     want = oracle.block_sparse_attention(qp, kp, vp, idx, cnt, 128, g, rows=rows)
     got = _np(o[b, h])[perm[rows]]
     assert_attn_close(got, want, kind)
+
+
+# --------------------------------------------------------------------------
+# tiled mode with 32- and 64-token tiles (a block is the tile itself)
+# --------------------------------------------------------------------------
+
+@pytest.mark.parametrize("D,grid,tiles,values", [
+    (128, (4, 16, 32), [(1, 4, 16), (1, 8, 8)], "smooth"),    # 64-token candidates, as in SPADE's own configs
+    (64, (4, 16, 32), [(1, 4, 16), (1, 8, 8)], "integer"),
+    (64, (4, 8, 16), [(2, 4, 4), (1, 4, 8)], "integer"),      # 32-token candidates
+])
+def test_small_block_tiled_attention_matches_permuted_path_and_oracle(D, grid, tiles, values):
+    """Blocks of 32 and 64 tokens read as TMA boxes from T-major tensors equal
+    permute -> attention -> unpermute bit for bit, and the oracle."""
+    B, H = 1, 3
+    S = grid[0] * grid[1] * grid[2]
+    block = tiles[0][0] * tiles[0][1] * tiles[0][2]
+    nb = S // block
+    if values == "integer":
+        q, k, v = (integer_grid((B, H, S, D), 91 + i, torch.bfloat16, DEV) for i in range(3))
+    else:
+        q, k, v = smooth_qkv(B, H, grid, D, seed=92, device=DEV)
+    choice = torch.tensor([1, 0, 1], dtype=torch.int32, device=DEV)
+    idx, cnt = _random_lists(nb, min(nb, 5), B * H, seed=D + nb + block)
+    ti = torch.as_tensor(idx, device=DEV).view(B, H, nb, -1)
+    tc = torch.as_tensor(cnt, device=DEV).view(B, H, nb)
+    o = vsa.block_sparse_attention_tiled(q, k, v, grid, tiles, choice, ti, tc, out_dtype=torch.float32)
+    qp, kp, vp = (vsa.permute(x, grid, tiles, choice) for x in (q, k, v))
+    op = vsa.block_sparse_attention(qp, kp, vp, ti, tc, block, out_dtype=torch.float32)
+    assert torch.equal(o, vsa.unpermute(op, grid, tiles, choice))
+    for h, c in enumerate(choice.tolist()):
+        perm = oracle.tile_permutation(grid, tiles[c])
+        qo, ko, vo = (oracle.permute_rows(_np(x[0, h]), perm) for x in (q, k, v))
+        want = oracle.block_sparse_attention(qo, ko, vo, idx[h], cnt[h], block)
+        assert_attn_close(_np(o[0, h])[perm], want, f"head {h}")
+
+
+def test_spade_64_token_candidates_tiled_equals_explicit():
+    """The whole composition with SPADE's 64-token candidates: tiled mode (boxes)
+    and the explicit permute path give the same bits, and the lists match the
+    oracle's on integer-grid values."""
+    grid, tiles = (4, 16, 32), [(1, 4, 16)]
+    S = grid[0] * grid[1] * grid[2]
+    q, k, v = (integer_grid((1, 2, S, 128), 93 + i, torch.bfloat16, DEV) for i in range(3))
+    o, mid = vsa.spade_attention(q, k, v, grid, tiles, topk=4, out_dtype=torch.float32, return_intermediates=True)
+    oe = vsa.spade_attention(q, k, v, grid, tiles, topk=4, out_dtype=torch.float32, tiled=False)
+    assert torch.equal(o, oe)
+    for h in range(2):
+        res = oracle.spade_head(_np(q[0, h]), _np(k[0, h]), _np(v[0, h]), grid, tiles, 4)
+        assert np.array_equal(mid["idx"][0, h].cpu().numpy(), res["idx"])
+        assert_attn_close(_np(o[0, h]), res["out"], f"head {h}")
