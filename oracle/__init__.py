@@ -43,6 +43,7 @@ def lib():
         L.orc_block_minmax.argtypes = [P, i64, i32, i32, P, P]
         L.orc_block_scores.argtypes = [P, P, P, P, i64, i32, P]
         L.orc_topk_block_list.argtypes = [P, i64, i32, i32, i32, i32, P, P]
+        L.orc_topp_block_list.argtypes = [P, i64, dbl, dbl, i32, i32, i32, P, P]
         L.orc_topk_block_list.restype = i32
         L.orc_tile_neighbourhood_list.argtypes = [i32] * 11 + [P, P, P]
         L.orc_tile_neighbourhood_list.restype = i32
@@ -215,6 +216,23 @@ def topk_block_list(score, k: int, n_sink: int = 1, diag_halfwidth: int = 0,
     rc = lib().orc_topk_block_list(_ptr(s), nb, k, n_sink, diag_halfwidth, cap, _ptr(idx), _ptr(cnt))
     if rc != 0:
         raise ValueError("cap too small for the top-k list")
+    return idx, cnt
+
+
+def topp_block_list(score, p: float, scale: float, n_sink: int = 1, diag_halfwidth: int = 0,
+                    cap: Optional[int] = None):
+    """Top-p (mass budget) lists: per row, the shortest prefix in descending
+    score order (ties: lower index) whose softmax(scale * score) mass reaches
+    p, plus the sink and diagonal blocks (see orc_topp_block_list)."""
+    s = np.ascontiguousarray(score, np.float64)
+    nb = s.shape[0]
+    cap = nb if cap is None else cap
+    idx = np.empty((nb, cap), np.int32)
+    cnt = np.empty(nb, np.int32)
+    rc = lib().orc_topp_block_list(_ptr(s), nb, ctypes.c_double(p), ctypes.c_double(scale), n_sink,
+                                   diag_halfwidth, cap, _ptr(idx), _ptr(cnt))
+    if rc != 0:
+        raise ValueError("cap too small for the top-p list")
     return idx, cnt
 
 

@@ -284,6 +284,56 @@ int orc_topk_block_list(const double *score, int64_t nb, int k, int n_sink,
     return rc;
 }
 
+/* Top-p (mass budget) block list  ["Adaptive tiling (SPADE)", function
+ * table: top_p_block_mask is named as one of the functions the recipe
+ * composes with, with no definition.  Reading: a row's probabilities are
+ * softmax(scale * s) over its key blocks; the kept blocks are the shortest
+ * prefix of the row in descending score order (equal scores: lower index
+ * first) whose probabilities sum to at least p, and the sink and diagonal
+ * blocks are ORed in as for top-k.]  Same output layout as
+ * orc_topk_block_list.  Returns 0, or -1 if a row needs more than cap slots. */
+int orc_topp_block_list(const double *score, int64_t nb, double p, double scale, int n_sink,
+                        int diag_halfwidth, int cap, int32_t *idx, int32_t *cnt)
+{
+    orc_scored *row = (orc_scored *)malloc(sizeof(orc_scored) * (size_t)nb);
+    unsigned char *keep = (unsigned char *)malloc((size_t)nb);
+    int rc = 0;
+    for (int64_t i = 0; i < nb; ++i) {
+        double m = -INFINITY;
+        for (int64_t j = 0; j < nb; ++j) {
+            row[j].score = score[i * nb + j];
+            row[j].j = j;
+            if (row[j].score > m) m = row[j].score;
+        }
+        double z = 0.0;
+        for (int64_t j = 0; j < nb; ++j) z += exp(scale * (score[i * nb + j] - m));
+        qsort(row, (size_t)nb, sizeof(orc_scored), orc_cmp_scored);
+        memset(keep, 0, (size_t)nb);
+        double acc = 0.0;
+        for (int64_t r = 0; r < nb; ++r) {
+            keep[row[r].j] = 1;
+            acc += exp(scale * (row[r].score - m));
+            if (acc >= p * z) break;
+        }
+        for (int64_t j = 0; j < nb; ++j) {
+            if (j < n_sink) keep[j] = 1;
+            if (llabs(j - i) <= diag_halfwidth) keep[j] = 1;
+        }
+        int c = 0;
+        for (int64_t j = 0; j < nb; ++j)
+            if (keep[j]) {
+                if (c < cap) idx[i * cap + c] = (int32_t)j;
+                ++c;
+            }
+        if (c > cap) rc = -1;
+        for (int s2 = c; s2 < cap; ++s2) idx[i * cap + s2] = -1;
+        cnt[i] = c;
+    }
+    free(keep);
+    free(row);
+    return rc;
+}
+
 /* ----------------------------------------------------------------------- */
 /* Structured masks as block lists  [ADR step 1: spatial_only_mask,         */
 /* temporal_only_mask, sliding_tile_block_mask]                             */

@@ -465,3 +465,73 @@ def test_padded_cohesion_by_brute_force():
             pairs = [n[i] @ n[j] for i in range(len(n)) for j in range(len(n)) if i != j]
             vals.append(float(np.mean(pairs)))
         assert abs(got[c] - np.mean(vals)) < 1e-12, (c, got[c], np.mean(vals))
+
+
+# --------------------------------------------------------------------------
+# top-p (mass budget) lists: the pages name top_p_block_mask only; the
+# reading (softmax(scale * score) mass, shortest descending prefix reaching
+# p, ties to the lower index, static blocks ORed in) is pinned by properties
+# that do not restate the algorithm
+# --------------------------------------------------------------------------
+
+def _topp_sets(score, p, scale, n_sink=0, dw=-1):
+    idx, cnt = oracle.topp_block_list(score, p, scale, n_sink, dw)
+    return [set(idx[i, :cnt[i]].tolist()) for i in range(score.shape[0])]
+
+
+def _probs(row, scale):
+    e = np.exp(scale * (row - row.max()))
+    return e / e.sum()
+
+
+@pytest.mark.parametrize("seed", [0, 1, 2])
+def test_topp_is_the_smallest_upper_set_reaching_p(seed):
+    rng = np.random.default_rng(seed)
+    nb = 23
+    score = rng.normal(size=(nb, nb)) * 4
+    for p in (0.05, 0.3, 0.6, 0.9, 0.999):
+        for i, kept in enumerate(_topp_sets(score, p, 0.7)):
+            pr = _probs(score[i], 0.7)
+            rest = set(range(nb)) - kept
+            # an upper set: no dropped block scores above a kept one
+            assert not rest or min(score[i, list(kept)]) >= max(score[i, list(rest)])
+            # it reaches p, and without its lowest block it would not
+            assert pr[list(kept)].sum() >= p - 1e-12
+            low = min(kept, key=lambda j: (score[i, j], -j))
+            assert pr[list(kept - {low})].sum() < p + 1e-12
+
+
+def test_topp_closed_forms():
+    rng = np.random.default_rng(5)
+    nb = 17
+    score = rng.normal(size=(nb, nb))
+    # p = 1 keeps every block; a vanishing p keeps the row's maximum alone
+    assert all(k == set(range(nb)) for k in _topp_sets(score, 1.0, 1.0))
+    assert all(k == {int(np.argmax(score[i]))} for i, k in enumerate(_topp_sets(score, 1e-12, 1.0)))
+    # scale 0: uniform probabilities, so the mass budget is a count budget: the
+    # ceil(p nb) highest scores, i.e. the top-k list with k = ceil(p nb)
+    for p in (0.1, 0.5, 0.77):
+        k = int(np.ceil(p * nb - 1e-9))
+        ti, tc = oracle.topk_block_list(score, k, 0, -1)
+        assert _topp_sets(score, p, 0.0) == [set(ti[i, :tc[i]].tolist()) for i in range(nb)]
+    # equal scores rank the lower index first
+    tie = np.zeros((4, 4))
+    assert _topp_sets(tie, 0.5, 1.0)[0] == {0, 1}
+
+
+def test_topp_invariances_and_static_blocks():
+    rng = np.random.default_rng(6)
+    nb = 19
+    score = rng.normal(size=(nb, nb)) * 2
+    base = _topp_sets(score, 0.6, 1.3)
+    assert _topp_sets(score + 7.5, 0.6, 1.3) == base           # softmax is shift invariant
+    assert _topp_sets(score * 2.0, 0.6, 0.65) == base          # only scale * score matters
+    prev = None
+    for p in (0.2, 0.4, 0.6, 0.8):                             # monotone in p
+        cur = _topp_sets(score, p, 1.3)
+        if prev is not None:
+            assert all(a <= b for a, b in zip(prev, cur))
+        prev = cur
+    with_static = _topp_sets(score, 0.6, 1.3, n_sink=2, dw=1)
+    for i, (k, ks) in enumerate(zip(base, with_static)):
+        assert ks == k | {0, 1} | {j for j in range(nb) if abs(j - i) <= 1}
