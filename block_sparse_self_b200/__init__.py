@@ -61,6 +61,7 @@ def lib() -> ctypes.CDLL:
         "vsa_block_summaries_tiled": ([P, I, I, I, I, I, D3, P, I, P, I, P, P, P], I),
         "vsa_block_scores": ([P, P, P, P, I, I, I, I, I, P, P], I),
         "vsa_topk_block_mask": ([P, I, I, I, I, I, I, P, P, I, P], I),
+        "vsa_topp_block_mask": ([P, I, I, I, F, F, I, I, P, P, I, P], I),
         "vsa_structured_block_list": ([I, D3, D3, D3, I, P, P, I, P, P], I),
         "vsa_block_sparse_attention": ([P, P, P, P, I, I, I, I, I, I, P, P, I, I, I, F, P], I),
         "vsa_block_sparse_attention_tiled": ([P, P, P, P, I, I, I, I, I, D3, P, I, P, P, P, I, I, I, F, P], I),
@@ -291,6 +292,23 @@ def topk_block_mask(scores: torch.Tensor, k: int, n_sink_blocks: int = 1, diag_h
     return idx, cnt
 
 
+def topp_block_mask(scores: torch.Tensor, p: float, scale: float, n_sink_blocks: int = 1, diag_halfwidth: int = 0,
+                    cap: Optional[int] = None):
+    """(idx [B,H,nb,cap] int32, cnt [B,H,nb] int32): per row the shortest
+    descending-score prefix whose softmax(scale * scores) mass reaches p, plus
+    sink and diagonal blocks, ascending, -1 padded (see include/vsa.h)."""
+    _cuda(scores, "scores")
+    if scores.dtype != torch.float32 or scores.dim() != 4 or scores.shape[-1] != scores.shape[-2]:
+        raise ValueError("scores must be fp32 [B, H, nb, nb]")
+    B, H, nb, _ = scores.shape
+    cap = nb if cap is None else int(cap)
+    idx = torch.empty(B, H, nb, max(cap, 1), dtype=torch.int32, device=scores.device)
+    cnt = torch.empty(B, H, nb, dtype=torch.int32, device=scores.device)
+    _check(lib().vsa_topp_block_mask(_ptr(scores), B, H, nb, float(p), float(scale), int(n_sink_blocks),
+                                     int(diag_halfwidth), _ptr(idx), _ptr(cnt), cap, _stream(scores.device)))
+    return idx, cnt
+
+
 _KINDS = {"spatial": MASK_SPATIAL, "temporal": MASK_TEMPORAL, "sliding_tile": MASK_SLIDING_TILE}
 
 
@@ -438,9 +456,17 @@ def topk_budget(nb: int, budget: float) -> int:
     return max(1, int(math.floor(budget * nb)))
 
 
+def _select_blocks(scores, kk, n_sink_blocks, diag_halfwidth, top_p, top_p_scale, D):
+    if top_p is None:
+        return topk_block_mask(scores, kk, n_sink_blocks, diag_halfwidth)
+    sc = (1.0 / math.sqrt(D)) if top_p_scale is None else float(top_p_scale)
+    return topp_block_mask(scores, top_p, sc, n_sink_blocks, diag_halfwidth)
+
+
 def spade_attention(q, k, v, grid, tiles, budget: Optional[float] = None, topk: Optional[int] = None,
                     n_sink_blocks: int = 1, diag_halfwidth: int = 0, scale: Optional[float] = None,
-                    out_dtype=None, return_intermediates: bool = False, tiled: Optional[bool] = None):
+                    out_dtype=None, return_intermediates: bool = False, tiled: Optional[bool] = None,
+                    top_p: Optional[float] = None, top_p_scale: Optional[float] = None):
     """Adaptive tiling -> permutation -> min/max block scores -> top-k + sink +
     diagonal -> block-sparse attention -> inverse permutation, all on the GPU.
 
@@ -450,6 +476,10 @@ def spade_attention(q, k, v, grid, tiles, budget: Optional[float] = None, topk: 
     padding holds no query of the cohesion, takes part in the summaries as
     zero tokens and is masked as keys; the result holds the real tokens only.
     Padded grids run in tiled mode, which masks the padding keys.
+
+    top_p selects key blocks by mass instead of count (topp_block_mask), with
+    probabilities softmax(top_p_scale * scores), top_p_scale defaulting to
+    1/sqrt(D); budget and topk are then unused.
 
     tiled=True runs the permutation inside the summaries and attention kernels
     (no permuted copies; blocks of 32, 64 or 128 tokens, see tiled_supported); tiled=False
@@ -480,7 +510,7 @@ def spade_attention(q, k, v, grid, tiles, budget: Optional[float] = None, topk: 
         qmax, qmin = block_summaries_tiled(q, grid, tiles, choice, block)
         kmax, kmin = block_summaries_tiled(k, grid, tiles, choice, block)
         scores = block_scores(qmax, qmin, kmax, kmin)
-        idx, cnt = topk_block_mask(scores, kk, n_sink_blocks, diag_halfwidth)
+        idx, cnt = _select_blocks(scores, kk, n_sink_blocks, diag_halfwidth, top_p, top_p_scale, D)
         o = block_sparse_attention_tiled(qb, kb, vb, grid, tiles, choice, idx, cnt, scale, out_dtype)
         if return_intermediates:
             qp, kp, vp, op = (permute(x, grid, tiles, choice) for x in (q, k, v, o))
@@ -489,7 +519,7 @@ def spade_attention(q, k, v, grid, tiles, budget: Optional[float] = None, topk: 
         qmax, qmin = block_summaries(qp, block)
         kmax, kmin = block_summaries(kp, block)
         scores = block_scores(qmax, qmin, kmax, kmin)
-        idx, cnt = topk_block_mask(scores, kk, n_sink_blocks, diag_halfwidth)
+        idx, cnt = _select_blocks(scores, kk, n_sink_blocks, diag_halfwidth, top_p, top_p_scale, D)
         op = block_sparse_attention(qp, kp, vp, idx, cnt, block, 0, scale, out_dtype)
         o = unpermute(op, grid, tiles, choice)
     if return_intermediates:

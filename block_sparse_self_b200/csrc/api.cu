@@ -341,6 +341,25 @@ vsa_status vsa_topk_block_mask(const float *scores, int B, int n_heads, int nb, 
                       "topk launch");
 }
 
+vsa_status vsa_topp_block_mask(const float *scores, int B, int n_heads, int nb, float p, float scale,
+                               int n_sink_blocks, int diag_halfwidth, int32_t *idx, int32_t *cnt, int cap,
+                               void *stream) {
+    VSA_REQUIRE(B >= 1 && n_heads >= 1, "B and n_heads must be >= 1");
+    VSA_REQUIRE(nb >= 1, "nb must be >= 1, got %d", nb);
+    VSA_REQUIRE(p > 0.f && p <= 1.f, "p must be in (0, 1], got %g", static_cast<double>(p));
+    VSA_REQUIRE(scale >= 0.f && scale < 3.0e38f, "scale must be finite and >= 0, got %g", static_cast<double>(scale));
+    VSA_REQUIRE(n_sink_blocks >= 0 && n_sink_blocks <= nb, "n_sink_blocks must be in [0, nb], got %d",
+                n_sink_blocks);
+    VSA_REQUIRE(diag_halfwidth >= -1, "diag_halfwidth must be >= -1 (-1 = no diagonal), got %d", diag_halfwidth);
+    VSA_REQUIRE(cap >= nb, "cap (%d) must be >= nb (%d): a top-p list can hold every block", cap, nb);
+    VSA_REQUIRE(aligned4(scores) && aligned4(idx) && aligned4(cnt),
+                "scores, idx and cnt must be non-NULL 4-byte aligned device pointers");
+    if (nb > 1024) return fail(VSA_ERR_UNSUPPORTED, "top-p lists support rows of at most 1024 blocks, got %d", nb);
+    return check_cuda(launch_topp(scores, B * n_heads, nb, p, scale, n_sink_blocks, diag_halfwidth, idx, cnt, cap,
+                                  as_stream(stream)),
+                      "topp launch");
+}
+
 vsa_status vsa_structured_block_list(vsa_mask_kind kind, vsa_dims3 grid, vsa_dims3 tile, vsa_dims3 radius, int block,
                                      int32_t *idx, int32_t *cnt, int cap, int *group_size_out, void *stream) {
     VSA_REQUIRE(grid.t > 0 && grid.h > 0 && grid.w > 0, "grid dimensions must be positive");

@@ -223,6 +223,26 @@ vsa_status vsa_topk_block_mask(const float *scores, int B, int n_heads, int nb, 
                                int n_sink_blocks, int diag_halfwidth, int32_t *idx,
                                int32_t *cnt, int cap, void *stream);
 
+/* Top-p (mass budget) key-block lists.  "Adaptive tiling (SPADE)" names
+ * top_p_block_mask among the functions its recipe composes with but does not
+ * define it; this is the reading used here.  For each row (b, head, i):
+ * probabilities softmax_j(scale * scores[bh, i, j]); the kept blocks are the
+ * shortest prefix of the row in descending score order (equal scores: lower
+ * index first) whose probabilities sum to at least p; then, as for
+ * vsa_topk_block_mask, blocks j < n_sink_blocks and |j - i| <= diag_halfwidth
+ * (-1: none) are ORed in, and the list is written in ascending order with
+ * -1 in unused slots.
+ *   scores  [B, n_heads, nb, nb] fp32 (vsa_block_scores)
+ *   p       in (0, 1]; scale >= 0 (0 makes every block equally likely, so the
+ *           list is the top-k list with k = ceil(p * nb))
+ *   idx     [B, n_heads, nb, cap] int32 with cap >= nb; cnt [B, n_heads, nb]
+ * Masses are accumulated in fp32: a block whose inclusion changes the
+ * prefix mass across p by less than about 1e-6 * (row mass) may be taken or
+ * left.  Rows of more than 1024 blocks return VSA_ERR_UNSUPPORTED.          */
+vsa_status vsa_topp_block_mask(const float *scores, int B, int n_heads, int nb, float p, float scale,
+                               int n_sink_blocks, int diag_halfwidth, int32_t *idx, int32_t *cnt, int cap,
+                               void *stream);
+
 /* ------------------------------------------------------------------------ */
 /* Structured static masks as block lists.  "ADR-0001", step 1
  * (spatial_only_mask, temporal_only_mask, sliding_tile_block_mask).

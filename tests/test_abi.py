@@ -129,6 +129,22 @@ def test_padded_grid_argument_errors(L):
     assert L.vsa_padded_grid(Dims3(2048, 2048, 1024), huge, nh, ctypes.byref(out)) == vsa.ERR_INVALID_ARGUMENT
 
 
+def test_topp_argument_errors(L):
+    idx, cnt = FAKE, ctypes.c_void_p(0x20000)
+    ok = dict(B=1, H=1, nb=8, p=0.5, scale=1.0, sink=1, dw=0, cap=8)
+    def call(**kw):
+        a = dict(ok, **kw)
+        return L.vsa_topp_block_mask(FAKE, a["B"], a["H"], a["nb"], a["p"], a["scale"], a["sink"], a["dw"],
+                                     idx, cnt, a["cap"], NULL)
+    assert call(p=0.0) == vsa.ERR_INVALID_ARGUMENT
+    assert call(p=1.5) == vsa.ERR_INVALID_ARGUMENT
+    assert call(scale=-1.0) == vsa.ERR_INVALID_ARGUMENT
+    assert call(cap=7) == vsa.ERR_INVALID_ARGUMENT     # a list can hold every block
+    assert call(sink=9) == vsa.ERR_INVALID_ARGUMENT
+    assert call(dw=-2) == vsa.ERR_INVALID_ARGUMENT
+    assert call(nb=2000, cap=2000) == vsa.ERR_UNSUPPORTED
+
+
 def test_structured_list_argument_errors(L):
     g = ctypes.c_int(0)
     grid = Dims3(32, 48, 80)

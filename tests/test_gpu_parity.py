@@ -598,3 +598,72 @@ def test_spade_64_token_candidates_tiled_equals_explicit():
         res = oracle.spade_head(_np(q[0, h]), _np(k[0, h]), _np(v[0, h]), grid, tiles, 4)
         assert np.array_equal(mid["idx"][0, h].cpu().numpy(), res["idx"])
         assert_attn_close(_np(o[0, h]), res["out"], f"head {h}")
+
+
+# --------------------------------------------------------------------------
+# top-p (mass budget) lists
+# --------------------------------------------------------------------------
+
+def _check_topp_row(kept, row, p, scale, what):
+    """kept must be an upper set of the row (ties by lower index) whose mass
+    reaches p while it would not without its last block, within fp32 error."""
+    nb = row.shape[0]
+    e = np.exp(scale * (row - row.max()))
+    pr = e / e.sum()
+    order = sorted(range(nb), key=lambda j: (-row[j], j))
+    n = len(kept)
+    assert kept == set(order[:n]), what
+    tol = 1e-5
+    assert pr[order[:n]].sum() >= p - tol, what
+    assert n == 1 or pr[order[:n - 1]].sum() < p + tol, what
+
+
+@pytest.mark.parametrize("nb", [1, 5, 33, 240, 960])
+@pytest.mark.parametrize("p,scale", [(0.1, 0.3), (0.5, 0.05), (0.9, 0.3), (0.99, 1.0)])
+def test_topp_lists_against_oracle(nb, p, scale):
+    scores = random_scores((1, 2, nb, nb), seed=nb + int(p * 100), device=DEV) * 4.0
+    idx, cnt = vsa.topp_block_mask(scores, p, scale, n_sink_blocks=0, diag_halfwidth=-1)
+    s = _np(scores).astype(np.float64)
+    same = 0
+    for h in range(2):
+        oi, oc = oracle.topp_block_list(s[0, h], p, scale, 0, -1)
+        gi, gc = idx[0, h].cpu().numpy(), cnt[0, h].cpu().numpy()
+        for i in range(nb):
+            kept = set(gi[i, :gc[i]].tolist())
+            assert (gi[i, :gc[i]] == np.sort(gi[i, :gc[i]])).all() and (gi[i, gc[i]:] == -1).all()
+            _check_topp_row(kept, s[0, h, i], p, scale, (h, i))
+            same += int(gc[i] == oc[i] and (gi[i, :gc[i]] == oi[i, :oc[i]]).all())
+    assert same >= 0.98 * 2 * nb   # a block whose mass straddles p within fp32 error may differ
+
+
+def test_topp_static_blocks_and_uniform_case():
+    nb = 96
+    scores = random_scores((1, 1, nb, nb), seed=7, device=DEV) * 4.0
+    s = _np(scores).astype(np.float64)[0, 0]
+    idx, cnt = vsa.topp_block_mask(scores, 0.3, 0.2, n_sink_blocks=2, diag_halfwidth=1)
+    oi, oc = oracle.topp_block_list(s, 0.3, 0.2, 2, 1)
+    gi, gc = idx[0, 0].cpu().numpy(), cnt[0, 0].cpu().numpy()
+    for i in range(nb):
+        assert {0, 1} | {j for j in range(max(0, i - 1), min(nb, i + 2))} <= set(gi[i, :gc[i]].tolist())
+    assert (np.array([np.array_equal(gi[i, :gc[i]], oi[i, :oc[i]]) for i in range(nb)])).mean() >= 0.98
+    # scale 0: every block equally likely, so the list is the top-k list, k = ceil(p nb)
+    p = 0.37   # p * nb = 35.52
+    ui, uc = vsa.topp_block_mask(scores, p, 0.0, n_sink_blocks=0, diag_halfwidth=-1)
+    ki, kc = vsa.topk_block_mask(scores, 36, n_sink_blocks=0, diag_halfwidth=-1, cap=nb)
+    assert torch.equal(uc, kc) and torch.equal(ui, ki)
+
+
+def test_spade_top_p_end_to_end():
+    w = WORKLOADS["tiny_s256"]
+    q, k, v = make_qkv(w, device=DEV)
+    o, mid = vsa.spade_attention(q, k, v, w.grid, list(w.tiles), top_p=0.6, top_p_scale=0.25,
+                                 out_dtype=torch.float32, return_intermediates=True)
+    for h in range(w.heads):
+        s = _np(mid["scores"][0, h]).astype(np.float64)
+        oi, oc = oracle.topp_block_list(s, 0.6, 0.25, 1, 0)
+        gi, gc = mid["idx"][0, h].cpu().numpy(), mid["cnt"][0, h].cpu().numpy()
+        assert np.array_equal(gc, oc) and all(np.array_equal(gi[i, :gc[i]], oi[i, :oc[i]]) for i in range(len(gc)))
+        perm = oracle.tile_permutation(w.grid, w.tiles[0])
+        qo, ko, vo = (oracle.permute_rows(_np(x[0, h]), perm) for x in (q, k, v))
+        want = oracle.block_sparse_attention(qo, ko, vo, oi, oc, w.block)
+        assert_attn_close(_np(o[0, h])[perm], want, f"head {h}")
