@@ -25,6 +25,7 @@ import dataclasses
 import datetime
 import hashlib
 import json
+import math
 import os
 import statistics
 import subprocess
@@ -546,6 +547,27 @@ def run_ours(args, w):
             extra["explicit_permute_" + w.name] = {"ms_per_step": ex_ms, "phase_ms": ex.phase_ms(),
                                                    "same_output": bool(torch.equal(ex.last["o"], step.last["o"]))}
             del ex
+        # top-p (mass budget) lists on the same scores, in place of the top-k lists
+        import block_sparse_self_b200 as vsa
+        sc = step.last["scores"]
+        p_mass, p_scale = 0.5, 1.0 / math.sqrt(w.D)
+        tp = {}
+        for _ in range(3):
+            vsa.topp_block_mask(sc, p_mass, p_scale)
+        ev = [torch.cuda.Event(enable_timing=True) for _ in range(2)]
+        ev[0].record()
+        n_rep = 5
+        for _ in range(n_rep):
+            ti, tc = vsa.topp_block_mask(sc, p_mass, p_scale)
+        ev[1].record()
+        torch.cuda.synchronize()
+        tp["ms_per_call"] = ev[0].elapsed_time(ev[1]) / n_rep
+        tp["p"], tp["scale"] = p_mass, p_scale
+        tp["mean_blocks_per_row"] = float(tc.float().mean().item())
+        tp["bytes"] = float(sc.numel() * 4 + ti.numel() * 4 + tc.numel() * 4)
+        tp["gbs"] = tp["bytes"] / tp["ms_per_call"] / 1e6
+        extra["topp_lists_" + w.name] = tp
+        del ti, tc
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
