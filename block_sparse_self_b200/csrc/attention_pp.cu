@@ -689,10 +689,563 @@ vsa_status run_pp(const AttnLaunch &L, int *status, cudaStream_t st) {
     return check_cuda(cudaGetLastError(), "attention launch (two tiles)");
 }
 
+// One query tile and one key block per CTA (lists of a single block, such as
+// the temporal-only mask's diagonal): Q, K and V tiles, one S and one O in
+// 256 tensor-memory columns, so two CTAs share an SM and one's loads overlap
+// the other's MMAs and softmax.  The two-tile kernel above cannot hide its
+// set-up and drain behind one block per tile.
+template <int D>
+struct OneCfg {
+    static constexpr int KSLABS = D / 64;
+    static constexpr int SLAB = 128 * 128;         // 128 rows x 128 bytes
+    static constexpr int TILE_BYTES = SLAB * KSLABS;  // Q, K or V tile of 128 rows
+    static constexpr int NK = 1;                   // K ring depth
+    static constexpr int NV = 1;                   // V ring depth
+    static constexpr int NS = 1;                   // S buffers in tensor memory
+    static constexpr int O_COL = NS * 128;         // O after the S buffers
+    static constexpr int N_BARS = 1 + 2 * NK + 2 * NV + NS + 2 + NS + 1;
+    static constexpr int SMEM = 1024 + (1 + NK + NV) * TILE_BYTES + N_BARS * 8 + 64;
+    static_assert(SMEM <= 232448, "shared memory");
+    static constexpr int TMEM_COLS = 256;
+    static_assert(O_COL + D <= TMEM_COLS, "tensor memory");
+    static_assert(2 * (SMEM + 1024) <= 233472, "two CTAs per SM");
+};
+constexpr int kOneThreads = 192;  // warps 0-3 softmax/epilogue, 4 TMA producer, 5 MMA issuer and TMEM owner
+
+template <int D, bool WINDOW, bool TILED, bool PAD>
+__global__ void __launch_bounds__(kOneThreads, 2)
+attn_one_kernel(const __grid_constant__ MapSet maps, const PPArgs a) {
+    using C = OneCfg<D>;
+    constexpr int BN = 128;
+    constexpr int NS = C::NS;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *base = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    uint8_t *sQ = base;                                  // [TILE]
+    uint8_t *sK = sQ + C::TILE_BYTES;                    // [NK][TILE]
+    uint8_t *sV = sK + C::NK * C::TILE_BYTES;            // [NV][TILE]
+    uint64_t *q_full = reinterpret_cast<uint64_t *>(sV + C::NV * C::TILE_BYTES);
+    uint64_t *k_full = q_full + 1;
+    uint64_t *k_empty = k_full + C::NK;
+    uint64_t *v_full = k_empty + C::NK;
+    uint64_t *v_empty = v_full + C::NV;
+    uint64_t *s_full = v_empty + C::NV;   // [NS]: S(j) in buffer j % NS
+    uint64_t *p_full = s_full + NS;       // [2]: P(j) written, block parity j & 1
+    uint64_t *pv_done = p_full + 2;       // [NS]: PV(j) complete, buffer j % NS
+    uint64_t *mma_done = pv_done + NS;
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(mma_done + 1);
+    volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
+    int *list_ok = reinterpret_cast<int *>(tmem_slot + 2);
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int bh = blockIdx.y;
+    const int S = a.S;
+    TileSched sc = make_sched<WINDOW>(a, blockIdx.x, bh);
+
+    if (threadIdx.x == 0) {
+        mbar_init(q_full, 1);
+        for (int s = 0; s < C::NK; ++s) {
+            mbar_init(&k_full[s], 1);
+            mbar_init(&k_empty[s], 1);
+        }
+        for (int s = 0; s < C::NV; ++s) {
+            mbar_init(&v_full[s], 1);
+            mbar_init(&v_empty[s], 1);
+        }
+        for (int b = 0; b < NS; ++b) {
+            mbar_init(&s_full[b], 1);
+            mbar_init(&pv_done[b], 1);
+        }
+        mbar_init(&p_full[0], 4);
+        mbar_init(&p_full[1], 4);
+        mbar_init(mma_done, 1);
+        *abort_flag = 0;
+        fence_mbar_init();
+    }
+    if constexpr (!WINDOW) {
+        if (warp == 0 && sc.qt >= 0) {  // validate the list
+            bool ok = sc.n >= 1 && sc.n <= a.cap;
+            if (ok) {
+                for (int j = lane; j < sc.n; j += 32) {
+                    const int v = __ldg(sc.list + j);
+                    ok = ok && v >= 0 && v < a.nb && (j == 0 || __ldg(sc.list + j - 1) < v);
+                }
+            }
+            ok = __all_sync(0xffffffffu, ok);
+            // written only here (read after the barrier below)
+            if (lane == 0) *list_ok = ok ? 1 : 0;
+        }
+    }
+    if (warp == 5) {
+        tmem_alloc(tmem_slot, OneCfg<D>::TMEM_COLS);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+    bool bad = false;
+    if (sc.qt < 0) sc.n = 0;
+    if constexpr (!WINDOW) {
+        if (sc.qt >= 0 && !*list_ok) {
+            bad = true;
+            sc.n = 0;
+            if (threadIdx.x == 0) report(a.status, DEV_RUNTIME);
+        }
+    }
+    int tc = 0;  // tiled mode: this head's tiling
+    if constexpr (TILED) {
+        if (a.choice) tc = __ldg(a.choice + bh);
+        if (tc < 0 || tc >= a.tiles.n) {  // the head is left unwritten
+            if (threadIdx.x == 0) report(a.status, DEV_RUNTIME);
+            sc.n = 0;
+            sc.qt = -1;
+            tc = 0;
+        }
+    }
+    const int tt = a.tiles.t[tc], th = a.tiles.h[tc], tw = a.tiles.w[tc];
+    if constexpr (PAD) {
+        if (sc.qt >= 0) {  // a query box wholly in the padding has no row to write
+            const BoxCoord c = box_of(static_cast<uint32_t>(sc.qt), a.geom[tc], th, tw);
+            if (c.t >= a.real.T || c.h >= a.real.H || c.w >= a.real.W) {
+                sc.qt = -1;
+                sc.n = 0;
+            }
+        }
+    }
+    const CUtensorMap *tmQ = &maps.q[tc], *tmK = &maps.k[tc], *tmV = &maps.v[tc];
+    // one 128-row tile of Q, K or V: block b of this head
+    auto load_tile = [&](uint8_t *dst, const CUtensorMap *map, uint64_t *bar, int b) {
+        if constexpr (TILED) {
+            const BoxCoord c = box_of(static_cast<uint32_t>(b), a.geom[tc], th, tw);
+            for (int s = 0; s < C::KSLABS; ++s) tma_load_5d(dst + s * C::SLAB, map, bar, s * 64, c.w, c.h, c.t, bh);
+        } else {
+            for (int s = 0; s < C::KSLABS; ++s) tma_load_3d(dst + s * C::SLAB, map, bar, s * 64, b * BN, bh);
+        }
+    };
+    const int n = sc.n;
+
+    if (warp == 4) {
+        // ================= TMA producer =================
+        // order: Q, K(0), K(1), then V(j), K(j+2) for j = 0, 1, ... (the order the MMAs use them)
+        if (lane == 0 && n > 0) {
+            tma_prefetch_desc(tmQ);
+            tma_prefetch_desc(tmK);
+            tma_prefetch_desc(tmV);
+            mbar_arrive_expect_tx(q_full, C::TILE_BYTES);
+            load_tile(sQ, tmQ, q_full, sc.qt);
+            uint32_t kc = 0, vc = 0;
+            bool ok = true;
+            auto load = [&](bool is_k, int j) -> bool {
+                uint32_t &c = is_k ? kc : vc;
+                const int depth = is_k ? C::NK : C::NV;
+                const int slot = c % depth;
+                uint64_t *full = is_k ? &k_full[slot] : &v_full[slot];
+                uint64_t *empty = is_k ? &k_empty[slot] : &v_empty[slot];
+                if (c >= static_cast<uint32_t>(depth) && !mbar_wait(empty, ((c / depth) - 1) & 1, abort_flag))
+                    return false;
+                uint8_t *dst = (is_k ? sK : sV) + slot * C::TILE_BYTES;
+                mbar_arrive_expect_tx(full, C::TILE_BYTES);
+                load_tile(dst, is_k ? tmK : tmV, full, kblock_of<WINDOW>(sc, j));
+                ++c;
+                return true;
+            };
+            ok = load(true, 0);
+            if (ok && n > 1) ok = load(true, 1);
+            for (int j = 0; ok && j < n; ++j) {
+                ok = load(false, j);
+                if (ok && j + 2 < n) ok = load(true, j + 2);
+            }
+            if (!ok) {
+                if (!*abort_flag) { report(a.status, DEV_TIMEOUT); *abort_flag = 1; }
+                // let the loads already issued land before the CTA exits
+                mbar_wait(q_full, 0, nullptr);
+                for (uint32_t c = kc > static_cast<uint32_t>(C::NK) ? kc - C::NK : 0; c < kc; ++c)
+                    mbar_wait(&k_full[c % C::NK], (c / C::NK) & 1, nullptr);
+                for (uint32_t c = vc > static_cast<uint32_t>(C::NV) ? vc - C::NV : 0; c < vc; ++c)
+                    mbar_wait(&v_full[c % C::NV], (c / C::NV) & 1, nullptr);
+            }
+        }
+        __syncwarp();
+    } else if (warp == 5) {
+        // ================= MMA issuer =================
+        // QK(0) QK(1) | PV(j) QK(j+2) | j = 0, 1, ...: S(j) lives in buffer
+        // j % NS, and a QK^T into a buffer first waits for the PV that read the
+        // P over it (with one buffer and lists of one block, QK(0) then PV(0)).
+        if (lane == 0) {
+            constexpr uint32_t idesc_qk = idesc_bf16_f32(128, BN, false);
+            constexpr uint32_t idesc_pv = idesc_bf16_f32(128, D, true);
+            // Descriptor bases, built once.  The start-address field holds
+            // addr >> 4 in 14 bits and every shared address here is < 256 KB,
+            // so advancing a descriptor by a byte offset is a plain add of
+            // offset >> 4 with no carry out of the field.
+            const uint64_t dQ = sdesc_sw128(smem_u32(sQ), 16, 1024);
+            const uint64_t dK = sdesc_sw128(smem_u32(sK), 16, 1024);
+            const uint64_t dV = sdesc_sw128(smem_u32(sV), C::SLAB, 1024);
+            constexpr uint64_t kTile16 = C::TILE_BYTES >> 4;
+            uint32_t kc = 0, vc = 0;
+            bool ok = true;
+            auto qk = [&](int j) -> bool {
+                const int slot = kc % C::NK, b = j % NS;
+                if (!mbar_wait(&k_full[slot], (kc / C::NK) & 1, abort_flag)) return false;
+                if (j >= NS && !mbar_wait(&pv_done[b], ((j - NS) / NS) & 1, abort_flag)) return false;
+                tc_fence_after();
+                const uint64_t k0 = dK + slot * kTile16;
+                const uint32_t d = tmem + b * 128;
+                #pragma unroll
+                for (int kk = 0; kk < D / 16; ++kk) {
+                    const uint64_t off = static_cast<uint64_t>(((kk >> 2) * C::SLAB + (kk & 3) * 32) >> 4);
+                    umma_bf16(d, dQ + off, k0 + off, idesc_qk, kk > 0 ? 1u : 0u);
+                }
+                umma_commit(&s_full[b]);
+                umma_commit(&k_empty[slot]);
+                ++kc;
+                return true;
+            };
+            auto pv = [&](int j) -> bool {
+                const int slot = vc % C::NV, b = j % NS;
+                if (!mbar_wait(&p_full[j & 1], (j >> 1) & 1, abort_flag)) return false;
+                if (!mbar_wait(&v_full[slot], (vc / C::NV) & 1, abort_flag)) return false;
+                tc_fence_after();
+                const uint64_t v0 = dV + slot * kTile16;
+                const uint32_t d = tmem + C::O_COL, pa = tmem + b * 128;
+                const uint32_t acc0 = j > 0 ? 1u : 0u;
+                #pragma unroll
+                for (int kk = 0; kk < BN / 16; ++kk)
+                    umma_bf16_ts(d, pa + kk * 8, v0 + static_cast<uint64_t>((kk * 2048) >> 4), idesc_pv,
+                                 kk > 0 ? 1u : acc0);
+                umma_commit(&pv_done[b]);
+                umma_commit(&v_empty[slot]);
+                ++vc;
+                return true;
+            };
+            if (n > 0) {
+                ok = mbar_wait(q_full, 0, abort_flag);
+                if (ok) ok = qk(0);
+                if (ok && n > 1) ok = qk(1);
+                for (int j = 0; ok && j < n; ++j) {
+                    ok = pv(j);
+                    if (ok && j + 2 < n) ok = qk(j + 2);
+                }
+                if (!ok && !*abort_flag) { report(a.status, DEV_TIMEOUT); *abort_flag = 1; }
+            }
+            umma_commit(mma_done);
+            mbar_wait(mma_done, 0, nullptr);
+        }
+        __syncwarp();
+    } else {
+        // ================= softmax + epilogue (warps 0-3) =================
+        const int wq = warp;                      // TMEM lane quadrant
+        const int row = wq * 32 + lane;           // row of the tile
+        const int q0 = (sc.qt < 0 ? 0 : sc.qt) * BN;
+        const int rg = q0 + row;
+        bool row_valid = sc.qt >= 0 && rg < S;
+        // output row: the permuted position itself, or its T-major token in tiled mode
+        uint32_t orow_in_head = rg;
+        if constexpr (PAD) {
+            int pt, ph, pw;
+            tile_coords(rg, a.H, a.W, tt, th, tw, pt, ph, pw);
+            const int tok = real_token(pt, ph, pw, a.real);
+            row_valid = row_valid && tok >= 0;
+            orow_in_head = tok < 0 ? 0u : static_cast<uint32_t>(tok);
+        } else if constexpr (TILED) {
+            orow_in_head = tile_token(rg, a.H, a.W, tt, th, tw);
+        }
+        const uint32_t t_lane = tmem + (static_cast<uint32_t>(wq * 32) << 16);
+        const uint32_t o_col = C::O_COL;
+        const float sl2 = a.scale_log2;
+        float m_ref = -INFINITY, l_sum = 0.f;
+        bool ok = true;
+        for (int j = 0; j < n; ++j) {
+            const uint32_t s_col = (j % NS) * 128;
+            if (!__all_sync(0xffffffffu, mbar_wait(&s_full[j % NS], (j / NS) & 1, abort_flag))) { ok = false; break; }
+            tc_fence_after();
+            uint32_t x[BN];
+            #pragma unroll
+            for (int c = 0; c < BN / 32; ++c)
+                tmem_ld32(t_lane + s_col + 32 * c, *reinterpret_cast<uint32_t(*)[32]>(&x[32 * c]));
+            tmem_ld_wait();
+            // padded grid: which of the key block's 128 columns are real tokens
+            // (column u * 32 + lane in bit lane of kv[u]); all ones off the edge
+            uint32_t kv[4] = {~0u, ~0u, ~0u, ~0u};
+            bool key_edge = false;
+            if constexpr (PAD) {
+                {
+                    const PPArgs::BoxGeom &g = a.geom[tc];
+                    const BoxCoord c = box_of(static_cast<uint32_t>(kblock_of<WINDOW>(sc, j)), g, th, tw);
+                    key_edge = c.t + g.bt > a.real.T || c.h + th > a.real.H || c.w + tw > a.real.W;
+                    if (key_edge) {
+                        #pragma unroll
+                        for (int u = 0; u < 4; ++u) {
+                            const uint32_t col = static_cast<uint32_t>(u * 32 + lane);
+                            const uint32_t dt = fdiv(col, g.bhw), r2 = col - dt * g.bhw.d;
+                            const uint32_t dh = fdiv(r2, g.bw), dw = r2 - dh * g.bw.d;
+                            kv[u] = __ballot_sync(0xffffffffu, c.t + static_cast<int>(dt) < a.real.T &&
+                                                                   c.h + static_cast<int>(dh) < a.real.H &&
+                                                                   c.w + static_cast<int>(dw) < a.real.W);
+                        }
+                    }
+                }
+            }
+            auto apply_mask = [&]() {
+                if constexpr (WINDOW) {
+                    const int ks = kblock_of<WINDOW>(sc, j) * BN;
+                    const int qe = min(q0 + BN, S);
+                    const bool full = (ks + BN <= S) &&
+                                      (a.dense || ks + BN <= a.sink || max(qe - 1 - ks, ks + BN - 1 - q0) <= a.half);
+                    if (!full) {
+                        #pragma unroll
+                        for (int c = 0; c < BN; ++c) {
+                            const int kc2 = ks + c;
+                            const int dd = rg > kc2 ? rg - kc2 : kc2 - rg;
+                            if (!(kc2 < S && (a.dense || kc2 < a.sink || dd <= a.half)))
+                                x[c] = __float_as_uint(-INFINITY);
+                        }
+                    }
+                } else {
+                    if (a.group > 0) {
+                        const int ks = kblock_of<WINDOW>(sc, j) * BN;
+                        // key ks + c is in the row's group iff it lies in [g0, g0 + group)
+                        const int g0 = (rg / a.group) * a.group - ks;
+                        #pragma unroll
+                        for (int c = 0; c < BN; ++c)
+                            if (c < g0 || c >= g0 + a.group) x[c] = __float_as_uint(-INFINITY);
+                    } else if (a.gstride > 1) {
+                        const int ks = kblock_of<WINDOW>(sc, j) * BN;
+                        // key ks + c is in the row's group iff (ks + c - rg) is a multiple of gstride
+                        const int r0 = (rg - ks) & (a.gstride - 1);
+                        #pragma unroll
+                        for (int c = 0; c < BN; ++c)
+                            if ((c & (a.gstride - 1)) != r0) x[c] = __float_as_uint(-INFINITY);
+                    }
+                    if (key_edge) {
+                        #pragma unroll
+                        for (int c = 0; c < BN; ++c)
+                            if (!((kv[c >> 5] >> (c & 31)) & 1u)) x[c] = __float_as_uint(-INFINITY);
+                    }
+                }
+            };
+            apply_mask();
+            // P = 2^(scale*log2e*S - m_use) in place (bf16 pairs), returns the row sum
+            // The arguments use two-wide fp32 instructions: the exponentials are
+            // bound by the exponential unit, and fewer issue slots here leave more
+            // to the other tile's warp on the sub-partition.  The row sum adds the
+            // bf16-rounded P that the PV MMA multiplies, so O / l is a convex
+            // combination of V rows: a row held by a few keys then carries no
+            // rounding error in its weights' total.  The mixed-precision adds take
+            // each half of the packed pair as it is; unpacking the pair first for
+            // two-wide adds measured a few percent slower.
+            auto exp_pass = [&](float m_use) -> float {
+                const uint64_t sl2x2 = f32x2(sl2, sl2), nmx2 = f32x2(-m_use, -m_use);
+                float s0 = 0.f, s1 = 0.f, s2 = 0.f, s3 = 0.f;
+                #pragma unroll
+                for (int q = 0; q < BN / 2; ++q) {
+                    float a0, a1;
+                    f32x2_split(fma_f32x2(f32x2(__uint_as_float(x[2 * q]), __uint_as_float(x[2 * q + 1])), sl2x2, nmx2),
+                                a0, a1);
+                    const uint32_t pk = pack_bf16x2(ex2_approx(a0), ex2_approx(a1));
+                    if (q & 1) add_bf16x2_f32(pk, s2, s3);
+                    else add_bf16x2_f32(pk, s0, s1);
+                    x[q] = pk;   // P, packed in place (q <= 2q)
+                }
+                return (s0 + s2) + (s1 + s3);
+            };
+            auto raw_max = [&]() -> float {
+                float m4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+                #pragma unroll
+                for (int c = 0; c < BN; c += 8) {
+                    #pragma unroll
+                    for (int u = 0; u < 4; ++u)
+                        m4[u] = fmax3(m4[u], __uint_as_float(x[c + 2 * u]), __uint_as_float(x[c + 2 * u + 1]));
+                }
+                return fmaxf(fmaxf(m4[0], m4[1]), fmaxf(m4[2], m4[3]));
+            };
+            // first visible keys of this row: take the block max before the exponentials
+            if (m_ref == -INFINITY) m_ref = raw_max() * sl2;  // may stay -inf
+            // The running max is lazy: every P is at most the row sum, so a sum
+            // above kMaxRowSum (or inf) means the row's max grew; then O and l are
+            // rescaled and the block is redone from S, still intact in TMEM.
+            float rs = 0.f;
+            #pragma unroll 1
+            for (int pass = 0; pass < 2; ++pass) {
+                rs = exp_pass(m_ref == -INFINITY ? 0.f : m_ref);
+                const bool need = !(rs <= kMaxRowSum);
+                if (pass == 1 || !__any_sync(0xffffffffu, need)) break;
+                #pragma unroll
+                for (int c = 0; c < BN / 32; ++c)
+                    tmem_ld32(t_lane + s_col + 32 * c, *reinterpret_cast<uint32_t(*)[32]>(&x[32 * c]));
+                tmem_ld_wait();
+                apply_mask();
+                const float m_new = need ? fmaxf(m_ref, raw_max() * sl2) : m_ref;
+                if (j > 0) {
+                    if (!__all_sync(0xffffffffu, mbar_wait(&pv_done[(j - 1) % NS], ((j - 1) / NS) & 1, abort_flag))) {
+                        ok = false;
+                    } else {
+                        tc_fence_after();
+                        const float alpha = (m_new > m_ref && m_ref != -INFINITY) ? ex2_approx(m_ref - m_new) : 1.f;
+                        #pragma unroll 1
+                        for (int c = 0; c < D / 8; ++c) {
+                            uint32_t o[8];
+                            tmem_ld8(t_lane + o_col + 8 * c, o);
+                            tmem_ld_wait();
+                            #pragma unroll
+                            for (int e = 0; e < 8; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * alpha);
+                            tmem_st8(t_lane + o_col + 8 * c, o);
+                        }
+                        tmem_st_wait();
+                        l_sum *= alpha;
+                    }
+                }
+                if (!__all_sync(0xffffffffu, ok)) break;
+                m_ref = m_new;
+            }
+            if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
+            l_sum += rs;
+            // P over the first 64 columns of this tile's S
+            tmem_st32(t_lane + s_col, *reinterpret_cast<const uint32_t(*)[32]>(&x[0]));
+            tmem_st32(t_lane + s_col + 32, *reinterpret_cast<const uint32_t(*)[32]>(&x[32]));
+            tmem_st_wait();
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&p_full[j & 1]);
+        }
+        if (!ok && !*abort_flag) { report(a.status, DEV_TIMEOUT); *abort_flag = 1; }
+
+        // ---- epilogue: O / l -> global ----
+        const size_t orow = static_cast<size_t>(bh) * a.S_out + orow_in_head;
+        bool have_o = ok && n > 0;
+        if (have_o && !__all_sync(0xffffffffu, mbar_wait(&pv_done[(n - 1) % NS], ((n - 1) / NS) & 1, abort_flag))) {
+            have_o = false;
+            if (!*abort_flag) { report(a.status, DEV_TIMEOUT); *abort_flag = 1; }
+        }
+        if (have_o) {
+            tc_fence_after();
+            const float inv = l_sum > 0.f ? 1.f / l_sum : 0.f;
+            #pragma unroll
+            for (int c = 0; c < D / 32; ++c) {
+                uint32_t o[32];
+                tmem_ld32(t_lane + o_col + 32 * c, o);
+                tmem_ld_wait();
+                if (row_valid) {
+                    if (a.out_f32) {
+                        float4 *dst = reinterpret_cast<float4 *>(static_cast<float *>(a.out) + orow * D + 32 * c);
+                        #pragma unroll
+                        for (int e = 0; e < 8; ++e)
+                            dst[e] = make_float4(__uint_as_float(o[4 * e]) * inv, __uint_as_float(o[4 * e + 1]) * inv,
+                                                 __uint_as_float(o[4 * e + 2]) * inv, __uint_as_float(o[4 * e + 3]) * inv);
+                    } else {
+                        uint4 *dst = reinterpret_cast<uint4 *>(static_cast<__nv_bfloat16 *>(a.out) + orow * D + 32 * c);
+                        #pragma unroll
+                        for (int e = 0; e < 4; ++e) {
+                            const uint32_t *u = &o[8 * e];
+                            dst[e] = make_uint4(pack_bf16x2(__uint_as_float(u[0]) * inv, __uint_as_float(u[1]) * inv),
+                                                pack_bf16x2(__uint_as_float(u[2]) * inv, __uint_as_float(u[3]) * inv),
+                                                pack_bf16x2(__uint_as_float(u[4]) * inv, __uint_as_float(u[5]) * inv),
+                                                pack_bf16x2(__uint_as_float(u[6]) * inv, __uint_as_float(u[7]) * inv));
+                        }
+                    }
+                }
+            }
+            if (row_valid && l_sum <= 0.f) report(a.status, DEV_RUNTIME);
+        } else if (row_valid && bad) {
+            if (a.out_f32) {
+                float4 *dst = reinterpret_cast<float4 *>(static_cast<float *>(a.out) + orow * D);
+                for (int e = 0; e < D / 4; ++e) dst[e] = make_float4(0.f, 0.f, 0.f, 0.f);
+            } else {
+                uint4 *dst = reinterpret_cast<uint4 *>(static_cast<__nv_bfloat16 *>(a.out) + orow * D);
+                for (int e = 0; e < D / 8; ++e) dst[e] = make_uint4(0u, 0u, 0u, 0u);
+            }
+        }
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 5) {
+        tc_fence_after();
+        tmem_dealloc(tmem, OneCfg<D>::TMEM_COLS);
+    }
+}
+
+template <int D, bool TILED, bool PAD = false>
+vsa_status run_one(const AttnLaunch &L, int *status, cudaStream_t st) {
+    constexpr bool WINDOW = false;
+    using C = OneCfg<D>;
+    MapSet maps = {};  // copied into the launch parameters
+    bool ok = true;
+    if constexpr (TILED) {
+        for (int c = 0; c < L.tiles.n; ++c) {
+            const int m = L.tiles.t[c] * L.tiles.h[c] * L.tiles.w[c] / 128;
+            const int bt = L.tiles.t[c] / m, bhh = L.tiles.h[c], bw = L.tiles.w[c];
+            // the real tensors: boxes reaching past them read zeros
+            ok = ok && make_box_map(&maps.q[c], L.q, D, L.T, L.Hg, L.Wg, L.BH, bt, bhh, bw) &&
+                 make_box_map(&maps.k[c], L.k, D, L.T, L.Hg, L.Wg, L.BH, bt, bhh, bw) &&
+                 make_box_map(&maps.v[c], L.v, D, L.T, L.Hg, L.Wg, L.BH, bt, bhh, bw);
+        }
+    } else {
+        ok = make_tile_map(&maps.q[0], L.q, D, L.S, L.BH, 128) && make_tile_map(&maps.k[0], L.k, D, L.S, L.BH, 128) &&
+             make_tile_map(&maps.v[0], L.v, D, L.S, L.BH, 128);
+    }
+    if (!ok) return fail(VSA_ERR_CUDA, "cuTensorMapEncodeTiled failed (driver entry point or arguments)");
+    auto kern = attn_one_kernel<D, WINDOW, TILED, PAD>;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
+    if (e != cudaSuccess) return check_cuda(e, "cudaFuncSetAttribute(attention, one key block)");
+    PPArgs a;
+    const int positions = TILED ? L.Tp * L.Hp * L.Wp : L.S;
+    a.S = positions;
+    a.S_out = L.S;
+    a.nq = (positions + 127) / 128;
+    a.idx = L.idx;
+    a.cnt = L.cnt;
+    a.cap = L.cap;
+    a.list_per_head = L.list_per_head;
+    a.group = L.group;
+    a.gstride = L.gstride;
+    a.nb = L.nb;
+    a.half = L.half;
+    a.sink = L.sink;
+    a.dense = L.dense;
+    a.scale_log2 = L.scale * 1.4426950408889634f;
+    a.out = L.o;
+    a.out_f32 = L.out_f32;
+    a.status = status;
+    a.H = TILED ? L.Hp : L.Hg;
+    a.W = TILED ? L.Wp : L.Wg;
+    a.real = RealGrid{L.T, L.Hg, L.Wg};
+    a.tiles = L.tiles;
+    a.choice = L.choice;
+    if (!TILED) a.tiles.n = 1;
+    for (int c = 0; c < kMaxTiles; ++c) {
+        auto &g = a.geom[c];
+        if (TILED && c < L.tiles.n) {
+            const int tt = L.tiles.t[c], th = L.tiles.h[c], tw = L.tiles.w[c];
+            const int m = tt * th * tw / 128;
+            g.m = make_fastdiv(m);
+            g.nthw = make_fastdiv((L.Hp / th) * (L.Wp / tw));
+            g.ntw = make_fastdiv(L.Wp / tw);
+            g.bhw = make_fastdiv(th * tw);
+            g.bw = make_fastdiv(tw);
+            g.bt = tt / m;
+        } else {
+            g.m = g.nthw = g.ntw = g.bhw = g.bw = make_fastdiv(1);
+            g.bt = 1;
+        }
+    }
+    dim3 grid(a.nq, L.BH);
+    kern<<<grid, kOneThreads, C::SMEM, st>>>(maps, a);
+    return check_cuda(cudaGetLastError(), "attention launch (one key block)");
+}
+
 }  // namespace
 
 vsa_status launch_attention_pp(const AttnLaunch &L, int *status, cudaStream_t st) {
     if (L.window) return L.D == 128 ? run_pp<128, true, false>(L, status, st) : run_pp<64, true, false>(L, status, st);
+    if (L.cap == 1) {  // lists of one key block
+        if (L.tiled) {
+            if (L.Tp * L.Hp * L.Wp != L.S)
+                return L.D == 128 ? run_one<128, true, true>(L, status, st) : run_one<64, true, true>(L, status, st);
+            return L.D == 128 ? run_one<128, true>(L, status, st) : run_one<64, true>(L, status, st);
+        }
+        return L.D == 128 ? run_one<128, false>(L, status, st) : run_one<64, false>(L, status, st);
+    }
     if (L.tiled) {
         if (L.Tp * L.Hp * L.Wp != L.S)  // a zero-padded grid
             return L.D == 128 ? run_pp<128, false, true, true>(L, status, st) : run_pp<64, false, true, true>(L, status, st);

@@ -667,3 +667,53 @@ def test_spade_top_p_end_to_end():
         qo, ko, vo = (oracle.permute_rows(_np(x[0, h]), perm) for x in (q, k, v))
         want = oracle.block_sparse_attention(qo, ko, vo, oi, oc, w.block)
         assert_attn_close(_np(o[0, h])[perm], want, f"head {h}")
+
+
+# --------------------------------------------------------------------------
+# lists of one key block: the one-block kernel (two CTAs per SM)
+# --------------------------------------------------------------------------
+
+@pytest.mark.parametrize("mode,grid", [("permuted", (4, 8, 16)), ("tiled", (4, 8, 16)), ("padded", (5, 12, 20))])
+def test_one_block_lists_match_two_tile_kernel_and_oracle(mode, grid):
+    """One-slot lists run through the one-key-block kernel; the same lists in
+    two slots (cnt 1, second slot -1) run through the two-tile kernel.  Both
+    must give the same bits, and the oracle's result."""
+    tiles = [(1, 8, 16), (2, 8, 8), (4, 4, 8)]
+    B, H, D = 1, 3, 128
+    S = grid[0] * grid[1] * grid[2]
+    pg = vsa.padded_grid(grid, tiles)
+    nb = pg[0] * pg[1] * pg[2] // 128
+    q, k, v = smooth_qkv(B, H, grid, D, seed=95, device=DEV)
+    rng = np.random.default_rng(96)
+    # padded grid: the diagonal block (it holds the query itself, so every real
+    # query has a real key); otherwise random blocks for heads 1 and 2
+    idx1 = np.stack([np.arange(nb) if h == 0 or mode == "padded" else rng.integers(0, nb, nb)
+                     for h in range(H)]).astype(np.int32)
+    cnt = np.ones((H, nb), np.int32)
+    ti1 = torch.as_tensor(idx1, device=DEV).view(B, H, nb, 1)
+    ti2 = torch.as_tensor(np.concatenate([idx1[..., None], np.full((H, nb, 1), -1, np.int32)], -1),
+                          device=DEV).view(B, H, nb, 2)
+    tc = torch.as_tensor(cnt, device=DEV).view(B, H, nb)
+    if mode == "permuted":
+        qp, kp, vp = (vsa.permute(x, grid, tiles[:1]) for x in (q, k, v))
+        o1 = vsa.block_sparse_attention(qp, kp, vp, ti1, tc, 128, out_dtype=torch.float32)
+        o2 = vsa.block_sparse_attention(qp, kp, vp, ti2, tc, 128, out_dtype=torch.float32)
+        assert torch.equal(o1, o2)
+        for h in range(H):
+            want = oracle.block_sparse_attention(_np(qp[0, h]), _np(kp[0, h]), _np(vp[0, h]), idx1[h][:, None],
+                                                 cnt[h], 128)
+            assert_attn_close(_np(o1[0, h]), want, f"head {h}")
+        return
+    choice = torch.tensor([0, 1, 2], dtype=torch.int32, device=DEV)
+    o1 = vsa.block_sparse_attention_tiled(q, k, v, grid, tiles, choice, ti1, tc, out_dtype=torch.float32)
+    o2 = vsa.block_sparse_attention_tiled(q, k, v, grid, tiles, choice, ti2, tc, out_dtype=torch.float32)
+    assert torch.equal(o1, o2)
+    for h, c in enumerate(choice.tolist()):
+        perm = oracle.tile_permutation(pg, tiles[c])
+        real = oracle.real_tokens(grid, pg)
+        qo, ko, vo = (oracle.permute_rows(oracle.pad_grid(_np(x[0, h]), grid, pg), perm) for x in (q, k, v))
+        want_p = oracle.block_sparse_attention(qo, ko, vo, idx1[h][:, None], cnt[h], 128,
+                                               key_ok=real[perm].astype(np.uint8) if mode == "padded" else None)
+        want = np.zeros((pg[0] * pg[1] * pg[2], D))
+        want[perm] = want_p
+        assert_attn_close(_np(o1[0, h]), want[real], f"head {h}")
