@@ -1169,6 +1169,9 @@ template <int D, bool TILED, bool PAD = false>
 vsa_status run_one(const AttnLaunch &L, int *status, cudaStream_t st) {
     constexpr bool WINDOW = false;
     using C = OneCfg<D>;
+    // with one S buffer, QK(1) would wait for PV(0), which is issued after it:
+    // lists of more than one block belong to the two-tile kernel
+    if (L.cap != 1) return fail(VSA_ERR_UNSUPPORTED, "the one-key-block kernel takes lists of one block");
     MapSet maps = {};  // copied into the launch parameters
     bool ok = true;
     if constexpr (TILED) {
