@@ -670,18 +670,9 @@ vsa_status launch_attention(const AttnLaunch &L, int *status, cudaStream_t st) {
         if (L.block == 64) return pad ? run<64, 64, false, true, true>(L, status, st) : run<64, 64, false, true>(L, status, st);
         return pad ? run<64, 32, false, true, true>(L, status, st) : run<64, 32, false, true>(L, status, st);
     }
-    if (L.window) {
-        if (L.D == 128) return run<128, 128, true>(L, status, st);
-        return run<64, 128, true>(L, status, st);
-    }
-    if (L.D == 128) {
-        if (L.block == 128) return run<128, 128, false>(L, status, st);
-        if (L.block == 64) return run<128, 64, false>(L, status, st);
-        return run<128, 32, false>(L, status, st);
-    }
-    if (L.block == 128) return run<64, 128, false>(L, status, st);
-    if (L.block == 64) return run<64, 64, false>(L, status, st);
-    return run<64, 32, false>(L, status, st);
+    // 32- and 64-token blocks in permuted order (windows always use 128-token tiles)
+    if (L.D == 128) return L.block == 64 ? run<128, 64, false>(L, status, st) : run<128, 32, false>(L, status, st);
+    return L.block == 64 ? run<64, 64, false>(L, status, st) : run<64, 32, false>(L, status, st);
 }
 
 }  // namespace vsa
