@@ -708,6 +708,8 @@ def test_one_block_lists_match_two_tile_kernel_and_oracle(mode, grid):
     o1 = vsa.block_sparse_attention_tiled(q, k, v, grid, tiles, choice, ti1, tc, out_dtype=torch.float32)
     o2 = vsa.block_sparse_attention_tiled(q, k, v, grid, tiles, choice, ti2, tc, out_dtype=torch.float32)
     assert torch.equal(o1, o2)
+    ob = vsa.block_sparse_attention_tiled(q, k, v, grid, tiles, choice, ti1, tc, out_dtype=torch.bfloat16)
+    assert torch.equal(ob, o1.to(torch.bfloat16))
     for h, c in enumerate(choice.tolist()):
         perm = oracle.tile_permutation(pg, tiles[c])
         real = oracle.real_tokens(grid, pg)
