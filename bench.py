@@ -459,7 +459,7 @@ def extra_workloads(steps: int):
     for kind in w.structured:
         stile = vsa.structured_tile(kind, w.grid, w.sliding_tile)
         idx, cnt, g = vsa.structured_block_list(kind, w.grid, 128, w.sliding_tile, w.sliding_radius,
-                                                cap=1 if kind == "temporal" else None)
+                                                cap=1 if kind == "temporal" and 128 % w.grid[0] == 0 else None)
         if stile[1] == w.grid[1] and stile[2] == w.grid[2]:
             mode = "t-major"
             fn = lambda: vsa.block_sparse_attention(q, k, v, idx, cnt, 128, g)  # noqa: E731

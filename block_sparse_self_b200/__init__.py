@@ -588,10 +588,10 @@ def structured_attention(q, k, v, kind: str, grid, block: int = 128, tile=(4, 8,
                          scale: Optional[float] = None, out_dtype=None):
     """A structured static mask as block-sparse attention, in and out in T-major order."""
     st = structured_tile(kind, grid, tile)
-    # temporal-only lists hold the diagonal block alone: a one-slot list lets
-    # the attention use its one-key-block kernel
-    idx, cnt, g = structured_block_list(kind, grid, block, tile, radius, device=q.device,
-                                        cap=1 if kind == "temporal" else None)
+    # when T divides the block, temporal-only lists hold the diagonal block
+    # alone: a one-slot list lets the attention use its one-key-block kernel
+    one = kind == "temporal" and block % grid[0] == 0
+    idx, cnt, g = structured_block_list(kind, grid, block, tile, radius, device=q.device, cap=1 if one else None)
     if st[1] == grid[1] and st[2] == grid[2]:  # whole frames: the tile-contiguous order is T-major itself
         return block_sparse_attention(q, k, v, idx, cnt, block, g, scale, out_dtype)
     T = grid[0]

@@ -719,3 +719,19 @@ def test_one_block_lists_match_two_tile_kernel_and_oracle(mode, grid):
         want = np.zeros((pg[0] * pg[1] * pg[2], D))
         want[perm] = want_p
         assert_attn_close(_np(o1[0, h]), want[real], f"head {h}")
+
+
+def test_temporal_mask_with_more_frames_than_a_block():
+    """T = 256 frames: a temporal tile is two blocks, so the lists hold two
+    blocks and the composition must not ask for one-slot lists."""
+    grid = (256, 1, 2)
+    q, k, v = smooth_qkv(1, 1, grid, 64, seed=99, device=DEV)
+    o = vsa.structured_attention(q, k, v, "temporal", grid, 128, out_dtype=torch.float32)
+    t, r = oracle.structured_tile("temporal", grid)
+    idx, cnt, g = oracle.tile_neighbourhood_list(grid, t, r, 128)
+    perm = oracle.tile_permutation(grid, t)
+    qp, kp, vp = (oracle.permute_rows(_np(x[0, 0]), perm) for x in (q, k, v))
+    op = oracle.block_sparse_attention(qp, kp, vp, idx, cnt, 128, g)
+    want = np.empty_like(op)
+    want[perm] = op
+    assert_attn_close(_np(o[0, 0]), want, "T = 256")
