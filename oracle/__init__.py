@@ -47,6 +47,8 @@ def lib():
         L.orc_topk_block_list.restype = i32
         L.orc_tile_neighbourhood_list.argtypes = [i32] * 11 + [P, P, P]
         L.orc_tile_neighbourhood_list.restype = i32
+        L.orc_centered_tile_neighbourhood_list.argtypes = [i32] * 11 + [P, P, P]
+        L.orc_centered_tile_neighbourhood_list.restype = i32
         L.orc_window_attention.argtypes = [P, P, P, i64, i32, i32, i32, dbl, i32, P, i64, P]
         L.orc_block_sparse_attention.argtypes = [P, P, P, i64, i32, i32, P, P, i32, i32, dbl, P, P, i64, P]
         L.orc_window_key_ranges.argtypes = [i64] * 5 + [P]
@@ -236,23 +238,27 @@ def topp_block_list(score, p: float, scale: float, n_sink: int = 1, diag_halfwid
     return idx, cnt
 
 
-STRUCTURED_KINDS = ("spatial", "temporal", "sliding_tile")
+STRUCTURED_KINDS = ("spatial", "temporal", "sliding_tile", "sliding_tile_centered")
 
 
 def structured_tile(kind: str, grid, tile=(4, 8, 8), radius=(1, 1, 1)):
     """(tile, radius) of a structured mask: spatial_only = same frame,
-    temporal_only = same (h, w), sliding_tile = tile neighbourhood."""
+    temporal_only = same (h, w), sliding_tile = tile neighbourhood clipped at
+    the border, sliding_tile_centered = a window of 2r+1 tiles shifted to fit."""
     T, H, W = grid
     if kind == "spatial":
         return (1, H, W), (0, 0, 0)
     if kind == "temporal":
         return (T, 1, 1), (0, 0, 0)
-    if kind == "sliding_tile":
+    if kind in ("sliding_tile", "sliding_tile_centered"):
         return tuple(tile), tuple(radius)
     raise ValueError(kind)
 
 
-def tile_neighbourhood_list(grid, tile, radius, block: int, cap: Optional[int] = None):
+def tile_neighbourhood_list(grid, tile, radius, block: int, cap: Optional[int] = None, centered: bool = False):
+    """Block list of a tile-neighbourhood mask in the tile-contiguous order of
+    `tile`: clipped at the grid border, or with `centered` a window of
+    min(2r+1, n) tiles per axis moved inside the grid."""
     T, H, W = grid
     S = T * H * W
     nb = S // block
@@ -262,8 +268,8 @@ def tile_neighbourhood_list(grid, tile, radius, block: int, cap: Optional[int] =
     idx = np.empty((nb, cap), np.int32)
     cnt = np.empty(nb, np.int32)
     g = ctypes.c_int(0)
-    rc = lib().orc_tile_neighbourhood_list(T, H, W, *tile, *radius, block, cap,
-                                           _ptr(idx), _ptr(cnt), ctypes.byref(g))
+    fn = lib().orc_centered_tile_neighbourhood_list if centered else lib().orc_tile_neighbourhood_list
+    rc = fn(T, H, W, *tile, *radius, block, cap, _ptr(idx), _ptr(cnt), ctypes.byref(g))
     if rc != 0:
         raise ValueError(f"unsupported tile/radius/block combination (rc={rc})")
     if trim:

@@ -336,24 +336,52 @@ int orc_topp_block_list(const double *score, int64_t nb, double p, double scale,
 
 /* ----------------------------------------------------------------------- */
 /* Structured masks as block lists  [ADR step 1: spatial_only_mask,         */
-/* temporal_only_mask, sliding_tile_block_mask]                             */
+/* temporal_only_mask, sliding_tile_block_mask, sliding_tile_centered_mask]  */
 /* ----------------------------------------------------------------------- */
 
 /* Tile-neighbourhood mask: query token i sees key token j iff their tiles'
  * coordinates differ by at most (rt, rh, rw) along (t, h, w), with no
  * wrap-around or shift at the grid border.  spatial_only is tile (1,H,W)
  * radius 0 (same frame), temporal_only is tile (T,1,1) radius 0 (same (h,w)),
- * the sliding-tile mask is a tile with radius 1.  In the tile-contiguous
- * order, with blocks of `block` tokens:
+ * the sliding-tile mask is a tile with radius 1.
+ *
+ * The centred form (sliding_tile_centered_mask) keeps the window's size
+ * fixed instead: along an axis of n tiles a query tile c sees the
+ * w = min(2r + 1, n) consecutive tiles starting at c - r, the start moved
+ * into [0, n - w] when the window would cross the border.  Away from the
+ * border the two forms agree.
+ *
+ * In the tile-contiguous order, with blocks of `block` tokens:
  *   - if a tile is a whole number of blocks, query block i lists every block
  *     of every neighbouring tile (ascending), group size 0;
  *   - if a block is a whole number of tiles and the radius is 0, query block
  *     i lists only itself and a key is visible iff it shares the query's
  *     group of tile-volume tokens (group size = tile volume).
  * Returns 0, -1 for an unsupported combination, -2 if cap is too small.   */
-int orc_tile_neighbourhood_list(int T, int H, int W, int tt, int th, int tw,
-                                int rt, int rh, int rw, int block, int cap,
-                                int32_t *idx, int32_t *cnt, int *group_size)
+
+/* The key tiles [*lo, *hi] a query tile c sees along one axis of n tiles. */
+static void orc_axis_window(int c, int r, int n, int centered, int *lo, int *hi)
+{
+    if (!centered) {
+        *lo = c - r;
+        *hi = c + r;
+        if (*lo < 0) *lo = 0;
+        if (*hi > n - 1) *hi = n - 1;
+        return;
+    }
+    int w = 2 * r + 1;
+    if (w > n) w = n;
+    int start = c - r;
+    if (start > n - w) start = n - w;
+    if (start < 0) start = 0;
+    *lo = start;
+    *hi = start + w - 1;
+}
+
+static int orc_neighbourhood(int T, int H, int W, int tt, int th, int tw,
+                             int rt, int rh, int rw, int centered, int block,
+                             int cap, int32_t *idx, int32_t *cnt,
+                             int *group_size)
 {
     int64_t S = (int64_t)T * H * W;
     int64_t vol = (int64_t)tt * th * tw;
@@ -367,21 +395,20 @@ int orc_tile_neighbourhood_list(int T, int H, int W, int tt, int th, int tw,
             int ct = (int)(tile / ((int64_t)nth * ntw));
             int ch = (int)((tile / ntw) % nth);
             int cw = (int)(tile % ntw);
+            int t0, t1, h0, h1, w0, w1;
+            orc_axis_window(ct, rt, ntt, centered, &t0, &t1);
+            orc_axis_window(ch, rh, nth, centered, &h0, &h1);
+            orc_axis_window(cw, rw, ntw, centered, &w0, &w1);
             int c = 0;
-            for (int at = ct - rt; at <= ct + rt; ++at) {
-                if (at < 0 || at >= ntt) continue;
-                for (int ah = ch - rh; ah <= ch + rh; ++ah) {
-                    if (ah < 0 || ah >= nth) continue;
-                    for (int aw = cw - rw; aw <= cw + rw; ++aw) {
-                        if (aw < 0 || aw >= ntw) continue;
+            for (int at = t0; at <= t1; ++at)
+                for (int ah = h0; ah <= h1; ++ah)
+                    for (int aw = w0; aw <= w1; ++aw) {
                         int64_t nt = ((int64_t)at * nth + ah) * ntw + aw;
                         for (int64_t q = 0; q < bpt; ++q) {
                             if (c >= cap) return -2;
                             idx[i * cap + c++] = (int32_t)(nt * bpt + q);
                         }
                     }
-                }
-            }
             for (int s = c; s < cap; ++s) idx[i * cap + s] = -1;
             cnt[i] = c;
         }
@@ -398,6 +425,23 @@ int orc_tile_neighbourhood_list(int T, int H, int W, int tt, int th, int tw,
         return 0;
     }
     return -1;
+}
+
+int orc_tile_neighbourhood_list(int T, int H, int W, int tt, int th, int tw,
+                                int rt, int rh, int rw, int block, int cap,
+                                int32_t *idx, int32_t *cnt, int *group_size)
+{
+    return orc_neighbourhood(T, H, W, tt, th, tw, rt, rh, rw, 0, block, cap,
+                             idx, cnt, group_size);
+}
+
+int orc_centered_tile_neighbourhood_list(int T, int H, int W, int tt, int th,
+                                         int tw, int rt, int rh, int rw,
+                                         int block, int cap, int32_t *idx,
+                                         int32_t *cnt, int *group_size)
+{
+    return orc_neighbourhood(T, H, W, tt, th, tw, rt, rh, rw, 1, block, cap,
+                             idx, cnt, group_size);
 }
 
 /* ----------------------------------------------------------------------- */

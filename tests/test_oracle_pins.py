@@ -293,6 +293,75 @@ def test_sliding_tile_list_is_the_clipped_tile_neighbourhood():
         assert np.all(np.diff(idx[i, :cnt[i]]) > 0)
 
 
+def _nearest_start(c, r, n):
+    """Brute force: of the in-grid windows of min(2r+1, n) tiles, the one whose
+    start is nearest the centred start c - r."""
+    w = min(2 * r + 1, n)
+    starts = range(0, n - w + 1)
+    s = min(starts, key=lambda s0: abs(s0 - (c - r)))
+    return s, s + w - 1
+
+
+_CENTERED_CASES = [((6, 12, 12), (2, 4, 4), (1, 1, 1), 16),   # 3 x 3 x 3 tiles: every window is the grid
+                   ((8, 20, 12), (2, 4, 4), (1, 1, 1), 32),   # 4 x 5 x 3 tiles
+                   ((8, 24, 8), (1, 4, 4), (2, 1, 0), 16),    # 8 x 6 x 2 tiles, unequal radii
+                   ((4, 8, 16), (1, 2, 2), (1, 2, 3), 4)]     # 4 x 4 x 8 tiles, a radius beyond the grid
+
+
+@pytest.mark.parametrize("grid,tile,radius,block", _CENTERED_CASES)
+def test_centered_sliding_tile_is_the_nearest_in_grid_window(grid, tile, radius, block):
+    idx, cnt, g = oracle.tile_neighbourhood_list(grid, tile, radius, block, centered=True)
+    perm = oracle.tile_permutation(grid, tile)
+    got = _expand_list_to_tmajor(idx, cnt, g, block, perm)
+    t, h, w = _coords(grid)
+    cs = [t // tile[0], h // tile[1], w // tile[2]]
+    ns = [grid[a] // tile[a] for a in range(3)]
+    want = np.ones_like(got)
+    for a in range(3):
+        lohi = np.array([_nearest_start(c, radius[a], ns[a]) for c in range(ns[a])])
+        lo, hi = lohi[cs[a], 0], lohi[cs[a], 1]
+        want &= (cs[a][None, :] >= lo[:, None]) & (cs[a][None, :] <= hi[:, None])
+    assert g == 0 and np.array_equal(got, want)
+    # every query sees the same number of key tiles, itself among them
+    per_tile = np.prod([min(2 * radius[a] + 1, ns[a]) for a in range(3)])
+    assert np.all(cnt == per_tile * (np.prod(tile) // block))
+    assert np.all(np.diag(got))
+    for i in range(len(cnt)):
+        assert np.all(np.diff(idx[i, :cnt[i]]) > 0)
+
+
+@pytest.mark.parametrize("grid,tile,radius,block", _CENTERED_CASES)
+def test_centered_sliding_tile_agrees_with_clipped_inside_and_is_mirror_symmetric(grid, tile, radius, block):
+    ci, cc, _ = oracle.tile_neighbourhood_list(grid, tile, radius, block, centered=True)
+    pi, pc, _ = oracle.tile_neighbourhood_list(grid, tile, radius, block)
+    ns = [grid[a] // tile[a] for a in range(3)]
+    bpt = np.prod(tile) // block
+    for i in range(len(cc)):
+        tl = i // bpt
+        c = (tl // (ns[1] * ns[2]), (tl // ns[2]) % ns[1], tl % ns[2])
+        inside = all(radius[a] <= c[a] <= ns[a] - 1 - radius[a] for a in range(3))
+        if inside:
+            assert cc[i] == pc[i] and np.array_equal(ci[i, :cc[i]], pi[i, :pc[i]])
+        else:
+            # the clipped window is the centred one cut at the border
+            assert set(pi[i, :pc[i]]) <= set(ci[i, :cc[i]])
+    perm = oracle.tile_permutation(grid, tile)
+    m = _expand_list_to_tmajor(ci, cc, 0, block, perm)
+    t, h, w = _coords(grid)
+    T, H, W = grid
+    for refl in ((T - 1 - t) * H * W + h * W + w, t * H * W + (H - 1 - h) * W + w, t * H * W + h * W + (W - 1 - w)):
+        assert np.array_equal(m[np.ix_(refl, refl)], m)
+
+
+def test_centered_sliding_tile_is_not_symmetric_at_the_border():
+    # 4 tiles along w, radius 1: tile 0 sees tiles 0..2, tile 2 sees 1..3
+    grid, tile, block = (1, 4, 16), (1, 4, 4), 16
+    ci, cc, _ = oracle.tile_neighbourhood_list(grid, tile, (0, 0, 1), block, centered=True)
+    assert [list(ci[i, :cc[i]]) for i in range(4)] == [[0, 1, 2], [0, 1, 2], [1, 2, 3], [1, 2, 3]]
+    pi, pc, _ = oracle.tile_neighbourhood_list(grid, tile, (0, 0, 1), block)
+    assert [list(pi[i, :pc[i]]) for i in range(4)] == [[0, 1], [0, 1, 2], [1, 2, 3], [2, 3]]
+
+
 # --------------------------------------------------------------------------
 # attention (windowed_attention / full_attention; recipe note: dropped blocks)
 # --------------------------------------------------------------------------
