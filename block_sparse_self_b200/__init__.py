@@ -28,7 +28,7 @@ HEADER_PATH = os.path.join(os.path.dirname(_HERE), "include", "vsa.h")
 
 OK, ERR_INVALID_ARGUMENT, ERR_RUNTIME, ERR_CUDA, ERR_UNSUPPORTED, ERR_TIMEOUT = range(6)
 BF16, F32 = 0, 1
-MASK_SPATIAL, MASK_TEMPORAL, MASK_SLIDING_TILE = 0, 1, 2
+MASK_SPATIAL, MASK_TEMPORAL, MASK_SLIDING_TILE, MASK_SLIDING_TILE_CENTERED = 0, 1, 2, 3
 
 
 class Dims3(ctypes.Structure):
@@ -309,13 +309,15 @@ def topp_block_mask(scores: torch.Tensor, p: float, scale: float, n_sink_blocks:
     return idx, cnt
 
 
-_KINDS = {"spatial": MASK_SPATIAL, "temporal": MASK_TEMPORAL, "sliding_tile": MASK_SLIDING_TILE}
+_KINDS = {"spatial": MASK_SPATIAL, "temporal": MASK_TEMPORAL, "sliding_tile": MASK_SLIDING_TILE,
+          "sliding_tile_centered": MASK_SLIDING_TILE_CENTERED}
 
 
 def structured_tile(kind: str, grid, tile=(4, 8, 8)):
     """The tile whose tile-contiguous order a structured list is expressed in."""
     T, Hg, Wg = grid
-    return {"spatial": (1, Hg, Wg), "temporal": (T, 1, 1), "sliding_tile": tuple(tile)}[kind]
+    return {"spatial": (1, Hg, Wg), "temporal": (T, 1, 1), "sliding_tile": tuple(tile),
+            "sliding_tile_centered": tuple(tile)}[kind]
 
 
 def structured_block_list(kind: str, grid, block: int = 128, tile=(4, 8, 8), radius=(1, 1, 1),

@@ -372,7 +372,8 @@ vsa_status vsa_structured_block_list(vsa_mask_kind kind, vsa_dims3 grid, vsa_dim
         tile = vsa_dims3{grid.t, 1, 1};
         radius = vsa_dims3{0, 0, 0};
     } else {
-        VSA_REQUIRE(kind == VSA_MASK_SLIDING_TILE, "unknown mask kind %d", static_cast<int>(kind));
+        VSA_REQUIRE(kind == VSA_MASK_SLIDING_TILE || kind == VSA_MASK_SLIDING_TILE_CENTERED, "unknown mask kind %d",
+                    static_cast<int>(kind));
     }
     VSA_REQUIRE(tile.t > 0 && tile.h > 0 && tile.w > 0, "tile must be positive");
     VSA_REQUIRE(grid.t % tile.t == 0 && grid.h % tile.h == 0 && grid.w % tile.w == 0,
@@ -403,8 +404,14 @@ vsa_status vsa_structured_block_list(vsa_mask_kind kind, vsa_dims3 grid, vsa_dim
     }
     VSA_REQUIRE(cap >= longest, "cap (%d) must be >= the longest list (%lld)", cap, longest);
     *group_size_out = group;
+    // A radius of n - 1 tiles already spans an axis of n tiles in both forms;
+    // clamping keeps the kernel's c +- r and 2r + 1 within int.
+    radius.t = radius.t < grid.t / tile.t ? radius.t : grid.t / tile.t - 1;
+    radius.h = radius.h < grid.h / tile.h ? radius.h : grid.h / tile.h - 1;
+    radius.w = radius.w < grid.w / tile.w ? radius.w : grid.w / tile.w - 1;
     return check_cuda(launch_structured(grid.t, grid.h, grid.w, tile.t, tile.h, tile.w, radius.t, radius.h,
-                                        radius.w, block, idx, cnt, cap, as_stream(stream)),
+                                        radius.w, kind == VSA_MASK_SLIDING_TILE_CENTERED, block, idx, cnt, cap,
+                                        as_stream(stream)),
                       "structured_block_list launch");
 }
 

@@ -45,8 +45,8 @@ cudaError_t launch_topk(const float *scores, int BH, int nb, int k, int n_sink, 
                         int32_t *cnt, int cap, cudaStream_t st);
 cudaError_t launch_topp(const float *scores, int BH, int nb, float p, float scale, int n_sink, int diag_hw,
                         int32_t *idx, int32_t *cnt, int cap, cudaStream_t st);
-cudaError_t launch_structured(int T, int H, int W, int tt, int th, int tw, int rt, int rh, int rw, int block,
-                              int32_t *idx, int32_t *cnt, int cap, cudaStream_t st);
+cudaError_t launch_structured(int T, int H, int W, int tt, int th, int tw, int rt, int rh, int rw, bool centered,
+                              int block, int32_t *idx, int32_t *cnt, int cap, cudaStream_t st);
 
 struct SelectGeom {
     int Rt, Rh, Rw;   // region = per-axis lcm of the candidate tiles

@@ -51,7 +51,9 @@ typedef struct { int32_t t, h, w; } vsa_dims3;
 typedef enum {
     VSA_MASK_SPATIAL = 0,      /* same frame: tile (1, Hg, Wg), radius 0      */
     VSA_MASK_TEMPORAL = 1,     /* same (h, w): tile (T, 1, 1), radius 0       */
-    VSA_MASK_SLIDING_TILE = 2  /* tiles whose coordinates differ by <= radius */
+    VSA_MASK_SLIDING_TILE = 2, /* tiles whose coordinates differ by <= radius */
+    VSA_MASK_SLIDING_TILE_CENTERED = 3 /* 2 radius + 1 tiles per axis, shifted
+                                          inside the grid at the border     */
 } vsa_mask_kind;
 
 /* Message for the last non-OK status returned on this host thread ("" if none). */
@@ -245,14 +247,19 @@ vsa_status vsa_topp_block_mask(const float *scores, int B, int n_heads, int nb, 
 
 /* ------------------------------------------------------------------------ */
 /* Structured static masks as block lists.  "ADR-0001", step 1
- * (spatial_only_mask, temporal_only_mask, sliding_tile_block_mask).
+ * (spatial_only_mask, temporal_only_mask, sliding_tile_block_mask,
+ * sliding_tile_centered_mask).
  *
  * The mask is a tile neighbourhood: token i sees token j iff the coordinates
  * of their tiles differ by at most the radius along (t, h, w), clipped at the
  * grid border.  SPATIAL uses tile (1, Hg, Wg) and radius 0 (same frame);
  * TEMPORAL uses tile (T, 1, 1) and radius 0 (same (h, w)); SLIDING_TILE uses
- * the given tile and radius.  `tile` and `radius` are ignored for SPATIAL
- * and TEMPORAL.  The list is expressed in the tile-contiguous order of that
+ * the given tile and radius.  SLIDING_TILE_CENTERED keeps the window's size
+ * instead of clipping it: along an axis of n tiles, query tile c sees the
+ * w = min(2 r + 1, n) tiles from start min(max(c - r, 0), n - w) on, so every
+ * query sees the same number of tiles and the mask is not symmetric at the
+ * border (the source names this mask only; this is the reading taken).
+ * `tile` and `radius` are ignored for SPATIAL and TEMPORAL.  The list is expressed in the tile-contiguous order of that
  * tile (use vsa_permute with the same tile):
  *   - tile volume a multiple of block: query block i lists every block of
  *     every neighbouring tile, ascending; *group_size_out = 0;

@@ -156,6 +156,13 @@ def test_structured_list_argument_errors(L):
                                        50, ctypes.byref(g), NULL) == vsa.ERR_INVALID_ARGUMENT  # longest list is 54
     assert L.vsa_structured_block_list(7, grid, Dims3(4, 8, 8), Dims3(1, 1, 1), 128, idx, cnt, 960,
                                        ctypes.byref(g), NULL) == vsa.ERR_INVALID_ARGUMENT
+    # the centred window holds the same 54 blocks for every query
+    assert L.vsa_structured_block_list(vsa.MASK_SLIDING_TILE_CENTERED, grid, Dims3(4, 8, 8), Dims3(1, 1, 1), 128,
+                                       idx, cnt, 53, ctypes.byref(g), NULL) == vsa.ERR_INVALID_ARGUMENT
+    assert L.vsa_structured_block_list(vsa.MASK_SLIDING_TILE_CENTERED, grid, Dims3(2, 3, 4), Dims3(1, 1, 1), 128,
+                                       idx, cnt, 960, ctypes.byref(g), NULL) == vsa.ERR_UNSUPPORTED
+    assert L.vsa_structured_block_list(vsa.MASK_SLIDING_TILE_CENTERED, grid, Dims3(4, 8, 8), Dims3(-1, 1, 1), 128,
+                                       idx, cnt, 960, ctypes.byref(g), NULL) == vsa.ERR_INVALID_ARGUMENT
 
 
 def test_python_binding_rejects_cpu_tensors():

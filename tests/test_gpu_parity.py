@@ -206,7 +206,7 @@ def test_topk_threshold_search_paths(nb, kind):
 @pytest.mark.parametrize("grid,block,tile", [((32, 48, 80), 128, (4, 8, 8)), ((8, 4, 8), 32, (2, 2, 8)),
                                              ((6, 12, 16), 64, (2, 4, 8))])
 def test_structured_lists_match_oracle(grid, block, tile):
-    for kind in ("spatial", "temporal", "sliding_tile"):
+    for kind in ("spatial", "temporal", "sliding_tile", "sliding_tile_centered"):
         try:
             idx, cnt, g = vsa.structured_block_list(kind, grid, block, tile=tile, radius=(1, 1, 1))
         except NotImplementedError:   # e.g. temporal groups of 6 tokens in blocks of 64
@@ -215,7 +215,8 @@ def test_structured_lists_match_oracle(grid, block, tile):
                 oracle.tile_neighbourhood_list(grid, t, r, block)
             continue
         t, r = oracle.structured_tile(kind, grid, tile, (1, 1, 1))
-        oi, oc, og = oracle.tile_neighbourhood_list(grid, t, r, block, cap=idx.shape[1])
+        oi, oc, og = oracle.tile_neighbourhood_list(grid, t, r, block, cap=idx.shape[1],
+                                                    centered=kind == "sliding_tile_centered")
         assert g == og
         assert np.array_equal(cnt.cpu().numpy(), oc)
         assert np.array_equal(idx.cpu().numpy(), oi)
@@ -531,14 +532,33 @@ def test_window_full_size_sampled():
         assert_attn_close(_np(o[0, h])[rows], want, f"head {h}")
 
 
-@pytest.mark.parametrize("kind", ["spatial", "temporal", "sliding_tile"])
+@pytest.mark.parametrize("grid,block,tile,radius", [
+    ((8, 16, 32), 128, (2, 8, 8), (1, 1, 1)),    # 4 x 2 x 4 tiles of one 128-token block, through TMA boxes
+    ((6, 16, 40), 64, (1, 8, 8), (2, 0, 1)),     # 64-token tiles through permuted copies, unequal radii
+])
+def test_sliding_tile_centered_attention_every_row(grid, block, tile, radius):
+    """All rows of the centred sliding-tile mask against the oracle, for shapes
+    where most query tiles sit at a border and the window is shifted."""
+    q, k, v = smooth_qkv(1, 2, grid, 64, seed=77, device=DEV)
+    for kind in ("sliding_tile_centered", "sliding_tile"):
+        o = vsa.structured_attention(q, k, v, kind, grid, block, tile=tile, radius=radius, out_dtype=torch.float32)
+        idx, cnt, g = oracle.tile_neighbourhood_list(grid, tile, radius, block,
+                                                     centered=kind == "sliding_tile_centered")
+        perm = oracle.tile_permutation(grid, tile)
+        for h in range(2):
+            qp, kp, vp = (oracle.permute_rows(_np(x[0, h]), perm) for x in (q, k, v))
+            want = oracle.block_sparse_attention(qp, kp, vp, idx, cnt, block, g)
+            assert_attn_close(_np(o[0, h])[perm], want, f"{kind} head {h}")
+
+
+@pytest.mark.parametrize("kind", ["spatial", "temporal", "sliding_tile", "sliding_tile_centered"])
 def test_structured_full_size_sampled(kind):
     w = WORKLOADS["structured_s122880"]
     q, k, v = make_qkv(w, device=DEV, B=2, heads=2)
     o = vsa.structured_attention(q, k, v, kind, w.grid, 128, tile=w.sliding_tile, radius=w.sliding_radius,
                                  out_dtype=torch.float32)
     t, r = oracle.structured_tile(kind, w.grid, w.sliding_tile, w.sliding_radius)
-    idx, cnt, g = oracle.tile_neighbourhood_list(w.grid, t, r, 128)
+    idx, cnt, g = oracle.tile_neighbourhood_list(w.grid, t, r, 128, centered=kind == "sliding_tile_centered")
     perm = oracle.tile_permutation(w.grid, t)
     b, h = 1, 1
     qp, kp, vp = (oracle.permute_rows(_np(x[b, h]), perm) for x in (q, k, v))

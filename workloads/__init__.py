@@ -57,7 +57,7 @@ class Workload:
     window: Optional[int] = None
     sink: int = 0
     chunk: Optional[int] = None
-    structured: Tuple[str, ...] = ()  # "spatial", "temporal", "sliding_tile"
+    structured: Tuple[str, ...] = ()  # "spatial", "temporal", "sliding_tile", "sliding_tile_centered"
     sliding_tile: Dims3 = (4, 8, 8)
     sliding_radius: Dims3 = (1, 1, 1)
 
@@ -114,7 +114,7 @@ WORKLOADS = {
     "structured_s122880": Workload(
         name="structured_s122880", B=2, heads=24, grid=(32, 48, 80), D=128,
         dtype=torch.bfloat16, values="smooth", seed_base=4000,
-        structured=("spatial", "temporal", "sliding_tile")),
+        structured=("spatial", "temporal", "sliding_tile", "sliding_tile_centered")),
 }
 
 
