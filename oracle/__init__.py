@@ -49,6 +49,8 @@ def lib():
         L.orc_tile_neighbourhood_list.restype = i32
         L.orc_centered_tile_neighbourhood_list.argtypes = [i32] * 11 + [P, P, P]
         L.orc_centered_tile_neighbourhood_list.restype = i32
+        L.orc_sampled_probs.argtypes = [P, P, i64, i32, P, i32, dbl, P]
+        L.orc_pattern_masses.argtypes = [P, i32, i32, i32, P, i32, P]
         L.orc_window_attention.argtypes = [P, P, P, i64, i32, i32, i32, dbl, i32, P, i64, P]
         L.orc_block_sparse_attention.argtypes = [P, P, P, i64, i32, i32, P, P, i32, i32, dbl, P, P, i64, P]
         L.orc_window_key_ranges.argtypes = [i64] * 5 + [P]
@@ -275,6 +277,41 @@ def tile_neighbourhood_list(grid, tile, radius, block: int, cap: Optional[int] =
     if trim:
         idx = idx[:, :int(cnt.max())].copy()
     return idx, cnt, int(g.value)
+
+
+# --------------------------------------------------------------------------
+# head profile: spatial or temporal pattern per head
+# --------------------------------------------------------------------------
+
+PATTERN_KINDS = ("spatial", "temporal")
+
+
+def sampled_probs(q, k, rows, scale=None):
+    """Attention probabilities [R, S] of the sampled query rows of one head."""
+    q, k = _f32(q), _f32(k)
+    S, D = q.shape
+    r = np.ascontiguousarray(rows, np.int32)
+    probs = np.empty((len(r), S), np.float64)
+    lib().orc_sampled_probs(_ptr(q), _ptr(k), S, D, _ptr(r), len(r), default_scale(D, scale), _ptr(probs))
+    return probs
+
+
+def pattern_masses(probs, grid, rows):
+    """[R, 2]: each sampled row's probability mass on its own frame (spatial)
+    and on its own (h, w) position (temporal)."""
+    T, H, W = grid
+    probs = np.ascontiguousarray(probs, np.float64)
+    r = np.ascontiguousarray(rows, np.int32)
+    mass = np.empty((len(r), 2), np.float64)
+    lib().orc_pattern_masses(_ptr(probs), T, H, W, _ptr(r), len(r), _ptr(mass))
+    return mass
+
+
+def classify_head(q, k, grid, rows, scale=None):
+    """(kind, mean masses [2]) of one head: the pattern holding the larger mean
+    mass over the sampled rows, 0 = spatial, 1 = temporal, ties to spatial."""
+    mass = pattern_masses(sampled_probs(q, k, rows, scale), grid, rows).mean(axis=0)
+    return (0 if mass[0] >= mass[1] else 1), mass
 
 
 # --------------------------------------------------------------------------

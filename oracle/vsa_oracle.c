@@ -11,7 +11,10 @@
  *
  * Sources (page title, section):
  *  [ADR]  "ADR-0001: Sparse-attention roadmap for video DiTs", Conventions
- *         (T-major token order) and step 1 / step 6 (video masks, permutation).
+ *         (T-major token order) and step 1 / step 2 / step 6 (video masks,
+ *         head profile, permutation).
+ *  [SVG]  "SVG implementation for LTX 2", overview (heads profiled on query
+ *         tokens, spatial or temporal pattern per head).
  *  [WIN]  "fastvideo/mlx_runtime/windowed_attention.py", module docstring
  *         ("Window policy"), _default_scale, _key_ranges_for_block,
  *         windowed_attention.
@@ -442,6 +445,58 @@ int orc_centered_tile_neighbourhood_list(int T, int H, int W, int tt, int th,
 {
     return orc_neighbourhood(T, H, W, tt, th, tw, rt, rh, rw, 1, block, cap,
                              idx, cnt, group_size);
+}
+
+/* ----------------------------------------------------------------------- */
+/* Head profile  [ADR step 2: classify_heads_from_qk, classify_heads_from_  */
+/* probs, classify; SVG overview: each head is profiled on sampled query    */
+/* tokens and given the spatial or the temporal pattern]                    */
+/* ----------------------------------------------------------------------- */
+
+/* Attention probabilities of the sampled query rows over every key of one
+ * head: probs[r][j] = softmax_j(scale * q[rows[r]] . k[j]).  T-major q, k
+ * of S = T*H*W rows.                                                        */
+void orc_sampled_probs(const float *q, const float *k, int64_t S, int D,
+                       const int32_t *rows, int R, double scale, double *probs)
+{
+    #pragma omp parallel for schedule(dynamic, 1)
+    for (int r = 0; r < R; ++r) {
+        const float *qi = q + (int64_t)rows[r] * D;
+        double *p = probs + (int64_t)r * S;
+        double mx = -INFINITY;
+        for (int64_t j = 0; j < S; ++j) {
+            double s = 0.0;
+            for (int d = 0; d < D; ++d) s += (double)qi[d] * (double)k[j * D + d];
+            p[j] = scale * s;
+            if (p[j] > mx) mx = p[j];
+        }
+        double sum = 0.0;
+        for (int64_t j = 0; j < S; ++j) {
+            p[j] = exp(p[j] - mx);
+            sum += p[j];
+        }
+        for (int64_t j = 0; j < S; ++j) p[j] /= sum;
+    }
+}
+
+/* The probability mass each sampled row puts inside the two structured
+ * patterns: mass[r][0] on the keys of its own frame (spatial_only_mask),
+ * mass[r][1] on the keys at its own (h, w) (temporal_only_mask).           */
+void orc_pattern_masses(const double *probs, int T, int H, int W,
+                        const int32_t *rows, int R, double *mass)
+{
+    int64_t S = (int64_t)T * H * W, HW = (int64_t)H * W;
+    for (int r = 0; r < R; ++r) {
+        int64_t i = rows[r];
+        int64_t ti = i / HW, pi = i % HW;
+        double sp = 0.0, tp = 0.0;
+        for (int64_t j = 0; j < S; ++j) {
+            if (j / HW == ti) sp += probs[(int64_t)r * S + j];
+            if (j % HW == pi) tp += probs[(int64_t)r * S + j];
+        }
+        mass[2 * r] = sp;
+        mass[2 * r + 1] = tp;
+    }
 }
 
 /* ----------------------------------------------------------------------- */

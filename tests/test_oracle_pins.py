@@ -363,6 +363,88 @@ def test_centered_sliding_tile_is_not_symmetric_at_the_border():
 
 
 # --------------------------------------------------------------------------
+# head profile (ADR step 2; SVG: spatial or temporal pattern per head)
+# --------------------------------------------------------------------------
+
+def test_head_profile_uniform_attention_masses_are_the_pattern_sizes():
+    # q = 0: every key has the same logit, so a pattern's mass is its size / S
+    grid = (5, 3, 4)
+    S, HW = 60, 12
+    k = np.random.default_rng(3).standard_normal((S, 16)).astype(np.float32)
+    q = np.zeros((S, 16), np.float32)
+    rows = [0, 7, 59, 31]
+    mass = oracle.pattern_masses(oracle.sampled_probs(q, k, rows), grid, rows)
+    assert np.allclose(mass[:, 0], HW / S, rtol=0, atol=1e-15)
+    assert np.allclose(mass[:, 1], 5 / S, rtol=0, atol=1e-15)
+
+
+@pytest.mark.parametrize("alpha", [0.5, 2.0, 6.0])
+def test_head_profile_closed_forms_of_one_hot_fields(alpha):
+    grid = (4, 4, 4)
+    T, HW, S = 4, 16, 64
+    t, h, w = _coords(grid)
+    hw = h * 4 + w
+    rows = [0, 21, 42, 63]
+    e = math.exp(alpha)
+    # frame-coded field: logit alpha inside the query's frame, 0 elsewhere
+    q = np.zeros((S, 16), np.float32)
+    k = np.zeros((S, 16), np.float32)
+    q[np.arange(S), t] = alpha
+    k[np.arange(S), t] = 1.0
+    kind, mass = oracle.classify_head(q, k, grid, rows, scale=1.0)
+    z = HW * e + (S - HW)
+    assert kind == 0
+    assert mass[0] == pytest.approx(HW * e / z, rel=1e-13)
+    assert mass[1] == pytest.approx((e + T - 1) / z, rel=1e-13)
+    # position-coded field: logit alpha at the query's (h, w), 0 elsewhere
+    q[:] = 0.0
+    k[:] = 0.0
+    q[np.arange(S), hw] = alpha
+    k[np.arange(S), hw] = 1.0
+    kind, mass = oracle.classify_head(q, k, grid, rows, scale=1.0)
+    z = T * e + (S - T)
+    sp, tp = (e + HW - 1) / z, T * e / z
+    assert mass[1] == pytest.approx(tp, rel=1e-13)
+    assert mass[0] == pytest.approx(sp, rel=1e-13)
+    # a weak position code still leaves more mass on the 16-token frame than on
+    # the 4 keys at the query's position
+    assert kind == (0 if sp >= tp else 1) and kind == (1 if alpha >= 2 else 0)
+
+
+def test_head_profile_matches_torch_softmax_and_coordinate_masks():
+    grid = (6, 4, 5)
+    S = 120
+    rng = np.random.default_rng(11)
+    q = (rng.standard_normal((S, 32)) * 0.7).astype(np.float32)
+    k = (rng.standard_normal((S, 32)) * 0.7).astype(np.float32)
+    rows = np.array([0, 1, 19, 20, 64, 119], np.int32)
+    scale = 0.3
+    logits = torch.as_tensor(q, dtype=torch.float64)[rows] @ torch.as_tensor(k, dtype=torch.float64).T * scale
+    want_p = torch.softmax(logits, dim=-1).numpy()
+    got_p = oracle.sampled_probs(q, k, rows, scale)
+    assert np.allclose(got_p, want_p, rtol=1e-12, atol=1e-15)
+    t, h, w = _coords(grid)
+    same_t = t[rows][:, None] == t[None, :]
+    same_hw = (h[rows][:, None] == h[None, :]) & (w[rows][:, None] == w[None, :])
+    mass = oracle.pattern_masses(got_p, grid, rows)
+    assert np.allclose(mass[:, 0], (want_p * same_t).sum(1), rtol=1e-12)
+    assert np.allclose(mass[:, 1], (want_p * same_hw).sum(1), rtol=1e-12)
+    # the patterns meet only at the query itself
+    self_p = want_p[np.arange(len(rows)), rows]
+    assert np.all(mass >= 0) and np.all(mass <= 1 + 1e-12)
+    assert np.all(mass[:, 0] + mass[:, 1] - self_p <= 1 + 1e-12)
+
+
+def test_head_profile_tie_goes_to_spatial():
+    # T = H*W and uniform attention: both patterns hold 4/16 of every row
+    grid = (4, 2, 2)
+    q = np.zeros((16, 8), np.float32)
+    k = np.random.default_rng(5).standard_normal((16, 8)).astype(np.float32)
+    kind, mass = oracle.classify_head(q, k, grid, [0, 5, 10, 15])
+    assert mass[0] == mass[1] and kind == 0
+
+
+# --------------------------------------------------------------------------
 # attention (windowed_attention / full_attention; recipe note: dropped blocks)
 # --------------------------------------------------------------------------
 
