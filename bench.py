@@ -569,6 +569,24 @@ def run_ours(args, w):
         tp["gbs"] = tp["bytes"] / tp["ms_per_call"] / 1e6
         extra["topp_lists_" + w.name] = tp
         del ti, tc
+        # head profile (spatial or temporal pattern per head) on 128 sampled query rows:
+        # K is read once per head (the bound); Q contributes only the sampled rows
+        rows = vsa.sample_query_rows(w.S, 128, seed=0, device=q.device)
+        for _ in range(3):
+            vsa.head_profile(q, k, w.grid, rows)
+        ev[0].record()
+        for _ in range(n_rep):
+            hk, hm = vsa.head_profile(q, k, w.grid, rows)
+        ev[1].record()
+        torch.cuda.synchronize()
+        hp_ms = ev[0].elapsed_time(ev[1]) / n_rep
+        hp_bytes = float(k.numel() * 2 + BH * 128 * w.D * 2)
+        extra["head_profile_" + w.name] = {
+            "ms_per_call": hp_ms, "rows": 128, "bytes": hp_bytes, "gbs": hp_bytes / hp_ms / 1e6,
+            "frac_hbm": hp_bytes / hp_ms / 1e6 / hbm,
+            "tflops": 2.0 * 2 * 128 * w.S * w.D * BH / hp_ms / 1e9,
+            "temporal_heads": int(hk.sum().item()), "heads": BH}
+        del hk, hm
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:

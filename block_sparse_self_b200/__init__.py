@@ -66,6 +66,8 @@ def lib() -> ctypes.CDLL:
         "vsa_block_sparse_attention": ([P, P, P, P, I, I, I, I, I, I, P, P, I, I, I, F, P], I),
         "vsa_block_sparse_attention_tiled": ([P, P, P, P, I, I, I, I, I, D3, P, I, P, P, P, I, I, I, F, P], I),
         "vsa_window_attention": ([P, P, P, P, I, I, I, I, I, I, I, F, I, P], I),
+        "vsa_head_profile_workspace_size": ([I, I, I, I], SZ),
+        "vsa_head_profile": ([P, P, I, I, I, I, D3, P, I, F, P, P, P, SZ, P], I),
         "vsa_cast_f32_to_bf16": ([P, P, I64, P], I),
         "vsa_debug_wait_timeout": ([I64, P], I),
     }
@@ -337,6 +339,44 @@ def structured_block_list(kind: str, grid, block: int = 128, tile=(4, 8, 8), rad
     _check(lib().vsa_structured_block_list(_KINDS[kind], Dims3(*grid), Dims3(*tile), Dims3(*radius), block,
                                            _ptr(idx), _ptr(cnt), cap, ctypes.byref(g), _stream(idx.device)))
     return idx, cnt, int(g.value)
+
+
+PATTERN_KINDS = ("spatial", "temporal")
+
+
+def sample_query_rows(S: int, n_rows: int = 128, seed: int = 0, device="cuda") -> torch.Tensor:
+    """A seeded draw of distinct query positions for the head profile (int32 [n_rows])."""
+    if not 1 <= n_rows <= min(128, S):
+        raise ValueError(f"n_rows must be in [1, min(128, S)], got {n_rows}")
+    g = torch.Generator(device="cpu")
+    g.manual_seed(int(seed))
+    rows = torch.randperm(S, generator=g)[:n_rows].sort().values
+    return rows.to(device=device, dtype=torch.int32)
+
+
+def head_profile(q, k, grid, rows=None, scale: Optional[float] = None, n_rows: int = 128, seed: int = 0):
+    """Per-(b, head) attention mass on the spatial (same frame) and temporal
+    (same (h, w)) patterns over sampled query rows, and the head's kind
+    (0 = spatial, 1 = temporal): (kind int32 [B, H], masses fp32 [B, H, 2]).
+    `rows` (int32 [R], R <= 128) defaults to sample_query_rows(S, n_rows, seed)."""
+    B, H, S, D = _bhsd(q, "q")
+    if tuple(k.shape) != (B, H, S, D):
+        raise ValueError(f"q/k shapes must match exactly; got q={tuple(q.shape)}, k={tuple(k.shape)}")
+    qb, kb = _bf16(q, "q"), _bf16(k, "k")
+    if rows is None:
+        rows = sample_query_rows(S, min(n_rows, S), seed, q.device)
+    _cuda(rows, "rows")
+    if rows.dtype != torch.int32 or rows.dim() != 1:
+        raise ValueError("rows must be a 1-D int32 tensor")
+    rows = rows.contiguous()
+    masses = torch.empty(B, H, 2, dtype=torch.float32, device=q.device)
+    kind = torch.empty(B, H, dtype=torch.int32, device=q.device)
+    ws_bytes = lib().vsa_head_profile_workspace_size(B, H, S, D)
+    ws = torch.empty(max(ws_bytes, 256) // 4 + 1, dtype=torch.float32, device=q.device)
+    _check(lib().vsa_head_profile(_ptr(qb), _ptr(kb), B, H, S, D, Dims3(*grid), _ptr(rows), rows.numel(),
+                                  0.0 if scale is None else float(scale), _ptr(masses), _ptr(kind), _ptr(ws),
+                                  ws.numel() * 4, _stream(q.device)))
+    return kind, masses
 
 
 def _bf16(t: torch.Tensor, name: str) -> torch.Tensor:

@@ -415,6 +415,32 @@ vsa_status vsa_structured_block_list(vsa_mask_kind kind, vsa_dims3 grid, vsa_dim
                       "structured_block_list launch");
 }
 
+size_t vsa_head_profile_workspace_size(int B, int n_heads, int S, int D) {
+    if (B < 1 || n_heads < 1 || S < 1 || (D != 64 && D != 128)) return 0;
+    return vsa::profile_workspace_bytes(B * n_heads, S, D);
+}
+
+vsa_status vsa_head_profile(const void *q, const void *k, int B, int n_heads, int S, int D, vsa_dims3 grid,
+                            const int32_t *rows, int R, float scale, float *masses, int32_t *kind, void *workspace,
+                            size_t workspace_bytes, void *stream) {
+    VSA_TRY(check_bhsd(B, n_heads, S, D));
+    VSA_TRY(check_d(D));
+    VSA_REQUIRE(S < (1 << 30), "S must be < 2^30, got %d", S);
+    VSA_TRY(check_grid(grid, S));
+    VSA_REQUIRE(aligned16(q) && aligned16(k), "q and k must be non-NULL 16-byte aligned device pointers");
+    VSA_REQUIRE(R >= 1 && R <= 128, "R (sampled rows) must be in [1, 128], got %d", R);
+    VSA_REQUIRE(aligned4(rows), "rows must be a non-NULL 4-byte aligned device pointer");
+    VSA_REQUIRE(aligned4(masses) && aligned4(kind), "masses and kind must be non-NULL 4-byte aligned device pointers");
+    VSA_REQUIRE(scale == scale && scale < 3.0e38f, "scale must be finite");
+    const size_t need = vsa_head_profile_workspace_size(B, n_heads, S, D);
+    VSA_REQUIRE(aligned16(workspace), "workspace must be a non-NULL 16-byte aligned device pointer");
+    VSA_REQUIRE(workspace_bytes >= need, "workspace holds %zu bytes, %zu needed", workspace_bytes, need);
+    const float sc = scale > 0.f ? scale : 1.0f / sqrtf(static_cast<float>(D));
+    return check_cuda(launch_head_profile(q, k, B * n_heads, S, D, grid.h * grid.w, rows, R, sc, workspace, masses,
+                                          kind, status_or_null(), as_stream(stream)),
+                      "head_profile launch");
+}
+
 static vsa_status check_attention_common(const void *q, const void *k, const void *v, void *o, vsa_dtype out_dtype,
                                          int B, int n_heads, int S, int D, float scale) {
     VSA_TRY(check_bhsd(B, n_heads, S, D));

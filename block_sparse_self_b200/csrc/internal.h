@@ -99,6 +99,14 @@ bool make_scores_store_map(CUtensorMap *m, float *ptr, int nb, int BH);
 
 cudaError_t launch_wait_timeout(uint64_t limit_ns, int *status, cudaStream_t st);
 
+// Head profile (profile.cu): CTAs per head over the key tiles, and the scratch
+// (gathered sample tiles, then per-part row partials) that launch needs.
+int profile_split(int BH, int S);
+size_t profile_workspace_bytes(int BH, int S, int D);
+cudaError_t launch_head_profile(const void *q, const void *k, int BH, int S, int D, int HW, const int32_t *rows,
+                                int R, float scale, void *workspace, float *masses, int32_t *kind, int *status,
+                                cudaStream_t st);
+
 // Address and size of the file-scope scratch array that
 // vsa_select_tiling_noalloc uses (looked up once per device).
 vsa_status select_static_scratch(float **ptr, size_t *bytes);

@@ -351,6 +351,41 @@ vsa_status vsa_window_attention(const void *q, const void *k, const void *v, voi
                                 void *stream);
 
 /* ------------------------------------------------------------------------ */
+/* Head profile: spatial or temporal pattern per head.  "ADR-0001", step 2
+ * (classify_heads_from_qk, classify_heads_from_probs, classify: the profiler
+ * consumes Q and K only) and "SVG implementation for LTX 2", overview (each
+ * head is profiled on query tokens and given the spatial or the temporal
+ * attention pattern).  The pages give the names and that purpose only; the
+ * reading taken here:
+ *   for each sampled query row i (T-major position rows[r]) of a (b, head),
+ *   p_ij = softmax_j(scale * q_i . k_j) over all S keys;
+ *   mass_spatial(i)  = sum of p_ij over the keys of i's frame
+ *                      (the spatial_only mask),
+ *   mass_temporal(i) = sum of p_ij over the keys at i's (h, w)
+ *                      (the temporal_only mask);
+ *   masses[bh] = (mean_i mass_spatial, mean_i mass_temporal);
+ *   kind[bh]   = 1 (temporal) if its mean mass is larger, else 0 (spatial).
+ * QK^T runs on the tensor cores (bf16 inputs, fp32 accumulation); the
+ * softmax sums are fp32, so masses are within about 1e-5 of exact and heads
+ * whose two masses differ by less than that may take either kind.
+ *   q, k      [B, n_heads, S, D] bf16, T-major over grid (T, Hg, Wg)
+ *   rows      [R] int32 device array of query positions in [0, S), shared
+ *             by every (b, head); 1 <= R <= 128 (the sample is an input:
+ *             callers draw it).  A position out of range sets
+ *             VSA_ERR_RUNTIME in the device status word (that row is
+ *             profiled as a zero query).
+ *   scale     softmax scale; <= 0 selects 1/sqrt(D)
+ *   masses    [B*n_heads, 2] fp32 output;  kind [B*n_heads] int32 output
+ *   workspace device scratch of vsa_head_profile_workspace_size(...) bytes,
+ *             16-byte aligned; contents need not be initialised.
+ * D in {64, 128}; S < 2^30.                                                */
+size_t vsa_head_profile_workspace_size(int B, int n_heads, int S, int D);
+vsa_status vsa_head_profile(const void *q, const void *k, int B, int n_heads, int S, int D,
+                            vsa_dims3 grid, const int32_t *rows, int R, float scale,
+                            float *masses, int32_t *kind, void *workspace,
+                            size_t workspace_bytes, void *stream);
+
+/* ------------------------------------------------------------------------ */
 /* Round-to-nearest-even fp32 -> bf16 conversion of n elements (x, y device).
  * Used to feed fp32 tensors to the bf16 attention calls.                  */
 vsa_status vsa_cast_f32_to_bf16(const float *x, void *y, int64_t n, void *stream);
