@@ -51,6 +51,7 @@ def lib():
         L.orc_centered_tile_neighbourhood_list.restype = i32
         L.orc_sampled_probs.argtypes = [P, P, i64, i32, P, i32, dbl, P]
         L.orc_pattern_masses.argtypes = [P, i32, i32, i32, P, i32, P]
+        L.orc_centroid_compensated_attention.argtypes = [P, P, P, i64, i32, P, P, i32, i32, P, dbl, P, i64, P]
         L.orc_window_attention.argtypes = [P, P, P, i64, i32, i32, i32, dbl, i32, P, i64, P]
         L.orc_block_sparse_attention.argtypes = [P, P, P, i64, i32, i32, P, P, i32, i32, dbl, P, P, i64, P]
         L.orc_window_key_ranges.argtypes = [i64] * 5 + [P]
@@ -332,6 +333,26 @@ def window_attention(q, k, v, window: int, sink: int = 0, scale=None, rows=None)
     out = np.empty((len(r), D), np.float64)
     lib().orc_window_attention(_ptr(q), _ptr(k), _ptr(v), S, D, window, sink,
                                default_scale(D, scale), 0, _ptr(r), len(r), _ptr(out))
+    return out
+
+
+def centroid_compensated_attention(q, k, v, q_labels, k_labels, block_mask, scale=None, rows=None):
+    """centroid_compensated_attention for one head [S, D]: kept key blocks
+    exactly, each skipped key block as its mean key and mean value weighted by
+    its size.  q_labels / k_labels give each token's block, block_mask
+    [n_q_blocks, n_k_blocks] (bool) the kept pairs.  Returns rows x D doubles."""
+    q, k, v = _f32(q), _f32(k), _f32(v)
+    S, D = q.shape
+    ql = np.ascontiguousarray(q_labels, np.int32)
+    kl = np.ascontiguousarray(k_labels, np.int32)
+    m = np.ascontiguousarray(block_mask, np.uint8)
+    n_qb, n_kb = m.shape
+    if len(ql) != S or len(kl) != S or ql.min() < 0 or ql.max() >= n_qb or kl.min() < 0 or kl.max() >= n_kb:
+        raise ValueError("labels must give every token a block of block_mask")
+    r = _rows(rows, S)
+    out = np.empty((len(r), D), np.float64)
+    lib().orc_centroid_compensated_attention(_ptr(q), _ptr(k), _ptr(v), S, D, _ptr(ql), _ptr(kl), n_qb, n_kb,
+                                             _ptr(m), default_scale(D, scale), _ptr(r), len(r), _ptr(out))
     return out
 
 

@@ -589,6 +589,89 @@ void orc_block_sparse_attention(const float *q, const float *k, const float *v,
     }
 }
 
+/* centroid_compensated_attention [SPADE Recipe: the attention call with
+ * q_labels, k_labels and the block mask; "compensate skipped blocks instead
+ * of dropping them"].  The pages give the call and its arguments only.  The
+ * reading: query i (block a = q_labels[i]) attends exactly to every key t
+ * whose block k_labels[t] is kept (block_mask[a][k_labels[t]] != 0); each
+ * skipped key block b with n_b > 0 keys takes part as one centroid key
+ * kbar_b (the mean of its keys) with value vbar_b (the mean of its values)
+ * and weight n_b:
+ *   o_i = (sum_kept e^{s(q_i, k_t)} v_t + sum_skipped n_b e^{s(q_i, kbar_b)} vbar_b)
+ *       / (sum_kept e^{s(q_i, k_t)}     + sum_skipped n_b e^{s(q_i, kbar_b)}),
+ * s(q, k) = scale q . k.  A skipped block whose keys are all equal then
+ * contributes exactly what it would have if kept.  All in double.          */
+void orc_centroid_compensated_attention(const float *q, const float *k, const float *v,
+                                        int64_t S, int D, const int32_t *q_labels,
+                                        const int32_t *k_labels, int n_qb, int n_kb,
+                                        const unsigned char *block_mask, double scale,
+                                        const int64_t *rows, int64_t n_rows, double *out)
+{
+    /* the centroids */
+    double *kbar = (double *)calloc((size_t)n_kb * D, sizeof(double));
+    double *vbar = (double *)calloc((size_t)n_kb * D, sizeof(double));
+    int64_t *nb = (int64_t *)calloc((size_t)n_kb, sizeof(int64_t));
+    for (int64_t t = 0; t < S; ++t) {
+        int b = k_labels[t];
+        nb[b] += 1;
+        for (int d = 0; d < D; ++d) {
+            kbar[(int64_t)b * D + d] += (double)k[t * D + d];
+            vbar[(int64_t)b * D + d] += (double)v[t * D + d];
+        }
+    }
+    for (int b = 0; b < n_kb; ++b)
+        if (nb[b] > 0)
+            for (int d = 0; d < D; ++d) {
+                kbar[(int64_t)b * D + d] /= (double)nb[b];
+                vbar[(int64_t)b * D + d] /= (double)nb[b];
+            }
+    #pragma omp parallel
+    {
+        /* logits of the S keys, then of the n_kb centroids */
+        double *logit = (double *)malloc(sizeof(double) * (size_t)(S + n_kb));
+        #pragma omp for schedule(dynamic, 4)
+        for (int64_t r = 0; r < n_rows; ++r) {
+            int64_t i = rows[r];
+            const unsigned char *keep = block_mask + (int64_t)q_labels[i] * n_kb;
+            double mx = -INFINITY;
+            for (int64_t t = 0; t < S; ++t) {
+                if (!keep[k_labels[t]]) continue;
+                double s = 0.0;
+                for (int d = 0; d < D; ++d) s += (double)q[i * D + d] * (double)k[t * D + d];
+                logit[t] = scale * s;
+                if (logit[t] > mx) mx = logit[t];
+            }
+            for (int b = 0; b < n_kb; ++b) {
+                if (keep[b] || nb[b] == 0) continue;
+                double s = 0.0;
+                for (int d = 0; d < D; ++d) s += (double)q[i * D + d] * kbar[(int64_t)b * D + d];
+                logit[S + b] = scale * s;
+                if (logit[S + b] > mx) mx = logit[S + b];
+            }
+            double den = 0.0;
+            double *o = out + r * D;
+            for (int d = 0; d < D; ++d) o[d] = 0.0;
+            for (int64_t t = 0; t < S; ++t) {
+                if (!keep[k_labels[t]]) continue;
+                double w = exp(logit[t] - mx);
+                den += w;
+                for (int d = 0; d < D; ++d) o[d] += w * (double)v[t * D + d];
+            }
+            for (int b = 0; b < n_kb; ++b) {
+                if (keep[b] || nb[b] == 0) continue;
+                double w = (double)nb[b] * exp(logit[S + b] - mx);
+                den += w;
+                for (int d = 0; d < D; ++d) o[d] += w * vbar[(int64_t)b * D + d];
+            }
+            for (int d = 0; d < D; ++d) o[d] /= den;
+        }
+        free(logit);
+    }
+    free(nb);
+    free(vbar);
+    free(kbar);
+}
+
 /* _key_ranges_for_block: ordered, non-overlapping key ranges [start, end)
  * that query rows [qs, qe) need: the local window over every row, plus the
  * sinks [0, sink), merged into one range when they touch.  Writes up to two

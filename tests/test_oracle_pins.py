@@ -686,3 +686,85 @@ def test_topp_invariances_and_static_blocks():
     with_static = _topp_sets(score, 0.6, 1.3, n_sink=2, dw=1)
     for i, (k, ks) in enumerate(zip(base, with_static)):
         assert ks == k | {0, 1} | {j for j in range(nb) if abs(j - i) <= 1}
+
+
+# --------------------------------------------------------------------------
+# centroid-compensated attention (SPADE Recipe: skipped blocks compensated)
+# --------------------------------------------------------------------------
+
+def _labels_irregular(S, seed):
+    """Block labels with blocks of unequal sizes (1 to 12 tokens), in order."""
+    rng = np.random.default_rng(seed)
+    sizes = []
+    while sum(sizes) < S:
+        sizes.append(int(rng.integers(1, 13)))
+    sizes[-1] -= sum(sizes) - S
+    return np.repeat(np.arange(len(sizes)), sizes).astype(np.int32), len(sizes)
+
+
+def test_compensated_attention_with_every_block_kept_is_dense():
+    q, k, v = _qkv(96, 16, 40)
+    lab = (np.arange(96) // 16).astype(np.int32)
+    got = oracle.centroid_compensated_attention(q, k, v, lab, lab, np.ones((6, 6), bool), scale=0.25)
+    assert np.allclose(got, _sdpa64(q, k, v, 0.25), rtol=0, atol=1e-12)
+
+
+@pytest.mark.parametrize("seed", [0, 1, 2])
+def test_compensated_attention_is_exact_when_block_keys_are_equal(seed):
+    # every key of a block is the same vector (values differ): a skipped block's
+    # centroid then stands for its keys exactly, whatever the mask
+    S, D = 120, 16
+    rng = np.random.default_rng(100 + seed)
+    kl, nkb = _labels_irregular(S, seed)
+    ql = (np.arange(S) // 10).astype(np.int32)
+    q = rng.standard_normal((S, D)).astype(np.float32)
+    kb = rng.standard_normal((nkb, D)).astype(np.float32)
+    k = kb[kl]
+    v = rng.standard_normal((S, D)).astype(np.float32)
+    mask = rng.random((12, nkb)) < 0.3
+    mask[0] = False       # query block 0 keeps nothing: centroids only
+    mask[1] = True        # query block 1 keeps everything
+    got = oracle.centroid_compensated_attention(q, k, v, ql, kl, mask, scale=0.5)
+    assert np.allclose(got, _sdpa64(q, k, v, 0.5), rtol=0, atol=1e-12)
+
+
+def test_compensated_attention_with_nothing_kept_is_attention_over_weighted_centroids():
+    S, D = 90, 8
+    q, k, v = _qkv(S, D, 50)
+    kl, nkb = _labels_irregular(S, 7)
+    ql = np.zeros(S, np.int32)
+    got = oracle.centroid_compensated_attention(q, k, v, ql, kl, np.zeros((1, nkb), bool), scale=0.7)
+    n = np.bincount(kl, minlength=nkb).astype(np.float64)
+    kbar = np.stack([k[kl == b].astype(np.float64).mean(0) for b in range(nkb)])
+    vbar = np.stack([v[kl == b].astype(np.float64).mean(0) for b in range(nkb)])
+    # a weight n_b on a key is an additive log(n_b) on its logit
+    bias = torch.as_tensor(np.log(n))[None, None, None, :].expand(1, 1, S, nkb)
+    want = torch.nn.functional.scaled_dot_product_attention(
+        torch.as_tensor(q, dtype=torch.float64)[None, None], torch.as_tensor(kbar)[None, None],
+        torch.as_tensor(vbar)[None, None], attn_mask=bias, scale=0.7)[0, 0].numpy()
+    assert np.allclose(got, want, rtol=0, atol=1e-12)
+
+
+def test_compensated_attention_reduces_to_dropped_blocks_when_skipped_weights_vanish():
+    # queries positive, skipped blocks' keys strongly negative: their centroid
+    # weights underflow next to the kept keys, leaving the recipe note's
+    # dropped-block attention
+    S, D, block = 64, 8, 16
+    rng = np.random.default_rng(9)
+    q = rng.uniform(0.5, 1.0, (S, D)).astype(np.float32)
+    k = rng.uniform(-0.5, 0.5, (S, D)).astype(np.float32)
+    v = rng.standard_normal((S, D)).astype(np.float32)
+    lab = (np.arange(S) // block).astype(np.int32)
+    mask = np.eye(4, dtype=bool)
+    mask[:, 0] = True
+    for b in (1, 2, 3):
+        k[lab == b] -= 40.0
+    got = oracle.centroid_compensated_attention(q, k, v, lab, lab, mask, scale=1.0)
+    idx = np.full((4, 2), -1, np.int32)
+    cnt = np.zeros(4, np.int32)
+    for a in range(4):
+        js = np.flatnonzero(mask[a])
+        idx[a, :len(js)] = js
+        cnt[a] = len(js)
+    want = oracle.block_sparse_attention(q, k, v, idx, cnt, block, 0, scale=1.0)
+    assert np.allclose(got, want, rtol=0, atol=1e-12)
