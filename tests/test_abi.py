@@ -189,3 +189,27 @@ def test_python_binding_rejects_cpu_tensors():
         vsa.window_attention(q, q, q, window=8)
     with pytest.raises(ValueError):
         vsa.permute(q, (2, 8, 8), [(1, 8, 8)])
+
+
+def test_sample_query_rows_is_a_seeded_sorted_distinct_draw():
+    import torch
+    r = vsa.sample_query_rows(1000, 128, seed=3, device="cpu")
+    assert r.dtype == torch.int32 and r.shape == (128,)
+    assert torch.all(r[1:] > r[:-1]) and int(r.min()) >= 0 and int(r.max()) < 1000
+    assert torch.equal(r, vsa.sample_query_rows(1000, 128, seed=3, device="cpu"))
+    assert not torch.equal(r, vsa.sample_query_rows(1000, 128, seed=4, device="cpu"))
+    assert vsa.sample_query_rows(50, 50, device="cpu").tolist() == list(range(50))
+    with pytest.raises(ValueError):
+        vsa.sample_query_rows(1000, 129, device="cpu")
+    with pytest.raises(ValueError):
+        vsa.sample_query_rows(10, 11, device="cpu")
+
+
+def test_head_profile_and_centred_kind_reject_bad_host_arguments():
+    import torch
+    q = torch.zeros(1, 1, 128, 64)
+    with pytest.raises(ValueError):   # CPU tensors never reach the library
+        vsa.head_profile(q, q, (2, 8, 8))
+    with pytest.raises(ValueError):
+        vsa.structured_block_list("sliding_tile_centred", (8, 16, 16), 128)   # the kind is spelt "centered"
+    assert vsa.structured_tile("sliding_tile_centered", (8, 16, 16), (2, 8, 8)) == (2, 8, 8)
