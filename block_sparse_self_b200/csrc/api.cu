@@ -9,6 +9,7 @@
 #include <stdarg.h>
 #include <stdio.h>
 
+#include <mutex>
 #include <string>
 
 #include "common.cuh"
@@ -36,16 +37,38 @@ vsa_status check_cuda(cudaError_t e, const char *what) {
     return fail(VSA_ERR_CUDA, "%s: %s", what, cudaGetErrorString(e));
 }
 
-int *device_status_word() {
-    static int *ptrs[128] = {};
+vsa_status cached_symbol_address(SymbolCache &cache, cudaStream_t st, cudaError_t (*lookup)(void **), void **out) {
     int dev = 0;
-    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 128) return nullptr;
-    if (!ptrs[dev]) {
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return check_cuda(e, "cudaGetDevice");
+    if (dev < 0 || dev >= SymbolCache::kDevices) return fail(VSA_ERR_UNSUPPORTED, "device ordinal %d out of range", dev);
+    // Outside a capture the address is looked up again, so a context that was
+    // torn down and created anew (cudaDeviceReset, a released primary
+    // context) is never served a stale address.  During a capture the lookup
+    // is skipped (it may have to load the module) and the last address seen
+    // on the device is used.
+    cudaStreamCaptureStatus cs = cudaStreamCaptureStatusNone;
+    const bool capturing = cudaStreamIsCapturing(st, &cs) != cudaSuccess || cs != cudaStreamCaptureStatusNone;
+    std::lock_guard<std::mutex> lock(cache.mu);
+    if (!capturing || !cache.addr[dev]) {
         void *p = nullptr;
-        if (cudaGetSymbolAddress(&p, g_status_word) != cudaSuccess) return nullptr;
-        ptrs[dev] = static_cast<int *>(p);
+        e = lookup(&p);
+        if (e != cudaSuccess) return check_cuda(e, "cudaGetSymbolAddress");
+        cache.addr[dev] = p;
     }
-    return ptrs[dev];
+    *out = cache.addr[dev];
+    return VSA_OK;
+}
+
+namespace {
+cudaError_t status_word_lookup(void **p) { return cudaGetSymbolAddress(p, g_status_word); }
+}  // namespace
+
+int *device_status_word(cudaStream_t st) {
+    static SymbolCache cache;
+    void *p = nullptr;
+    if (cached_symbol_address(cache, st, status_word_lookup, &p) != VSA_OK) return nullptr;
+    return static_cast<int *>(p);
 }
 
 }  // namespace vsa
@@ -132,7 +155,7 @@ bool overlaps(const void *a, size_t na, const void *b, size_t nb) {
         if (_s != VSA_OK) return _s;      \
     } while (0)
 
-int *status_or_null() { return device_status_word(); }
+int *status_or_null(void *stream) { return device_status_word(as_stream(stream)); }
 
 }  // namespace
 
@@ -198,7 +221,7 @@ vsa_status vsa_select_tiling(const void *q, vsa_dtype dtype, int B, int n_heads,
     VSA_REQUIRE(workspace_bytes >= need, "workspace holds %zu bytes, %zu needed", workspace_bytes, need);
     return check_cuda(launch_select_tiling(q, esize_of(dtype), B * n_heads, D, grid.t, grid.h, grid.w, pg.t, pg.h,
                                            pg.w, ts, g, choice, sics, static_cast<float *>(workspace),
-                                           status_or_null(), as_stream(stream)),
+                                           status_or_null(stream), as_stream(stream)),
                       "select_tiling launch");
 }
 
@@ -227,9 +250,9 @@ vsa_status vsa_select_tiling_noalloc(const void *q, vsa_dtype dtype, int B, int 
                 need, VSA_SELECT_TILING_NOALLOC_MAX_BYTES);
     float *scratch = nullptr;
     size_t scratch_bytes = 0;
-    VSA_TRY(select_static_scratch(&scratch, &scratch_bytes));
+    VSA_TRY(select_static_scratch(&scratch, &scratch_bytes, as_stream(stream)));
     return check_cuda(launch_select_tiling(q, esize_of(dtype), B * n_heads, D, grid.t, grid.h, grid.w, pg.t, pg.h,
-                                           pg.w, ts, g, choice, sics, scratch, status_or_null(), as_stream(stream)),
+                                           pg.w, ts, g, choice, sics, scratch, status_or_null(stream), as_stream(stream)),
                       "select_tiling (no-alloc) launch");
 }
 
@@ -251,7 +274,7 @@ static vsa_status permute_common(const void *src, void *dst, vsa_dtype dtype, in
     const size_t tbytes = static_cast<size_t>(B) * n_heads * S * row, pbytes = static_cast<size_t>(B) * n_heads * Sp * row;
     VSA_REQUIRE(!overlaps(src, inverse ? pbytes : tbytes, dst, inverse ? tbytes : pbytes), "x and y must not overlap");
     return check_cuda(launch_permute(src, dst, esize_of(dtype), B * n_heads, D, grid.t, grid.h, grid.w, pg.t, pg.h,
-                                     pg.w, ts, choice, inverse, status_or_null(), as_stream(stream)),
+                                     pg.w, ts, choice, inverse, status_or_null(stream), as_stream(stream)),
                       inverse ? "unpermute launch" : "permute launch");
 }
 
@@ -300,7 +323,7 @@ vsa_status vsa_block_summaries_tiled(const void *x, vsa_dtype dtype, int B, int 
     VSA_REQUIRE(Sp / block <= 0x7fffffffLL && static_cast<long long>(B) * n_heads <= 65535,
                 "too many blocks or heads");
     return check_cuda(launch_summaries_tiled(x, esize_of(dtype), B * n_heads, D, grid.t, grid.h, grid.w, pg.t, pg.h,
-                                             pg.w, ts, choice, x_max, x_min, status_or_null(), as_stream(stream),
+                                             pg.w, ts, choice, x_max, x_min, status_or_null(stream), as_stream(stream),
                                              block),
                       "block_summaries_tiled launch");
 }
@@ -315,7 +338,7 @@ vsa_status vsa_block_scores(const void *q_max, const void *q_min, const void *k_
     VSA_REQUIRE(aligned4(scores), "scores must be a non-NULL 4-byte aligned device pointer");
     VSA_REQUIRE(static_cast<long long>(nb) <= 65535LL * 64, "nb too large");
     if (dtype == VSA_BF16)  // tensor cores: exact bf16 products, fp32 accumulation
-        return check_cuda(launch_scores_tc(q_max, q_min, k_max, k_min, B * n_heads, nb, D, scores, status_or_null(),
+        return check_cuda(launch_scores_tc(q_max, q_min, k_max, k_min, B * n_heads, nb, D, scores, status_or_null(stream),
                                            as_stream(stream)),
                           "block_scores launch");
     return check_cuda(launch_scores(q_max, q_min, k_max, k_min, esize_of(dtype), B * n_heads, nb, D, scores,
@@ -437,7 +460,7 @@ vsa_status vsa_head_profile(const void *q, const void *k, int B, int n_heads, in
     VSA_REQUIRE(workspace_bytes >= need, "workspace holds %zu bytes, %zu needed", workspace_bytes, need);
     const float sc = scale > 0.f ? scale : 1.0f / sqrtf(static_cast<float>(D));
     return check_cuda(launch_head_profile(q, k, B * n_heads, S, D, grid.h * grid.w, rows, R, sc, workspace, masses,
-                                          kind, status_or_null(), as_stream(stream)),
+                                          kind, status_or_null(stream), as_stream(stream)),
                       "head_profile launch");
 }
 
@@ -475,7 +498,7 @@ vsa_status vsa_block_sparse_attention(const void *q, const void *k, const void *
     L.idx = idx; L.cnt = cnt; L.cap = cap; L.list_per_head = list_per_head ? 1 : 0;
     L.group = group_size; L.nb = S / block;
     L.scale = scale > 0.f ? scale : 1.0f / sqrtf(static_cast<float>(D));
-    return launch_attention(L, status_or_null(), as_stream(stream));
+    return launch_attention(L, status_or_null(stream), as_stream(stream));
 }
 
 vsa_status vsa_block_sparse_attention_tiled(const void *q, const void *k, const void *v, void *o,
@@ -527,7 +550,7 @@ vsa_status vsa_block_sparse_attention_tiled(const void *q, const void *k, const 
     L.Tp = pg.t; L.Hp = pg.h; L.Wp = pg.w;
     L.tiles = ts;
     L.choice = choice;
-    return launch_attention(L, status_or_null(), as_stream(stream));
+    return launch_attention(L, status_or_null(stream), as_stream(stream));
 }
 
 vsa_status vsa_window_attention(const void *q, const void *k, const void *v, void *o, vsa_dtype out_dtype, int B,
@@ -548,7 +571,7 @@ vsa_status vsa_window_attention(const void *q, const void *k, const void *v, voi
     L.half = window / 2;
     L.sink = sink;
     L.scale = scale > 0.f ? scale : 1.0f / sqrtf(static_cast<float>(D));
-    return launch_attention(L, status_or_null(), as_stream(stream));
+    return launch_attention(L, status_or_null(stream), as_stream(stream));
 }
 
 vsa_status vsa_cast_f32_to_bf16(const float *x, void *y, int64_t n, void *stream) {
@@ -561,7 +584,7 @@ vsa_status vsa_cast_f32_to_bf16(const float *x, void *y, int64_t n, void *stream
 
 vsa_status vsa_debug_wait_timeout(int64_t timeout_ns, void *stream) {
     VSA_REQUIRE(timeout_ns >= 0 && timeout_ns <= 10000000000LL, "timeout_ns must be in [0, 1e10]");
-    return check_cuda(launch_wait_timeout(static_cast<uint64_t>(timeout_ns), status_or_null(), as_stream(stream)),
+    return check_cuda(launch_wait_timeout(static_cast<uint64_t>(timeout_ns), status_or_null(stream), as_stream(stream)),
                       "wait_timeout launch");
 }
 

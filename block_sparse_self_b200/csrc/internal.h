@@ -5,6 +5,8 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include <mutex>
+
 #include "../../include/vsa.h"
 
 namespace vsa {
@@ -13,8 +15,19 @@ namespace vsa {
 vsa_status fail(vsa_status s, const char *fmt, ...);
 // Map a CUDA error to VSA_ERR_CUDA (with its message), or VSA_OK.
 vsa_status check_cuda(cudaError_t e, const char *what);
-// Device address of the status word of the current device.
-int *device_status_word();
+// Per-device cache of a __device__ symbol's address (see cached_symbol_address).
+struct SymbolCache {
+    static constexpr int kDevices = 128;
+    std::mutex mu;
+    void *addr[kDevices] = {};
+};
+// Device address of a file-scope __device__ symbol on the current device.
+// `lookup` calls cudaGetSymbolAddress in the symbol's own file.  It runs on
+// every call whose stream is not capturing; during a capture the address
+// cached by the last such call on the device is used.
+vsa_status cached_symbol_address(SymbolCache &cache, cudaStream_t st, cudaError_t (*lookup)(void **), void **out);
+// Device address of the status word of the current device (nullptr on error).
+int *device_status_word(cudaStream_t st);
 
 constexpr int kMaxTiles = 8;
 struct TileSet {
@@ -108,7 +121,7 @@ cudaError_t launch_head_profile(const void *q, const void *k, int BH, int S, int
                                 cudaStream_t st);
 
 // Address and size of the file-scope scratch array that
-// vsa_select_tiling_noalloc uses (looked up once per device).
-vsa_status select_static_scratch(float **ptr, size_t *bytes);
+// vsa_select_tiling_noalloc uses (see cached_symbol_address).
+vsa_status select_static_scratch(float **ptr, size_t *bytes, cudaStream_t st);
 
 }  // namespace vsa

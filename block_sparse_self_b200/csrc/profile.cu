@@ -348,8 +348,13 @@ __global__ void profile_finish_kernel(const float4 *__restrict__ partial, int np
             lsp += v.z * f;
         }
         const float2 t = tpart[static_cast<size_t>(bh) * 128 + r];
-        fsp = lsp / l;
-        ftp = t.y * ex2_approx(t.x - mx) / l;
+        // l is 0 only when every part of the row gave up on a wait (the
+        // status word then holds VSA_ERR_TIMEOUT): the row adds nothing
+        // rather than a NaN
+        if (l > 0.f) {
+            fsp = lsp / l;
+            ftp = t.y * ex2_approx(t.x - mx) / l;
+        }
     }
     fsp = warp_sum(fsp);
     ftp = warp_sum(ftp);

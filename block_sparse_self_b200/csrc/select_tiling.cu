@@ -366,22 +366,17 @@ namespace vsa {
 
 // Device address of g_select_scratch on the current device.  In host code the
 // array's name is only a host-side stand-in, so the address is looked up with
-// cudaGetSymbolAddress once per device (with that device current) and cached.
-vsa_status select_static_scratch(float **ptr, size_t *bytes) {
-    static std::mutex mu;
-    static float *addr[128] = {};
-    int dev = 0;
-    cudaError_t e = cudaGetDevice(&dev);
-    if (e != cudaSuccess) return check_cuda(e, "cudaGetDevice");
-    if (dev < 0 || dev >= 128) return fail(VSA_ERR_UNSUPPORTED, "device ordinal %d out of range", dev);
-    std::lock_guard<std::mutex> lock(mu);
-    if (!addr[dev]) {
-        void *p = nullptr;
-        e = cudaGetSymbolAddress(&p, g_select_scratch);
-        if (e != cudaSuccess) return check_cuda(e, "cudaGetSymbolAddress(select_tiling scratch)");
-        addr[dev] = static_cast<float *>(p);
-    }
-    *ptr = addr[dev];
+// cudaGetSymbolAddress, with the device current, by cached_symbol_address.
+namespace {
+cudaError_t select_scratch_lookup(void **p) { return cudaGetSymbolAddress(p, g_select_scratch); }
+}  // namespace
+
+vsa_status select_static_scratch(float **ptr, size_t *bytes, cudaStream_t st) {
+    static SymbolCache cache;
+    void *p = nullptr;
+    const vsa_status s = cached_symbol_address(cache, st, select_scratch_lookup, &p);
+    if (s != VSA_OK) return s;
+    *ptr = static_cast<float *>(p);
     *bytes = kStaticScratchBytes;
     return VSA_OK;
 }

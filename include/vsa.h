@@ -128,9 +128,12 @@ vsa_status vsa_select_tiling(const void *q, vsa_dtype dtype, int B, int n_heads,
  * library holds until the process exits; a request whose scratch
  * (vsa_select_tiling_workspace_size) exceeds it returns
  * VSA_ERR_INVALID_ARGUMENT without launching anything.  The call allocates
- * nothing.  The first call on a device looks the array's device address up
- * (cudaGetSymbolAddress, with that device current) and caches it; make that
- * first call before any stream capture.  All calls share the one array:
+ * nothing.  A call whose stream is not capturing looks the array's device
+ * address up (cudaGetSymbolAddress, with that device current), so a context
+ * that was torn down and created anew on the device is never handed an old
+ * address; a call whose stream is capturing uses the address that the last
+ * such call on the device found, so make one call on the device before any
+ * stream capture.  All calls share the one array:
  * every scratch entry a call reads is written earlier in the same call, so
  * nothing has to start at zero, but calls whose work overlaps on the GPU
  * (different streams, or different host threads on one device) race on it

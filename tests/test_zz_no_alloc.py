@@ -57,11 +57,15 @@ def test_noalloc_matches_the_workspace_variant_on_two_calls_in_a_row():
 
 
 def test_noalloc_rejects_requests_larger_than_its_scratch():
-    """384 (b, head) pairs x 240 regions x 3 candidates x 4 bytes > 1 MiB: the
-    call must refuse before launching anything (the pointer is never read)."""
+    """256 heads x 240 regions x 3 candidates x 8 bytes (a SICS sum and a tile
+    count each) is 1.47 MB, above the 1 MiB array: the call must refuse before
+    launching anything (the fake pointers are never read).  The shape is valid
+    for every other check, and the workspace variant would accept it."""
     arr = (Dims3 * 3)(*[Dims3(*t) for t in TILES])
+    grid = Dims3(32, 48, 80)
+    need = vsa.lib().vsa_select_tiling_workspace_size(1, 256, grid, arr, 3)
+    assert need > 1 << 20
     fake = ctypes.c_void_p(1 << 20)
-    st = vsa.lib().vsa_select_tiling_noalloc(fake, vsa.BF16, 16, 24, 122880, 128, Dims3(32, 48, 80), arr, 3,
-                                             fake, None, None)
+    st = vsa.lib().vsa_select_tiling_noalloc(fake, vsa.BF16, 1, 256, 122880, 64, grid, arr, 3, fake, None, None)
     assert st == vsa.ERR_INVALID_ARGUMENT
     assert "at most" in vsa.last_error()
