@@ -14,6 +14,11 @@ Two value distributions are provided:
 * ``integer_grid`` -- i.i.d. values from {-4, ..., 4} / 4.  Every value is
   exact in bf16 and every product and short sum of them is exact in fp32, so
   block scores are exact and index outputs can be compared bit for bit.
+* ``quantized_smooth_qkv`` -- the smooth fields below rounded onto that same
+  {-4..4}/4 grid (per head, about two grid steps per standard deviation,
+  clipped): exact scores like ``integer_grid``, but with the spatial or
+  temporal cohesion of the smooth fields, so tiling choices have clear
+  margins.
 * ``smooth_qkv`` -- Q and K are smooth 3-D random fields over (t, h, w): per
   head 16 random low-frequency plane waves, mixed per channel with random
   amplitude and phase, plus N(0, 0.5^2) noise, then scaled per head so that
@@ -46,7 +51,7 @@ class Workload:
     grid: Dims3
     D: int
     dtype: torch.dtype
-    values: str                       # "integer" or "smooth" / "smooth_adaptive"
+    values: str                       # "integer", "smooth" or "smooth_adaptive" ("integer_adaptive" on request)
     seed_base: int
     tiles: Tuple[Dims3, ...] = ()
     block: int = 128
@@ -207,6 +212,24 @@ def smooth_qkv(B: int, heads: int, grid: Dims3, D: int, seed: int,
     return q, k, v
 
 
+def quantized_smooth_qkv(B: int, heads: int, grid: Dims3, D: int, seed: int,
+                         kinds: Optional[Sequence[str]] = None, dtype=torch.bfloat16,
+                         device="cpu", steps_per_std: float = 2.0):
+    """smooth_qkv's Q and K rounded onto the {-4..4}/4 grid (per (b, head):
+    x / std(x) * steps_per_std, rounded, clipped to [-4, 4], divided by 4),
+    and i.i.d. integer-grid V.  Every value is exact in bf16."""
+    q, k, _ = smooth_qkv(B, heads, grid, D, seed, kinds=kinds, dtype=torch.float32, device=device)
+
+    def grid_values(x):
+        sd = x.flatten(2).std(dim=-1).clamp_min(1e-12)[..., None, None]
+        # + 0.0 turns the -0.0 that rounding small negatives gives into +0.0
+        return (torch.round(x / sd * steps_per_std).clamp(-4, 4) / 4.0 + 0.0).to(dtype)
+
+    S = grid[0] * grid[1] * grid[2]
+    v = integer_grid((B, heads, S, D), seed + 2, dtype, device)
+    return grid_values(q), grid_values(k), v
+
+
 def make_qkv(workload: Workload, device="cpu", values: Optional[str] = None,
              B: Optional[int] = None, heads: Optional[int] = None):
     """Q, K, V for a workload (optionally overriding value kind or sizes)."""
@@ -218,9 +241,12 @@ def make_qkv(workload: Workload, device="cpu", values: Optional[str] = None,
         s = workload.seed_base
         return tuple(integer_grid(shape, s + o, workload.dtype, device)
                      for o in (0, 1, 2))
-    kinds = head_kinds(workload) if values == "smooth_adaptive" else None
+    kinds = head_kinds(workload) if values in ("smooth_adaptive", "integer_adaptive") else None
     if kinds is not None:
         kinds = kinds[: B * heads] + ["generic"] * max(0, B * heads - len(kinds))
+    if values == "integer_adaptive":
+        return quantized_smooth_qkv(B, heads, workload.grid, workload.D, workload.seed_base,
+                                    kinds=kinds, dtype=workload.dtype, device=device)
     return smooth_qkv(B, heads, workload.grid, workload.D, workload.seed_base,
                       kinds=kinds, dtype=workload.dtype, device=device)
 
