@@ -68,6 +68,10 @@ def lib() -> ctypes.CDLL:
         "vsa_window_attention": ([P, P, P, P, I, I, I, I, I, I, I, F, I, P], I),
         "vsa_head_profile_workspace_size": ([I, I, I, I], SZ),
         "vsa_head_profile": ([P, P, I, I, I, I, D3, P, I, F, P, P, P, SZ, P], I),
+        "vsa_centroid_compensated_attention_workspace_size": ([I, I, I, I, I], SZ),
+        "vsa_centroid_compensated_attention": ([P, P, P, P, I, I, I, I, I, I, P, P, I, I, F, P, SZ, P], I),
+        "vsa_spade_attention_host_workspace_size": ([I, I, I, I, D3, P, I, I, I, I, I, I], SZ),
+        "vsa_spade_attention_host": ([P, P, P, P, I, I, I, I, I, D3, P, I, I, I, I, F, I, P, SZ, P], I),
         "vsa_cast_f32_to_bf16": ([P, P, I64, P], I),
         "vsa_debug_wait_timeout": ([I64, P], I),
     }
@@ -420,6 +424,34 @@ def block_sparse_attention(q, k, v, idx, cnt, block: int, group_size: int = 0, s
     return o
 
 
+def centroid_compensated_attention(q, k, v, idx, cnt, block: int = 128, scale: Optional[float] = None,
+                                   out_dtype=None) -> torch.Tensor:
+    """Block-sparse attention (tile-contiguous order, 128-token blocks) in which
+    every key block a query block's list skips still takes part, as one key:
+    the block's mean key, with its mean value, weighted by its key count (see
+    include/vsa.h for the reading of the pages' call)."""
+    B, H, S, D = _bhsd(q, "q")
+    if tuple(k.shape) != (B, H, S, D) or tuple(v.shape) != (B, H, S, D):
+        raise ValueError(f"q/k/v shapes must match exactly; got q={tuple(q.shape)}, k={tuple(k.shape)}, "
+                         f"v={tuple(v.shape)}")
+    odt = _out_dtype(out_dtype, q)
+    qb, kb, vb = _bf16(q, "q"), _bf16(k, "k"), _bf16(v, "v")
+    _cuda(idx, "idx")
+    _cuda(cnt, "cnt")
+    if idx.dtype != torch.int32 or cnt.dtype != torch.int32:
+        raise ValueError("idx and cnt must be int32")
+    oc = BF16 if odt == torch.bfloat16 else F32
+    need = lib().vsa_centroid_compensated_attention_workspace_size(B, H, S, D, oc)
+    if need == 0:
+        raise ValueError(f"no workspace size for B={B}, H={H}, S={S}, D={D} (S must be a multiple of 128, D 64 or 128)")
+    ws = torch.empty(need, dtype=torch.uint8, device=q.device)
+    o = torch.empty(B, H, S, D, dtype=odt, device=q.device)
+    _check(lib().vsa_centroid_compensated_attention(
+        _ptr(qb), _ptr(kb), _ptr(vb), _ptr(o), oc, B, H, S, D, int(block), _ptr(idx), _ptr(cnt), int(idx.shape[-1]),
+        1 if idx.dim() == 4 else 0, 0.0 if scale is None else float(scale), _ptr(ws), need, _stream(q.device)))
+    return o
+
+
 def block_sparse_attention_tiled(q, k, v, grid, tiles, choice, idx, cnt, scale: Optional[float] = None,
                                  out_dtype=None, group_stride: int = 0) -> torch.Tensor:
     """unpermute(block_sparse_attention(permute(q), permute(k), permute(v), idx, cnt, block)) in one
@@ -571,58 +603,48 @@ def spade_attention(q, k, v, grid, tiles, budget: Optional[float] = None, topk: 
 
 
 def spade_attention_host(q, k, v, grid, tiles, out: Optional[torch.Tensor] = None, chunks: int = 8,
-                         device=None, **kwargs) -> torch.Tensor:
-    """spade_attention for inputs and output in (pinned) host memory.
-
-    The B*H (batch, head) rows are taken in `chunks` groups.  Each group's
-    copy to the device, its attention and the copy of its output back run on
-    separate streams, so the copies of one group overlap the kernels of
-    another.  Every (batch, head) is independent of the others, so the result
-    equals spade_attention on the whole batch.  Returns `out` (allocated
-    pinned when not given) once the last copy back has finished.  Keyword
-    arguments go to spade_attention (budget, topk, n_sink_blocks, ...).
-    """
+                         device=None, budget: Optional[float] = None, topk: Optional[int] = None,
+                         n_sink_blocks: int = 1, diag_halfwidth: int = 0, scale: Optional[float] = None,
+                         out_dtype=None) -> torch.Tensor:
+    """spade_attention for bf16 inputs and an output in (pinned) host memory,
+    through vsa_spade_attention_host: the B*H (batch, head) rows are taken in
+    `chunks` groups whose copies to the device and back overlap the kernels
+    of other groups (see include/vsa.h).  Allocates the device workspace and
+    `out` (pinned) when not given, and returns `out` once the call's stream
+    has finished with it."""
     for t, nm in ((q, "q"), (k, "k"), (v, "v")):
         if not isinstance(t, torch.Tensor) or t.is_cuda or not t.is_contiguous():
             raise ValueError(f"{nm} must be a contiguous host tensor")
+        if t.dtype != torch.bfloat16:
+            raise ValueError(f"{nm} must be bfloat16")
     B, H, S, D = _bhsd(q, "q")
     if tuple(k.shape) != (B, H, S, D) or tuple(v.shape) != (B, H, S, D):
         raise ValueError("q/k/v shapes must match exactly")
-    odt = _out_dtype(kwargs.get("out_dtype"), q)
+    odt = _out_dtype(out_dtype, q)
     if out is None:
         out = torch.empty(q.shape, dtype=odt, pin_memory=True)
     elif out.shape != q.shape or out.dtype != odt or out.is_cuda or not out.is_contiguous():
         raise ValueError("out must be a contiguous host tensor of q's shape and the output dtype")
+    tiles = [tuple(t) for t in tiles]
+    block = min(128, tiles[0][0] * tiles[0][1] * tiles[0][2])
+    nb = _grid_tokens(padded_grid(grid, tiles)) // block
+    kk = topk if topk is not None else topk_budget(nb, budget if budget is not None else 0.17)
     dev = torch.device("cuda", torch.cuda.current_device()) if device is None else torch.device(device)
-    BH = B * H
-    n_chunks = max(1, min(int(chunks), BH))
-    bounds = [(BH * g // n_chunks, BH * (g + 1) // n_chunks) for g in range(n_chunks)]
-    rows = max(b - a for a, b in bounds)
-    flat = [x.view(BH, S, D) for x in (q, k, v)]
-    oflat = out.view(BH, S, D)
-    comp = torch.cuda.current_stream(dev)
-    h2d, d2h = torch.cuda.Stream(dev), torch.cuda.Stream(dev)
-    slots = [[torch.empty(rows, S, D, dtype=q.dtype, device=dev) for _ in range(3)] for _ in range(2)]
-    used = [None, None]  # per slot: event after the attention that last read it
-    for g, (a, b) in enumerate(bounds):
-        n, slot = b - a, g % 2
-        with torch.cuda.stream(h2d):
-            if used[slot] is not None:
-                h2d.wait_event(used[slot])
-            for src, dst in zip(flat, slots[slot]):
-                dst[:n].copy_(src[a:b], non_blocking=True)
-            ready = h2d.record_event()
-        comp.wait_event(ready)
-        qd, kd, vd = (x[:n].view(1, n, S, D) for x in slots[slot])
-        o = spade_attention(qd, kd, vd, grid, tiles, **kwargs)
-        used[slot] = comp.record_event()
-        with torch.cuda.stream(d2h):
-            d2h.wait_event(used[slot])
-            oflat[a:b].copy_(o.view(n, S, D), non_blocking=True)
-            o.record_stream(d2h)
-    for x in slots[0] + slots[1]:
-        x.record_stream(comp)
-    d2h.synchronize()
+    arr, n = _tiles_arg(tiles)
+    g = Dims3(*grid)
+    oc = BF16 if odt == torch.bfloat16 else F32
+    need = lib().vsa_spade_attention_host_workspace_size(B, H, S, D, g, arr, n, int(kk), int(n_sink_blocks),
+                                                         int(diag_halfwidth), oc, int(chunks))
+    if need == 0:
+        raise ValueError(f"no valid workspace size for these arguments ({last_error() or 'check the shapes'})")
+    ws = torch.empty(need, dtype=torch.uint8, device=dev)
+    with torch.cuda.device(dev):
+        st = torch.cuda.current_stream(dev)
+        _check(lib().vsa_spade_attention_host(_ptr(q), _ptr(k), _ptr(v), _ptr(out), oc, B, H, S, D, g, arr, n,
+                                              int(kk), int(n_sink_blocks), int(diag_halfwidth),
+                                              0.0 if scale is None else float(scale), int(chunks), _ptr(ws), need,
+                                              ctypes.c_void_p(st.cuda_stream)))
+        st.synchronize()
     return out
 
 

@@ -301,6 +301,42 @@ vsa_status vsa_block_sparse_attention(const void *q, const void *k, const void *
                                       const int32_t *cnt, int cap, int list_per_head,
                                       int group_size, float scale, void *stream);
 
+/* Block-sparse attention with centroid compensation.  "Adaptive tiling
+ * (SPADE)", Recipe: the attention call centroid_compensated_attention(q, k,
+ * v, q_labels, k_labels, block_mask), with dropping the skipped blocks named
+ * as the alternative in its recipe note.  The pages give the call and its
+ * arguments only; the reading taken here: query i attends exactly to the
+ * keys of the blocks its list names, and every other key block b (n_b keys)
+ * takes part as one key, the mean kbar_b of its keys, with value the mean
+ * vbar_b of its values and weight n_b:
+ *   o_i = (sum_kept e^{s(q_i,k_t)} v_t + sum_skipped n_b e^{s(q_i,kbar_b)} vbar_b)
+ *       / (sum_kept e^{s(q_i,k_t)}     + sum_skipped n_b e^{s(q_i,kbar_b)}),
+ * s(q, k) = scale q . k.  Blocks are those of the tile-contiguous order
+ * (labels = position / block), so a block whose keys are all equal
+ * contributes exactly what it would if kept.
+ *   q, k, v  [B, n_heads, S, D] bf16 (tile-contiguous order); o in out_dtype
+ *   idx/cnt  block lists as for vsa_block_sparse_attention (list_per_head)
+ *   block    128 (S % 128 == 0); at most 8192 blocks per head
+ *   workspace DEVICE scratch of vsa_centroid_compensated_attention_workspace_size
+ *            bytes, 256-byte aligned, not overlapping o: the centroids (as
+ *            bf16 pairs hi + lo, about 16 significant bits), each row's
+ *            softmax state over its kept keys and, for a bf16 output, the
+ *            fp32 output of the kept keys
+ * The kept keys run on the block-sparse attention kernel; a second tcgen05
+ * pass attends each query tile to the centroids its list skips and merges
+ * the two softmaxes exactly.  Lists are checked as for
+ * vsa_block_sparse_attention (rows of an invalid list are written as zeros,
+ * VSA_ERR_RUNTIME).  A bf16 output is the fp32 result rounded once.  D in
+ * {64, 128}.                                                               */
+size_t vsa_centroid_compensated_attention_workspace_size(int B, int n_heads, int S, int D,
+                                                         vsa_dtype out_dtype);
+vsa_status vsa_centroid_compensated_attention(const void *q, const void *k, const void *v, void *o,
+                                              vsa_dtype out_dtype, int B, int n_heads, int S,
+                                              int D, int block, const int32_t *idx,
+                                              const int32_t *cnt, int cap, int list_per_head,
+                                              float scale, void *workspace, size_t workspace_bytes,
+                                              void *stream);
+
 /* Block-sparse attention on T-major q, k, v and o, with each (b, head) in its
  * own tiling and no permuted copies ("Adaptive tiling (SPADE)", Recipe: the
  * permutation, attention and inverse permutation in one pass).  Block i of
@@ -387,6 +423,49 @@ vsa_status vsa_head_profile(const void *q, const void *k, int B, int n_heads, in
                             vsa_dims3 grid, const int32_t *rows, int R, float scale,
                             float *masses, int32_t *kind, void *workspace,
                             size_t workspace_bytes, void *stream);
+
+/* ------------------------------------------------------------------------ */
+/* The whole SPADE path for Q, K, V and O in HOST memory.  "Adaptive tiling
+ * (SPADE)", Recipe: per (b, head) the tiling choice (skipped with one
+ * candidate), the tile-contiguous order, the min/max block scores, the top-k
+ * lists with the sink and diagonal blocks, block-sparse attention and the
+ * return to T-major order -- the composition of vsa_select_tiling,
+ * vsa_block_summaries_tiled, vsa_block_scores, vsa_topk_block_mask and
+ * vsa_block_sparse_attention_tiled, whose result it equals bit for bit.
+ *
+ * The (b, head) rows are taken in `groups` groups (at most B*n_heads).  Each
+ * group's Q, K, V are copied into the workspace, its steps run on `stream`,
+ * and its O is copied back, with the copies on two streams of the call's own:
+ * the copies of one group overlap the kernels of another.  Host buffers
+ * should be page-locked (cudaHostAlloc / cudaHostRegister); pageable memory
+ * works but its copies do not overlap.
+ *   q, k, v  HOST [B, n_heads, S, D] bf16, T-major over grid (S = T*Hg*Wg)
+ *   o        HOST [B, n_heads, S, D] in out_dtype (VSA_BF16 or VSA_F32)
+ *   tiles    HOST array of n_tiles (1..8) candidate tiles of one volume V:
+ *            32 or 64 (a block is the tile) or a multiple of 128 whose blocks
+ *            are whole (h, w) planes (the conditions of
+ *            vsa_block_sparse_attention_tiled); grids the tiles do not divide
+ *            are padded as vsa_padded_grid says
+ *   topk     k key blocks per query block, 1 <= k <= nb (nb = padded tokens
+ *            / block); n_sink_blocks, diag_halfwidth as for
+ *            vsa_topk_block_mask; scale <= 0 selects 1/sqrt(D)
+ *   workspace DEVICE scratch of vsa_spade_attention_host_workspace_size(...)
+ *            bytes (same arguments), 256-byte aligned, owned by the caller
+ * The call enqueues its work and returns: `stream` reaches the end of the
+ * call once every copy into o has landed, so synchronise `stream` before
+ * reading o, and do not reuse the workspace on another stream before then.
+ * Argument errors return before any copy is issued; an error that a device
+ * step reports for a group stops the call there (earlier groups' copies
+ * have been issued) and is returned.  D in {64, 128}.                      */
+size_t vsa_spade_attention_host_workspace_size(int B, int n_heads, int S, int D, vsa_dims3 grid,
+                                               const vsa_dims3 *tiles, int n_tiles, int topk,
+                                               int n_sink_blocks, int diag_halfwidth,
+                                               vsa_dtype out_dtype, int groups);
+vsa_status vsa_spade_attention_host(const void *q, const void *k, const void *v, void *o,
+                                    vsa_dtype out_dtype, int B, int n_heads, int S, int D,
+                                    vsa_dims3 grid, const vsa_dims3 *tiles, int n_tiles, int topk,
+                                    int n_sink_blocks, int diag_halfwidth, float scale, int groups,
+                                    void *workspace, size_t workspace_bytes, void *stream);
 
 /* ------------------------------------------------------------------------ */
 /* Round-to-nearest-even fp32 -> bf16 conversion of n elements (x, y device).

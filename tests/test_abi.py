@@ -213,3 +213,67 @@ def test_head_profile_and_centred_kind_reject_bad_host_arguments():
     with pytest.raises(ValueError):
         vsa.structured_block_list("sliding_tile_centred", (8, 16, 16), 128)   # the kind is spelt "centered"
     assert vsa.structured_tile("sliding_tile_centered", (8, 16, 16), (2, 8, 8)) == (2, 8, 8)
+
+
+def test_spade_attention_host_argument_errors(L):
+    """The host-buffer path refuses bad arguments before creating a stream or
+    issuing a copy (the host pointers here are never read)."""
+    arr, n = _tiles((1, 8, 16), (2, 8, 8), (4, 4, 8))
+    g = Dims3(8, 16, 32)
+
+    def size(**kw):
+        a = dict(B=1, H=3, S=4096, D=128, k=4, sink=1, dw=0, out=vsa.BF16, groups=2)
+        a.update(kw)
+        return L.vsa_spade_attention_host_workspace_size(a["B"], a["H"], a["S"], a["D"], g, arr, n, a["k"],
+                                                         a["sink"], a["dw"], a["out"], a["groups"])
+
+    need = size()
+    assert need > 3 * 2 * 2 * 4096 * 128 * 2   # two slots of q, k, v and the output slots
+    assert size(groups=0) == 0 and size(k=33) == 0 and size(k=0) == 0
+
+    def call(**kw):
+        a = dict(q=FAKE, k=FAKE, v=FAKE, o=FAKE, out=vsa.BF16, B=1, H=3, S=4096, D=128, topk=4, sink=1, dw=0,
+                 scale=0.0, groups=2, ws=ctypes.c_void_p(1 << 20), wsb=need)
+        a.update(kw)
+        return L.vsa_spade_attention_host(a["q"], a["k"], a["v"], a["o"], a["out"], a["B"], a["H"], a["S"], a["D"],
+                                          g, arr, n, a["topk"], a["sink"], a["dw"], a["scale"], a["groups"], a["ws"],
+                                          a["wsb"], NULL)
+    assert call(q=NULL) == vsa.ERR_INVALID_ARGUMENT
+    assert call(out=5) == vsa.ERR_INVALID_ARGUMENT
+    assert call(topk=33) == vsa.ERR_INVALID_ARGUMENT
+    assert "k must be in [1, nb]" in vsa.last_error()
+    assert call(groups=0) == vsa.ERR_INVALID_ARGUMENT
+    assert call(wsb=need - 1) == vsa.ERR_INVALID_ARGUMENT
+    assert "needed" in vsa.last_error()
+    assert call(ws=ctypes.c_void_p((1 << 20) + 16)) == vsa.ERR_INVALID_ARGUMENT
+    assert call(S=4095) == vsa.ERR_INVALID_ARGUMENT
+    assert call(sink=-1) == vsa.ERR_INVALID_ARGUMENT
+    assert call(dw=-2) == vsa.ERR_INVALID_ARGUMENT
+    assert call(scale=float("inf")) == vsa.ERR_INVALID_ARGUMENT
+    assert call(D=96, wsb=1 << 40) == vsa.ERR_UNSUPPORTED
+
+
+def test_compensated_attention_argument_errors(L):
+    def call(**kw):
+        a = dict(q=FAKE, k=ctypes.c_void_p(0x100000), v=ctypes.c_void_p(0x200000), o=ctypes.c_void_p(0x400000),
+                 out=vsa.F32, B=1, H=2, S=512, D=64, block=128, cap=2, per_head=1, scale=0.0,
+                 ws=ctypes.c_void_p(1 << 24), wsb=None)
+        a.update(kw)
+        wsb = a["wsb"] if a["wsb"] is not None else L.vsa_centroid_compensated_attention_workspace_size(
+            a["B"], a["H"], max(a["S"], 128), a["D"] if a["D"] in (64, 128) else 64, a["out"] if a["out"] in (0, 1) else 1)
+        return L.vsa_centroid_compensated_attention(a["q"], a["k"], a["v"], a["o"], a["out"], a["B"], a["H"], a["S"],
+                                                    a["D"], a["block"], FAKE, FAKE, a["cap"], a["per_head"],
+                                                    a["scale"], a["ws"], wsb, NULL)
+    f32 = L.vsa_centroid_compensated_attention_workspace_size(1, 2, 512, 64, vsa.F32)
+    bf = L.vsa_centroid_compensated_attention_workspace_size(1, 2, 512, 64, vsa.BF16)
+    assert bf >= f32 + 2 * 512 * 64 * 4          # a bf16 output also holds the kept keys' fp32 output
+    assert L.vsa_centroid_compensated_attention_workspace_size(1, 2, 500, 64, vsa.F32) == 0
+    assert call(block=64) == vsa.ERR_UNSUPPORTED
+    assert call(S=500) == vsa.ERR_INVALID_ARGUMENT
+    assert call(cap=0) == vsa.ERR_INVALID_ARGUMENT
+    assert call(D=96) == vsa.ERR_UNSUPPORTED
+    assert call(wsb=f32 - 1) == vsa.ERR_INVALID_ARGUMENT
+    assert "needed" in vsa.last_error()
+    assert call(ws=ctypes.c_void_p((1 << 24) + 16)) == vsa.ERR_INVALID_ARGUMENT
+    assert call(ws=ctypes.c_void_p(0x400000)) == vsa.ERR_INVALID_ARGUMENT  # workspace over o
+    assert call(o=FAKE) == vsa.ERR_INVALID_ARGUMENT                        # o over q
