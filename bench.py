@@ -489,6 +489,39 @@ def extra_workloads(steps: int):
     return out
 
 
+def compensated_line(w, q, k, v, idx, cnt, n_rep: int):
+    """Centroid-compensated attention against the plain block-sparse attention
+    on the same permuted inputs and lists.  Algorithmic FLOPs: 4 * 128 * 128 * D
+    per listed block pair plus 4 * 128 * D per (query block, skipped block)
+    centroid."""
+    import block_sparse_self_b200 as vsa
+    choice = vsa.select_tiling(q, w.grid, list(w.tiles))
+    qp, kp, vp = (vsa.permute(x, w.grid, list(w.tiles), choice) for x in (q, k, v))
+
+    def timed(fn):
+        for _ in range(3):
+            fn()
+        torch.cuda.synchronize()
+        s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        s.record()
+        for _ in range(n_rep):
+            fn()
+        e.record()
+        torch.cuda.synchronize()
+        return s.elapsed_time(e) / n_rep
+
+    comp_ms = timed(lambda: vsa.centroid_compensated_attention(qp, kp, vp, idx, cnt))
+    plain_ms = timed(lambda: vsa.block_sparse_attention(qp, kp, vp, idx, cnt, 128))
+    pairs = float(cnt.to(torch.int64).sum().item())
+    BH, nb = w.B * w.heads, w.nb
+    skipped = BH * nb * nb - pairs
+    flops = pairs * 4.0 * 128 * 128 * w.D + skipped * 4.0 * 128 * w.D
+    del qp, kp, vp
+    return {"ms_per_call": comp_ms, "tflops": flops / comp_ms / 1e9, "plain_attention_ms": plain_ms,
+            "compensation_overhead": comp_ms / plain_ms - 1.0, "skipped_blocks_per_row": skipped / (BH * nb),
+            "out_dtype": "bf16", "layout": "permuted copies in each head's chosen tiling"}
+
+
 def run_ours(args, w):
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
@@ -558,6 +591,11 @@ def run_ours(args, w):
             extra["explicit_permute_" + w.name] = {"ms_per_step": ex_ms, "phase_ms": ex.phase_ms(),
                                                    "same_output": bool(torch.equal(ex.last["o"], step.last["o"]))}
             del ex
+        # centroid-compensated attention on the same lists: the kept blocks as
+        # above plus every skipped block as its centroid (explicit permuted
+        # copies in each head's tiling; bf16 output)
+        extra["compensated_" + w.name] = compensated_line(w, q, k, v, step.last["idx"], step.last["cnt"],
+                                                          max(3, args.steps // 2))
         # top-p (mass budget) lists on the same scores, in place of the top-k lists
         import block_sparse_self_b200 as vsa
         sc = step.last["scores"]

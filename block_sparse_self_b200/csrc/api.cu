@@ -553,6 +553,40 @@ vsa_status vsa_block_sparse_attention_tiled(const void *q, const void *k, const 
     return launch_attention(L, status_or_null(stream), as_stream(stream));
 }
 
+size_t vsa_centroid_compensated_attention_workspace_size(int B, int n_heads, int S, int D, vsa_dtype out_dtype) {
+    if (B < 1 || n_heads < 1 || S < 128 || S % 128 != 0 || (D != 64 && D != 128)) return 0;
+    if (out_dtype != VSA_BF16 && out_dtype != VSA_F32) return 0;
+    return compensated_workspace_bytes(B * n_heads, S, D, out_dtype == VSA_F32);
+}
+
+vsa_status vsa_centroid_compensated_attention(const void *q, const void *k, const void *v, void *o,
+                                              vsa_dtype out_dtype, int B, int n_heads, int S, int D, int block,
+                                              const int32_t *idx, const int32_t *cnt, int cap, int list_per_head,
+                                              float scale, void *workspace, size_t workspace_bytes, void *stream) {
+    VSA_TRY(check_attention_common(q, k, v, o, out_dtype, B, n_heads, S, D, scale));
+    if (block != 128) return fail(VSA_ERR_UNSUPPORTED, "compensated attention takes 128-token blocks, got %d", block);
+    VSA_REQUIRE(S % block == 0, "block (%d) must divide S (%d)", block, S);
+    VSA_REQUIRE(aligned4(idx) && aligned4(cnt), "idx and cnt must be non-NULL 4-byte aligned device pointers");
+    VSA_REQUIRE(cap >= 1, "cap must be >= 1, got %d", cap);
+    if (S / block > 8192) return fail(VSA_ERR_UNSUPPORTED, "compensated attention supports at most 8192 blocks per head");
+    const size_t need = vsa_centroid_compensated_attention_workspace_size(B, n_heads, S, D, out_dtype);
+    VSA_REQUIRE(workspace != nullptr && (reinterpret_cast<uintptr_t>(workspace) & 255u) == 0,
+                "workspace must be a non-NULL 256-byte aligned device pointer");
+    VSA_REQUIRE(workspace_bytes >= need, "workspace holds %zu bytes, %zu needed", workspace_bytes, need);
+    VSA_REQUIRE(!overlaps(workspace, need, o, static_cast<size_t>(B) * n_heads * S * D * esize_of(out_dtype)),
+                "workspace must not overlap o");
+    AttnLaunch L{};
+    L.q = q; L.k = k; L.v = v; L.o = o;
+    L.out_f32 = out_dtype == VSA_F32;
+    L.BH = B * n_heads; L.S = S; L.D = D;
+    L.block = block;
+    L.window = false;
+    L.idx = idx; L.cnt = cnt; L.cap = cap; L.list_per_head = list_per_head ? 1 : 0;
+    L.group = 0; L.nb = S / block;
+    L.scale = scale > 0.f ? scale : 1.0f / sqrtf(static_cast<float>(D));
+    return launch_compensated(L, workspace, status_or_null(stream), as_stream(stream));
+}
+
 vsa_status vsa_window_attention(const void *q, const void *k, const void *v, void *o, vsa_dtype out_dtype, int B,
                                 int n_heads, int S, int D, int window, int sink, float scale, int chunk,
                                 void *stream) {

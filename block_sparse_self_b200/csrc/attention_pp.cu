@@ -51,6 +51,7 @@ struct PPArgs {
     float scale_log2;
     void *out;
     int out_f32;
+    float2 *stats;  // optional per-row (m, l), see AttnLaunch
     int *status;
     // tiled mode: T-major tensors, per-head tiling (all of volume 128 * m)
     int H, W;         // the padded grid's frame (equal to the real one when nothing is padded)
@@ -602,7 +603,9 @@ attn_pp_kernel(const __grid_constant__ MapSet maps, const PPArgs a) {
                 }
             }
             if (row_valid && l_sum <= 0.f) report(a.status, DEV_RUNTIME);
+            if (a.stats && row_valid) a.stats[static_cast<size_t>(bh) * a.S + rg] = make_float2(m_ref, l_sum);
         } else if (row_valid && bad[t]) {
+            if (a.stats) a.stats[static_cast<size_t>(bh) * a.S + rg] = make_float2(-INFINITY, 0.f);
             if (a.out_f32) {
                 float4 *dst = reinterpret_cast<float4 *>(static_cast<float *>(a.out) + orow * D);
                 for (int e = 0; e < D / 4; ++e) dst[e] = make_float4(0.f, 0.f, 0.f, 0.f);
@@ -661,6 +664,7 @@ vsa_status run_pp(const AttnLaunch &L, int *status, cudaStream_t st) {
     a.scale_log2 = L.scale * 1.4426950408889634f;
     a.out = L.o;
     a.out_f32 = L.out_f32;
+    a.stats = L.stats;
     a.status = status;
     a.H = TILED ? L.Hp : L.Hg;
     a.W = TILED ? L.Wp : L.Wg;
@@ -1146,7 +1150,9 @@ attn_one_kernel(const __grid_constant__ MapSet maps, const PPArgs a) {
                 }
             }
             if (row_valid && l_sum <= 0.f) report(a.status, DEV_RUNTIME);
+            if (a.stats && row_valid) a.stats[static_cast<size_t>(bh) * a.S + rg] = make_float2(m_ref, l_sum);
         } else if (row_valid && bad) {
+            if (a.stats) a.stats[static_cast<size_t>(bh) * a.S + rg] = make_float2(-INFINITY, 0.f);
             if (a.out_f32) {
                 float4 *dst = reinterpret_cast<float4 *>(static_cast<float *>(a.out) + orow * D);
                 for (int e = 0; e < D / 4; ++e) dst[e] = make_float4(0.f, 0.f, 0.f, 0.f);
@@ -1209,6 +1215,7 @@ vsa_status run_one(const AttnLaunch &L, int *status, cudaStream_t st) {
     a.scale_log2 = L.scale * 1.4426950408889634f;
     a.out = L.o;
     a.out_f32 = L.out_f32;
+    a.stats = L.stats;
     a.status = status;
     a.H = TILED ? L.Hp : L.Hg;
     a.W = TILED ? L.Wp : L.Wg;

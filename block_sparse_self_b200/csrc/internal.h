@@ -96,6 +96,10 @@ struct AttnLaunch {
     int Tp, Hp, Wp;     // tiled mode: the padded grid the tiles cut (block lists over its positions)
     TileSet tiles;
     const int32_t *choice;
+    // optional: per row (position p of head bh at stats[bh * positions + p])
+    // the softmax state behind the normalised output, in the log2 domain:
+    // (m, l) with l = sum over the visible keys of 2^(scale log2e q.k - m)
+    float2 *stats;
 };
 vsa_status launch_attention(const AttnLaunch &a, int *status, cudaStream_t st);
 // Two query tiles per CTA (128-token blocks only); launch_attention routes to it.
@@ -119,6 +123,10 @@ size_t profile_workspace_bytes(int BH, int S, int D);
 cudaError_t launch_head_profile(const void *q, const void *k, int BH, int S, int D, int HW, const int32_t *rows,
                                 int R, float scale, void *workspace, float *masses, int32_t *kind, int *status,
                                 cudaStream_t st);
+
+// Skipped key blocks compensated by their centroids (compensated.cu).
+size_t compensated_workspace_bytes(int BH, int S, int D, int out_f32);
+vsa_status launch_compensated(const AttnLaunch &a, void *workspace, int *status, cudaStream_t st);
 
 // Address and size of the file-scope scratch array that
 // vsa_select_tiling_noalloc uses (see cached_symbol_address).
