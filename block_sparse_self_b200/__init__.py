@@ -61,6 +61,7 @@ def lib() -> ctypes.CDLL:
         "vsa_block_summaries_tiled": ([P, I, I, I, I, I, D3, P, I, P, I, P, P, P], I),
         "vsa_block_scores": ([P, P, P, P, I, I, I, I, I, P, P], I),
         "vsa_topk_block_mask": ([P, I, I, I, I, I, I, P, P, I, P], I),
+        "vsa_block_scores_topk": ([P, P, P, P, I, I, I, I, I, I, I, I, P, P, I, P], I),
         "vsa_topp_block_mask": ([P, I, I, I, F, F, I, I, P, P, I, P], I),
         "vsa_structured_block_list": ([I, D3, D3, D3, I, P, P, I, P, P], I),
         "vsa_block_sparse_attention": ([P, P, P, P, I, I, I, I, I, I, P, P, I, I, I, F, P], I),
@@ -295,6 +296,24 @@ def topk_block_mask(scores: torch.Tensor, k: int, n_sink_blocks: int = 1, diag_h
     cnt = torch.empty(B, H, nb, dtype=torch.int32, device=scores.device)
     _check(lib().vsa_topk_block_mask(_ptr(scores), B, H, nb, int(k), int(n_sink_blocks), int(diag_halfwidth),
                                      _ptr(idx), _ptr(cnt), cap, _stream(scores.device)))
+    return idx, cnt
+
+
+def block_scores_topk(q_max, q_min, k_max, k_min, k: int, n_sink_blocks: int = 1, diag_halfwidth: int = 0,
+                      cap: Optional[int] = None):
+    """topk_block_mask(block_scores(q_max, q_min, k_max, k_min), k, ...) in one
+    kernel, without the score matrix: (idx [B,H,nb,cap] int32, cnt [B,H,nb] int32)."""
+    for t, nm in ((q_max, "q_max"), (q_min, "q_min"), (k_max, "k_max"), (k_min, "k_min")):
+        _cuda(t, nm)
+        if t.shape != q_max.shape or t.dtype != q_max.dtype:
+            raise ValueError("summaries must share shape and dtype")
+    B, H, nb, D = _bhsd(q_max, "q_max")
+    cap = list_cap(nb, k, n_sink_blocks, diag_halfwidth) if cap is None else int(cap)
+    idx = torch.empty(B, H, nb, max(cap, 1), dtype=torch.int32, device=q_max.device)
+    cnt = torch.empty(B, H, nb, dtype=torch.int32, device=q_max.device)
+    _check(lib().vsa_block_scores_topk(_ptr(q_max), _ptr(q_min), _ptr(k_max), _ptr(k_min),
+                                       _dtype_code(q_max, "q_max"), B, H, nb, D, int(k), int(n_sink_blocks),
+                                       int(diag_halfwidth), _ptr(idx), _ptr(cnt), cap, _stream(q_max.device)))
     return idx, cnt
 
 

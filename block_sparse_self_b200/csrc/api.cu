@@ -364,6 +364,31 @@ vsa_status vsa_topk_block_mask(const float *scores, int B, int n_heads, int nb, 
                       "topk launch");
 }
 
+vsa_status vsa_block_scores_topk(const void *q_max, const void *q_min, const void *k_max, const void *k_min,
+                                 vsa_dtype dtype, int B, int n_heads, int nb, int D, int k, int n_sink_blocks,
+                                 int diag_halfwidth, int32_t *idx, int32_t *cnt, int cap, void *stream) {
+    VSA_REQUIRE(esize_of(dtype) != 0, "dtype must be VSA_BF16 or VSA_F32");
+    VSA_TRY(check_bhsd(B, n_heads, nb, D));
+    VSA_TRY(check_d(D));
+    VSA_REQUIRE(k >= 1 && k <= nb, "k must be in [1, nb] = [1, %d], got %d", nb, k);
+    VSA_REQUIRE(n_sink_blocks >= 0 && n_sink_blocks <= nb, "n_sink_blocks must be in [0, nb], got %d",
+                n_sink_blocks);
+    VSA_REQUIRE(diag_halfwidth >= -1, "diag_halfwidth must be >= -1 (-1 = no diagonal), got %d", diag_halfwidth);
+    long long most = static_cast<long long>(k) + n_sink_blocks + (diag_halfwidth >= 0 ? 2LL * diag_halfwidth + 1 : 0);
+    if (most > nb) most = nb;
+    VSA_REQUIRE(cap >= most, "cap (%d) must be >= min(nb, k + n_sink + 2*diag_halfwidth + 1) = %lld", cap, most);
+    VSA_REQUIRE(aligned16(q_max) && aligned16(q_min) && aligned16(k_max) && aligned16(k_min),
+                "summaries must be non-NULL 16-byte aligned device pointers");
+    VSA_REQUIRE(aligned4(idx) && aligned4(cnt), "idx and cnt must be non-NULL 4-byte aligned device pointers");
+    if (dtype != VSA_BF16) return fail(VSA_ERR_UNSUPPORTED, "the fused scores and lists take bf16 summaries");
+    if (nb > scores_topk_max_blocks())
+        return fail(VSA_ERR_UNSUPPORTED, "the fused scores and lists take rows of at most %d blocks, got %d",
+                    scores_topk_max_blocks(), nb);
+    return check_cuda(launch_scores_topk(q_max, q_min, k_max, k_min, B * n_heads, nb, D, k, n_sink_blocks,
+                                         diag_halfwidth, idx, cnt, cap, status_or_null(stream), as_stream(stream)),
+                      "scores_topk launch");
+}
+
 vsa_status vsa_topp_block_mask(const float *scores, int B, int n_heads, int nb, float p, float scale,
                                int n_sink_blocks, int diag_halfwidth, int32_t *idx, int32_t *cnt, int cap,
                                void *stream) {

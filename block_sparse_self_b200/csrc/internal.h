@@ -56,6 +56,11 @@ cudaError_t launch_scores_tc(const void *qmax, const void *qmin, const void *kma
                              int D, float *scores, int *status, cudaStream_t st);
 cudaError_t launch_topk(const float *scores, int BH, int nb, int k, int n_sink, int diag_hw, int32_t *idx,
                         int32_t *cnt, int cap, cudaStream_t st);
+// Scores and top-k lists in one kernel (bf16 summaries, nb <= scores_topk_max_blocks()).
+int scores_topk_max_blocks();
+cudaError_t launch_scores_topk(const void *qmax, const void *qmin, const void *kmax, const void *kmin, int BH, int nb,
+                               int D, int k, int n_sink, int diag_hw, int32_t *idx, int32_t *cnt, int cap, int *status,
+                               cudaStream_t st);
 cudaError_t launch_topp(const float *scores, int BH, int nb, float p, float scale, int n_sink, int diag_hw,
                         int32_t *idx, int32_t *cnt, int cap, cudaStream_t st);
 cudaError_t launch_structured(int T, int H, int W, int tt, int th, int tw, int rt, int rh, int rw, bool centered,

@@ -228,6 +228,20 @@ vsa_status vsa_topk_block_mask(const float *scores, int B, int n_heads, int nb, 
                                int n_sink_blocks, int diag_halfwidth, int32_t *idx,
                                int32_t *cnt, int cap, void *stream);
 
+/* vsa_block_scores followed by vsa_topk_block_mask in one kernel: the
+ * scores of a row stay on the chip and are never written ("Adaptive tiling
+ * (SPADE)", Dense by design: its speed comes from a fused estimator).  The
+ * arguments and the lists (idx, cnt, cap) are those of the two calls; the
+ * scores are the same fp32 sums of exact bf16 products, so on
+ * small-integer-valued summaries the lists equal the two calls' bit for bit
+ * (elsewhere fp32 rounding may order near-equal scores differently).
+ * bf16 summaries only and nb <= 1024 (VSA_ERR_UNSUPPORTED otherwise); D in
+ * {64, 128}.                                                              */
+vsa_status vsa_block_scores_topk(const void *q_max, const void *q_min, const void *k_max,
+                                 const void *k_min, vsa_dtype dtype, int B, int n_heads, int nb,
+                                 int D, int k, int n_sink_blocks, int diag_halfwidth, int32_t *idx,
+                                 int32_t *cnt, int cap, void *stream);
+
 /* Top-p (mass budget) key-block lists.  "Adaptive tiling (SPADE)" names
  * top_p_block_mask among the functions its recipe composes with but does not
  * define it; this is the reading used here.  For each row (b, head, i):

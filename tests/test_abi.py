@@ -277,3 +277,20 @@ def test_compensated_attention_argument_errors(L):
     assert call(ws=ctypes.c_void_p((1 << 24) + 16)) == vsa.ERR_INVALID_ARGUMENT
     assert call(ws=ctypes.c_void_p(0x400000)) == vsa.ERR_INVALID_ARGUMENT  # workspace over o
     assert call(o=FAKE) == vsa.ERR_INVALID_ARGUMENT                        # o over q
+
+
+def test_fused_scores_topk_argument_errors(L):
+    def call(**kw):
+        a = dict(dt=vsa.BF16, B=1, H=2, nb=240, D=128, k=24, sink=1, dw=0, cap=26)
+        a.update(kw)
+        return L.vsa_block_scores_topk(FAKE, FAKE, FAKE, FAKE, a["dt"], a["B"], a["H"], a["nb"], a["D"], a["k"],
+                                       a["sink"], a["dw"], FAKE, FAKE, a["cap"], NULL)
+    assert call(k=0) == vsa.ERR_INVALID_ARGUMENT
+    assert call(k=241) == vsa.ERR_INVALID_ARGUMENT
+    assert call(cap=25) == vsa.ERR_INVALID_ARGUMENT
+    assert call(sink=-1) == vsa.ERR_INVALID_ARGUMENT
+    assert call(dw=-2) == vsa.ERR_INVALID_ARGUMENT
+    assert call(dt=vsa.F32) == vsa.ERR_UNSUPPORTED
+    assert call(nb=1025, k=100, cap=102) == vsa.ERR_UNSUPPORTED
+    assert "at most 1024" in vsa.last_error()
+    assert call(D=96) == vsa.ERR_UNSUPPORTED

@@ -173,12 +173,14 @@ def test_topk_lists_bit_exact(nb, levels):
 
 
 @pytest.mark.parametrize("nb", [200, 960, 1000])
-@pytest.mark.parametrize("kind", ["negative", "narrow", "wide_ties", "spread"])
+@pytest.mark.parametrize("kind", ["negative", "narrow", "wide_ties", "spread", "infinite", "clustered"])
 def test_topk_threshold_search_paths(nb, kind):
     """Score rows that drive the threshold search down each of its paths: all
     negative (padded slots share the threshold's prefix), values within a few
     ulps of each other (many keys share every prefix), exact ties wider than
-    the candidate buffer, and magnitudes spread over many octaves."""
+    the candidate buffer, magnitudes spread over many octaves (most of a
+    row's histogram in its end bins), infinite scores (no finite value range
+    to bin) and two far-apart clusters (the threshold's bin crowded)."""
     g = torch.Generator(DEV).manual_seed(nb + len(kind))
     x = torch.randn(2, 1, nb, nb, generator=g, device=DEV)
     if kind == "negative":
@@ -187,6 +189,13 @@ def test_topk_threshold_search_paths(nb, kind):
         sc = 1.0 + x * 1e-6
     elif kind == "wide_ties":
         sc = torch.where(x > -0.5, torch.full_like(x, 2.5), x)  # ~70% of each row ties at the top
+    elif kind == "infinite":
+        sc = x.clone()
+        sc[..., 5] = float("inf")
+        sc[..., 9] = float("-inf")
+        sc[..., 11] = float("inf")
+    elif kind == "clustered":
+        sc = torch.where(x > 0.3, 1e6 + x, x)
     else:
         sc = torch.sign(x) * torch.exp2(x * 20.0)
     sc = sc.contiguous()
@@ -197,6 +206,55 @@ def test_topk_threshold_search_paths(nb, kind):
                                             cap=idx.shape[-1])
             assert np.array_equal(idx.view(2, nb, -1)[bh].cpu().numpy(), oi), (kind, nb, k, bh)
             assert np.array_equal(cnt.view(2, nb)[bh].cpu().numpy(), oc)
+
+
+@pytest.mark.parametrize("nb,D", [(1, 64), (33, 128), (240, 128), (300, 64), (960, 128), (1024, 64)])
+def test_fused_scores_topk_bit_exact(nb, D):
+    """The fused scores-and-lists kernel on integer-grid summaries (exact
+    scores): lists equal the oracle's and the separate scores -> top-k path's
+    bit for bit, for several budgets, sink counts and diagonal widths."""
+    summ = [integer_grid((2, 2, nb, D), 40 + i, torch.bfloat16, DEV) for i in range(4)]
+    settings = [(max(1, nb // 10), 1, 0), (1, 0, -1), (nb, 1, 0), (max(1, nb // 6), min(3, nb), 2)]
+    for k, n_sink, dw in settings:
+        fi, fc = vsa.block_scores_topk(*summ, k, n_sink, dw)
+        si, sc_ = vsa.topk_block_mask(vsa.block_scores(*summ), k, n_sink, dw)
+        assert torch.equal(fi, si) and torch.equal(fc, sc_), (nb, D, k, n_sink, dw)
+        for bh in range(4):
+            s = oracle.block_scores(*(_np(x.view(4, nb, D)[bh]) for x in summ))
+            oi, oc = oracle.topk_block_list(s, k, n_sink, dw, cap=fi.shape[-1])
+            assert np.array_equal(fi.view(4, nb, -1)[bh].cpu().numpy(), oi), (nb, k, n_sink, dw, bh)
+            assert np.array_equal(fc.view(4, nb)[bh].cpu().numpy(), oc)
+
+
+def test_fused_scores_topk_adaptive_full_size():
+    """The S = 122880 adaptive step's summaries (smooth fields, 24 heads, k =
+    96): the fused kernel's lists against the separate path's and, where they
+    differ, as valid top-k sets under the oracle's scores within the fp32
+    allowance."""
+    w = WORKLOADS["spade_adaptive_s122880"]
+    q, k, v = make_qkv(w, device=DEV)
+    choice = vsa.select_tiling(q, w.grid, list(w.tiles))
+    summ = [*vsa.block_summaries_tiled(q, w.grid, list(w.tiles), choice, 128),
+            *vsa.block_summaries_tiled(k, w.grid, list(w.tiles), choice, 128)]
+    fi, fc = vsa.block_scores_topk(*summ, w.k)
+    si, sc_ = vsa.topk_block_mask(vsa.block_scores(*summ), w.k)
+    same = (fi == si).all(-1)
+    print(f"rows whose fused list differs from the separate path's: {int((~same).sum())} of {same.numel()}")
+    for h in torch.nonzero(~same.all(-1).view(-1)).flatten().tolist()[:3]:
+        res = {"qmax": _np(summ[0][0, h]).astype(np.float64), "qmin": _np(summ[1][0, h]).astype(np.float64),
+               "kmax": _np(summ[2][0, h]).astype(np.float64), "kmin": _np(summ[3][0, h]).astype(np.float64)}
+        s = oracle.block_scores(res["qmax"], res["qmin"], res["kmax"], res["kmin"])
+        bound = SCORE_EPS * _abs_terms(res)
+        gi, gc = fi[0, h].cpu().numpy(), fc[0, h].cpu().numpy()
+        for i in range(w.nb):
+            sel = set(gi[i, :gc[i]].tolist())
+            forced = {0, i}
+            assert forced <= sel and w.k <= len(sel) <= w.k + len(forced)
+            order = np.lexsort((np.arange(w.nb), -s[i]))
+            kth = order[w.k - 1]
+            tol = bound[i] + bound[i, kth]
+            assert all(s[i, j] >= s[i, kth] - tol[j] for j in sel - forced), (h, i)
+            assert all(s[i, j] <= s[i, kth] + tol[j] for j in set(range(w.nb)) - sel), (h, i)
 
 
 # --------------------------------------------------------------------------
