@@ -395,7 +395,10 @@ def window_tile_pairs(S: int, window: int, sink: int, bn: int = 128) -> int:
     return total
 
 
-def extra_workloads(steps: int):
+EXTRAS = ("window", "fixed", "padded", "structured", "explicit", "compensated", "topp", "profile")
+
+
+def extra_workloads(steps: int, want=EXTRAS):
     """Secondary lines: window (S=30720), SPADE fixed tiling (S=30720), SPADE
     adaptive on a padded 16 x 45 x 80 grid (S=57600), structured masks on a
     CFG pair (S=122880), and dense SDPA context."""
@@ -415,6 +418,19 @@ def extra_workloads(steps: int):
         return s.elapsed_time(e) / n
 
     # window attention: computed 128x128 tiles counted by the kernel's enumeration
+    if "window" in want:
+        window_line(out, timed)
+    if "fixed" in want:
+        fixed_line(out, timed, steps)
+    if "padded" in want:
+        padded_line(out, timed, steps)
+    if "structured" in want:
+        structured_lines(out, timed, steps)
+    return out
+
+
+def window_line(out, timed):
+    import block_sparse_self_b200 as vsa
     w = WORKLOADS["window_s30720"]
     q, k, v = make_qkv(w, device="cuda")
     ms = timed(lambda: vsa.window_attention(q, k, v, w.window, w.sink, chunk_size=w.chunk))
@@ -425,7 +441,8 @@ def extra_workloads(steps: int):
     out[w.name]["dense_sdpa_ms_context"] = dense
     del q, k, v
 
-    # SPADE fixed tiling
+
+def fixed_line(out, timed, steps):
     w = WORKLOADS["spade_fixed_s30720"]
     q, k, v = make_qkv(w, device="cuda")
     st = SpadeStep(w, q, k, v)
@@ -436,10 +453,13 @@ def extra_workloads(steps: int):
                    "attn_tflops": fl / ph["attention"] / 1e9, "phase_ms": ph}
     del q, k, v, st
 
+
+def padded_line(out, timed, steps):
     # SPADE with adaptive tiling on a grid the candidates do not divide
     # (16 x 45 x 80, zero-padded to 16 x 48 x 80 inside the kernels; every
     # 128-position query block of it holds real tokens, so the counted blocks
     # are the computed ones)
+    import block_sparse_self_b200 as vsa
     w = WORKLOADS["spade_adaptive_pad_s57600"]
     q, k, v = make_qkv(w, device="cuda")
     st = SpadeStep(w, q, k, v)
@@ -451,6 +471,9 @@ def extra_workloads(steps: int):
                    "padded_grid": list(vsa.padded_grid(w.grid, w.tiles))}
     del q, k, v, st
 
+
+def structured_lines(out, timed, steps):
+    import block_sparse_self_b200 as vsa
     # structured masks on a CFG pair.  The attention kernel runs in the mode
     # structured_attention picks: T-major directly for whole-frame tiles
     # (spatial), through TMA boxes for sliding tiles, and for the temporal
@@ -486,7 +509,6 @@ def extra_workloads(steps: int):
         fn = None
         qp = kp = vp = None
     out[w.name] = res
-    return out
 
 
 def compensated_line(w, q, k, v, idx, cnt, n_rep: int):
@@ -583,9 +605,10 @@ def run_ours(args, w):
                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h}
 
     extra = None
-    if rank == 0 and world == 1 and not args.no_extra:
-        extra = extra_workloads(max(3, args.steps // 2))
-        if step.tiled:  # the same step with explicit permuted copies, for comparison
+    want = () if args.no_extra else tuple(args.extras.split(","))
+    if rank == 0 and world == 1 and want:
+        extra = extra_workloads(max(3, args.steps // 2), want)
+        if step.tiled and "explicit" in want:  # the same step with explicit permuted copies, for comparison
             ex = SpadeStep(wr, q, k, v, tiled=False)
             ex_ms = time_steps(ex, max(3, args.steps // 2), 3, False)
             extra["explicit_permute_" + w.name] = {"ms_per_step": ex_ms, "phase_ms": ex.phase_ms(),
@@ -594,47 +617,49 @@ def run_ours(args, w):
         # centroid-compensated attention on the same lists: the kept blocks as
         # above plus every skipped block as its centroid (explicit permuted
         # copies in each head's tiling; bf16 output)
-        extra["compensated_" + w.name] = compensated_line(w, q, k, v, step.last["idx"], step.last["cnt"],
-                                                          max(3, args.steps // 2))
-        # top-p (mass budget) lists on the same scores, in place of the top-k lists
-        import block_sparse_self_b200 as vsa
-        sc = step.last["scores"]
-        p_mass, p_scale = 0.5, 1.0 / math.sqrt(w.D)
-        tp = {}
-        for _ in range(3):
-            vsa.topp_block_mask(sc, p_mass, p_scale)
+        if "compensated" in want:
+            extra["compensated_" + w.name] = compensated_line(w, q, k, v, step.last["idx"], step.last["cnt"],
+                                                              max(3, args.steps // 2))
         ev = [torch.cuda.Event(enable_timing=True) for _ in range(2)]
-        ev[0].record()
         n_rep = 5
-        for _ in range(n_rep):
-            ti, tc = vsa.topp_block_mask(sc, p_mass, p_scale)
-        ev[1].record()
-        torch.cuda.synchronize()
-        tp["ms_per_call"] = ev[0].elapsed_time(ev[1]) / n_rep
-        tp["p"], tp["scale"] = p_mass, p_scale
-        tp["mean_blocks_per_row"] = float(tc.float().mean().item())
-        tp["bytes"] = float(sc.numel() * 4 + ti.numel() * 4 + tc.numel() * 4)
-        tp["gbs"] = tp["bytes"] / tp["ms_per_call"] / 1e6
-        extra["topp_lists_" + w.name] = tp
-        del ti, tc
-        # head profile (spatial or temporal pattern per head) on 128 sampled query rows:
-        # K is read once per head (the bound); Q contributes only the sampled rows
-        rows = vsa.sample_query_rows(w.S, 128, seed=0, device=q.device)
-        for _ in range(3):
-            vsa.head_profile(q, k, w.grid, rows)
-        ev[0].record()
-        for _ in range(n_rep):
-            hk, hm = vsa.head_profile(q, k, w.grid, rows)
-        ev[1].record()
-        torch.cuda.synchronize()
-        hp_ms = ev[0].elapsed_time(ev[1]) / n_rep
-        hp_bytes = float(k.numel() * 2 + BH * 128 * w.D * 2)
-        extra["head_profile_" + w.name] = {
-            "ms_per_call": hp_ms, "rows": 128, "bytes": hp_bytes, "gbs": hp_bytes / hp_ms / 1e6,
-            "frac_hbm": hp_bytes / hp_ms / 1e6 / hbm,
-            "tflops": 2.0 * 2 * 128 * w.S * w.D * BH / hp_ms / 1e9,
-            "temporal_heads": int(hk.sum().item()), "heads": BH}
-        del hk, hm
+        if "topp" in want:
+            # top-p (mass budget) lists on the same scores, in place of the top-k lists
+            sc = step.last["scores"]
+            p_mass, p_scale = 0.5, 1.0 / math.sqrt(w.D)
+            tp = {}
+            for _ in range(3):
+                vsa.topp_block_mask(sc, p_mass, p_scale)
+            ev[0].record()
+            for _ in range(n_rep):
+                ti, tc = vsa.topp_block_mask(sc, p_mass, p_scale)
+            ev[1].record()
+            torch.cuda.synchronize()
+            tp["ms_per_call"] = ev[0].elapsed_time(ev[1]) / n_rep
+            tp["p"], tp["scale"] = p_mass, p_scale
+            tp["mean_blocks_per_row"] = float(tc.float().mean().item())
+            tp["bytes"] = float(sc.numel() * 4 + ti.numel() * 4 + tc.numel() * 4)
+            tp["gbs"] = tp["bytes"] / tp["ms_per_call"] / 1e6
+            extra["topp_lists_" + w.name] = tp
+            del ti, tc
+        if "profile" in want:
+            # head profile (spatial or temporal pattern per head) on 128 sampled query rows:
+            # K is read once per head (the bound); Q contributes only the sampled rows
+            rows = vsa.sample_query_rows(w.S, 128, seed=0, device=q.device)
+            for _ in range(3):
+                vsa.head_profile(q, k, w.grid, rows)
+            ev[0].record()
+            for _ in range(n_rep):
+                hk, hm = vsa.head_profile(q, k, w.grid, rows)
+            ev[1].record()
+            torch.cuda.synchronize()
+            hp_ms = ev[0].elapsed_time(ev[1]) / n_rep
+            hp_bytes = float(k.numel() * 2 + BH * 128 * w.D * 2)
+            extra["head_profile_" + w.name] = {
+                "ms_per_call": hp_ms, "rows": 128, "bytes": hp_bytes, "gbs": hp_bytes / hp_ms / 1e6,
+                "frac_hbm": hp_bytes / hp_ms / 1e6 / hbm,
+                "tflops": 2.0 * 2 * 128 * w.S * w.D * BH / hp_ms / 1e9,
+                "temporal_heads": int(hk.sum().item()), "heads": BH}
+            del hk, hm
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
@@ -670,12 +695,17 @@ def main():
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=sorted(WORKLOADS))
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-extra", action="store_true")
+    ap.add_argument("--extras", default=",".join(EXTRAS),
+                    help="comma-separated secondary lines to run (%s); --no-extra runs none" % ",".join(EXTRAS))
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--heads", type=int, default=None,
                     help="run the workload with this many heads (smaller cases for profilers; not a bench line)")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
+    unknown = set(args.extras.split(",")) - set(EXTRAS)
+    if unknown:
+        ap.error(f"unknown --extras {sorted(unknown)}; choose from {EXTRAS}")
     w = WORKLOADS[args.workload]
     if args.heads is not None:
         if args.heads < 1:

@@ -405,44 +405,6 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
     return *reinterpret_cast<uint32_t *>(&v);
 }
 
-__device__ __forceinline__ uint64_t mul_f32x2(uint64_t a, uint64_t b) {
-    uint64_t r;
-    asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
-    return r;
-}
-
-// 2^a0 and 2^a1 as a packed bf16 pair from one half-precision exponential
-// instruction (two results), for moving work off the exponential unit.  The
-// argument is split as a = n + f, n = round(a) by adding and subtracting
-// 1.5 * 2^23 (the fp32 sum rounds to an integer), f = a - n in [-1/2, 1/2]
-// (exact); 2^f comes from ex2.approx.f16x2 on f rounded to half precision,
-// and 2^n is written into an fp32 exponent field as (n + 127) << 23, which
-// the integer part of the rounding sum already holds in its low bits.  a is
-// clamped to [-127, 64] first: n = -127 encodes as +0 (so a masked -inf key
-// gives exactly 0) and 2^64 is far above every row-sum limit.
-__device__ __forceinline__ uint32_t ex2_bf16x2_split(float a0, float a1) {
-    a0 = fminf(fmaxf(a0, -127.f), 64.f);
-    a1 = fminf(fmaxf(a1, -127.f), 64.f);
-    const uint64_t a = f32x2(a0, a1);
-    const uint64_t t = add_f32x2(a, f32x2(12582912.f, 12582912.f));
-    const uint64_t nf = add_f32x2(t, f32x2(-12582912.f, -12582912.f));
-    float f0, f1, t0, t1;
-    f32x2_split(fma_f32x2(nf, f32x2(-1.f, -1.f), a), f0, f1);
-    f32x2_split(t, t0, t1);
-    uint32_t h, e;
-    asm("cvt.rn.f16x2.f32 %0, %1, %2;" : "=r"(h) : "f"(f1), "f"(f0));
-    asm("ex2.approx.f16x2 %0, %1;" : "=r"(e) : "r"(h));
-    float e0, e1;
-    asm("{\n\t.reg .f16 lo, hi;\n\tmov.b32 {lo, hi}, %2;\n\tcvt.f32.f16 %0, lo;\n\tcvt.f32.f16 %1, hi;\n\t}"
-        : "=f"(e0), "=f"(e1)
-        : "r"(e));
-    const uint32_t s0 = __float_as_uint(t0) * 8388608u + 0x3f800000u;  // (n + 127) << 23, mod 2^32
-    const uint32_t s1 = __float_as_uint(t1) * 8388608u + 0x3f800000u;
-    float p0, p1;
-    f32x2_split(mul_f32x2(f32x2(e0, e1), f32x2(__uint_as_float(s0), __uint_as_float(s1))), p0, p1);
-    return pack_bf16x2(p0, p1);
-}
-
 // acc_lo += low bf16 of pk, acc_hi += high bf16 of pk: sm_100 mixed-precision
 // adds (the bf16 operand widens exactly, then one fp32 rounding), with no
 // separate unpacking of the pair.
