@@ -308,11 +308,21 @@ def pattern_masses(probs, grid, rows):
     return mass
 
 
-def classify_head(q, k, grid, rows, scale=None):
-    """(kind, mean masses [2]) of one head: the pattern holding the larger mean
-    mass over the sampled rows, 0 = spatial, 1 = temporal, ties to spatial."""
+PROFILE_RULES = ("mass", "mass_per_key")
+
+
+def classify_head(q, k, grid, rows, scale=None, rule="mass"):
+    """(kind, mean masses [2]) of one head, 0 = spatial, 1 = temporal, ties to
+    spatial.  rule "mass": the pattern holding the larger mean mass over the
+    sampled rows.  rule "mass_per_key": the larger mean mass per key of the
+    pattern, spatial mass / (H W) against temporal mass / T (the attention a
+    query pays each key of its frame, or each key at its (h, w))."""
+    if rule not in PROFILE_RULES:
+        raise ValueError(f"rule must be one of {PROFILE_RULES}")
     mass = pattern_masses(sampled_probs(q, k, rows, scale), grid, rows).mean(axis=0)
-    return (0 if mass[0] >= mass[1] else 1), mass
+    T, H, W = grid
+    sp, tp = (mass[0], mass[1]) if rule == "mass" else (mass[0] / (H * W), mass[1] / T)
+    return (0 if sp >= tp else 1), mass
 
 
 # --------------------------------------------------------------------------

@@ -411,6 +411,53 @@ def test_head_profile_closed_forms_of_one_hot_fields(alpha):
     assert kind == (0 if sp >= tp else 1) and kind == (1 if alpha >= 2 else 0)
 
 
+@pytest.mark.parametrize("alpha", [0.05, 0.5, 2.0, 6.0])
+def test_head_profile_mass_per_key_rule_closed_forms(alpha):
+    """The per-key rule compares spatial mass / (H W) with temporal mass / T.
+    With a frame code every key of the frame holds e^alpha / z and the keys at
+    the query's (h, w) hold (e^alpha + T - 1) / (T z) on average, so the head is
+    spatial for every alpha > 0; with a position code it is temporal for every
+    alpha > 0 (the mass rule calls weak position codes spatial, see above)."""
+    grid = (4, 4, 4)
+    T, HW, S = 4, 16, 64
+    t, h, w = _coords(grid)
+    hw = h * 4 + w
+    rows = [0, 21, 42, 63]
+    q = np.zeros((S, 16), np.float32)
+    k = np.zeros((S, 16), np.float32)
+    q[np.arange(S), t] = alpha
+    k[np.arange(S), t] = 1.0
+    kind, mass = oracle.classify_head(q, k, grid, rows, scale=1.0, rule="mass_per_key")
+    assert kind == 0 and mass[0] / HW > mass[1] / T
+    q[:] = 0.0
+    k[:] = 0.0
+    q[np.arange(S), hw] = alpha
+    k[np.arange(S), hw] = 1.0
+    kind, mass = oracle.classify_head(q, k, grid, rows, scale=1.0, rule="mass_per_key")
+    assert kind == 1 and mass[1] / T > mass[0] / HW
+    assert kind == oracle.classify_head(q, k, grid, rows, scale=1.0, rule="mass")[0] or alpha < 2
+
+
+def test_head_profile_mass_per_key_uniform_tie_and_equal_sizes():
+    # q = 0: every key carries 1/S, so both patterns hold 1/S per key exactly
+    # (1/64 and its multiples are exact): a tie, which goes to spatial
+    grid = (4, 4, 4)
+    k = np.random.default_rng(7).standard_normal((64, 8)).astype(np.float32)
+    q = np.zeros((64, 8), np.float32)
+    kind, mass = oracle.classify_head(q, k, grid, [0, 9, 33, 63], rule="mass_per_key")
+    assert mass[0] / 16 == mass[1] / 4 and kind == 0
+    # T = H W: the two rules are one
+    grid = (4, 2, 2)
+    rng = np.random.default_rng(8)
+    for _ in range(5):
+        q = rng.standard_normal((16, 8)).astype(np.float32)
+        k = rng.standard_normal((16, 8)).astype(np.float32)
+        assert (oracle.classify_head(q, k, grid, [0, 3, 9], rule="mass_per_key")[0]
+                == oracle.classify_head(q, k, grid, [0, 3, 9], rule="mass")[0])
+    with pytest.raises(ValueError):
+        oracle.classify_head(q, k, grid, [0], rule="density")
+
+
 def test_head_profile_matches_torch_softmax_and_coordinate_masks():
     grid = (6, 4, 5)
     S = 120
