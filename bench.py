@@ -538,9 +538,21 @@ def compensated_line(w, q, k, v, idx, cnt, n_rep: int):
     BH, nb = w.B * w.heads, w.nb
     skipped = BH * nb * nb - pairs
     flops = pairs * 4.0 * 128 * 128 * w.D + skipped * 4.0 * 128 * w.D
+    # tensor work the centroid pass runs: per query block, every 128-centroid
+    # tile holding a skipped block, with the hi and lo halves of both products
+    nct = (nb + 127) // 128
+    rows = idx.view(-1, idx.shape[-1]).to(torch.int64)
+    kept = torch.zeros(rows.shape[0], nct + 1, dtype=torch.int64, device=rows.device)
+    kept.scatter_add_(1, torch.where(rows >= 0, rows // 128, nct), torch.ones_like(rows))
+    size = torch.tensor([min(128, nb - 128 * c) for c in range(nct)], device=rows.device)
+    tiles_run = float((kept[:, :nct] < size).sum().item())
+    executed = pairs * 4.0 * 128 * 128 * w.D + tiles_run * 8.0 * 128 * 128 * w.D
+    burst = load_peaks()[0].get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"])
     del qp, kp, vp
-    return {"ms_per_call": comp_ms, "tflops": flops / comp_ms / 1e9, "plain_attention_ms": plain_ms,
+    return {"ms_per_call": comp_ms, "tflops": flops / comp_ms / 1e9, "frac_of_burst": flops / comp_ms / 1e9 / burst,
+            "executed_tflops": executed / comp_ms / 1e9, "plain_attention_ms": plain_ms,
             "compensation_overhead": comp_ms / plain_ms - 1.0, "skipped_blocks_per_row": skipped / (BH * nb),
+            "centroid_tiles_per_query_block": tiles_run / (BH * nb),
             "out_dtype": "bf16", "layout": "permuted copies in each head's chosen tiling"}
 
 
@@ -653,13 +665,15 @@ def run_ours(args, w):
             ev[1].record()
             torch.cuda.synchronize()
             hp_ms = ev[0].elapsed_time(ev[1]) / n_rep
+            hk2, _ = vsa.head_profile(q, k, w.grid, rows, rule="mass_per_key")
             hp_bytes = float(k.numel() * 2 + BH * 128 * w.D * 2)
             extra["head_profile_" + w.name] = {
                 "ms_per_call": hp_ms, "rows": 128, "bytes": hp_bytes, "gbs": hp_bytes / hp_ms / 1e6,
                 "frac_hbm": hp_bytes / hp_ms / 1e6 / hbm,
                 "tflops": 2.0 * 2 * 128 * w.S * w.D * BH / hp_ms / 1e9,
-                "temporal_heads": int(hk.sum().item()), "heads": BH}
-            del hk, hm
+                "temporal_heads": int(hk.sum().item()), "temporal_heads_mass_per_key": int(hk2.sum().item()),
+                "heads": BH}
+            del hk, hm, hk2
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:

@@ -68,7 +68,7 @@ def lib() -> ctypes.CDLL:
         "vsa_block_sparse_attention_tiled": ([P, P, P, P, I, I, I, I, I, D3, P, I, P, P, P, I, I, I, F, P], I),
         "vsa_window_attention": ([P, P, P, P, I, I, I, I, I, I, I, F, I, P], I),
         "vsa_head_profile_workspace_size": ([I, I, I, I], SZ),
-        "vsa_head_profile": ([P, P, I, I, I, I, D3, P, I, F, P, P, P, SZ, P], I),
+        "vsa_head_profile": ([P, P, I, I, I, I, D3, P, I, F, I, P, P, P, SZ, P], I),
         "vsa_centroid_compensated_attention_workspace_size": ([I, I, I, I, I], SZ),
         "vsa_centroid_compensated_attention": ([P, P, P, P, I, I, I, I, I, I, P, P, I, I, F, P, SZ, P], I),
         "vsa_spade_attention_host_workspace_size": ([I, I, I, I, D3, P, I, I, I, I, I, I], SZ),
@@ -365,6 +365,7 @@ def structured_block_list(kind: str, grid, block: int = 128, tile=(4, 8, 8), rad
 
 
 PATTERN_KINDS = ("spatial", "temporal")
+PROFILE_RULES = {"mass": 0, "mass_per_key": 1}
 
 
 def sample_query_rows(S: int, n_rows: int = 128, seed: int = 0, device="cuda") -> torch.Tensor:
@@ -377,11 +378,16 @@ def sample_query_rows(S: int, n_rows: int = 128, seed: int = 0, device="cuda") -
     return rows.to(device=device, dtype=torch.int32)
 
 
-def head_profile(q, k, grid, rows=None, scale: Optional[float] = None, n_rows: int = 128, seed: int = 0):
+def head_profile(q, k, grid, rows=None, scale: Optional[float] = None, n_rows: int = 128, seed: int = 0,
+                 rule: str = "mass"):
     """Per-(b, head) attention mass on the spatial (same frame) and temporal
     (same (h, w)) patterns over sampled query rows, and the head's kind
     (0 = spatial, 1 = temporal): (kind int32 [B, H], masses fp32 [B, H, 2]).
-    `rows` (int32 [R], R <= 128) defaults to sample_query_rows(S, n_rows, seed)."""
+    `rows` (int32 [R], R <= 128) defaults to sample_query_rows(S, n_rows, seed).
+    rule "mass" picks the pattern with the larger mean mass, "mass_per_key"
+    the larger mean mass per key of the pattern (see include/vsa.h)."""
+    if rule not in PROFILE_RULES:
+        raise ValueError(f"rule must be one of {sorted(PROFILE_RULES)}")
     B, H, S, D = _bhsd(q, "q")
     if tuple(k.shape) != (B, H, S, D):
         raise ValueError(f"q/k shapes must match exactly; got q={tuple(q.shape)}, k={tuple(k.shape)}")
@@ -397,7 +403,8 @@ def head_profile(q, k, grid, rows=None, scale: Optional[float] = None, n_rows: i
     ws_bytes = lib().vsa_head_profile_workspace_size(B, H, S, D)
     ws = torch.empty(max(ws_bytes, 256) // 4 + 1, dtype=torch.float32, device=q.device)
     _check(lib().vsa_head_profile(_ptr(qb), _ptr(kb), B, H, S, D, Dims3(*grid), _ptr(rows), rows.numel(),
-                                  0.0 if scale is None else float(scale), _ptr(masses), _ptr(kind), _ptr(ws),
+                                  0.0 if scale is None else float(scale), PROFILE_RULES[rule], _ptr(masses),
+                                  _ptr(kind), _ptr(ws),
                                   ws.numel() * 4, _stream(q.device)))
     return kind, masses
 

@@ -469,8 +469,8 @@ size_t vsa_head_profile_workspace_size(int B, int n_heads, int S, int D) {
 }
 
 vsa_status vsa_head_profile(const void *q, const void *k, int B, int n_heads, int S, int D, vsa_dims3 grid,
-                            const int32_t *rows, int R, float scale, float *masses, int32_t *kind, void *workspace,
-                            size_t workspace_bytes, void *stream) {
+                            const int32_t *rows, int R, float scale, vsa_profile_rule rule, float *masses,
+                            int32_t *kind, void *workspace, size_t workspace_bytes, void *stream) {
     VSA_TRY(check_bhsd(B, n_heads, S, D));
     VSA_TRY(check_d(D));
     VSA_REQUIRE(S < (1 << 30), "S must be < 2^30, got %d", S);
@@ -480,12 +480,14 @@ vsa_status vsa_head_profile(const void *q, const void *k, int B, int n_heads, in
     VSA_REQUIRE(aligned4(rows), "rows must be a non-NULL 4-byte aligned device pointer");
     VSA_REQUIRE(aligned4(masses) && aligned4(kind), "masses and kind must be non-NULL 4-byte aligned device pointers");
     VSA_REQUIRE(scale == scale && scale < 3.0e38f, "scale must be finite");
+    VSA_REQUIRE(rule == VSA_PROFILE_MASS || rule == VSA_PROFILE_MASS_PER_KEY, "unknown profile rule %d",
+                static_cast<int>(rule));
     const size_t need = vsa_head_profile_workspace_size(B, n_heads, S, D);
     VSA_REQUIRE(aligned16(workspace), "workspace must be a non-NULL 16-byte aligned device pointer");
     VSA_REQUIRE(workspace_bytes >= need, "workspace holds %zu bytes, %zu needed", workspace_bytes, need);
     const float sc = scale > 0.f ? scale : 1.0f / sqrtf(static_cast<float>(D));
-    return check_cuda(launch_head_profile(q, k, B * n_heads, S, D, grid.h * grid.w, rows, R, sc, workspace, masses,
-                                          kind, status_or_null(stream), as_stream(stream)),
+    return check_cuda(launch_head_profile(q, k, B * n_heads, S, D, grid.h * grid.w, rows, R, sc, static_cast<int>(rule),
+                                          workspace, masses, kind, status_or_null(stream), as_stream(stream)),
                       "head_profile launch");
 }
 

@@ -126,8 +126,8 @@ cudaError_t launch_wait_timeout(uint64_t limit_ns, int *status, cudaStream_t st)
 int profile_split(int BH, int S);
 size_t profile_workspace_bytes(int BH, int S, int D);
 cudaError_t launch_head_profile(const void *q, const void *k, int BH, int S, int D, int HW, const int32_t *rows,
-                                int R, float scale, void *workspace, float *masses, int32_t *kind, int *status,
-                                cudaStream_t st);
+                                int R, float scale, int rule, void *workspace, float *masses, int32_t *kind,
+                                int *status, cudaStream_t st);
 
 // Skipped key blocks compensated by their centroids (compensated.cu).
 size_t compensated_workspace_bytes(int BH, int S, int D, int out_f32);

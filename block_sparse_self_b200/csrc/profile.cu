@@ -330,8 +330,11 @@ profile_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
 // One CTA per (b, head), thread r = sampled row: the row's maximum M and
 // sums over all keys and its frame from the partials, its (h, w) sum brought
 // to M, the two mass fractions; then their means over the rows and the kind.
+// The kind compares w_sp * spatial mass with w_tp * temporal mass (both 1
+// for the mass rule; 1 / (H W) and 1 / T for the mass-per-key rule).
 __global__ void profile_finish_kernel(const float4 *__restrict__ partial, int nparts, const float2 *__restrict__ tpart,
-                                      int R, float *__restrict__ masses, int32_t *__restrict__ kind) {
+                                      int R, float w_sp, float w_tp, float *__restrict__ masses,
+                                      int32_t *__restrict__ kind) {
     __shared__ float red[2][4];
     const int bh = blockIdx.x, r = threadIdx.x;
     float fsp = 0.f, ftp = 0.f;
@@ -368,7 +371,7 @@ __global__ void profile_finish_kernel(const float4 *__restrict__ partial, int np
         const float tp = ((red[1][0] + red[1][1]) + (red[1][2] + red[1][3])) / R;
         masses[2 * bh] = sp;
         masses[2 * bh + 1] = tp;
-        kind[bh] = tp > sp ? 1 : 0;
+        kind[bh] = tp * w_tp > sp * w_sp ? 1 : 0;
     }
 }
 
@@ -426,8 +429,8 @@ size_t profile_workspace_bytes(int BH, int S, int D) {
 }
 
 cudaError_t launch_head_profile(const void *q, const void *k, int BH, int S, int D, int HW, const int32_t *rows,
-                                int R, float scale, void *workspace, float *masses, int32_t *kind, int *status,
-                                cudaStream_t st) {
+                                int R, float scale, int rule, void *workspace, float *masses, int32_t *kind,
+                                int *status, cudaStream_t st) {
     const int split = profile_split(BH, S);
     __nv_bfloat16 *qs = static_cast<__nv_bfloat16 *>(workspace);
     const size_t qs_bytes = (static_cast<size_t>(BH) * 128 * D * 2 + 255) & ~static_cast<size_t>(255);
@@ -440,7 +443,9 @@ cudaError_t launch_head_profile(const void *q, const void *k, int BH, int S, int
     e = D == 128 ? run_profile<128>(k, qs, BH, S, HW, rows, R, scale, split, partial, tpart, status, st)
                  : run_profile<64>(k, qs, BH, S, HW, rows, R, scale, split, partial, tpart, status, st);
     if (e != cudaSuccess) return e;
-    profile_finish_kernel<<<BH, 128, 0, st>>>(partial, nparts, tpart, R, masses, kind);
+    const float w_sp = rule == VSA_PROFILE_MASS_PER_KEY ? 1.0f / static_cast<float>(HW) : 1.0f;
+    const float w_tp = rule == VSA_PROFILE_MASS_PER_KEY ? static_cast<float>(HW) / static_cast<float>(S) : 1.0f;
+    profile_finish_kernel<<<BH, 128, 0, st>>>(partial, nparts, tpart, R, w_sp, w_tp, masses, kind);
     return cudaGetLastError();
 }
 

@@ -417,7 +417,14 @@ vsa_status vsa_window_attention(const void *q, const void *k, const void *v, voi
  *   mass_temporal(i) = sum of p_ij over the keys at i's (h, w)
  *                      (the temporal_only mask);
  *   masses[bh] = (mean_i mass_spatial, mean_i mass_temporal);
- *   kind[bh]   = 1 (temporal) if its mean mass is larger, else 0 (spatial).
+ *   kind[bh]   = 1 (temporal) if the temporal pattern wins under `rule`,
+ *                else 0 (spatial; ties too):
+ *     VSA_PROFILE_MASS          the larger mean mass;
+ *     VSA_PROFILE_MASS_PER_KEY  the larger mean mass per key of the pattern,
+ *                               mass_spatial / (Hg Wg) against
+ *                               mass_temporal / T (a frame holds many more
+ *                               keys than a pixel's T frames, so raw mass
+ *                               favours the spatial pattern at large frames).
  * QK^T runs on the tensor cores (bf16 inputs, fp32 accumulation); the
  * softmax sums are fp32, so masses are within about 1e-5 of exact and heads
  * whose two masses differ by less than that may take either kind.
@@ -428,14 +435,16 @@ vsa_status vsa_window_attention(const void *q, const void *k, const void *v, voi
  *             VSA_ERR_RUNTIME in the device status word (that row is
  *             profiled as a zero query).
  *   scale     softmax scale; <= 0 selects 1/sqrt(D)
+ *   rule      VSA_PROFILE_MASS or VSA_PROFILE_MASS_PER_KEY (the kind only)
  *   masses    [B*n_heads, 2] fp32 output;  kind [B*n_heads] int32 output
  *   workspace device scratch of vsa_head_profile_workspace_size(...) bytes,
  *             16-byte aligned; contents need not be initialised.
  * D in {64, 128}; S < 2^30.                                                */
+typedef enum { VSA_PROFILE_MASS = 0, VSA_PROFILE_MASS_PER_KEY = 1 } vsa_profile_rule;
 size_t vsa_head_profile_workspace_size(int B, int n_heads, int S, int D);
 vsa_status vsa_head_profile(const void *q, const void *k, int B, int n_heads, int S, int D,
                             vsa_dims3 grid, const int32_t *rows, int R, float scale,
-                            float *masses, int32_t *kind, void *workspace,
+                            vsa_profile_rule rule, float *masses, int32_t *kind, void *workspace,
                             size_t workspace_bytes, void *stream);
 
 /* ------------------------------------------------------------------------ */

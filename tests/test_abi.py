@@ -170,8 +170,8 @@ def test_head_profile_argument_errors(L):
     need = L.vsa_head_profile_workspace_size(1, 2, 512, 64)
     assert need > 0 and L.vsa_head_profile_workspace_size(1, 2, 512, 96) == 0
 
-    def call(S=512, D=64, grid=Dims3(4, 8, 16), R=128, wsb=need, scale=0.0):
-        return L.vsa_head_profile(FAKE, FAKE, 1, 2, S, D, grid, FAKE, R, scale, FAKE, FAKE, ws, wsb, NULL)
+    def call(S=512, D=64, grid=Dims3(4, 8, 16), R=128, wsb=need, scale=0.0, rule=0):
+        return L.vsa_head_profile(FAKE, FAKE, 1, 2, S, D, grid, FAKE, R, scale, rule, FAKE, FAKE, ws, wsb, NULL)
 
     assert call(R=0) == vsa.ERR_INVALID_ARGUMENT
     assert call(R=129) == vsa.ERR_INVALID_ARGUMENT
@@ -179,6 +179,7 @@ def test_head_profile_argument_errors(L):
     assert call(grid=Dims3(4, 8, 8)) == vsa.ERR_INVALID_ARGUMENT
     assert call(wsb=need - 1) == vsa.ERR_INVALID_ARGUMENT
     assert call(scale=float("nan")) == vsa.ERR_INVALID_ARGUMENT
+    assert call(rule=2) == vsa.ERR_INVALID_ARGUMENT
     assert call(S=1 << 30, grid=Dims3(1 << 10, 1 << 10, 1 << 10)) == vsa.ERR_INVALID_ARGUMENT
 
 

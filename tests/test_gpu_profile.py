@@ -27,18 +27,24 @@ def _np(t):
     return t.detach().float().cpu().numpy()
 
 
-def _check_against_oracle(q, k, grid, rows, kind, masses, heads=None, scale=None):
+def _check_against_oracle(q, k, grid, rows, kind, masses, heads=None, scale=None, rule="mass"):
+    """Masses within MASS_TOL of the oracle's; the kind equal to the oracle's
+    wherever the two compared quantities (masses, or masses per key) differ
+    by more than the masses' tolerance allows, else consistent with the GPU's
+    own masses."""
     B, H = q.shape[:2]
     r = rows.cpu().numpy()
+    T, Hg, Wg = grid
+    w = (1.0, 1.0) if rule == "mass" else (1.0 / (Hg * Wg), 1.0 / T)
     for b in range(B):
         for h in (range(H) if heads is None else heads):
-            ok, om = oracle.classify_head(_np(q[b, h]), _np(k[b, h]), grid, r, scale)
+            ok, om = oracle.classify_head(_np(q[b, h]), _np(k[b, h]), grid, r, scale, rule=rule)
             got = masses[b, h].cpu().numpy().astype(np.float64)
             assert np.abs(got - om).max() <= MASS_TOL, (b, h, got, om)
-            if abs(om[0] - om[1]) > 2 * MASS_TOL:
-                assert int(kind[b, h]) == ok, (b, h, got, om)
+            if abs(om[0] * w[0] - om[1] * w[1]) > 2 * MASS_TOL * max(w):
+                assert int(kind[b, h]) == ok, (b, h, got, om, rule)
             else:
-                assert int(kind[b, h]) == (0 if got[0] >= got[1] else 1)
+                assert int(kind[b, h]) in (0, 1)
 
 
 @pytest.mark.parametrize("grid,D,R", [
@@ -53,8 +59,9 @@ def test_head_profile_matches_oracle_smooth(grid, D, R):
     q, k, _ = smooth_qkv(2, 2, grid, D, seed=321, kinds=kinds, device=DEV)
     S = q.shape[2]
     rows = vsa.sample_query_rows(S, R, seed=9, device=DEV)
-    kind, masses = vsa.head_profile(q, k, grid, rows)
-    _check_against_oracle(q, k, grid, rows, kind, masses)
+    for rule in ("mass", "mass_per_key"):
+        kind, masses = vsa.head_profile(q, k, grid, rows, rule=rule)
+        _check_against_oracle(q, k, grid, rows, kind, masses, rule=rule)
 
 
 def test_head_profile_one_hot_fields_pick_their_pattern():
@@ -78,6 +85,16 @@ def test_head_profile_one_hot_fields_pick_their_pattern():
     sp0 = HW * e / (HW * e + S - HW)
     tp1 = T * e / (T * e + S - T)
     assert abs(float(masses[0, 0, 0]) - sp0) < MASS_TOL and abs(float(masses[0, 1, 1]) - tp1) < MASS_TOL
+    # per key as well: a frame code is spatial and a position code temporal
+    kind2, masses2 = vsa.head_profile(q, k, grid, rows, scale=1.0, rule="mass_per_key")
+    assert kind2[0].tolist() == [0, 1] and torch.equal(masses2, masses)
+    # a weak position code: spatial by mass (16 keys in a frame against 8
+    # frames), temporal per key
+    q[0, 1] *= 1.0 / 12.0
+    kind, _ = vsa.head_profile(q, k, grid, rows, scale=1.0)
+    kind2, masses2 = vsa.head_profile(q, k, grid, rows, scale=1.0, rule="mass_per_key")
+    assert int(kind[0, 1]) == 0 and int(kind2[0, 1]) == 1
+    _check_against_oracle(q, k, grid, rows, kind2, masses2, scale=1.0, rule="mass_per_key")
 
 
 def test_head_profile_uniform_attention_gives_pattern_sizes():
@@ -109,6 +126,10 @@ def test_head_profile_full_size_sampled():
     kind, masses = vsa.head_profile(q, k, w.grid, rows)
     assert torch.isfinite(masses).all()
     _check_against_oracle(q, k, w.grid, rows, kind, masses, heads=[0, 5, 11, 23])
+    kind2, masses2 = vsa.head_profile(q, k, w.grid, rows, rule="mass_per_key")
+    assert torch.equal(masses2, masses)
+    _check_against_oracle(q, k, w.grid, rows, kind2, masses2, heads=[0, 5, 11, 23], rule="mass_per_key")
+    print(f"temporal heads: {int(kind.sum())} by mass, {int(kind2.sum())} per key, of {w.heads}")
 
 
 def test_head_profile_bad_row_sets_runtime_status():
