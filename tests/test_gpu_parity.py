@@ -505,6 +505,22 @@ def test_spade_attention_host_buffers_match_device(chunks):
     assert not got.is_cuda and torch.equal(got, want.cpu())
 
 
+@pytest.mark.parametrize("grid,tiles,chunks,out", [
+    ((4, 9, 16), [(1, 8, 16), (2, 8, 8), (4, 4, 8)], 4, torch.float32),   # padded to (4, 16, 16)
+    ((4, 8, 16), [(2, 8, 8)], 2, torch.bfloat16),                        # one candidate: no tiling choice
+    ((4, 8, 16), [(1, 4, 16), (1, 8, 8)], 64, torch.float32),           # 64-token tiles; more groups than heads
+])
+def test_spade_attention_host_more_shapes(grid, tiles, chunks, out):
+    """The host-buffer entry point on a padded grid, with a single candidate,
+    with 64-token candidate tiles and with more groups than (b, head) rows:
+    the device composition's result bit for bit."""
+    q, k, v = smooth_qkv(1, 3, grid, 64, seed=78, device=DEV)
+    want = vsa.spade_attention(q, k, v, grid, tiles, topk=2, out_dtype=out)
+    qh, kh, vh = (x.cpu().pin_memory() for x in (q, k, v))
+    got = vsa.spade_attention_host(qh, kh, vh, grid, tiles, chunks=chunks, topk=2, out_dtype=out)
+    assert got.dtype == out and torch.equal(got, want.cpu())
+
+
 def _sample_blocks(nb, seed, n=16):
     rng = np.random.default_rng(seed)
     mid = rng.choice(np.arange(1, nb - 1), n - 2, replace=False)
