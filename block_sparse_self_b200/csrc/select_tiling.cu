@@ -140,15 +140,27 @@ __global__ void __launch_bounds__(kThreads, 4) sics_partial_kernel(const SelArgs
                         for (int e = 0; e < EPC; ++e) x[u * EPC + e] = fv[e];
                     }
                 }
-                float ss = 0.f;
+                // two-wide fp32 FMAs (each half rounds as the scalar FMA):
+                // the sum of squares in two interleaved partial sums, the
+                // unit vector's accumulation element by element as before
+                uint64_t ss2 = f32x2(0.f, 0.f);
                 #pragma unroll
-                for (int e = 0; e < EPL; ++e) ss = fmaf(x[e], x[e], ss);
+                for (int e = 0; e < EPL / 2; ++e) {
+                    const uint64_t xe = f32x2(x[2 * e], x[2 * e + 1]);
+                    ss2 = fma_f32x2(xe, xe, ss2);
+                }
+                float ss_lo, ss_hi;
+                f32x2_split(ss2, ss_lo, ss_hi);
+                float ss = ss_lo + ss_hi;
                 #pragma unroll
                 for (int off = LPT / 2; off > 0; off >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, off);
                 if (ss > 0.f) {
                     const float inv = rsqrtf(ss);
+                    const uint64_t inv2 = f32x2(inv, inv);
                     #pragma unroll
-                    for (int e = 0; e < EPL; ++e) acc[e] = fmaf(x[e], inv, acc[e]);
+                    for (int e = 0; e < EPL / 2; ++e)
+                        f32x2_split(fma_f32x2(f32x2(x[2 * e], x[2 * e + 1]), inv2, f32x2(acc[2 * e], acc[2 * e + 1])),
+                                    acc[2 * e], acc[2 * e + 1]);
                     m += 1.f;
                 }
             }
