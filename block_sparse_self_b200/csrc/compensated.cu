@@ -17,10 +17,10 @@
 //      so that the tensor cores see the centroids to about 16 bits.
 //   2. the block-sparse attention kernel over the kept blocks, writing its
 //      normalised output in fp32 and each row's softmax state (m, l).
-//   3. comp_pass_kernel: per query tile, S = Q kbar^T (hi and lo MMAs) over
-//      all centroids, kept blocks masked, an online softmax with the same
-//      lazy running max as the attention kernel, O = P vbar (hi and lo MMAs);
-//      then the two partial softmaxes are merged exactly:
+//   3. comp_pair_kernel: per pair of query tiles, S = Q kbar^T (hi and lo
+//      MMAs) over all centroids, kept blocks masked, an online softmax with
+//      the same lazy running max as the attention kernel, O = P vbar (hi and
+//      lo MMAs); then the two partial softmaxes are merged exactly:
 //        o = (l1 2^(m1-M) o1 + n_b 2^(m2-M) O2) / (l1 2^(m1-M) + n_b l2 2^(m2-M)),
 //      M = max(m1, m2), and written in the output dtype.
 #include "common.cuh"
@@ -94,25 +94,33 @@ __global__ void __launch_bounds__(256) centroid_kernel(const __nv_bfloat16 *__re
 // ---------------------------------------------------------------------------
 // 3. the centroid pass and the merge
 // ---------------------------------------------------------------------------
+// Two query tiles per CTA, as in the block-sparse attention kernel: warps 0-3
+// run tile A's softmax and merge, warps 4-7 tile B's, warp 8 the TMA loads,
+// warp 9 the MMAs and the tensor memory.  Both tiles walk every centroid tile
+// of the head, so each centroid tile (its kbar hi and lo parts, its vbar hi
+// and lo parts) is loaded once for the two of them; a tile's kept blocks and
+// the blocks past nb are masked.  Tensor memory: S_A, S_B (128 columns
+// each), O_A, O_B (D each); P is written over the first 64 columns of its S.
+// The MMAs go in the order QK_A(0) QK_B(0) | PV_A(c) QK_A(c+1) PV_B(c)
+// QK_B(c+1) | c = 0, 1, ..., so one tile's softmax runs while the other's
+// products do.
 template <int D>
-struct CompCfg {
+struct PairCfg {
     static constexpr int KSLABS = D / 64;
     static constexpr int SLAB = 128 * 128;            // 128 rows x 128 bytes
     static constexpr int TILE_BYTES = SLAB * KSLABS;  // one 128-row operand tile
-    static constexpr int NR = 2;                      // operand ring depth
-    static constexpr int O_COL = 128;                 // S at column 0, O after it
-    static constexpr int TMEM_COLS = 256;
-    static constexpr int N_BARS = 1 + 2 * NR + 1 + 1 + 1 + 1;
-    static constexpr int MASK_WORDS = kMaxCentroidTiles * 4;
-    static constexpr int SMEM = 1024 + (1 + NR) * TILE_BYTES + N_BARS * 8 + 64 + MASK_WORDS * 4 + kMaxCentroidTiles * 4;
-    static_assert(O_COL + D <= TMEM_COLS, "tensor memory");
-    static_assert(2 * (SMEM + 1024) <= 233472, "two CTAs per SM");
+    static constexpr int O_COL = 256;                 // S_A, S_B at 0 and 128; O_A, O_B at 256 and 256 + D
+    static constexpr int N_BARS = 1 + 4 + 3 * 2 + 1;
+    static constexpr int MASK_WORDS = kMaxCentroidTiles * 4;  // per tile: bit j set when block j is kept
+    // Q_A, Q_B, kbar hi, kbar lo, vbar hi, vbar lo
+    static constexpr int SMEM = 1024 + 6 * TILE_BYTES + N_BARS * 8 + 64 + 2 * MASK_WORDS * 4;
+    static_assert(SMEM <= 232448, "shared memory");
 };
-constexpr int kCompThreads = 192;  // warps 0-3 softmax/merge, 4 TMA producer, 5 MMA issuer and TMEM owner
+constexpr int kPairThreads = 320;
 constexpr float kCompMaxRowSum = 16777216.0f;
 
 struct CompArgs {
-    int S, nb, nct;            // positions per head, blocks per head, centroid tiles (ceil(nb / 128))
+    int S, nb, nct, nq;        // positions per head, blocks per head, centroid tiles, query tiles
     const int32_t *idx, *cnt;
     int cap, list_per_head;
     float scale_log2;
@@ -129,218 +137,224 @@ struct CompMaps {
 };
 
 template <int D>
-__global__ void __launch_bounds__(kCompThreads, 2)
-comp_pass_kernel(const __grid_constant__ CompMaps maps, const CompArgs a) {
-    using C = CompCfg<D>;
+__global__ void __launch_bounds__(kPairThreads, 1)
+comp_pair_kernel(const __grid_constant__ CompMaps maps, const CompArgs a) {
+    using C = PairCfg<D>;
     extern __shared__ uint8_t smem_raw[];
     uint8_t *base = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-    uint8_t *sQ = base;
-    uint8_t *sR = sQ + C::TILE_BYTES;  // [NR][TILE]
-    uint64_t *q_full = reinterpret_cast<uint64_t *>(sR + C::NR * C::TILE_BYTES);
-    uint64_t *r_full = q_full + 1;
-    uint64_t *r_empty = r_full + C::NR;
-    uint64_t *s_full = r_empty + C::NR;
-    uint64_t *p_full = s_full + 1;
-    uint64_t *pv_done = p_full + 1;
-    uint64_t *mma_done = pv_done + 1;
+    uint8_t *sQ = base;                               // [2][TILE]
+    uint8_t *sKh = sQ + 2 * C::TILE_BYTES;
+    uint8_t *sKl = sKh + C::TILE_BYTES;
+    uint8_t *sVh = sKl + C::TILE_BYTES;
+    uint8_t *sVl = sVh + C::TILE_BYTES;
+    uint64_t *q_full = reinterpret_cast<uint64_t *>(sVl + C::TILE_BYTES);
+    uint64_t *k_full = q_full + 1;
+    uint64_t *k_empty = k_full + 1;
+    uint64_t *v_full = k_empty + 1;
+    uint64_t *v_empty = v_full + 1;
+    uint64_t *s_full = v_empty + 1;   // [2]
+    uint64_t *p_full = s_full + 2;    // [2]
+    uint64_t *pv_done = p_full + 2;   // [2]
+    uint64_t *mma_done = pv_done + 2;
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(mma_done + 1);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
-    int *n_sched = reinterpret_cast<int *>(tmem_slot + 2);
-    int *list_ok = reinterpret_cast<int *>(tmem_slot + 3);
-    uint32_t *kept = reinterpret_cast<uint32_t *>(tmem_slot + 16);  // [MASK_WORDS] bit j: block j kept
-    int *sched = reinterpret_cast<int *>(kept + C::MASK_WORDS);     // centroid tiles with a skipped block
+    int *list_ok = reinterpret_cast<int *>(tmem_slot + 2);          // [2]
+    uint32_t *kept = reinterpret_cast<uint32_t *>(tmem_slot + 16);  // [2][MASK_WORDS]
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int qt = blockIdx.x, bh = blockIdx.y;
-    const size_t lrow = (a.list_per_head ? static_cast<size_t>(bh) * a.nb : 0) + qt;
-    const int32_t *list = a.idx + lrow * a.cap;
-    const int cnt = __ldg(a.cnt + lrow);
+    const int bh = blockIdx.y;
+    int qt[2];
+    const int32_t *list[2] = {nullptr, nullptr};
+    int cnt[2] = {0, 0};
+    bool valid[2];
+    for (int t = 0; t < 2; ++t) {
+        qt[t] = 2 * blockIdx.x + t;
+        valid[t] = qt[t] < a.nq;
+        if (valid[t]) {
+            const size_t lrow = (a.list_per_head ? static_cast<size_t>(bh) * a.nb : 0) + qt[t];
+            list[t] = a.idx + lrow * a.cap;
+            cnt[t] = __ldg(a.cnt + lrow);
+        }
+    }
 
     if (threadIdx.x == 0) {
         mbar_init(q_full, 1);
-        for (int s = 0; s < C::NR; ++s) {
-            mbar_init(&r_full[s], 1);
-            mbar_init(&r_empty[s], 1);
+        mbar_init(k_full, 1);
+        mbar_init(k_empty, 1);
+        mbar_init(v_full, 1);
+        mbar_init(v_empty, 1);
+        for (int t = 0; t < 2; ++t) {
+            mbar_init(&s_full[t], 1);
+            mbar_init(&p_full[t], 4);
+            mbar_init(&pv_done[t], 1);
         }
-        mbar_init(s_full, 1);
-        mbar_init(p_full, 4);
-        mbar_init(pv_done, 1);
         mbar_init(mma_done, 1);
         *abort_flag = 0;
         fence_mbar_init();
     }
-    for (int i = threadIdx.x; i < C::MASK_WORDS; i += blockDim.x) kept[i] = 0u;
-    if (warp == 0) {  // validate the list as the attention kernel does
-        bool ok = cnt >= 1 && cnt <= a.cap;
+    for (int i = threadIdx.x; i < 2 * C::MASK_WORDS; i += blockDim.x) kept[i] = 0u;
+    if (warp < 2) {  // warp t validates tile t's list as the attention kernel does
+        const int t = warp;
+        bool ok = valid[t] && cnt[t] >= 1 && cnt[t] <= a.cap;
         if (ok) {
-            for (int j = lane; j < cnt; j += 32) {
-                const int b = __ldg(list + j);
-                ok = ok && b >= 0 && b < a.nb && (j == 0 || __ldg(list + j - 1) < b);
+            for (int j = lane; j < cnt[t]; j += 32) {
+                const int b = __ldg(list[t] + j);
+                ok = ok && b >= 0 && b < a.nb && (j == 0 || __ldg(list[t] + j - 1) < b);
             }
         }
         ok = __all_sync(0xffffffffu, ok);
-        if (lane == 0) *list_ok = ok ? 1 : 0;
+        if (lane == 0) list_ok[t] = ok ? 1 : 0;
     }
-    if (warp == 5) {
-        tmem_alloc(tmem_slot, C::TMEM_COLS);
+    if (warp == 9) {
+        tmem_alloc(tmem_slot, 512);
         tmem_relinquish();
     }
     __syncthreads();
-    if (*list_ok) {
-        for (int j = threadIdx.x; j < cnt; j += blockDim.x) {
-            const int b = __ldg(list + j);
-            atomicOr(&kept[b >> 5], 1u << (b & 31));
-        }
-    }
-    __syncthreads();
-    if (threadIdx.x == 0) {
-        // the centroid tiles that hold at least one skipped block (none if the
-        // list is invalid: the output then keeps the main pass's zeros)
-        int n = 0;
-        if (*list_ok) {
-            for (int c = 0; c < a.nct; ++c) {
-                bool any = false;
-                for (int w = 0; w < 4; ++w) {
-                    const int b0 = c * kBlock + w * 32;
-                    if (b0 >= a.nb) break;
-                    const int valid = a.nb - b0 >= 32 ? 32 : a.nb - b0;
-                    const uint32_t vm = valid == 32 ? ~0u : ((1u << valid) - 1u);
-                    any = any || ((~kept[c * 4 + w]) & vm) != 0u;
-                }
-                if (any) sched[n++] = c;
+    bool act[2];
+    for (int t = 0; t < 2; ++t) {
+        act[t] = valid[t] && list_ok[t];
+        if (valid[t] && !list_ok[t] && threadIdx.x == 0) report(a.status, DEV_RUNTIME);
+        if (act[t])
+            for (int j = threadIdx.x; j < cnt[t]; j += blockDim.x) {
+                const int b = __ldg(list[t] + j);
+                atomicOr(&kept[t * C::MASK_WORDS + (b >> 5)], 1u << (b & 31));
             }
-        } else {
-            report(a.status, DEV_RUNTIME);
-        }
-        *n_sched = n;
     }
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
-    const int n = *n_sched;
+    const int nct = a.nct;
+    const bool any = act[0] || act[1];
+    const int last = act[1] ? 1 : 0;  // the tile whose MMAs are the last readers of a centroid tile
 
-    if (warp == 4) {
+    if (warp == 8) {
         // ================= TMA producer =================
-        // per scheduled centroid tile: kbar hi, kbar lo (for QK), vbar hi, vbar lo (for PV)
-        if (lane == 0 && n > 0) {
-            tma_prefetch_desc(&maps.q);
-            mbar_arrive_expect_tx(q_full, C::TILE_BYTES);
-            for (int s = 0; s < C::KSLABS; ++s)
-                tma_load_3d(sQ + s * C::SLAB, &maps.q, q_full, s * 64, qt * kBlock, bh);
-            const CUtensorMap *ops[4] = {&maps.khi, &maps.klo, &maps.vhi, &maps.vlo};
-            uint32_t lc = 0;
-            bool ok = true;
-            for (int j = 0; ok && j < n; ++j) {
-                const int c = sched[j];
-                for (int op = 0; ok && op < 4; ++op, ++lc) {
-                    const int slot = lc % C::NR;
-                    if (lc >= static_cast<uint32_t>(C::NR) &&
-                        !mbar_wait(&r_empty[slot], ((lc / C::NR) - 1) & 1, abort_flag)) {
-                        ok = false;
-                        break;
-                    }
-                    mbar_arrive_expect_tx(&r_full[slot], C::TILE_BYTES);
+        if (lane == 0 && any) {
+            tma_prefetch_desc(&maps.khi);
+            tma_prefetch_desc(&maps.vhi);
+            mbar_arrive_expect_tx(q_full, (act[0] + act[1]) * C::TILE_BYTES);
+            for (int t = 0; t < 2; ++t)
+                if (act[t])
                     for (int s = 0; s < C::KSLABS; ++s)
-                        tma_load_3d(sR + slot * C::TILE_BYTES + s * C::SLAB, ops[op], &r_full[slot], s * 64,
-                                    c * kBlock, bh);
+                        tma_load_3d(sQ + t * C::TILE_BYTES + s * C::SLAB, &maps.q, q_full, s * 64, qt[t] * kBlock, bh);
+            int kl = 0, vl = 0;  // centroid tiles whose K, V parts were issued
+            bool ok = true;
+            for (int c = 0; ok && c < nct; ++c) {
+                if (c > 0 && !mbar_wait(k_empty, (c - 1) & 1, abort_flag)) { ok = false; break; }
+                mbar_arrive_expect_tx(k_full, 2 * C::TILE_BYTES);
+                for (int s = 0; s < C::KSLABS; ++s) {
+                    tma_load_3d(sKh + s * C::SLAB, &maps.khi, k_full, s * 64, c * kBlock, bh);
+                    tma_load_3d(sKl + s * C::SLAB, &maps.klo, k_full, s * 64, c * kBlock, bh);
                 }
+                ++kl;
+                if (c > 0 && !mbar_wait(v_empty, (c - 1) & 1, abort_flag)) { ok = false; break; }
+                mbar_arrive_expect_tx(v_full, 2 * C::TILE_BYTES);
+                for (int s = 0; s < C::KSLABS; ++s) {
+                    tma_load_3d(sVh + s * C::SLAB, &maps.vhi, v_full, s * 64, c * kBlock, bh);
+                    tma_load_3d(sVl + s * C::SLAB, &maps.vlo, v_full, s * 64, c * kBlock, bh);
+                }
+                ++vl;
             }
             if (!ok) {
                 if (!*abort_flag) { report(a.status, DEV_TIMEOUT); *abort_flag = 1; }
                 // let the loads already issued land before the CTA exits
                 mbar_wait(q_full, 0, nullptr);
-                for (uint32_t c = lc > static_cast<uint32_t>(C::NR) ? lc - C::NR : 0; c < lc; ++c)
-                    mbar_wait(&r_full[c % C::NR], (c / C::NR) & 1, nullptr);
+                if (kl > 0) mbar_wait(k_full, (kl - 1) & 1, nullptr);
+                if (vl > 0) mbar_wait(v_full, (vl - 1) & 1, nullptr);
             }
         }
         __syncwarp();
-    } else if (warp == 5) {
+    } else if (warp == 9) {
         // ================= MMA issuer =================
-        // per tile j: QK(j) = Q khi^T + Q klo^T into S (after PV(j-1) has read
-        // the P over S), then PV(j) = P vhi + P vlo into O once P is written
-        if (lane == 0 && n > 0) {
+        if (lane == 0 && any) {
             constexpr uint32_t idesc_qk = idesc_bf16_f32(128, kBlock, false);
             constexpr uint32_t idesc_pv = idesc_bf16_f32(128, D, true);
             const uint64_t dQ = sdesc_sw128(smem_u32(sQ), 16, 1024);
-            const uint64_t dRk = sdesc_sw128(smem_u32(sR), 16, 1024);
-            const uint64_t dRv = sdesc_sw128(smem_u32(sR), C::SLAB, 1024);
+            const uint64_t dKh = sdesc_sw128(smem_u32(sKh), 16, 1024), dKl = sdesc_sw128(smem_u32(sKl), 16, 1024);
+            const uint64_t dVh = sdesc_sw128(smem_u32(sVh), C::SLAB, 1024), dVl = sdesc_sw128(smem_u32(sVl), C::SLAB, 1024);
             constexpr uint64_t kTile16 = C::TILE_BYTES >> 4;
-            uint32_t lc = 0;
-            bool ok = mbar_wait(q_full, 0, abort_flag);
-            for (int j = 0; ok && j < n; ++j) {
-                // QK(j)
-                const int s0 = lc % C::NR, s1 = (lc + 1) % C::NR;
-                ok = mbar_wait(&r_full[s0], (lc / C::NR) & 1, abort_flag) &&
-                     mbar_wait(&r_full[s1], ((lc + 1) / C::NR) & 1, abort_flag) &&
-                     (j == 0 || mbar_wait(pv_done, (j - 1) & 1, abort_flag));
-                if (!ok) break;
+            // S_t = Q_t kbar_hi^T + Q_t kbar_lo^T, once PV_t(c - 1) has read the P over S_t
+            auto qk = [&](int t, int c) -> bool {
+                if (!mbar_wait(k_full, c & 1, abort_flag)) return false;
+                if (c > 0 && !mbar_wait(&pv_done[t], (c - 1) & 1, abort_flag)) return false;
                 tc_fence_after();
+                const uint64_t q0 = dQ + t * kTile16;
+                const uint32_t d = tmem + t * 128;
                 #pragma unroll
                 for (int part = 0; part < 2; ++part) {
-                    const uint64_t k0 = dRk + ((part == 0 ? s0 : s1) * kTile16);
+                    const uint64_t k0 = part == 0 ? dKh : dKl;
                     #pragma unroll
                     for (int kk = 0; kk < D / 16; ++kk) {
                         const uint64_t off = static_cast<uint64_t>(((kk >> 2) * C::SLAB + (kk & 3) * 32) >> 4);
-                        umma_bf16(tmem, dQ + off, k0 + off, idesc_qk, (part > 0 || kk > 0) ? 1u : 0u);
+                        umma_bf16(d, q0 + off, k0 + off, idesc_qk, (part > 0 || kk > 0) ? 1u : 0u);
                     }
                 }
-                umma_commit(s_full);
-                umma_commit(&r_empty[s0]);
-                umma_commit(&r_empty[s1]);
-                lc += 2;
-                // PV(j)
-                const int s2 = lc % C::NR, s3 = (lc + 1) % C::NR;
-                ok = mbar_wait(p_full, j & 1, abort_flag) &&
-                     mbar_wait(&r_full[s2], (lc / C::NR) & 1, abort_flag) &&
-                     mbar_wait(&r_full[s3], ((lc + 1) / C::NR) & 1, abort_flag);
-                if (!ok) break;
+                umma_commit(&s_full[t]);
+                if (t == last) umma_commit(k_empty);
+                return true;
+            };
+            // O_t += P_t vbar_hi + P_t vbar_lo
+            auto pv = [&](int t, int c) -> bool {
+                if (!mbar_wait(&p_full[t], c & 1, abort_flag)) return false;
+                if (!mbar_wait(v_full, c & 1, abort_flag)) return false;
                 tc_fence_after();
+                const uint32_t d = tmem + C::O_COL + t * D, pa = tmem + t * 128;
                 #pragma unroll
                 for (int part = 0; part < 2; ++part) {
-                    const uint64_t v0 = dRv + ((part == 0 ? s2 : s3) * kTile16);
+                    const uint64_t v0 = part == 0 ? dVh : dVl;
                     #pragma unroll
                     for (int kk = 0; kk < kBlock / 16; ++kk)
-                        umma_bf16_ts(tmem + C::O_COL, tmem + kk * 8, v0 + static_cast<uint64_t>((kk * 2048) >> 4),
-                                     idesc_pv, (j > 0 || part > 0 || kk > 0) ? 1u : 0u);
+                        umma_bf16_ts(d, pa + kk * 8, v0 + static_cast<uint64_t>((kk * 2048) >> 4), idesc_pv,
+                                     (c > 0 || part > 0 || kk > 0) ? 1u : 0u);
                 }
-                umma_commit(pv_done);
-                umma_commit(&r_empty[s2]);
-                umma_commit(&r_empty[s3]);
-                lc += 2;
-            }
+                umma_commit(&pv_done[t]);
+                if (t == last) umma_commit(v_empty);
+                return true;
+            };
+            bool ok = mbar_wait(q_full, 0, abort_flag);
+            for (int t = 0; ok && t < 2; ++t)
+                if (act[t]) ok = qk(t, 0);
+            for (int c = 0; ok && c < nct; ++c)
+                for (int t = 0; ok && t < 2; ++t)
+                    if (act[t]) {
+                        ok = pv(t, c);
+                        if (ok && c + 1 < nct) ok = qk(t, c + 1);
+                    }
             if (!ok && !*abort_flag) { report(a.status, DEV_TIMEOUT); *abort_flag = 1; }
             umma_commit(mma_done);
             mbar_wait(mma_done, 0, nullptr);
         }
         __syncwarp();
     } else {
-        // ================= softmax over the centroids, then the merge (warps 0-3) =================
-        const int wq = warp, row = wq * 32 + lane;
-        const int rg = qt * kBlock + row;
+        // ================= softmax over the centroids, then the merge (warps 0-7) =================
+        const int t = warp >> 2, wq = warp & 3, row = wq * 32 + lane;
+        const int rg = (valid[t] ? qt[t] : 0) * kBlock + row;
         const uint32_t t_lane = tmem + (static_cast<uint32_t>(wq * 32) << 16);
+        const uint32_t s_col = t * 128, o_col = C::O_COL + t * D;
+        const uint32_t *kept_t = kept + t * C::MASK_WORDS;
         const float sl2 = a.scale_log2;
         float m_ref = -INFINITY, l_sum = 0.f;
         bool ok = true;
-        for (int j = 0; j < n; ++j) {
-            const int c = sched[j];
-            if (!__all_sync(0xffffffffu, mbar_wait(s_full, j & 1, abort_flag))) { ok = false; break; }
+        const int n = act[t] ? nct : 0;
+        for (int c = 0; c < n; ++c) {
+            if (!__all_sync(0xffffffffu, mbar_wait(&s_full[t], c & 1, abort_flag))) { ok = false; break; }
             tc_fence_after();
             uint32_t x[kBlock];
             #pragma unroll
             for (int u = 0; u < kBlock / 32; ++u)
-                tmem_ld32(t_lane + 32 * u, *reinterpret_cast<uint32_t(*)[32]>(&x[32 * u]));
+                tmem_ld32(t_lane + s_col + 32 * u, *reinterpret_cast<uint32_t(*)[32]>(&x[32 * u]));
             tmem_ld_wait();
             // a centroid takes part iff its block exists and is not kept
             uint32_t skip[4];
             #pragma unroll
             for (int w = 0; w < 4; ++w) {
                 const int b0 = c * kBlock + w * 32;
-                const int valid = a.nb - b0 >= 32 ? 32 : (a.nb - b0 > 0 ? a.nb - b0 : 0);
-                const uint32_t vm = valid == 32 ? ~0u : ((1u << valid) - 1u);
-                skip[w] = ~kept[c * 4 + w] & vm;
+                const int nv = a.nb - b0 >= 32 ? 32 : (a.nb - b0 > 0 ? a.nb - b0 : 0);
+                const uint32_t vm = nv == 32 ? ~0u : ((1u << nv) - 1u);
+                skip[w] = ~kept_t[c * 4 + w] & vm;
             }
-            // per 32 columns, a branch the whole CTA takes alike (the mask
+            // per 32 columns, a branch the whole tile takes alike (the mask
             // is the query tile's): most words skip every centroid
             auto apply_mask = [&]() {
                 #pragma unroll
@@ -378,7 +392,7 @@ comp_pass_kernel(const __grid_constant__ CompMaps maps, const CompArgs a) {
                 }
                 return fmaxf(fmaxf(m4[0], m4[1]), fmaxf(m4[2], m4[3]));
             };
-            if (m_ref == -INFINITY) m_ref = raw_max() * sl2;
+            if (m_ref == -INFINITY) m_ref = raw_max() * sl2;  // may stay -inf (every centroid of the tile kept)
             float rs = 0.f;
             #pragma unroll 1
             for (int pass = 0; pass < 2; ++pass) {
@@ -387,12 +401,12 @@ comp_pass_kernel(const __grid_constant__ CompMaps maps, const CompArgs a) {
                 if (pass == 1 || !__any_sync(0xffffffffu, need)) break;
                 #pragma unroll
                 for (int u = 0; u < kBlock / 32; ++u)
-                    tmem_ld32(t_lane + 32 * u, *reinterpret_cast<uint32_t(*)[32]>(&x[32 * u]));
+                    tmem_ld32(t_lane + s_col + 32 * u, *reinterpret_cast<uint32_t(*)[32]>(&x[32 * u]));
                 tmem_ld_wait();
                 apply_mask();
                 const float m_new = need ? fmaxf(m_ref, raw_max() * sl2) : m_ref;
-                if (j > 0) {
-                    if (!__all_sync(0xffffffffu, mbar_wait(pv_done, (j - 1) & 1, abort_flag))) {
+                if (c > 0) {
+                    if (!__all_sync(0xffffffffu, mbar_wait(&pv_done[t], (c - 1) & 1, abort_flag))) {
                         ok = false;
                     } else {
                         tc_fence_after();
@@ -400,11 +414,11 @@ comp_pass_kernel(const __grid_constant__ CompMaps maps, const CompArgs a) {
                         #pragma unroll 1
                         for (int u = 0; u < D / 8; ++u) {
                             uint32_t o[8];
-                            tmem_ld8(t_lane + C::O_COL + 8 * u, o);
+                            tmem_ld8(t_lane + o_col + 8 * u, o);
                             tmem_ld_wait();
                             #pragma unroll
                             for (int e = 0; e < 8; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * alpha);
-                            tmem_st8(t_lane + C::O_COL + 8 * u, o);
+                            tmem_st8(t_lane + o_col + 8 * u, o);
                         }
                         tmem_st_wait();
                         l_sum *= alpha;
@@ -415,62 +429,64 @@ comp_pass_kernel(const __grid_constant__ CompMaps maps, const CompArgs a) {
             }
             if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
             l_sum += rs;
-            tmem_st32(t_lane, *reinterpret_cast<const uint32_t(*)[32]>(&x[0]));
-            tmem_st32(t_lane + 32, *reinterpret_cast<const uint32_t(*)[32]>(&x[32]));
+            tmem_st32(t_lane + s_col, *reinterpret_cast<const uint32_t(*)[32]>(&x[0]));
+            tmem_st32(t_lane + s_col + 32, *reinterpret_cast<const uint32_t(*)[32]>(&x[32]));
             tmem_st_wait();
             tc_fence_before();
             __syncwarp();
-            if (lane == 0) mbar_arrive(p_full);
+            if (lane == 0) mbar_arrive(&p_full[t]);
         }
         if (!ok && !*abort_flag) { report(a.status, DEV_TIMEOUT); *abort_flag = 1; }
         bool have_c = ok && n > 0;
-        if (have_c && !__all_sync(0xffffffffu, mbar_wait(pv_done, (n - 1) & 1, abort_flag))) {
+        if (have_c && !__all_sync(0xffffffffu, mbar_wait(&pv_done[t], (n - 1) & 1, abort_flag))) {
             have_c = false;
             if (!*abort_flag) { report(a.status, DEV_TIMEOUT); *abort_flag = 1; }
         }
         if (have_c) tc_fence_after();
-        // ---- merge with the main pass and write the row ----
-        // main pass: o1 (normalised) with state (m1, l1); centroids: O2 (not
-        // normalised) with state (m2, l2), each centroid weighted by n_b
-        const size_t prow = static_cast<size_t>(bh) * a.S + rg;
-        const float2 st = a.stats[prow];
-        const float m2 = have_c ? m_ref : -INFINITY;
-        const float M = fmaxf(st.x, m2);
-        const float f1 = st.x == -INFINITY ? 0.f : ex2_approx(st.x - M);
-        const float f2 = m2 == -INFINITY ? 0.f : a.weight * ex2_approx(m2 - M);
-        const float w1 = st.y * f1;
-        const float den = w1 + f2 * (have_c ? l_sum : 0.f);
-        const float c1 = den > 0.f ? w1 / den : 0.f, c2 = den > 0.f ? f2 / den : 0.f;
-        const float *o1 = a.o1 + prow * D;
-        #pragma unroll 1
-        for (int u = 0; u < D / 8; ++u) {
-            uint32_t o2[8] = {0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u};
-            if (have_c) {
-                tmem_ld8(t_lane + C::O_COL + 8 * u, o2);
-                tmem_ld_wait();
-            }
-            const float4 fa = reinterpret_cast<const float4 *>(o1 + 8 * u)[0];
-            const float4 fb = reinterpret_cast<const float4 *>(o1 + 8 * u)[1];
-            const float r0 = c1 * fa.x + c2 * __uint_as_float(o2[0]), r1 = c1 * fa.y + c2 * __uint_as_float(o2[1]);
-            const float r2 = c1 * fa.z + c2 * __uint_as_float(o2[2]), r3 = c1 * fa.w + c2 * __uint_as_float(o2[3]);
-            const float r4 = c1 * fb.x + c2 * __uint_as_float(o2[4]), r5 = c1 * fb.y + c2 * __uint_as_float(o2[5]);
-            const float r6 = c1 * fb.z + c2 * __uint_as_float(o2[6]), r7 = c1 * fb.w + c2 * __uint_as_float(o2[7]);
-            if (a.out_f32) {
-                float4 *dst = reinterpret_cast<float4 *>(static_cast<float *>(a.out) + prow * D + 8 * u);
-                dst[0] = make_float4(r0, r1, r2, r3);
-                dst[1] = make_float4(r4, r5, r6, r7);
-            } else {
-                uint4 *dst = reinterpret_cast<uint4 *>(static_cast<__nv_bfloat16 *>(a.out) + prow * D + 8 * u);
-                *dst = make_uint4(pack_bf16x2(r0, r1), pack_bf16x2(r2, r3), pack_bf16x2(r4, r5), pack_bf16x2(r6, r7));
+        if (valid[t]) {
+            // ---- merge with the main pass and write the row ----
+            // main pass: o1 (normalised) with state (m1, l1); centroids: O2 (not
+            // normalised) with state (m2, l2), each centroid weighted by n_b
+            const size_t prow = static_cast<size_t>(bh) * a.S + rg;
+            const float2 st = a.stats[prow];
+            const float m2 = have_c ? m_ref : -INFINITY;
+            const float M = fmaxf(st.x, m2);
+            const float f1 = st.x == -INFINITY ? 0.f : ex2_approx(st.x - M);
+            const float f2 = m2 == -INFINITY ? 0.f : a.weight * ex2_approx(m2 - M);
+            const float w1 = st.y * f1;
+            const float den = w1 + f2 * (have_c ? l_sum : 0.f);
+            const float c1 = den > 0.f ? w1 / den : 0.f, c2 = den > 0.f ? f2 / den : 0.f;
+            const float *o1 = a.o1 + prow * D;
+            #pragma unroll 1
+            for (int u = 0; u < D / 8; ++u) {
+                uint32_t o2[8] = {0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u};
+                if (have_c) {
+                    tmem_ld8(t_lane + o_col + 8 * u, o2);
+                    tmem_ld_wait();
+                }
+                const float4 fa = reinterpret_cast<const float4 *>(o1 + 8 * u)[0];
+                const float4 fb = reinterpret_cast<const float4 *>(o1 + 8 * u)[1];
+                const float r0 = c1 * fa.x + c2 * __uint_as_float(o2[0]), r1 = c1 * fa.y + c2 * __uint_as_float(o2[1]);
+                const float r2 = c1 * fa.z + c2 * __uint_as_float(o2[2]), r3 = c1 * fa.w + c2 * __uint_as_float(o2[3]);
+                const float r4 = c1 * fb.x + c2 * __uint_as_float(o2[4]), r5 = c1 * fb.y + c2 * __uint_as_float(o2[5]);
+                const float r6 = c1 * fb.z + c2 * __uint_as_float(o2[6]), r7 = c1 * fb.w + c2 * __uint_as_float(o2[7]);
+                if (a.out_f32) {
+                    float4 *dst = reinterpret_cast<float4 *>(static_cast<float *>(a.out) + prow * D + 8 * u);
+                    dst[0] = make_float4(r0, r1, r2, r3);
+                    dst[1] = make_float4(r4, r5, r6, r7);
+                } else {
+                    uint4 *dst = reinterpret_cast<uint4 *>(static_cast<__nv_bfloat16 *>(a.out) + prow * D + 8 * u);
+                    *dst = make_uint4(pack_bf16x2(r0, r1), pack_bf16x2(r2, r3), pack_bf16x2(r4, r5), pack_bf16x2(r6, r7));
+                }
             }
         }
     }
 
     tc_fence_before();
     __syncthreads();
-    if (warp == 5) {
+    if (warp == 9) {
         tc_fence_after();
-        tmem_dealloc(tmem, C::TMEM_COLS);
+        tmem_dealloc(tmem, 512);
     }
 }
 
@@ -495,7 +511,7 @@ CompLayout comp_layout(int BH, int S, int D, int out_f32) {
 
 template <int D>
 vsa_status run_compensated(const AttnLaunch &L, void *workspace, int *status, cudaStream_t st) {
-    using C = CompCfg<D>;
+    using C = PairCfg<D>;
     const int nb = L.S / kBlock;
     const CompLayout lay = comp_layout(L.BH, L.S, D, L.out_f32);
     char *ws = static_cast<char *>(workspace);
@@ -524,13 +540,14 @@ vsa_status run_compensated(const AttnLaunch &L, void *workspace, int *status, cu
                     make_tile_map(&maps.klo, klo, D, nb, L.BH, 128) && make_tile_map(&maps.vhi, vhi, D, nb, L.BH, 128) &&
                     make_tile_map(&maps.vlo, vlo, D, nb, L.BH, 128);
     if (!ok) return fail(VSA_ERR_CUDA, "cuTensorMapEncodeTiled failed (driver entry point or arguments)");
-    auto kern = comp_pass_kernel<D>;
+    auto kern = comp_pair_kernel<D>;
     e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
     if (e != cudaSuccess) return check_cuda(e, "cudaFuncSetAttribute(compensation pass)");
     CompArgs a;
     a.S = L.S;
     a.nb = nb;
     a.nct = (nb + kBlock - 1) / kBlock;
+    a.nq = nb;
     a.idx = L.idx;
     a.cnt = L.cnt;
     a.cap = L.cap;
@@ -542,7 +559,7 @@ vsa_status run_compensated(const AttnLaunch &L, void *workspace, int *status, cu
     a.out = L.o;
     a.out_f32 = L.out_f32;
     a.status = status;
-    kern<<<dim3(nb, L.BH), kCompThreads, C::SMEM, st>>>(maps, a);
+    kern<<<dim3((nb + 1) / 2, L.BH), kPairThreads, C::SMEM, st>>>(maps, a);
     return check_cuda(cudaGetLastError(), "compensation pass launch");
 }
 
