@@ -295,3 +295,21 @@ def test_fused_scores_topk_argument_errors(L):
     assert call(nb=1025, k=100, cap=102) == vsa.ERR_UNSUPPORTED
     assert "at most 1024" in vsa.last_error()
     assert call(D=96) == vsa.ERR_UNSUPPORTED
+
+
+def test_header_is_plain_c(tmp_path):
+    """include/vsa.h is a C header: it compiles as C99 and as C++17 on its own,
+    with no CUDA or torch types in the signatures."""
+    import os
+    import shutil
+    import subprocess
+    header = os.path.abspath(vsa.HEADER_PATH)
+    src = tmp_path / "use.c"
+    src.write_text('#include "%s"\nint main(void) { return vsa_last_error() == 0; }\n' % header)
+    for compiler, std in (("gcc", "-std=c99"), ("g++", "-std=c++17")):
+        if shutil.which(compiler) is None:
+            pytest.skip(f"{compiler} not found")
+        lang = ["-x", "c++"] if compiler == "g++" else []
+        r = subprocess.run([compiler, std, "-Wall", "-Werror", "-fsyntax-only", *lang, str(src)],
+                           capture_output=True, text=True)
+        assert r.returncode == 0, r.stderr
