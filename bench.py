@@ -249,7 +249,7 @@ def time_steps(fn, steps: int, warmup: int, dist_on: bool):
     return s.elapsed_time(e) / steps
 
 
-def run_e2e(w, step, q, k, v, steps: int):
+def run_e2e(w, step, q, k, v, steps: int, groups: int = 8):
     """Same metric through the public API with host buffers: spade_attention_host
     takes Q, K, V in pinned host memory and returns O there; every step's H2D
     copies and D2H copy are inside the timed region (the call overlaps the
@@ -260,7 +260,7 @@ def run_e2e(w, step, q, k, v, steps: int):
     kw = dict(topk=w.k, n_sink_blocks=w.n_sink_blocks, diag_halfwidth=w.diag_halfwidth)
 
     def once():
-        vsa.spade_attention_host(qh, kh, vh, w.grid, list(w.tiles), out=oh, **kw)
+        vsa.spade_attention_host(qh, kh, vh, w.grid, list(w.tiles), out=oh, chunks=groups, **kw)
 
     once()
     torch.cuda.synchronize()
@@ -611,10 +611,11 @@ def run_ours(args, w):
 
     e2e = None
     if not args.no_e2e:
-        e_ms, h2d, d2h = run_e2e(w, step, q, k, v, max(2, args.steps // 2))
+        groups = args.e2e_groups if args.e2e_groups > 0 else w.B * w.heads
+        e_ms, h2d, d2h = run_e2e(w, step, q, k, v, max(2, args.steps // 2), groups)
         e_max = reduce_over_ranks(e_ms, "max", dist_on, "cuda")
         e2e = {"value": total_flops / e_max / 1e9, "unit": UNIT, "ms_per_step": e_max,
-               "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h}
+               "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "groups": groups}
 
     extra = None
     want = () if args.no_extra else tuple(args.extras.split(","))
@@ -708,6 +709,8 @@ def main():
     ap.add_argument("--impl", choices=("ours", "reference"), default="ours")
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=sorted(WORKLOADS))
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--e2e-groups", type=int, default=0,
+                    help="groups of (b, head) rows in the host-buffer run (0: one group per (b, head))")
     ap.add_argument("--no-extra", action="store_true")
     ap.add_argument("--extras", default=",".join(EXTRAS),
                     help="comma-separated secondary lines to run (%s); --no-extra runs none" % ",".join(EXTRAS))

@@ -628,16 +628,16 @@ def spade_attention(q, k, v, grid, tiles, budget: Optional[float] = None, topk: 
     return o
 
 
-def spade_attention_host(q, k, v, grid, tiles, out: Optional[torch.Tensor] = None, chunks: int = 8,
+def spade_attention_host(q, k, v, grid, tiles, out: Optional[torch.Tensor] = None, chunks: Optional[int] = None,
                          device=None, budget: Optional[float] = None, topk: Optional[int] = None,
                          n_sink_blocks: int = 1, diag_halfwidth: int = 0, scale: Optional[float] = None,
                          out_dtype=None) -> torch.Tensor:
     """spade_attention for bf16 inputs and an output in (pinned) host memory,
     through vsa_spade_attention_host: the B*H (batch, head) rows are taken in
-    `chunks` groups whose copies to the device and back overlap the kernels
-    of other groups (see include/vsa.h).  Allocates the device workspace and
-    `out` (pinned) when not given, and returns `out` once the call's stream
-    has finished with it."""
+    `chunks` groups (default: one per (batch, head)) whose copies to the
+    device and back overlap the kernels of other groups (see include/vsa.h).
+    Allocates the device workspace and `out` (pinned) when not given, and
+    returns `out` once the call's stream has finished with it."""
     for t, nm in ((q, "q"), (k, "k"), (v, "v")):
         if not isinstance(t, torch.Tensor) or t.is_cuda or not t.is_contiguous():
             raise ValueError(f"{nm} must be a contiguous host tensor")
@@ -646,6 +646,7 @@ def spade_attention_host(q, k, v, grid, tiles, out: Optional[torch.Tensor] = Non
     B, H, S, D = _bhsd(q, "q")
     if tuple(k.shape) != (B, H, S, D) or tuple(v.shape) != (B, H, S, D):
         raise ValueError("q/k/v shapes must match exactly")
+    chunks = B * H if chunks is None else int(chunks)
     odt = _out_dtype(out_dtype, q)
     if out is None:
         out = torch.empty(q.shape, dtype=odt, pin_memory=True)
