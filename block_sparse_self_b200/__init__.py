@@ -566,9 +566,15 @@ def _select_blocks(scores, kk, n_sink_blocks, diag_halfwidth, top_p, top_p_scale
 def spade_attention(q, k, v, grid, tiles, budget: Optional[float] = None, topk: Optional[int] = None,
                     n_sink_blocks: int = 1, diag_halfwidth: int = 0, scale: Optional[float] = None,
                     out_dtype=None, return_intermediates: bool = False, tiled: Optional[bool] = None,
-                    top_p: Optional[float] = None, top_p_scale: Optional[float] = None):
+                    top_p: Optional[float] = None, top_p_scale: Optional[float] = None,
+                    compensate: bool = False):
     """Adaptive tiling -> permutation -> min/max block scores -> top-k + sink +
     diagonal -> block-sparse attention -> inverse permutation, all on the GPU.
+
+    compensate=True takes the Recipe's attention call: every key block a
+    query block skips still takes part as its centroid
+    (centroid_compensated_attention); it runs on explicit permuted copies,
+    128-token blocks and grids the tiles divide.
 
     Every candidate tile must have the same volume (the block size).  With a
     single candidate the tiling choice is skipped (choice 0 for every head).
@@ -597,6 +603,12 @@ def spade_attention(q, k, v, grid, tiles, budget: Optional[float] = None, topk: 
     nb = _grid_tokens(pgrid) // block
     kk = topk if topk is not None else topk_budget(nb, budget if budget is not None else 0.17)
     can_tile = block in (32, 64, 128) and tiled_supported(tiles)
+    if compensate:
+        if block != 128:
+            raise NotImplementedError("compensated attention takes 128-token blocks")
+        if tiled:
+            raise ValueError("compensated attention runs on explicit permuted copies (tiled=False)")
+        tiled = False
     if tiled is None:
         tiled = can_tile
     elif tiled and not can_tile:
@@ -620,7 +632,10 @@ def spade_attention(q, k, v, grid, tiles, budget: Optional[float] = None, topk: 
         kmax, kmin = block_summaries(kp, block)
         scores = block_scores(qmax, qmin, kmax, kmin)
         idx, cnt = _select_blocks(scores, kk, n_sink_blocks, diag_halfwidth, top_p, top_p_scale, D)
-        op = block_sparse_attention(qp, kp, vp, idx, cnt, block, 0, scale, out_dtype)
+        if compensate:
+            op = centroid_compensated_attention(qp, kp, vp, idx, cnt, block, scale, out_dtype)
+        else:
+            op = block_sparse_attention(qp, kp, vp, idx, cnt, block, 0, scale, out_dtype)
         o = unpermute(op, grid, tiles, choice)
     if return_intermediates:
         return o, dict(choice=choice, qp=qp, kp=kp, vp=vp, qmax=qmax, qmin=qmin, kmax=kmax, kmin=kmin,
