@@ -600,8 +600,11 @@ vsa_status vsa_centroid_compensated_attention(const void *q, const void *k, cons
     VSA_REQUIRE(workspace != nullptr && (reinterpret_cast<uintptr_t>(workspace) & 255u) == 0,
                 "workspace must be a non-NULL 256-byte aligned device pointer");
     VSA_REQUIRE(workspace_bytes >= need, "workspace holds %zu bytes, %zu needed", workspace_bytes, need);
-    VSA_REQUIRE(!overlaps(workspace, need, o, static_cast<size_t>(B) * n_heads * S * D * esize_of(out_dtype)),
-                "workspace must not overlap o");
+    const size_t in_bytes = static_cast<size_t>(B) * n_heads * S * D * 2;
+    VSA_REQUIRE(!overlaps(workspace, need, o, static_cast<size_t>(B) * n_heads * S * D * esize_of(out_dtype)) &&
+                    !overlaps(workspace, need, q, in_bytes) && !overlaps(workspace, need, k, in_bytes) &&
+                    !overlaps(workspace, need, v, in_bytes),
+                "workspace must not overlap q, k, v or o");
     AttnLaunch L{};
     L.q = q; L.k = k; L.v = v; L.o = o;
     L.out_f32 = out_dtype == VSA_F32;

@@ -332,7 +332,7 @@ vsa_status vsa_block_sparse_attention(const void *q, const void *k, const void *
  *   idx/cnt  block lists as for vsa_block_sparse_attention (list_per_head)
  *   block    128 (S % 128 == 0); at most 8192 blocks per head
  *   workspace DEVICE scratch of vsa_centroid_compensated_attention_workspace_size
- *            bytes, 256-byte aligned, not overlapping o: the centroids (as
+ *            bytes, 256-byte aligned, not overlapping q, k, v or o: the centroids (as
  *            bf16 pairs hi + lo, about 16 significant bits), each row's
  *            softmax state over its kept keys and, for a bf16 output, the
  *            fp32 output of the kept keys

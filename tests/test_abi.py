@@ -277,6 +277,7 @@ def test_compensated_attention_argument_errors(L):
     assert "needed" in vsa.last_error()
     assert call(ws=ctypes.c_void_p((1 << 24) + 16)) == vsa.ERR_INVALID_ARGUMENT
     assert call(ws=ctypes.c_void_p(0x400000)) == vsa.ERR_INVALID_ARGUMENT  # workspace over o
+    assert call(ws=ctypes.c_void_p(0x100000)) == vsa.ERR_INVALID_ARGUMENT  # workspace over k
     assert call(o=FAKE) == vsa.ERR_INVALID_ARGUMENT                        # o over q
 
 
