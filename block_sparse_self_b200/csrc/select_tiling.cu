@@ -52,6 +52,69 @@ struct SelArgs {
     float *partial;     // [BH][n_regions][2][tiles.n]: SICS sums, then counts of tiles with a query
 };
 
+// Candidate tiles inside one region, candidate by candidate (the same item
+// layout in every region, precomputed on the host): warp w takes items w,
+// w + kWarps, ...; it sums the tile's cells, four channels per lane, and turns
+// |sum|^2 into the tile's SICS.  cell_sum is [cells][D], cell_cnt [cells].
+__device__ void region_tile_pass(const SelArgs &a, const float *cell_sum, const float *cell_cnt, float *tile_val,
+                                 float *tile_used, int warp, int lane) {
+    int item = 0;
+    for (int c = 0; c < a.tiles.n; ++c) {
+        const int kt = a.cpt_t[c], kh = a.cpt_h[c], kw = a.cpt_w[c];
+        for (int at = 0; at < a.tpr_t[c]; ++at)
+            for (int ah = 0; ah < a.tpr_h[c]; ++ah)
+                for (int aw = 0; aw < a.tpr_w[c]; ++aw, ++item) {
+                    if (item % kWarps != warp) continue;  // warp-uniform
+                    float sq = 0.f, m = 0.f;
+                    for (int d4 = lane; d4 < a.D / 4; d4 += 32) {
+                        float4 sum = make_float4(0.f, 0.f, 0.f, 0.f);
+                        for (int x = 0; x < kt; ++x)
+                            for (int y = 0; y < kh; ++y) {
+                                const int row = ((at * kt + x) * a.nch + ah * kh + y) * a.ncw + aw * kw;
+                                for (int z = 0; z < kw; ++z) {
+                                    const float4 v = reinterpret_cast<const float4 *>(cell_sum + (row + z) * a.D)[d4];
+                                    sum.x += v.x;
+                                    sum.y += v.y;
+                                    sum.z += v.z;
+                                    sum.w += v.w;
+                                }
+                            }
+                        sq = fmaf(sum.x, sum.x, sq);
+                        sq = fmaf(sum.y, sum.y, sq);
+                        sq = fmaf(sum.z, sum.z, sq);
+                        sq = fmaf(sum.w, sum.w, sq);
+                    }
+                    for (int x = 0; x < kt; ++x)
+                        for (int y = 0; y < kh; ++y) {
+                            const int row = ((at * kt + x) * a.nch + ah * kh + y) * a.ncw + aw * kw;
+                            for (int z = 0; z < kw; ++z) m += cell_cnt[row + z];
+                        }
+                    #pragma unroll
+                    for (int off = 16; off > 0; off >>= 1) sq += __shfl_down_sync(0xffffffffu, sq, off);
+                    if (lane == 0) {
+                        tile_val[item] = m >= 2.f ? (sq - m) / (m * (m - 1.f)) : 0.f;
+                        tile_used[item] = m >= 1.f ? 1.f : 0.f;
+                    }
+                }
+    }
+}
+
+// Candidate c's sum of tile SICS over this region and its count of tiles that
+// hold a non-zero query, into the [BH][n_regions][2][n_tiles] partials.
+__device__ void region_write(const SelArgs &a, const float *tile_val, const float *tile_used, int region, int bh,
+                             int c) {
+    const int first = a.item_first[c], n = a.item_first[c + 1] - first;
+    float s = 0.f, used = 0.f;
+    for (int i = 0; i < n; ++i) {
+        s += tile_val[first + i];
+        used += tile_used[first + i];
+    }
+    const int n_regions = a.nrt * a.nrh * a.nrw;
+    float *out = a.partial + (static_cast<size_t>(bh) * n_regions + region) * 2 * a.tiles.n;
+    out[c] = s;
+    out[a.tiles.n + c] = used;
+}
+
 // LPT lanes share a query row; each lane takes CPL of the row's 16-byte chunks,
 // chunk lt + LPT u (lt = lane % LPT), so one load instruction reads LPT
 // consecutive chunks of every row it touches.  Four CTAs per SM (64
@@ -119,7 +182,7 @@ __global__ void __launch_bounds__(kThreads, 4) sics_partial_kernel(const SelArgs
                 const uint4 *row = cell_q + static_cast<size_t>(cell_off[valid ? tok : 0]) * CPR;
                 #pragma unroll
                 for (int u = 0; u < CPL; ++u)
-                    raw[pb][u] = valid ? __ldcs(row + LPT * u) : make_uint4(0u, 0u, 0u, 0u);
+                    raw[pb][u] = valid ? ld_stream_l2_256(row + LPT * u) : make_uint4(0u, 0u, 0u, 0u);
             }
             #pragma unroll
             for (int pb = 0; pb < NB; ++pb) {
@@ -140,17 +203,27 @@ __global__ void __launch_bounds__(kThreads, 4) sics_partial_kernel(const SelArgs
                         for (int e = 0; e < EPC; ++e) x[u * EPC + e] = fv[e];
                     }
                 }
-                // two-wide fp32 FMAs (each half rounds as the scalar FMA):
-                // the sum of squares in two interleaved partial sums, the
-                // unit vector's accumulation element by element as before
-                uint64_t ss2 = f32x2(0.f, 0.f);
-                #pragma unroll
-                for (int e = 0; e < EPL / 2; ++e) {
-                    const uint64_t xe = f32x2(x[2 * e], x[2 * e + 1]);
-                    ss2 = fma_f32x2(xe, xe, ss2);
+                // the sum of squares in two interleaved partial sums; bf16
+                // rows square their packed pairs with mixed-precision FMAs, so
+                // the norm does not wait for the unpacking (2 % faster)
+                float ss_lo = 0.f, ss_hi = 0.f;
+                if constexpr (sizeof(T) == 2) {
+                    #pragma unroll
+                    for (int u = 0; u < CPL; ++u) {
+                        sq_bf16x2_f32(raw[pb][u].x, ss_lo, ss_hi);
+                        sq_bf16x2_f32(raw[pb][u].y, ss_lo, ss_hi);
+                        sq_bf16x2_f32(raw[pb][u].z, ss_lo, ss_hi);
+                        sq_bf16x2_f32(raw[pb][u].w, ss_lo, ss_hi);
+                    }
+                } else {
+                    uint64_t ss2 = f32x2(0.f, 0.f);
+                    #pragma unroll
+                    for (int e = 0; e < EPL / 2; ++e) {
+                        const uint64_t xe = f32x2(x[2 * e], x[2 * e + 1]);
+                        ss2 = fma_f32x2(xe, xe, ss2);
+                    }
+                    f32x2_split(ss2, ss_lo, ss_hi);
                 }
-                float ss_lo, ss_hi;
-                f32x2_split(ss2, ss_lo, ss_hi);
                 float ss = ss_lo + ss_hi;
                 #pragma unroll
                 for (int off = LPT / 2; off > 0; off >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, off);
@@ -182,62 +255,9 @@ __global__ void __launch_bounds__(kThreads, 4) sics_partial_kernel(const SelArgs
     }
     __syncthreads();
 
-    // candidate tiles inside this region, candidate by candidate (the same
-    // item layout in every region, precomputed on the host): sum the tile's
-    // cells, four channels per lane, and turn |sum|^2 into the tile's SICS
-    int item = 0;
-    for (int c = 0; c < a.tiles.n; ++c) {
-        const int kt = a.cpt_t[c], kh = a.cpt_h[c], kw = a.cpt_w[c];
-        for (int at = 0; at < a.tpr_t[c]; ++at)
-            for (int ah = 0; ah < a.tpr_h[c]; ++ah)
-                for (int aw = 0; aw < a.tpr_w[c]; ++aw, ++item) {
-                    if (item % kWarps != warp) continue;  // warp-uniform
-                    float sq = 0.f, m = 0.f;
-                    for (int d4 = lane; d4 < a.D / 4; d4 += 32) {
-                        float4 sum = make_float4(0.f, 0.f, 0.f, 0.f);
-                        for (int x = 0; x < kt; ++x)
-                            for (int y = 0; y < kh; ++y) {
-                                const int row = ((at * kt + x) * a.nch + ah * kh + y) * a.ncw + aw * kw;
-                                for (int z = 0; z < kw; ++z) {
-                                    const float4 v = reinterpret_cast<const float4 *>(cell_sum + (row + z) * a.D)[d4];
-                                    sum.x += v.x;
-                                    sum.y += v.y;
-                                    sum.z += v.z;
-                                    sum.w += v.w;
-                                }
-                            }
-                        sq = fmaf(sum.x, sum.x, sq);
-                        sq = fmaf(sum.y, sum.y, sq);
-                        sq = fmaf(sum.z, sum.z, sq);
-                        sq = fmaf(sum.w, sum.w, sq);
-                    }
-                    for (int x = 0; x < kt; ++x)
-                        for (int y = 0; y < kh; ++y) {
-                            const int row = ((at * kt + x) * a.nch + ah * kh + y) * a.ncw + aw * kw;
-                            for (int z = 0; z < kw; ++z) m += cell_cnt[row + z];
-                        }
-                    #pragma unroll
-                    for (int off = 16; off > 0; off >>= 1) sq += __shfl_down_sync(0xffffffffu, sq, off);
-                    if (lane == 0) {
-                        tile_val[item] = m >= 2.f ? (sq - m) / (m * (m - 1.f)) : 0.f;
-                        tile_used[item] = m >= 1.f ? 1.f : 0.f;
-                    }
-                }
-    }
+    region_tile_pass(a, cell_sum, cell_cnt, tile_val, tile_used, warp, lane);
     __syncthreads();
-    if (threadIdx.x < a.tiles.n) {
-        const int c = threadIdx.x;
-        const int first = a.item_first[c], n = a.item_first[c + 1] - first;
-        float s = 0.f, used = 0.f;
-        for (int i = 0; i < n; ++i) {
-            s += tile_val[first + i];
-            used += tile_used[first + i];
-        }
-        const int n_regions = a.nrt * a.nrh * a.nrw;
-        float *out = a.partial + (static_cast<size_t>(bh) * n_regions + region) * 2 * a.tiles.n;
-        out[c] = s;
-        out[a.tiles.n + c] = used;
-    }
+    if (threadIdx.x < a.tiles.n) region_write(a, tile_val, tile_used, region, bh, threadIdx.x);
 }
 
 struct FinalArgs {
@@ -275,6 +295,19 @@ __global__ void sics_final_kernel(const FinalArgs a) {
         if (lane == 0 && a.sics) a.sics[static_cast<size_t>(bh) * a.n_tiles + c] = mean;
     }
     if (lane == 0) a.choice[bh] = best_c;
+}
+
+cudaError_t launch_sics_final(const float *partial, int BH, int n_regions, int n_tiles, int32_t *choice, float *sics,
+                              cudaStream_t st) {
+    FinalArgs f;
+    f.partial = partial;
+    f.BH = BH;
+    f.n_regions = n_regions;
+    f.n_tiles = n_tiles;
+    f.choice = choice;
+    f.sics = sics;
+    sics_final_kernel<<<(BH + 7) / 8, 256, 0, st>>>(f);
+    return cudaGetLastError();
 }
 
 }  // namespace
@@ -329,11 +362,11 @@ cudaError_t launch_select_tiling(const void *q, int esize, int BH, int D, int T,
         a.cpt_w[c] = on ? tiles.w[c] / g.Cw : 0;
         a.item_first[c + 1] = a.item_first[c] + a.tpr_t[c] * a.tpr_h[c] * a.tpr_w[c];
     }
+    cudaError_t e = cudaSuccess;
     const size_t cvol = static_cast<size_t>(g.Ct) * g.Ch * g.Cw;
     const size_t smem = (static_cast<size_t>(g.cells) * D + g.cells + 2 * items) * sizeof(float) + cvol * sizeof(int);
     dim3 grid(g.n_regions, BH);
     const int lpt = D * esize / 16;
-    cudaError_t e = cudaSuccess;
 #define VSA_SICS_LAUNCH(TYPE, L, C)                                                                           \
     do {                                                                                                      \
         e = cudaFuncSetAttribute(sics_partial_kernel<TYPE, L, C>, cudaFuncAttributeMaxDynamicSharedMemorySize, \
@@ -353,15 +386,7 @@ cudaError_t launch_select_tiling(const void *q, int esize, int BH, int D, int T,
 #undef VSA_SICS_LAUNCH
     e = cudaGetLastError();
     if (e != cudaSuccess) return e;
-    FinalArgs f;
-    f.partial = partial;
-    f.BH = BH;
-    f.n_regions = g.n_regions;
-    f.n_tiles = tiles.n;
-    f.choice = choice;
-    f.sics = sics;
-    sics_final_kernel<<<(BH + 7) / 8, 256, 0, st>>>(f);
-    return cudaGetLastError();
+    return launch_sics_final(partial, BH, g.n_regions, tiles.n, choice, sics, st);
 }
 
 }  // namespace vsa

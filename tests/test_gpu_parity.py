@@ -302,6 +302,42 @@ def test_select_tiling_matches_oracle(dtype, D):
     assert flips <= 1
 
 
+# Region geometries of the tiling choice: the candidates' per-axis lcm region
+# and gcd cells in several shapes (one frame per 128-token box of the region,
+# several frames, a cell spanning several frames, a padded grid).
+SICS_TILE_SETS = [
+    ((8, 16, 32), [(1, 8, 16), (2, 8, 8), (4, 4, 8)]),   # 16 cells of 1 x 4 x 8
+    ((8, 16, 32), [(2, 4, 8), (4, 4, 4)]),               # cells two frames deep
+    ((16, 16, 32), [(4, 8, 16), (8, 8, 16)]),            # two cells of 512 tokens
+    ((8, 16, 16), [(4, 4, 8), (2, 8, 8)]),
+    ((8, 16, 32), [(1, 16, 8), (2, 8, 8)]),
+    ((6, 21, 36), [(1, 8, 16), (2, 8, 8), (4, 4, 8)]),   # padded grid: regions cross its edge
+]
+
+
+@pytest.mark.parametrize("D", [64, 128])
+@pytest.mark.parametrize("case", range(len(SICS_TILE_SETS)))
+def test_select_tiling_region_geometries(case, D):
+    """Each head's cohesion per candidate against the oracle's on several
+    region geometries, bf16 and fp32 inputs of the same values agreeing."""
+    grid, tiles = SICS_TILE_SETS[case]
+    kinds = ["spatial", "temporal", "generic", "spatial"]
+    q, _, _ = smooth_qkv(1, 4, grid, D, seed=300 + case, kinds=kinds, device=DEV)
+    choice, sics = vsa.select_tiling(q, grid, tiles, return_sics=True)
+    choice32, sics32 = vsa.select_tiling(q.float(), grid, tiles, return_sics=True)
+    np.testing.assert_allclose(_np(sics), _np(sics32), atol=2e-6, rtol=0)
+    pg = oracle.padded_grid(grid, tiles)
+    for h in range(4):
+        qh = _np(q[0, h])
+        if tuple(pg) != tuple(grid):
+            qh = oracle.pad_grid(qh, grid, pg)
+        oc, osc = oracle.select_tiling(qh, pg, tiles)
+        np.testing.assert_allclose(_np(sics[h]), osc, atol=2e-5, rtol=0)
+        if np.sort(osc)[-1] - np.sort(osc)[-2] > 1e-4:
+            assert int(choice[h]) == oc and int(choice32[h]) == oc, (h, osc)
+    assert torch.equal(choice, vsa.select_tiling_noalloc(q, grid, tiles))
+
+
 # --------------------------------------------------------------------------
 # attention
 # --------------------------------------------------------------------------
