@@ -45,6 +45,8 @@ struct SelArgs {
     int nrt, nrh, nrw;  // regions per axis of the padded grid
     int cells, items;
     FastDiv cell_hw, cell_w;  // Ch * Cw and Cw: token of a cell -> (dt, dh, dw)
+    FastDiv reg_hw, reg_w;    // nrh * nrw and nrw: region -> (rt, rh, rw)
+    FastDiv cel_hw, cel_w;    // nch * ncw and ncw: cell -> (ct, ch, cw)
     int nch, ncw;             // cells of a region along h and w
     int tpr_t[kMaxTiles], tpr_h[kMaxTiles], tpr_w[kMaxTiles];  // candidate c: its tiles per region axis
     int cpt_t[kMaxTiles], cpt_h[kMaxTiles], cpt_w[kMaxTiles];  // candidate c: cells per tile axis
@@ -135,9 +137,11 @@ __global__ void __launch_bounds__(kThreads, 4) sics_partial_kernel(const SelArgs
     const int region = blockIdx.x, bh = blockIdx.y;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int lt = lane % LPT;
-    const int rt = region / (a.nrh * a.nrw), rh = (region / a.nrw) % a.nrh, rw = region % a.nrw;
+    // multiply-shift divisions: a runtime division per coordinate cost about 5 %
+    const int rt = static_cast<int>(fdiv(static_cast<uint32_t>(region), a.reg_hw));
+    const int r_hw = region - rt * static_cast<int>(a.reg_hw.d);
+    const int rh = static_cast<int>(fdiv(static_cast<uint32_t>(r_hw), a.reg_w)), rw = r_hw - rh * a.nrw;
     const int t0 = rt * a.Rt, h0 = rh * a.Rh, w0 = rw * a.Rw;
-    const int nch = a.Rh / a.Ch, ncw = a.Rw / a.Cw;
     const int cvol = a.Ct * a.Ch * a.Cw;
     const size_t head = static_cast<size_t>(bh) * a.S;
     // every cell has the same shape: offsets of its tokens from its first one, once per CTA
@@ -151,7 +155,9 @@ __global__ void __launch_bounds__(kThreads, 4) sics_partial_kernel(const SelArgs
     const uint4 *q4 = reinterpret_cast<const uint4 *>(a.q);
 
     for (int cell = warp; cell < a.cells; cell += kWarps) {
-        const int ct = cell / (nch * ncw), ch = (cell / ncw) % nch, cw = cell % ncw;
+        const int ct = static_cast<int>(fdiv(static_cast<uint32_t>(cell), a.cel_hw));
+        const int c_hw = cell - ct * static_cast<int>(a.cel_hw.d);
+        const int ch = static_cast<int>(fdiv(static_cast<uint32_t>(c_hw), a.cel_w)), cw = c_hw - ch * a.ncw;
         const int tb = t0 + ct * a.Ct, hb = h0 + ch * a.Ch, wb = w0 + cw * a.Cw;
         // padded grids: a cell wholly past the real grid holds only zero tokens
         // (no loads), one across its edge tests each token (warp-uniform flags)
@@ -351,6 +357,10 @@ cudaError_t launch_select_tiling(const void *q, int esize, int BH, int D, int T,
     a.items = items;
     a.nch = g.Rh / g.Ch;
     a.ncw = g.Rw / g.Cw;
+    a.reg_hw = make_fastdiv(static_cast<uint32_t>(a.nrh * a.nrw));
+    a.reg_w = make_fastdiv(static_cast<uint32_t>(a.nrw));
+    a.cel_hw = make_fastdiv(static_cast<uint32_t>(a.nch * a.ncw));
+    a.cel_w = make_fastdiv(static_cast<uint32_t>(a.ncw));
     a.item_first[0] = 0;
     for (int c = 0; c < kMaxTiles; ++c) {
         const bool on = c < tiles.n;
