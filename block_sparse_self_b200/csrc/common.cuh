@@ -405,26 +405,6 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
     return *reinterpret_cast<uint32_t *>(&v);
 }
 
-// acc_lo += lo * lo, acc_hi += hi * hi for the two bf16 halves of pk: sm_100
-// mixed-precision FMAs (the product of two bf16 values is exact in fp32, so
-// each is one rounding, as an fp32 FMA on the widened values would give).
-__device__ __forceinline__ void sq_bf16x2_f32(uint32_t pk, float &acc_lo, float &acc_hi) {
-    asm("{\n\t.reg .b16 lo, hi;\n\tmov.b32 {lo, hi}, %2;\n\t"
-        "fma.rn.f32.bf16 %0, lo, lo, %0;\n\tfma.rn.f32.bf16 %1, hi, hi, %1;\n\t}"
-        : "+f"(acc_lo), "+f"(acc_hi)
-        : "r"(pk));
-}
-
-// 16 bytes from global memory read once: no L1 allocation, and the L2 fetches
-// the whole 256-byte line around it (a token row of D = 128 bf16 values).
-__device__ __forceinline__ uint4 ld_stream_l2_256(const uint4 *p) {
-    uint4 r;
-    asm volatile("ld.global.nc.L1::no_allocate.L2::256B.v4.u32 {%0, %1, %2, %3}, [%4];"
-                 : "=r"(r.x), "=r"(r.y), "=r"(r.z), "=r"(r.w)
-                 : "l"(p));
-    return r;
-}
-
 // acc_lo += low bf16 of pk, acc_hi += high bf16 of pk: sm_100 mixed-precision
 // adds (the bf16 operand widens exactly, then one fp32 rounding), with no
 // separate unpacking of the pair.
