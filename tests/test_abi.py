@@ -192,6 +192,25 @@ def test_python_binding_rejects_cpu_tensors():
         vsa.permute(q, (2, 8, 8), [(1, 8, 8)])
 
 
+def test_missing_library_fails_loudly():
+    """No CPU fallback: without libvsa.so every call raises (run in a child
+    process so this process keeps its loaded library)."""
+    import os
+    import subprocess
+    import sys
+    code = ("import block_sparse_self_b200 as v, torch\n"
+            "v.LIB_PATH = '/nonexistent/libvsa.so'\n"
+            "v._lib = None\n"
+            "try:\n"
+            "    v.lib()\n"
+            "except RuntimeError as e:\n"
+            "    print('raised:', e)\n")
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    r = subprocess.run([sys.executable, "-c", code], cwd=root, capture_output=True, text=True, timeout=300)
+    assert r.returncode == 0, r.stderr
+    assert "raised:" in r.stdout and "missing" in r.stdout
+
+
 def test_sample_query_rows_is_a_seeded_sorted_distinct_draw():
     import torch
     r = vsa.sample_query_rows(1000, 128, seed=3, device="cpu")
