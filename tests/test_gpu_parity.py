@@ -918,6 +918,56 @@ def test_one_block_lists_match_two_tile_kernel_and_oracle(mode, grid):
         assert_attn_close(_np(o1[0, h]), want[real], f"head {h}")
 
 
+def test_one_block_kernel_many_tiles_per_cta_with_invalid_lists():
+    """1024 query tiles of four heads in three tilings, with tiles whose list
+    is invalid (zeros and an error status) among them: the one-block kernel
+    gives the two-tile kernel's bits on the same lists, and the oracle's
+    result on sampled blocks."""
+    grid, tiles = (16, 32, 64), [(1, 8, 16), (2, 8, 8), (4, 4, 8)]
+    B, H, D = 1, 4, 128
+    nb = grid[0] * grid[1] * grid[2] // 128
+    q, k, v = smooth_qkv(B, H, grid, D, seed=97, device=DEV)
+    rng = np.random.default_rng(98)
+    idx1 = rng.integers(0, nb, (H, nb)).astype(np.int32)
+    cnt = np.ones((H, nb), np.int32)
+    choice = torch.tensor([0, 1, 2, 1], dtype=torch.int32, device=DEV)
+
+    def run(idx):
+        ti1 = torch.as_tensor(idx, device=DEV).view(B, H, nb, 1)
+        ti2 = torch.as_tensor(np.concatenate([idx[..., None], np.full((H, nb, 1), -1, np.int32)], -1),
+                              device=DEV).view(B, H, nb, 2)
+        tc = torch.as_tensor(cnt, device=DEV).view(B, H, nb)
+        o1 = vsa.block_sparse_attention_tiled(q, k, v, grid, tiles, choice, ti1, tc, out_dtype=torch.float32)
+        o2 = vsa.block_sparse_attention_tiled(q, k, v, grid, tiles, choice, ti2, tc, out_dtype=torch.float32)
+        return o1, o2
+
+    o1, o2 = run(idx1)
+    vsa.device_status()
+    assert torch.equal(o1, o2)
+    for h, c in enumerate(choice.tolist()):
+        perm = oracle.tile_permutation(grid, tiles[c])
+        qo, ko, vo = (oracle.permute_rows(_np(x[0, h]), perm) for x in (q, k, v))
+        blocks = [0, 1, 100, 201, nb - 1]
+        rows = np.concatenate([np.arange(b * 128, (b + 1) * 128) for b in blocks])
+        want = oracle.block_sparse_attention(qo, ko, vo, idx1[h][:, None], cnt[h], 128, rows=rows)
+        assert_attn_close(_np(o1[0, h])[perm[rows]], want, f"head {h}")
+    bad = idx1.copy()
+    bad[1, ::5] = nb          # out of range
+    bad[3, 3::7] = -1
+    o1b, o2b = run(bad)
+    with pytest.raises(RuntimeError):
+        vsa.device_status()
+    assert torch.equal(o1b, o2b)
+    for h, sel in ((1, slice(0, None, 5)), (3, slice(3, None, 7))):
+        perm = oracle.tile_permutation(grid, tiles[int(choice[h])])
+        dead = np.zeros(nb, bool)
+        dead[sel] = True
+        rows = perm[np.repeat(dead, 128)]
+        assert torch.count_nonzero(o1b[0, h, torch.as_tensor(rows, device=DEV)]) == 0
+        live = perm[np.repeat(~dead, 128)]
+        assert torch.equal(o1b[0, h, torch.as_tensor(live, device=DEV)], o1[0, h, torch.as_tensor(live, device=DEV)])
+
+
 def test_temporal_mask_with_more_frames_than_a_block():
     """T = 256 frames: a temporal tile is two blocks, so the lists hold two
     blocks and the composition must not ask for one-slot lists."""
