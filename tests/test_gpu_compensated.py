@@ -118,6 +118,22 @@ def test_compensated_shared_list_and_every_block_kept():
     assert torch.equal(oc, vsa.block_sparse_attention(q, k, v, full, fcnt, BLOCK, out_dtype=torch.float32))
 
 
+def test_compensated_one_block_lists():
+    """Lists of one block (the diagonal): the kept block runs through the
+    one-key-block kernel with its per-row softmax state, every other block
+    through the centroid pass."""
+    grid, D = (8, 16, 16), 128
+    S, nb, H = 2048, 16, 2
+    q, k, v = smooth_qkv(1, H, grid, D, seed=21, device=DEV)
+    idx = np.tile(np.arange(nb, dtype=np.int32)[None, :, None], (H, 1, 1))
+    cnt = np.ones((H, nb), np.int32)
+    o = vsa.centroid_compensated_attention(q, k, v, torch.tensor(idx, device=DEV).view(1, H, nb, 1),
+                                           torch.tensor(cnt, device=DEV).view(1, H, nb), out_dtype=torch.float32)
+    for h in range(H):
+        want = _oracle_rows(_np(q[0, h]), _np(k[0, h]), _np(v[0, h]), idx[h], cnt[h])
+        assert_close(_np(o[0, h]), want, f"head {h}")
+
+
 def test_compensated_equal_keys_within_blocks_is_dense_attention():
     """Keys (and values) equal within each block: every skipped block's
     centroid stands for it exactly, so the result is dense attention whatever

@@ -870,7 +870,8 @@ def test_spade_top_p_end_to_end():
 # lists of one key block: the one-block kernel (two CTAs per SM)
 # --------------------------------------------------------------------------
 
-@pytest.mark.parametrize("mode,grid", [("permuted", (4, 8, 16)), ("tiled", (4, 8, 16)), ("padded", (5, 12, 20))])
+@pytest.mark.parametrize("mode,grid", [("permuted", (4, 8, 16)), ("tiled", (4, 8, 16)), ("padded", (5, 12, 20)),
+                                       ("padded", (5, 44, 76))])   # 720 tiles: several per persistent CTA
 def test_one_block_lists_match_two_tile_kernel_and_oracle(mode, grid):
     """One-slot lists run through the one-key-block kernel; the same lists in
     two slots (cnt 1, second slot -1) run through the two-tile kernel.  Both
