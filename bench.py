@@ -513,12 +513,13 @@ def structured_lines(out, timed, steps):
 
 def compensated_line(w, q, k, v, idx, cnt, n_rep: int):
     """Centroid-compensated attention against the plain block-sparse attention
-    on the same permuted inputs and lists.  Algorithmic FLOPs: 4 * 128 * 128 * D
-    per listed block pair plus 4 * 128 * D per (query block, skipped block)
-    centroid."""
+    on the same inputs and lists, both in tiled mode (T-major q, k, v, each
+    head's chosen tiling, no permuted copies).  Algorithmic FLOPs: 4 * 128 *
+    128 * D per listed block pair plus 4 * 128 * D per (query block, skipped
+    block) centroid."""
     import block_sparse_self_b200 as vsa
-    choice = vsa.select_tiling(q, w.grid, list(w.tiles))
-    qp, kp, vp = (vsa.permute(x, w.grid, list(w.tiles), choice) for x in (q, k, v))
+    tiles = list(w.tiles)
+    choice = vsa.select_tiling(q, w.grid, tiles)
 
     def timed(fn):
         for _ in range(3):
@@ -532,8 +533,8 @@ def compensated_line(w, q, k, v, idx, cnt, n_rep: int):
         torch.cuda.synchronize()
         return s.elapsed_time(e) / n_rep
 
-    comp_ms = timed(lambda: vsa.centroid_compensated_attention(qp, kp, vp, idx, cnt))
-    plain_ms = timed(lambda: vsa.block_sparse_attention(qp, kp, vp, idx, cnt, 128))
+    comp_ms = timed(lambda: vsa.centroid_compensated_attention_tiled(q, k, v, w.grid, tiles, choice, idx, cnt))
+    plain_ms = timed(lambda: vsa.block_sparse_attention_tiled(q, k, v, w.grid, tiles, choice, idx, cnt))
     pairs = float(cnt.to(torch.int64).sum().item())
     BH, nb = w.B * w.heads, w.nb
     skipped = BH * nb * nb - pairs
@@ -548,12 +549,11 @@ def compensated_line(w, q, k, v, idx, cnt, n_rep: int):
     tiles_run = float((kept[:, :nct] < size).sum().item())
     executed = pairs * 4.0 * 128 * 128 * w.D + tiles_run * 8.0 * 128 * 128 * w.D
     burst = load_peaks()[0].get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"])
-    del qp, kp, vp
     return {"ms_per_call": comp_ms, "tflops": flops / comp_ms / 1e9, "frac_of_burst": flops / comp_ms / 1e9 / burst,
             "executed_tflops": executed / comp_ms / 1e9, "plain_attention_ms": plain_ms,
             "compensation_overhead": comp_ms / plain_ms - 1.0, "skipped_blocks_per_row": skipped / (BH * nb),
             "centroid_tiles_per_query_block": tiles_run / (BH * nb),
-            "out_dtype": "bf16", "layout": "permuted copies in each head's chosen tiling"}
+            "out_dtype": "bf16", "layout": "T-major, tiled (each head's chosen tiling, no permuted copies)"}
 
 
 def run_ours(args, w):

@@ -71,6 +71,8 @@ def lib() -> ctypes.CDLL:
         "vsa_head_profile": ([P, P, I, I, I, I, D3, P, I, F, I, P, P, P, SZ, P], I),
         "vsa_centroid_compensated_attention_workspace_size": ([I, I, I, I, I], SZ),
         "vsa_centroid_compensated_attention": ([P, P, P, P, I, I, I, I, I, I, P, P, I, I, F, P, SZ, P], I),
+        "vsa_centroid_compensated_attention_tiled": ([P, P, P, P, I, I, I, I, I, D3, P, I, P, P, P, I, I, F, P, SZ, P],
+                                                     I),
         "vsa_spade_attention_host_workspace_size": ([I, I, I, I, D3, P, I, I, I, I, I, I], SZ),
         "vsa_spade_attention_host": ([P, P, P, P, I, I, I, I, I, D3, P, I, I, I, I, F, I, P, SZ, P], I),
         "vsa_cast_f32_to_bf16": ([P, P, I64, P], I),
@@ -478,6 +480,35 @@ def centroid_compensated_attention(q, k, v, idx, cnt, block: int = 128, scale: O
     return o
 
 
+def centroid_compensated_attention_tiled(q, k, v, grid, tiles, choice, idx, cnt, scale: Optional[float] = None,
+                                         out_dtype=None) -> torch.Tensor:
+    """unpermute(centroid_compensated_attention(permute(q), permute(k), permute(v), idx, cnt)) with no
+    permuted copies: q, k, v and the result in T-major order, each head's 128-token blocks those of
+    tiles[choice[b, h]] (tiling 0 without a choice); the tiles must divide the grid."""
+    B, H, S, D = _bhsd(q, "q")
+    if tuple(k.shape) != (B, H, S, D) or tuple(v.shape) != (B, H, S, D):
+        raise ValueError(f"q/k/v shapes must match exactly; got q={tuple(q.shape)}, k={tuple(k.shape)}, "
+                         f"v={tuple(v.shape)}")
+    odt = _out_dtype(out_dtype, q)
+    qb, kb, vb = _bf16(q, "q"), _bf16(k, "k"), _bf16(v, "v")
+    _cuda(idx, "idx")
+    _cuda(cnt, "cnt")
+    if idx.dtype != torch.int32 or cnt.dtype != torch.int32:
+        raise ValueError("idx and cnt must be int32")
+    oc = BF16 if odt == torch.bfloat16 else F32
+    need = lib().vsa_centroid_compensated_attention_workspace_size(B, H, S, D, oc)
+    if need == 0:
+        raise ValueError(f"no workspace size for B={B}, H={H}, S={S}, D={D} (S must be a multiple of 128, D 64 or 128)")
+    arr, n = _tiles_arg(tiles)
+    ws = torch.empty(need, dtype=torch.uint8, device=q.device)
+    o = torch.empty(B, H, S, D, dtype=odt, device=q.device)
+    _check(lib().vsa_centroid_compensated_attention_tiled(
+        _ptr(qb), _ptr(kb), _ptr(vb), _ptr(o), oc, B, H, S, D, Dims3(*grid), arr, n, _choice_arg(choice, B * H),
+        _ptr(idx), _ptr(cnt), int(idx.shape[-1]), 1 if idx.dim() == 4 else 0, 0.0 if scale is None else float(scale),
+        _ptr(ws), need, _stream(q.device)))
+    return o
+
+
 def block_sparse_attention_tiled(q, k, v, grid, tiles, choice, idx, cnt, scale: Optional[float] = None,
                                  out_dtype=None, group_stride: int = 0) -> torch.Tensor:
     """unpermute(block_sparse_attention(permute(q), permute(k), permute(v), idx, cnt, block)) in one
@@ -573,8 +604,8 @@ def spade_attention(q, k, v, grid, tiles, budget: Optional[float] = None, topk: 
 
     compensate=True takes the Recipe's attention call: every key block a
     query block skips still takes part as its centroid
-    (centroid_compensated_attention); it runs on explicit permuted copies,
-    128-token blocks and grids the tiles divide.
+    (centroid_compensated_attention, or its tiled form); it needs 128-token
+    blocks and grids the tiles divide.
 
     Every candidate tile must have the same volume (the block size).  With a
     single candidate the tiling choice is skipped (choice 0 for every head).
@@ -606,9 +637,9 @@ def spade_attention(q, k, v, grid, tiles, budget: Optional[float] = None, topk: 
     if compensate:
         if block != 128:
             raise NotImplementedError("compensated attention takes 128-token blocks")
-        if tiled:
-            raise ValueError("compensated attention runs on explicit permuted copies (tiled=False)")
-        tiled = False
+        if tuple(pgrid) != tuple(grid):
+            raise NotImplementedError(f"compensated attention needs a grid the tiles divide; {tuple(grid)} "
+                                      f"is padded to {pgrid}")
     if tiled is None:
         tiled = can_tile
     elif tiled and not can_tile:
@@ -623,7 +654,10 @@ def spade_attention(q, k, v, grid, tiles, budget: Optional[float] = None, topk: 
         kmax, kmin = block_summaries_tiled(k, grid, tiles, choice, block)
         scores = block_scores(qmax, qmin, kmax, kmin)
         idx, cnt = _select_blocks(scores, kk, n_sink_blocks, diag_halfwidth, top_p, top_p_scale, D)
-        o = block_sparse_attention_tiled(qb, kb, vb, grid, tiles, choice, idx, cnt, scale, out_dtype)
+        if compensate:
+            o = centroid_compensated_attention_tiled(qb, kb, vb, grid, tiles, choice, idx, cnt, scale, out_dtype)
+        else:
+            o = block_sparse_attention_tiled(qb, kb, vb, grid, tiles, choice, idx, cnt, scale, out_dtype)
         if return_intermediates:
             qp, kp, vp, op = (permute(x, grid, tiles, choice) for x in (q, k, v, o))
     else:

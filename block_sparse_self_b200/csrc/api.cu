@@ -617,6 +617,63 @@ vsa_status vsa_centroid_compensated_attention(const void *q, const void *k, cons
     return launch_compensated(L, workspace, status_or_null(stream), as_stream(stream));
 }
 
+vsa_status vsa_centroid_compensated_attention_tiled(const void *q, const void *k, const void *v, void *o,
+                                                    vsa_dtype out_dtype, int B, int n_heads, int S, int D,
+                                                    vsa_dims3 grid, const vsa_dims3 *tiles, int n_tiles,
+                                                    const int32_t *choice, const int32_t *idx, const int32_t *cnt,
+                                                    int cap, int list_per_head, float scale, void *workspace,
+                                                    size_t workspace_bytes, void *stream) {
+    VSA_TRY(check_attention_common(q, k, v, o, out_dtype, B, n_heads, S, D, scale));
+    VSA_REQUIRE(aligned4(idx) && aligned4(cnt), "idx and cnt must be non-NULL 4-byte aligned device pointers");
+    VSA_REQUIRE(cap >= 1, "cap must be >= 1, got %d", cap);
+    VSA_REQUIRE(choice == nullptr || aligned4(choice), "choice must be NULL or 4-byte aligned");
+    VSA_TRY(check_grid(grid, S));
+    TileSet ts;
+    vsa_dims3 pg;
+    VSA_TRY(check_tiles(grid, tiles, n_tiles, &ts, &pg));
+    if (pg.t != grid.t || pg.h != grid.h || pg.w != grid.w)
+        return fail(VSA_ERR_UNSUPPORTED, "compensated attention in tiled mode needs a grid every tile divides");
+    const int vol = ts.t[0] * ts.h[0] * ts.w[0];
+    if (vol % 128 != 0)
+        return fail(VSA_ERR_UNSUPPORTED, "compensated attention takes 128-token blocks; the tiles hold %d tokens", vol);
+    for (int c = 0; c < n_tiles; ++c) {
+        VSA_REQUIRE(ts.t[c] * ts.h[c] * ts.w[c] == vol, "every tile must have the volume of tile 0 (%d); tile %d has %d",
+                    vol, c, ts.t[c] * ts.h[c] * ts.w[c]);
+        VSA_REQUIRE(ts.t[c] % (vol / 128) == 0,
+                    "tile %d: tile.t (%d) must be divisible by volume / 128 (%d) so each 128-token block is whole "
+                    "(h, w) planes",
+                    c, ts.t[c], vol / 128);
+        if (ts.t[c] / (vol / 128) > grid.t || ts.h[c] > grid.h || ts.w[c] > grid.w)
+            return fail(VSA_ERR_UNSUPPORTED, "tile %d: its 128-token box is larger than the grid", c);
+    }
+    if (S / 128 > 8192) return fail(VSA_ERR_UNSUPPORTED, "compensated attention supports at most 8192 blocks per head");
+    const size_t need = vsa_centroid_compensated_attention_workspace_size(B, n_heads, S, D, out_dtype);
+    VSA_REQUIRE(workspace != nullptr && (reinterpret_cast<uintptr_t>(workspace) & 255u) == 0,
+                "workspace must be a non-NULL 256-byte aligned device pointer");
+    VSA_REQUIRE(workspace_bytes >= need, "workspace holds %zu bytes, %zu needed", workspace_bytes, need);
+    const size_t in_bytes = static_cast<size_t>(B) * n_heads * S * D * 2;
+    VSA_REQUIRE(!overlaps(workspace, need, o, static_cast<size_t>(B) * n_heads * S * D * esize_of(out_dtype)) &&
+                    !overlaps(workspace, need, q, in_bytes) && !overlaps(workspace, need, k, in_bytes) &&
+                    !overlaps(workspace, need, v, in_bytes),
+                "workspace must not overlap q, k, v or o");
+    AttnLaunch L{};
+    L.q = q; L.k = k; L.v = v; L.o = o;
+    L.out_f32 = out_dtype == VSA_F32;
+    L.BH = B * n_heads; L.S = S; L.D = D;
+    L.block = 128;
+    L.window = false;
+    L.idx = idx; L.cnt = cnt; L.cap = cap; L.list_per_head = list_per_head ? 1 : 0;
+    L.group = 0; L.nb = S / 128;
+    L.scale = scale > 0.f ? scale : 1.0f / sqrtf(static_cast<float>(D));
+    L.tiled = true;
+    L.gstride = 0;
+    L.T = grid.t; L.Hg = grid.h; L.Wg = grid.w;
+    L.Tp = pg.t; L.Hp = pg.h; L.Wp = pg.w;
+    L.tiles = ts;
+    L.choice = choice;
+    return launch_compensated(L, workspace, status_or_null(stream), as_stream(stream));
+}
+
 vsa_status vsa_window_attention(const void *q, const void *k, const void *v, void *o, vsa_dtype out_dtype, int B,
                                 int n_heads, int S, int D, int window, int sink, float scale, int chunk,
                                 void *stream) {

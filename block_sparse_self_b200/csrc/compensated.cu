@@ -23,6 +23,10 @@
 //      lo MMAs); then the two partial softmaxes are merged exactly:
 //        o = (l1 2^(m1-M) o1 + n_b 2^(m2-M) O2) / (l1 2^(m1-M) + n_b l2 2^(m2-M)),
 //      M = max(m1, m2), and written in the output dtype.
+// Tiled mode takes q, k, v and o in T-major order, as the tiled attention
+// does: each head's blocks are those of its own tiling, the centroid kernel
+// and the pass read a block's rows where the tiling puts them (Q as 5-D TMA
+// boxes), and every output row goes to its T-major token.
 #include "common.cuh"
 #include "internal.h"
 
@@ -33,28 +37,53 @@ namespace {
 constexpr int kBlock = 128;        // tokens per block (and per centroid tile)
 constexpr int kMaxCentroidTiles = 64;  // nb <= 64 * 128 = 8192 blocks per head
 
+// Tiled mode: each head's tiling (candidate choice[bh], tiling 0 without a
+// choice); position p of its tile-contiguous order is T-major token
+// tile_token_fast(p, divs[c]), and query tile qt is the 128-token box at
+// part qt % m of tile qt / m (m = volume / 128, bt = tile.t / m frames).
+struct CompTiling {
+    int n;
+    const int32_t *choice;
+    TileDivs divs[kMaxTiles];
+    FastDiv m[kMaxTiles], nthw[kMaxTiles], ntw[kMaxTiles];
+    int bt[kMaxTiles], th[kMaxTiles], tw[kMaxTiles];
+};
+
+// the head's tiling, or -1 for a choice out of range (the head is left unwritten)
+__device__ __forceinline__ int comp_tiling(const CompTiling &tl, int bh) {
+    const int c = tl.choice ? __ldg(tl.choice + bh) : 0;
+    return (c < 0 || c >= tl.n) ? -1 : c;
+}
+
 // ---------------------------------------------------------------------------
 // 1. centroids
 // ---------------------------------------------------------------------------
 // One CTA per (key block, bh), 256 threads: thread t sums 16-byte chunk
 // t % (D / 8) of every (256 / (D / 8))-th row of the block, for K and V.
-template <int D>
+template <int D, bool TILED>
 __global__ void __launch_bounds__(256) centroid_kernel(const __nv_bfloat16 *__restrict__ k,
                                                        const __nv_bfloat16 *__restrict__ v, int S, int nb,
                                                        __nv_bfloat16 *__restrict__ khi, __nv_bfloat16 *__restrict__ klo,
-                                                       __nv_bfloat16 *__restrict__ vhi, __nv_bfloat16 *__restrict__ vlo) {
+                                                       __nv_bfloat16 *__restrict__ vhi, __nv_bfloat16 *__restrict__ vlo,
+                                                       const CompTiling tl) {
     constexpr int CPR = D / 8;            // 16-byte chunks per row
     constexpr int G = 256 / CPR;          // row groups
     __shared__ float red[2][G][D];
     const int b = blockIdx.x, bh = blockIdx.y;
     const int chunk = threadIdx.x % CPR, g = threadIdx.x / CPR;
-    const size_t base = (static_cast<size_t>(bh) * S + static_cast<size_t>(b) * kBlock) * D;
-    const uint4 *kr = reinterpret_cast<const uint4 *>(k + base);
-    const uint4 *vr = reinterpret_cast<const uint4 *>(v + base);
+    const uint4 *kr = reinterpret_cast<const uint4 *>(k + static_cast<size_t>(bh) * S * D);
+    const uint4 *vr = reinterpret_cast<const uint4 *>(v + static_cast<size_t>(bh) * S * D);
+    int c = 0;
+    if constexpr (TILED) {
+        c = comp_tiling(tl, bh);
+        if (c < 0) c = 0;  // the head is left unwritten downstream; read tiling 0 in bounds
+    }
     float ak[8] = {}, av[8] = {};
     #pragma unroll 4
     for (int r = g; r < kBlock; r += G) {
-        const uint4 xk = __ldg(kr + r * CPR + chunk), xv = __ldg(vr + r * CPR + chunk);
+        const uint32_t p = static_cast<uint32_t>(b * kBlock + r);
+        const size_t row = TILED ? tile_token_fast(p, tl.divs[c]) : p;
+        const uint4 xk = __ldg(kr + row * CPR + chunk), xv = __ldg(vr + row * CPR + chunk);
         const __nv_bfloat162 *pk = reinterpret_cast<const __nv_bfloat162 *>(&xk);
         const __nv_bfloat162 *pv = reinterpret_cast<const __nv_bfloat162 *>(&xv);
         #pragma unroll
@@ -133,12 +162,13 @@ struct CompArgs {
 };
 
 struct CompMaps {
-    CUtensorMap q, khi, klo, vhi, vlo;
+    CUtensorMap q[kMaxTiles];  // slot 0 only, or one per candidate tiling in tiled mode
+    CUtensorMap khi, klo, vhi, vlo;
 };
 
-template <int D>
+template <int D, bool TILED>
 __global__ void __launch_bounds__(kPairThreads, 1)
-comp_pair_kernel(const __grid_constant__ CompMaps maps, const CompArgs a) {
+comp_pair_kernel(const __grid_constant__ CompMaps maps, const CompArgs a, const CompTiling tl) {
     using C = PairCfg<D>;
     extern __shared__ uint8_t smem_raw[];
     uint8_t *base = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -163,13 +193,15 @@ comp_pair_kernel(const __grid_constant__ CompMaps maps, const CompArgs a) {
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int bh = blockIdx.y;
+    int tc = 0;  // tiled mode: this head's tiling (out of range: the head is left unwritten)
+    if constexpr (TILED) tc = comp_tiling(tl, bh);
     int qt[2];
     const int32_t *list[2] = {nullptr, nullptr};
     int cnt[2] = {0, 0};
     bool valid[2];
     for (int t = 0; t < 2; ++t) {
         qt[t] = 2 * blockIdx.x + t;
-        valid[t] = qt[t] < a.nq;
+        valid[t] = qt[t] < a.nq && tc >= 0;
         if (valid[t]) {
             const size_t lrow = (a.list_per_head ? static_cast<size_t>(bh) * a.nb : 0) + qt[t];
             list[t] = a.idx + lrow * a.cap;
@@ -192,6 +224,8 @@ comp_pair_kernel(const __grid_constant__ CompMaps maps, const CompArgs a) {
         *abort_flag = 0;
         fence_mbar_init();
     }
+    if (tc < 0 && threadIdx.x == 0) report(a.status, DEV_RUNTIME);
+    if (tc < 0) tc = 0;
     for (int i = threadIdx.x; i < 2 * C::MASK_WORDS; i += blockDim.x) kept[i] = 0u;
     if (warp < 2) {  // warp t validates tile t's list as the attention kernel does
         const int t = warp;
@@ -234,10 +268,22 @@ comp_pair_kernel(const __grid_constant__ CompMaps maps, const CompArgs a) {
             tma_prefetch_desc(&maps.khi);
             tma_prefetch_desc(&maps.vhi);
             mbar_arrive_expect_tx(q_full, (act[0] + act[1]) * C::TILE_BYTES);
-            for (int t = 0; t < 2; ++t)
-                if (act[t])
+            for (int t = 0; t < 2; ++t) {
+                if (!act[t]) continue;
+                if constexpr (TILED) {  // the 128-token box of query tile qt in this head's tiling
+                    const uint32_t tile = fdiv(static_cast<uint32_t>(qt[t]), tl.m[tc]);
+                    const uint32_t part = static_cast<uint32_t>(qt[t]) - tile * tl.m[tc].d;
+                    const uint32_t ct = fdiv(tile, tl.nthw[tc]), rem = tile - ct * tl.nthw[tc].d;
+                    const uint32_t ch = fdiv(rem, tl.ntw[tc]), cw = rem - ch * tl.ntw[tc].d;
+                    const int bw = static_cast<int>(cw) * tl.tw[tc], bhh = static_cast<int>(ch) * tl.th[tc];
+                    const int bt = static_cast<int>(ct * tl.m[tc].d + part) * tl.bt[tc];
                     for (int s = 0; s < C::KSLABS; ++s)
-                        tma_load_3d(sQ + t * C::TILE_BYTES + s * C::SLAB, &maps.q, q_full, s * 64, qt[t] * kBlock, bh);
+                        tma_load_5d(sQ + t * C::TILE_BYTES + s * C::SLAB, &maps.q[tc], q_full, s * 64, bw, bhh, bt, bh);
+                } else {
+                    for (int s = 0; s < C::KSLABS; ++s)
+                        tma_load_3d(sQ + t * C::TILE_BYTES + s * C::SLAB, &maps.q[0], q_full, s * 64, qt[t] * kBlock, bh);
+                }
+            }
             int kl = 0, vl = 0;  // centroid tiles whose K, V parts were issued
             bool ok = true;
             for (int c = 0; ok && c < nct; ++c) {
@@ -447,7 +493,10 @@ comp_pair_kernel(const __grid_constant__ CompMaps maps, const CompArgs a) {
             // ---- merge with the main pass and write the row ----
             // main pass: o1 (normalised) with state (m1, l1); centroids: O2 (not
             // normalised) with state (m2, l2), each centroid weighted by n_b
-            const size_t prow = static_cast<size_t>(bh) * a.S + rg;
+            const size_t prow = static_cast<size_t>(bh) * a.S + rg;  // the row's state: permuted position
+            // o1 and the output: the permuted row, or its T-major token in tiled mode
+            const size_t orow = TILED ? static_cast<size_t>(bh) * a.S + tile_token_fast(static_cast<uint32_t>(rg), tl.divs[tc])
+                                      : prow;
             const float2 st = a.stats[prow];
             const float m2 = have_c ? m_ref : -INFINITY;
             const float M = fmaxf(st.x, m2);
@@ -456,7 +505,7 @@ comp_pair_kernel(const __grid_constant__ CompMaps maps, const CompArgs a) {
             const float w1 = st.y * f1;
             const float den = w1 + f2 * (have_c ? l_sum : 0.f);
             const float c1 = den > 0.f ? w1 / den : 0.f, c2 = den > 0.f ? f2 / den : 0.f;
-            const float *o1 = a.o1 + prow * D;
+            const float *o1 = a.o1 + orow * D;
             #pragma unroll 1
             for (int u = 0; u < D / 8; ++u) {
                 uint32_t o2[8] = {0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u};
@@ -471,11 +520,11 @@ comp_pair_kernel(const __grid_constant__ CompMaps maps, const CompArgs a) {
                 const float r4 = c1 * fb.x + c2 * __uint_as_float(o2[4]), r5 = c1 * fb.y + c2 * __uint_as_float(o2[5]);
                 const float r6 = c1 * fb.z + c2 * __uint_as_float(o2[6]), r7 = c1 * fb.w + c2 * __uint_as_float(o2[7]);
                 if (a.out_f32) {
-                    float4 *dst = reinterpret_cast<float4 *>(static_cast<float *>(a.out) + prow * D + 8 * u);
+                    float4 *dst = reinterpret_cast<float4 *>(static_cast<float *>(a.out) + orow * D + 8 * u);
                     dst[0] = make_float4(r0, r1, r2, r3);
                     dst[1] = make_float4(r4, r5, r6, r7);
                 } else {
-                    uint4 *dst = reinterpret_cast<uint4 *>(static_cast<__nv_bfloat16 *>(a.out) + prow * D + 8 * u);
+                    uint4 *dst = reinterpret_cast<uint4 *>(static_cast<__nv_bfloat16 *>(a.out) + orow * D + 8 * u);
                     *dst = make_uint4(pack_bf16x2(r0, r1), pack_bf16x2(r2, r3), pack_bf16x2(r4, r5), pack_bf16x2(r6, r7));
                 }
             }
@@ -509,7 +558,7 @@ CompLayout comp_layout(int BH, int S, int D, int out_f32) {
     return L;
 }
 
-template <int D>
+template <int D, bool TILED>
 vsa_status run_compensated(const AttnLaunch &L, void *workspace, int *status, cudaStream_t st) {
     using C = PairCfg<D>;
     const int nb = L.S / kBlock;
@@ -522,9 +571,29 @@ vsa_status run_compensated(const AttnLaunch &L, void *workspace, int *status, cu
     auto *stats = reinterpret_cast<float2 *>(ws + lay.stats);
     float *o1 = L.out_f32 ? static_cast<float *>(L.o) : reinterpret_cast<float *>(ws + lay.o32);
 
-    centroid_kernel<D><<<dim3(nb, L.BH), 256, 0, st>>>(static_cast<const __nv_bfloat16 *>(L.k),
-                                                        static_cast<const __nv_bfloat16 *>(L.v), L.S, nb, khi, klo,
-                                                        vhi, vlo);
+    CompTiling tl = {};
+    tl.n = TILED ? L.tiles.n : 1;
+    tl.choice = TILED ? L.choice : nullptr;
+    for (int c = 0; c < kMaxTiles; ++c) {
+        if (TILED && c < L.tiles.n) {
+            const int tt = L.tiles.t[c], th = L.tiles.h[c], tw = L.tiles.w[c];
+            const int m = tt * th * tw / kBlock;
+            tl.divs[c] = make_tile_divs(L.Hg, L.Wg, tt, th, tw);
+            tl.m[c] = make_fastdiv(static_cast<uint32_t>(m));
+            tl.nthw[c] = make_fastdiv(static_cast<uint32_t>((L.Hg / th) * (L.Wg / tw)));
+            tl.ntw[c] = make_fastdiv(static_cast<uint32_t>(L.Wg / tw));
+            tl.bt[c] = tt / m;
+            tl.th[c] = th;
+            tl.tw[c] = tw;
+        } else {
+            tl.divs[c] = make_tile_divs(1, 1, 1, 1, 1);
+            tl.m[c] = tl.nthw[c] = tl.ntw[c] = make_fastdiv(1);
+            tl.bt[c] = tl.th[c] = tl.tw[c] = 1;
+        }
+    }
+    centroid_kernel<D, TILED><<<dim3(nb, L.BH), 256, 0, st>>>(static_cast<const __nv_bfloat16 *>(L.k),
+                                                               static_cast<const __nv_bfloat16 *>(L.v), L.S, nb, khi,
+                                                               klo, vhi, vlo, tl);
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return check_cuda(e, "centroid launch");
 
@@ -536,11 +605,16 @@ vsa_status run_compensated(const AttnLaunch &L, void *workspace, int *status, cu
     if (s != VSA_OK) return s;
 
     CompMaps maps = {};
-    const bool ok = make_tile_map(&maps.q, L.q, D, L.S, L.BH, 128) && make_tile_map(&maps.khi, khi, D, nb, L.BH, 128) &&
-                    make_tile_map(&maps.klo, klo, D, nb, L.BH, 128) && make_tile_map(&maps.vhi, vhi, D, nb, L.BH, 128) &&
-                    make_tile_map(&maps.vlo, vlo, D, nb, L.BH, 128);
+    bool ok = make_tile_map(&maps.khi, khi, D, nb, L.BH, 128) && make_tile_map(&maps.klo, klo, D, nb, L.BH, 128) &&
+              make_tile_map(&maps.vhi, vhi, D, nb, L.BH, 128) && make_tile_map(&maps.vlo, vlo, D, nb, L.BH, 128);
+    if (TILED) {
+        for (int c = 0; ok && c < L.tiles.n; ++c)
+            ok = make_box_map(&maps.q[c], L.q, D, L.T, L.Hg, L.Wg, L.BH, tl.bt[c], tl.th[c], tl.tw[c]);
+    } else {
+        ok = ok && make_tile_map(&maps.q[0], L.q, D, L.S, L.BH, 128);
+    }
     if (!ok) return fail(VSA_ERR_CUDA, "cuTensorMapEncodeTiled failed (driver entry point or arguments)");
-    auto kern = comp_pair_kernel<D>;
+    auto kern = comp_pair_kernel<D, TILED>;
     e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
     if (e != cudaSuccess) return check_cuda(e, "cudaFuncSetAttribute(compensation pass)");
     CompArgs a;
@@ -559,7 +633,7 @@ vsa_status run_compensated(const AttnLaunch &L, void *workspace, int *status, cu
     a.out = L.o;
     a.out_f32 = L.out_f32;
     a.status = status;
-    kern<<<dim3((nb + 1) / 2, L.BH), kPairThreads, C::SMEM, st>>>(maps, a);
+    kern<<<dim3((nb + 1) / 2, L.BH), kPairThreads, C::SMEM, st>>>(maps, a, tl);
     return check_cuda(cudaGetLastError(), "compensation pass launch");
 }
 
@@ -573,7 +647,11 @@ vsa_status launch_compensated(const AttnLaunch &L, void *workspace, int *status,
     if (L.S / kBlock > kMaxCentroidTiles * kBlock)
         return fail(VSA_ERR_UNSUPPORTED, "compensated attention supports at most %d blocks per head",
                     kMaxCentroidTiles * kBlock);
-    return L.D == 128 ? run_compensated<128>(L, workspace, status, st) : run_compensated<64>(L, workspace, status, st);
+    if (L.tiled)
+        return L.D == 128 ? run_compensated<128, true>(L, workspace, status, st)
+                          : run_compensated<64, true>(L, workspace, status, st);
+    return L.D == 128 ? run_compensated<128, false>(L, workspace, status, st)
+                      : run_compensated<64, false>(L, workspace, status, st);
 }
 
 }  // namespace vsa

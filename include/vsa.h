@@ -351,6 +351,22 @@ vsa_status vsa_centroid_compensated_attention(const void *q, const void *k, cons
                                               float scale, void *workspace, size_t workspace_bytes,
                                               void *stream);
 
+/* The same in tiled mode: q, k, v and o in T-major order over `grid`, each
+ * (b, head)'s blocks those of tiles[choice[bh]] (choice NULL: tile 0), as in
+ * vsa_block_sparse_attention_tiled: the result equals vsa_permute of q, k, v,
+ * vsa_centroid_compensated_attention and vsa_unpermute of o, bit for bit,
+ * with no permuted copies.  Every tile has one volume, a multiple of 128,
+ * with tile.t divisible by volume / 128; the tiles must divide the grid (no
+ * padding).  A choice out of range leaves that head unwritten and sets
+ * VSA_ERR_RUNTIME.  Workspace, lists and errors as above.                     */
+vsa_status vsa_centroid_compensated_attention_tiled(const void *q, const void *k, const void *v, void *o,
+                                                    vsa_dtype out_dtype, int B, int n_heads, int S, int D,
+                                                    vsa_dims3 grid, const vsa_dims3 *tiles, int n_tiles,
+                                                    const int32_t *choice, const int32_t *idx,
+                                                    const int32_t *cnt, int cap, int list_per_head,
+                                                    float scale, void *workspace, size_t workspace_bytes,
+                                                    void *stream);
+
 /* Block-sparse attention on T-major q, k, v and o, with each (b, head) in its
  * own tiling and no permuted copies ("Adaptive tiling (SPADE)", Recipe: the
  * permutation, attention and inverse permutation in one pass).  Block i of

@@ -300,6 +300,26 @@ def test_compensated_attention_argument_errors(L):
     assert call(o=FAKE) == vsa.ERR_INVALID_ARGUMENT                        # o over q
 
 
+def test_compensated_tiled_argument_errors(L):
+    q, k, v, o = (ctypes.c_void_p(0x100000 * (i + 1)) for i in range(4))
+    idx, cnt = ctypes.c_void_p(0x800000), ctypes.c_void_p(0x900000)
+    ws = ctypes.c_void_p(0x10000000)
+    big = 1 << 34
+
+    def call(grid=Dims3(8, 16, 16), tiles=((1, 8, 16), (2, 8, 8)), S=2048, D=64, cap=2, wsz=big, w=ws):
+        arr, n = _tiles(*tiles)
+        return L.vsa_centroid_compensated_attention_tiled(q, k, v, o, vsa.F32, 1, 1, S, D, grid, arr, n, None,
+                                                          idx, cnt, cap, 0, 0.0, w, wsz, None)
+
+    assert call(grid=Dims3(5, 12, 20), S=1200) == vsa.ERR_UNSUPPORTED            # padded grid
+    assert call(tiles=((1, 4, 16), (2, 4, 8))) == vsa.ERR_UNSUPPORTED            # 64-token tiles
+    assert call(tiles=((1, 8, 16), (1, 8, 8))) == vsa.ERR_INVALID_ARGUMENT       # volumes differ
+    assert call(S=2000) == vsa.ERR_INVALID_ARGUMENT                              # grid product != S
+    assert call(cap=0) == vsa.ERR_INVALID_ARGUMENT
+    assert call(wsz=16) == vsa.ERR_INVALID_ARGUMENT                              # workspace too small
+    assert call(w=ctypes.c_void_p(0x100000 * 2)) == vsa.ERR_INVALID_ARGUMENT     # workspace over k
+
+
 def test_fused_scores_topk_argument_errors(L):
     def call(**kw):
         a = dict(dt=vsa.BF16, B=1, H=2, nb=240, D=128, k=24, sink=1, dw=0, cap=26)

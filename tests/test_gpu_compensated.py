@@ -214,5 +214,50 @@ def test_spade_attention_compensated_composition():
         want = np.empty_like(want_p)
         want[perm] = want_p
         assert_close(_np(o[0, h]), want, f"head {h}")
-    with pytest.raises(ValueError):
-        vsa.spade_attention(q, k, v, grid, tiles, topk=3, compensate=True, tiled=True)
+    # tiled mode: no permuted copies, the same bits
+    ot = vsa.spade_attention(q, k, v, grid, tiles, topk=3, out_dtype=torch.float32, compensate=True, tiled=True)
+    oe = vsa.spade_attention(q, k, v, grid, tiles, topk=3, out_dtype=torch.float32, compensate=True, tiled=False)
+    assert torch.equal(ot, oe) and torch.equal(ot, o)
+
+
+@pytest.mark.parametrize("D,grid,cap", [(128, (8, 16, 32), 5), (64, (16, 16, 16), 1), (128, (8, 24, 32), 1)])
+def test_compensated_tiled_equals_permuted_path(D, grid, cap):
+    """T-major q, k, v through each head's tiling give unpermute of the
+    permuted path's result bit for bit, in both output dtypes, with lists of
+    several blocks (two-tile kernel) or of one (one-key-block kernel)."""
+    tiles = [(1, 8, 16), (2, 8, 8), (4, 4, 8)]
+    B, H = 2, 2
+    S = grid[0] * grid[1] * grid[2]
+    nb = S // BLOCK
+    q, k, v = smooth_qkv(B, H, grid, D, seed=S + cap, device=DEV)
+    choice = torch.tensor([2, 0, 1, 2], dtype=torch.int32, device=DEV)
+    if cap == 1:
+        idx = np.tile(np.arange(nb, dtype=np.int32)[None, None, :, None], (B, H, 1, 1))
+        cnt = np.ones((B, H, nb), np.int32)
+    else:
+        idx_h, cnt_h = _lists(nb, cap, B * H, seed=S, keep_forced_only={nb // 3})
+        idx, cnt = idx_h.reshape(B, H, nb, cap), cnt_h.reshape(B, H, nb)
+    ti, tc = torch.tensor(idx, device=DEV), torch.tensor(cnt, device=DEV)
+    for odt in (torch.float32, torch.bfloat16):
+        ot = vsa.centroid_compensated_attention_tiled(q, k, v, grid, tiles, choice, ti, tc, out_dtype=odt)
+        qp, kp, vp = (vsa.permute(x, grid, tiles, choice) for x in (q, k, v))
+        op = vsa.centroid_compensated_attention(qp, kp, vp, ti, tc, out_dtype=odt)
+        vsa.device_status()
+        assert torch.equal(ot, vsa.unpermute(op, grid, tiles, choice)), odt
+
+
+def test_compensated_tiled_bad_choice_sets_runtime_status():
+    grid, tiles, D = (8, 16, 16), [(1, 8, 16), (2, 8, 8)], 64
+    S, nb = 2048, 16
+    q, k, v = smooth_qkv(1, 2, grid, D, seed=8, device=DEV)
+    idx = torch.arange(nb, dtype=torch.int32, device=DEV).view(nb, 1).contiguous()
+    cnt = torch.ones(nb, dtype=torch.int32, device=DEV)
+    o = vsa.centroid_compensated_attention_tiled(q, k, v, grid, tiles, torch.tensor([1, 5], dtype=torch.int32,
+                                                                                    device=DEV), idx, cnt,
+                                                 out_dtype=torch.float32)
+    with pytest.raises(RuntimeError):
+        vsa.device_status()
+    good = vsa.centroid_compensated_attention_tiled(q[:, :1], k[:, :1], v[:, :1], grid, tiles,
+                                                    torch.tensor([1], dtype=torch.int32, device=DEV), idx, cnt,
+                                                    out_dtype=torch.float32)
+    assert torch.equal(o[:, :1], good)
