@@ -628,8 +628,8 @@ def run_ours(args, w):
                                                    "same_output": bool(torch.equal(ex.last["o"], step.last["o"]))}
             del ex
         # centroid-compensated attention on the same lists: the kept blocks as
-        # above plus every skipped block as its centroid (explicit permuted
-        # copies in each head's tiling; bf16 output)
+        # above plus every skipped block as its centroid (tiled mode, each
+        # head's tiling; bf16 output)
         if "compensated" in want:
             extra["compensated_" + w.name] = compensated_line(w, q, k, v, step.last["idx"], step.last["cnt"],
                                                               max(3, args.steps // 2))
