@@ -38,7 +38,7 @@ typedef enum {
     VSA_ERR_INVALID_ARGUMENT = 1, /* bad shape, size or option (ValueError)      */
     VSA_ERR_RUNTIME = 2,          /* violated invariant seen on the device        */
     VSA_ERR_CUDA = 3,             /* CUDA runtime / launch failure                */
-    VSA_ERR_UNSUPPORTED = 4,      /* valid request this build does not implement  */
+    VSA_ERR_UNSUPPORTED = 4,      /* valid request the library does not implement */
     VSA_ERR_TIMEOUT = 5           /* a bounded on-device wait gave up             */
 } vsa_status;
 
