@@ -614,6 +614,28 @@ def _check_choice(h, gpu_choice, cohesion):
     return False
 
 
+def _near_tied(cohesion):
+    """Candidate tilings the oracle cannot separate from its own choice (within
+    CHOICE_MARGIN of the best), its argmax first: the set of correct choices,
+    decided by the oracle alone."""
+    best = int(np.argmax(cohesion))
+    return [best] + [c for c in range(len(cohesion)) if c != best and cohesion[c] >= cohesion[best] - CHOICE_MARGIN]
+
+
+def _in_some_tiling(h, cohesion, check):
+    """check(c) raises AssertionError unless the GPU's results for head h are
+    the oracle's in candidate tiling c.  Passes if they are for one of the
+    near-tied tilings (scores alone may not tell them apart: on i.i.d. grid
+    values every block summary saturates and every score is 0)."""
+    failures = []
+    for c in _near_tied(cohesion):
+        try:
+            return check(c)
+        except AssertionError as e:
+            failures.append(f"tiling {c}: {e}")
+    raise AssertionError(f"head {h}: " + "; ".join(failures))
+
+
 @pytest.mark.parametrize("values", ["integer", "integer_adaptive"])
 def test_spade_adaptive_full_size_integer_lists(values):
     """24 heads, S = 122880, three candidate tilings, k = 96, on {-4..4}/4 grid
@@ -621,8 +643,9 @@ def test_spade_adaptive_full_size_integer_lists(values):
     ("integer_adaptive", whose heads have clear tiling preferences).  Scores
     are exact, so every head's whole score matrix and its whole lists must
     equal the oracle's bit for bit; the tiling choice must equal the oracle's
-    wherever its margin is clear; sampled query blocks of every head are
-    within the attention tolerance."""
+    wherever its margin is clear (where it is not, the GPU's results must be
+    the oracle's in one of the near-tied tilings); sampled query blocks of
+    every head are within the attention tolerance."""
     w = WORKLOADS["spade_adaptive_s122880"]
     q, k, v = make_qkv(w, device=DEV, values=values)
     o, mid = vsa.spade_attention(q, k, v, w.grid, list(w.tiles), topk=w.k, out_dtype=torch.float32,
@@ -634,12 +657,18 @@ def test_spade_adaptive_full_size_integer_lists(values):
         _, cohesion = oracle.select_tiling(qh, w.grid, list(w.tiles))
         clear += _check_choice(h, int(choice[h]), cohesion)
         blocks = _sample_blocks(w.nb, 300 + h, n=16 if h in (0, 13) else 4)
-        res = oracle.spade_head(qh, kh, vh, w.grid, [w.tiles[int(choice[h])]], w.k, query_blocks=blocks)
-        assert np.array_equal(_np(mid["scores"][0, h]).astype(np.float64), res["score"]), h
-        assert np.array_equal(mid["idx"][0, h].cpu().numpy(), res["idx"]), h
-        assert np.array_equal(mid["cnt"][0, h].cpu().numpy(), res["cnt"]), h
-        got = _np(mid["out_perm"][0, h])[res["rows"]]
-        assert_attn_close(got, res["out_perm"], f"head {h}")
+        got_scores = _np(mid["scores"][0, h]).astype(np.float64)
+        got_idx, got_cnt = mid["idx"][0, h].cpu().numpy(), mid["cnt"][0, h].cpu().numpy()
+        got_out = _np(mid["out_perm"][0, h])
+
+        def check(c):
+            res = oracle.spade_head(qh, kh, vh, w.grid, [w.tiles[c]], w.k, query_blocks=blocks)
+            assert np.array_equal(got_scores, res["score"]), "scores"
+            assert np.array_equal(got_idx, res["idx"]), "idx"
+            assert np.array_equal(got_cnt, res["cnt"]), "cnt"
+            assert_attn_close(got_out[res["rows"]], res["out_perm"], "attention")
+
+        _in_some_tiling(h, cohesion, check)
     if values == "integer_adaptive":
         assert clear == w.heads and len(set(choice.tolist())) >= 2
 
@@ -651,8 +680,9 @@ def test_spade_adaptive_full_size_sampled():
     the exact one; every list is a valid top-k set under the oracle's scores
     (a block may differ from the oracle's list only where its score and the
     k-th score lie within that allowance of each other); sampled query blocks
-    are compared with the oracle's attention over the GPU's own lists, so that
-    near-tie flips are not mistaken for attention error."""
+    whose list equals the oracle's are compared with the oracle's attention
+    over its own lists (a block whose list flipped at a near-tie was checked
+    valid above; at most one per head may be left out)."""
     w = WORKLOADS["spade_adaptive_s122880"]
     q, k, v = make_qkv(w, device=DEV)
     o, mid = vsa.spade_attention(q, k, v, w.grid, list(w.tiles), topk=w.k, out_dtype=torch.float32,
@@ -668,32 +698,44 @@ def test_spade_adaptive_full_size_sampled():
     differing_rows = 0
     for h in (0, 13, 22):
         qh, kh, vh = (_np(x[0, h]) for x in (q, k, v))
-        tile = w.tiles[int(choice[h])]
+        _, cohesion = oracle.select_tiling(qh, w.grid, list(w.tiles))
         blocks = _sample_blocks(w.nb, 100 + h)
-        res = oracle.spade_head(qh, kh, vh, w.grid, [tile], w.k, query_blocks=blocks[:1])
-        s, terms = res["score"], _abs_terms(res)
-        bound = SCORE_EPS * terms
-        err = np.abs(_np(mid["scores"][0, h]).astype(np.float64) - s)
-        assert (err <= bound).all(), f"head {h}: score error {np.max(err / np.maximum(terms, 1e-30)):.3e} x sum|terms|"
-        gi = mid["idx"][0, h].cpu().numpy()
-        gc = mid["cnt"][0, h].cpu().numpy()
-        for i in range(w.nb):
-            sel = set(gi[i, :gc[i]].tolist())
-            forced = {0, i}
-            assert forced <= sel and w.k <= len(sel) <= w.k + len(forced)
-            order = np.lexsort((np.arange(w.nb), -s[i]))      # descending score, ties: lower index
-            kth = order[w.k - 1]
-            tol = bound[i] + bound[i, kth]
-            assert all(s[i, j] >= s[i, kth] - tol[j] for j in sel - forced), (h, i)
-            assert all(s[i, j] <= s[i, kth] + tol[j] for j in set(range(w.nb)) - sel), (h, i)
-            differing_rows += int(not np.array_equal(gi[i], res["idx"][i]))
-        perm = oracle.tile_permutation(w.grid, tile)
-        qp, kp, vp = (oracle.permute_rows(x, perm) for x in (qh, kh, vh))
-        rows = np.concatenate([np.arange(b * 128, (b + 1) * 128) for b in blocks])
-        want = oracle.block_sparse_attention(qp, kp, vp, gi, gc, 128, 0, None, rows)
-        got = _np(mid["out_perm"][0, h])[rows]
-        for bi, b in enumerate(blocks):
-            assert_attn_close(got[bi * 128:(bi + 1) * 128], want[bi * 128:(bi + 1) * 128], f"head {h} block {b}")
+        got_scores = _np(mid["scores"][0, h]).astype(np.float64)
+        gi, gc = mid["idx"][0, h].cpu().numpy(), mid["cnt"][0, h].cpu().numpy()
+        got_out = _np(mid["out_perm"][0, h])
+
+        def check(c):
+            tile = w.tiles[c]
+            res = oracle.spade_head(qh, kh, vh, w.grid, [tile], w.k, query_blocks=blocks[:1])
+            s, terms = res["score"], _abs_terms(res)
+            bound = SCORE_EPS * terms
+            err = np.abs(got_scores - s)
+            assert (err <= bound).all(), f"score error {np.max(err / np.maximum(terms, 1e-30)):.3e} x sum|terms|"
+            differing = 0
+            for i in range(w.nb):
+                sel = set(gi[i, :gc[i]].tolist())
+                forced = {0, i}
+                assert forced <= sel and w.k <= len(sel) <= w.k + len(forced), i
+                order = np.lexsort((np.arange(w.nb), -s[i]))      # descending score, ties: lower index
+                kth = order[w.k - 1]
+                tol = bound[i] + bound[i, kth]
+                assert all(s[i, j] >= s[i, kth] - tol[j] for j in sel - forced), i
+                assert all(s[i, j] <= s[i, kth] + tol[j] for j in set(range(w.nb)) - sel), i
+                differing += int(not np.array_equal(gi[i], res["idx"][i]))
+            perm = oracle.tile_permutation(w.grid, tile)
+            qp, kp, vp = (oracle.permute_rows(x, perm) for x in (qh, kh, vh))
+            rows = np.concatenate([np.arange(b * 128, (b + 1) * 128) for b in blocks])
+            want = oracle.block_sparse_attention(qp, kp, vp, res["idx"], res["cnt"], 128, 0, None, rows)
+            got = got_out[rows]
+            compared = 0
+            for bi, b in enumerate(blocks):
+                if np.array_equal(gi[b], res["idx"][b]):
+                    assert_attn_close(got[bi * 128:(bi + 1) * 128], want[bi * 128:(bi + 1) * 128], f"block {b}")
+                    compared += 1
+            assert compared >= len(blocks) - 1, (compared, len(blocks))
+            return differing
+
+        differing_rows += _in_some_tiling(h, cohesion, check)
     print(f"rows whose list differs from the oracle's by near-ties: {differing_rows} of {3 * w.nb}")
 
 
