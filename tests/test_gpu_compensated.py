@@ -196,24 +196,36 @@ def test_compensated_adaptive_full_size_sampled():
 def test_spade_attention_compensated_composition():
     """spade_attention(compensate=True): tiling choice, permutation, scores,
     top-k lists and the compensated attention, back in T-major order, against
-    the oracle's steps on every head (integer-grid values: exact lists)."""
+    the oracle's steps on every head (integer-grid values: exact lists), in
+    the oracle's tiling or in one within 1e-5 of its best cohesion (the
+    tiling choice's fp32 resolution), a set the oracle alone decides."""
     grid, tiles = (8, 16, 16), [(1, 8, 16), (2, 8, 8), (4, 4, 8)]
     q = integer_grid((1, 3, 2048, 64), 51, torch.bfloat16, DEV)
     k = integer_grid((1, 3, 2048, 64), 52, torch.bfloat16, DEV)
     v = integer_grid((1, 3, 2048, 64), 53, torch.bfloat16, DEV)
     o, mid = vsa.spade_attention(q, k, v, grid, tiles, topk=3, out_dtype=torch.float32, compensate=True,
                                  return_intermediates=True)
-    choice = mid["choice"].cpu().numpy()
     for h in range(3):
         qh, kh, vh = (_np(x[0, h]) for x in (q, k, v))
-        res = oracle.spade_head(qh, kh, vh, grid, [tiles[int(choice[h])]], 3, query_blocks=[0])
-        assert np.array_equal(mid["idx"][0, h].cpu().numpy(), res["idx"])
-        perm = res["perm"]
-        qp, kp, vp = (oracle.permute_rows(x, perm) for x in (qh, kh, vh))
-        want_p = _oracle_rows(qp, kp, vp, res["idx"], res["cnt"])
-        want = np.empty_like(want_p)
-        want[perm] = want_p
-        assert_close(_np(o[0, h]), want, f"head {h}")
+        _, cohesion = oracle.select_tiling(qh, grid, tiles)
+        best = int(np.argmax(cohesion))
+        near = [best] + [c for c in range(len(tiles)) if c != best and cohesion[c] >= cohesion[best] - 1e-5]
+        failures = []
+        for c in near:
+            res = oracle.spade_head(qh, kh, vh, grid, [tiles[c]], 3, query_blocks=[0])
+            perm = res["perm"]
+            qp, kp, vp = (oracle.permute_rows(x, perm) for x in (qh, kh, vh))
+            want_p = _oracle_rows(qp, kp, vp, res["idx"], res["cnt"])
+            want = np.empty_like(want_p)
+            want[perm] = want_p
+            try:
+                assert np.array_equal(mid["idx"][0, h].cpu().numpy(), res["idx"]), "lists"
+                assert_close(_np(o[0, h]), want, "attention")
+                break
+            except AssertionError as e:
+                failures.append(f"tiling {c}: {e}")
+        else:
+            raise AssertionError(f"head {h}: " + "; ".join(failures))
     # tiled mode: no permuted copies, the same bits
     ot = vsa.spade_attention(q, k, v, grid, tiles, topk=3, out_dtype=torch.float32, compensate=True, tiled=True)
     oe = vsa.spade_attention(q, k, v, grid, tiles, topk=3, out_dtype=torch.float32, compensate=True, tiled=False)
