@@ -168,26 +168,40 @@ def test_compensated_invalid_list_writes_zeros_and_sets_status():
 
 
 def test_compensated_adaptive_full_size_sampled():
-    """The S = 122880 adaptive workload in each head's chosen tiling (explicit
-    permuted copies), top-k lists with k = 96: sampled query blocks of two
-    heads, one of them keeping only its sink and diagonal blocks."""
+    """The S = 122880 adaptive workload in each head's tiling (explicit
+    permuted copies) with its top-k lists, k = 96, both taken from the oracle
+    and given to the GPU as inputs: sampled query blocks of two heads, one of
+    them keeping only its sink and diagonal blocks."""
     w = WORKLOADS["spade_adaptive_s122880"]
-    q, k, v = make_qkv(w, device=DEV, heads=4)
-    choice = vsa.select_tiling(q, w.grid, list(w.tiles))
-    qp, kp, vp = (vsa.permute(x, w.grid, list(w.tiles), choice) for x in (q, k, v))
-    qmax, qmin = vsa.block_summaries(qp, BLOCK)
-    kmax, kmin = vsa.block_summaries(kp, BLOCK)
-    idx, cnt = vsa.topk_block_mask(vsa.block_scores(qmax, qmin, kmax, kmin), w.k)
+    H = 4
+    q, k, v = make_qkv(w, device=DEV, heads=H)
+    choices, perms, idx_o, cnt_o = [], [], [], []
+    for h in range(H):
+        qh, kh = _np(q[0, h]), _np(k[0, h])
+        c, _ = oracle.select_tiling(qh, w.grid, list(w.tiles))
+        perm = oracle.tile_permutation(w.grid, w.tiles[c])
+        qmax, qmin = oracle.block_minmax(oracle.permute_rows(qh, perm), BLOCK)
+        kmax, kmin = oracle.block_minmax(oracle.permute_rows(kh, perm), BLOCK)
+        i_, c_ = oracle.topk_block_list(oracle.block_scores(qmax, qmin, kmax, kmin), w.k)
+        choices.append(c)
+        perms.append(perm)
+        idx_o.append(i_)
+        cnt_o.append(c_)
+    idx_np, cnt_np = np.stack(idx_o), np.stack(cnt_o)
     # head 3: query block 500 keeps only its forced blocks (0 and 500)
-    idx[0, 3, 500].fill_(-1)
-    idx[0, 3, 500, :2] = torch.tensor([0, 500], dtype=torch.int32)
-    cnt[0, 3, 500] = 2
+    idx_np[3, 500] = -1
+    idx_np[3, 500, :2] = (0, 500)
+    cnt_np[3, 500] = 2
+    choice = torch.tensor(choices, dtype=torch.int32, device=DEV)
+    qp, kp, vp = (vsa.permute(x, w.grid, list(w.tiles), choice) for x in (q, k, v))
+    idx = torch.as_tensor(idx_np, device=DEV).view(1, H, w.nb, -1)
+    cnt = torch.as_tensor(cnt_np, device=DEV).view(1, H, w.nb)
     o = vsa.centroid_compensated_attention(qp, kp, vp, idx, cnt, out_dtype=torch.float32)
     for h in (1, 3):
         blocks = [0, 17, 500, 958, w.nb - 1]
         rows = np.concatenate([np.arange(b * BLOCK, (b + 1) * BLOCK) for b in blocks])
-        want = _oracle_rows(_np(qp[0, h]), _np(kp[0, h]), _np(vp[0, h]), idx[0, h].cpu().numpy(),
-                            cnt[0, h].cpu().numpy(), rows)
+        qo, ko, vo = (oracle.permute_rows(_np(x[0, h]), perms[h]) for x in (q, k, v))
+        want = _oracle_rows(qo, ko, vo, idx_np[h], cnt_np[h], rows)
         got = _np(o[0, h])[rows]
         for bi, b in enumerate(blocks):
             assert_close(got[bi * BLOCK:(bi + 1) * BLOCK], want[bi * BLOCK:(bi + 1) * BLOCK], f"head {h} block {b}")

@@ -898,12 +898,12 @@ def test_spade_top_p_end_to_end():
     o, mid = vsa.spade_attention(q, k, v, w.grid, list(w.tiles), top_p=0.6, top_p_scale=0.25,
                                  out_dtype=torch.float32, return_intermediates=True)
     for h in range(w.heads):
-        s = _np(mid["scores"][0, h]).astype(np.float64)
+        perm = oracle.tile_permutation(w.grid, w.tiles[0])
+        qo, ko, vo = (oracle.permute_rows(_np(x[0, h]), perm) for x in (q, k, v))
+        s = oracle.block_scores(*oracle.block_minmax(qo, w.block), *oracle.block_minmax(ko, w.block))
         oi, oc = oracle.topp_block_list(s, 0.6, 0.25, 1, 0)
         gi, gc = mid["idx"][0, h].cpu().numpy(), mid["cnt"][0, h].cpu().numpy()
         assert np.array_equal(gc, oc) and all(np.array_equal(gi[i, :gc[i]], oi[i, :oc[i]]) for i in range(len(gc)))
-        perm = oracle.tile_permutation(w.grid, w.tiles[0])
-        qo, ko, vo = (oracle.permute_rows(_np(x[0, h]), perm) for x in (q, k, v))
         want = oracle.block_sparse_attention(qo, ko, vo, oi, oc, w.block)
         assert_attn_close(_np(o[0, h])[perm], want, f"head {h}")
 
@@ -934,14 +934,17 @@ def test_one_block_lists_match_two_tile_kernel_and_oracle(mode, grid):
     ti2 = torch.as_tensor(np.concatenate([idx1[..., None], np.full((H, nb, 1), -1, np.int32)], -1),
                           device=DEV).view(B, H, nb, 2)
     tc = torch.as_tensor(cnt, device=DEV).view(B, H, nb)
+    opg = tuple(oracle.padded_grid(grid, tiles))   # the oracle's own padded grid
+    assert tuple(pg) == opg
     if mode == "permuted":
         qp, kp, vp = (vsa.permute(x, grid, tiles[:1]) for x in (q, k, v))
         o1 = vsa.block_sparse_attention(qp, kp, vp, ti1, tc, 128, out_dtype=torch.float32)
         o2 = vsa.block_sparse_attention(qp, kp, vp, ti2, tc, 128, out_dtype=torch.float32)
         assert torch.equal(o1, o2)
+        perm = oracle.tile_permutation(grid, tiles[0])
         for h in range(H):
-            want = oracle.block_sparse_attention(_np(qp[0, h]), _np(kp[0, h]), _np(vp[0, h]), idx1[h][:, None],
-                                                 cnt[h], 128)
+            qo, ko, vo = (oracle.permute_rows(_np(x[0, h]), perm) for x in (q, k, v))
+            want = oracle.block_sparse_attention(qo, ko, vo, idx1[h][:, None], cnt[h], 128)
             assert_attn_close(_np(o1[0, h]), want, f"head {h}")
         return
     choice = torch.tensor([0, 1, 2], dtype=torch.int32, device=DEV)
@@ -951,12 +954,12 @@ def test_one_block_lists_match_two_tile_kernel_and_oracle(mode, grid):
     ob = vsa.block_sparse_attention_tiled(q, k, v, grid, tiles, choice, ti1, tc, out_dtype=torch.bfloat16)
     assert torch.equal(ob, o1.to(torch.bfloat16))
     for h, c in enumerate(choice.tolist()):
-        perm = oracle.tile_permutation(pg, tiles[c])
-        real = oracle.real_tokens(grid, pg)
-        qo, ko, vo = (oracle.permute_rows(oracle.pad_grid(_np(x[0, h]), grid, pg), perm) for x in (q, k, v))
+        perm = oracle.tile_permutation(opg, tiles[c])
+        real = oracle.real_tokens(grid, opg)
+        qo, ko, vo = (oracle.permute_rows(oracle.pad_grid(_np(x[0, h]), grid, opg), perm) for x in (q, k, v))
         want_p = oracle.block_sparse_attention(qo, ko, vo, idx1[h][:, None], cnt[h], 128,
                                                key_ok=real[perm].astype(np.uint8) if mode == "padded" else None)
-        want = np.zeros((pg[0] * pg[1] * pg[2], D))
+        want = np.zeros((opg[0] * opg[1] * opg[2], D))
         want[perm] = want_p
         assert_attn_close(_np(o1[0, h]), want[real], f"head {h}")
 
